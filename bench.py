@@ -1,0 +1,447 @@
+#!/usr/bin/env python
+"""Throughput of Qwen Sparse Attention (QSA) on B200 through the C ABI.
+
+One step = one full QSA call over one batch of synthetic input: pooling,
+indexer scoring, top-k selection, sparse attention and the sigmoid gate
+(qsa_prefill for prefill workloads, qsa_decode for decode workloads).
+The metric counts selected-KV tokens: the sum over query tokens of the number
+of keys each query attends, |S(t)| = min(k, floor(n/B)) * B + n mod B.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                  [--impl ours|reference]
+
+Under torchrun every rank runs its own copy of the workload (independent
+problems, no collective on the data path: weak scaling); the reported value is
+all ranks' tokens over the slowest rank's device time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from block_sparse_attention_17_b200.workloads import (WORKLOADS, make_decode_inputs,  # noqa: E402
+                                                      make_prefill_inputs, resolve_seqlens)
+
+METRIC = "QSA selected-KV tokens/s (prefill, decode) + µs/decode step; % HBM/TC roofline"
+UNIT = "selected-KV tokens/s"
+DEFAULT_WORKLOAD = "prefill_bf16_t8192"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ------------------------------------------------------------------ helpers
+def selected_tokens(n: int, B: int, k: int) -> int:
+    nc = n // B
+    return min(k, nc) * B + n % B
+
+
+def workload_units(w):
+    """Selected-KV tokens per step and the list of visible lengths."""
+    if w.kind == "prefill":
+        seqlens, _ = resolve_seqlens(w)
+        ns = [p + 1 for L in seqlens for p in range(L)]
+    else:
+        ns = [w.kv_len - w.n_q + 1 + i for _ in range(w.batch) for i in range(w.n_q)]
+    return sum(selected_tokens(n, w.block_size, w.topk) for n in ns), ns
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def config_of(w, extra=None):
+    c = {"workload": w.name, "kind": w.kind, "dtype": w.dtype, "Hq": w.num_q_heads,
+         "Hkv": w.num_kv_heads, "head_dim": w.head_dim, "block_size": w.block_size,
+         "budget": w.budget, "idx_heads": w.idx_heads, "idx_dim": w.idx_dim, "seed": w.seed}
+    if w.kind == "prefill":
+        seqlens, _ = resolve_seqlens(w)
+        c.update(seqlens=list(seqlens), global_batch=len(seqlens), seq_len=max(seqlens))
+    else:
+        c.update(batch=w.batch, kv_len=w.kv_len, n_q=w.n_q, global_batch=w.batch,
+                 seq_len=w.kv_len)
+    if extra:
+        c.update(extra)
+    return c
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during timing."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_id: str):
+        self.device_id = device_id
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                   "-lms", "100"]
+            if self.device_id:
+                cmd += ["-i", self.device_id]
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[3:7]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------ cpu baseline
+def oracle_sample(w, inp, budget_s: float, max_queries=None, seed=0):
+    """Time the fp64 oracle, as it stands, on an evenly spread sample of the
+    workload's queries until about budget_s seconds of CPU work are done.
+    Returns (selected tokens processed, seconds, queries, cores)."""
+    from threadpoolctl import threadpool_limits
+    from oracle import qsa_oracle as O
+    rng = np.random.default_rng(seed)
+    if w.kind == "prefill":
+        T = int(inp["cu_seqlens"][-1])
+        order = rng.permutation(T)
+    else:
+        pairs = [(b, i) for b in range(w.batch) for i in range(w.n_q)]
+        order = [pairs[j] for j in rng.permutation(len(pairs))]
+    done, toks = 0, 0
+    chunk = 16
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        for c0 in range(0, len(order), chunk):
+            items = order[c0:c0 + chunk]
+            if w.kind == "prefill":
+                res = O.qsa_prefill(w, inp, queries=[int(x) for x in items])["queries"]
+            else:
+                res = O.qsa_decode(w, inp, pairs=[tuple(x) for x in items])["queries"]
+            toks += sum(r.tokens for r in res.values())
+            done += len(items)
+            el = time.perf_counter() - t0
+            if el >= budget_s or (max_queries and done >= max_queries):
+                break
+        el = time.perf_counter() - t0
+    return toks, el, done, 1
+
+
+# ------------------------------------------------------------------ ours
+def run_ours(args, w, rank, world, dist):
+    import torch
+    import block_sparse_attention_17_b200 as qsa
+    from block_sparse_attention_17_b200 import _lib
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    lib = _lib.lib()
+    peaks, peak_kind = load_peaks()
+    cfg = qsa.QSAConfig.from_workload(w)
+    dt = cfg.dtype
+    units, ns = workload_units(w)
+
+    t_gen = time.perf_counter()
+    inp = make_prefill_inputs(w) if w.kind == "prefill" else make_decode_inputs(w)
+    t_gen = time.perf_counter() - t_gen
+    host = {}
+    for name, arr in inp.items():
+        if not isinstance(arr, np.ndarray) or name == "seqlens":
+            continue
+        t = torch.from_numpy(np.ascontiguousarray(arr))
+        if arr.dtype == np.float32 and name != "iw":
+            t = t.to(dt)
+        host[name] = t.pin_memory()
+    d = {k: v.to(dev, non_blocking=True) for k, v in host.items()}
+    torch.cuda.synchronize()
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    ev_stage = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    arr_t = (ctypes_voidp_array([e.cuda_event for e in ev_stage]))
+
+    if w.kind == "prefill":
+        T = host["q"].shape[0]
+        out = torch.empty_like(d["q"])
+        ws = torch.empty(qsa.prefill_workspace_size(cfg, len(inp["seqlens"]), T,
+                                                    inp["max_seqlen"]), dtype=torch.uint8,
+                         device=dev)
+
+        def step(dd=d, o=out):
+            qsa.prefill(cfg, dd["q"], dd["k"], dd["v"], dd["iq"], dd["ik"], dd["iw"], dd["gate"],
+                        dd["cu_seqlens"], inp["max_seqlen"], out=o, workspace=ws)
+        flops = 4.0 * w.head_dim * w.num_q_heads * units
+        alg = {"bound": "tensor", "work": flops, "peak_key": "bf16_tflops", "unit": "TFLOP/s"}
+        in_names = ["q", "k", "v", "iq", "ik", "iw", "gate", "cu_seqlens"]
+    else:
+        kv = d["kv_len"]
+        pooled = qsa.pool_build(cfg, d["ik_cache"], (kv - w.n_q).to(torch.int32))
+        out = torch.empty_like(d["q"])
+        ws = torch.empty(qsa.decode_workspace_size(cfg, w.batch, w.n_q, inp["cap"]),
+                         dtype=torch.uint8, device=dev)
+        sel = torch.empty(w.batch, w.n_q, w.topk + 1, dtype=torch.int32, device=dev)
+        nsel = torch.empty(w.batch, w.n_q, dtype=torch.int32, device=dev)
+
+        def step(dd=d, o=out):
+            qsa.decode(cfg, dd["q"], dd["k_cache"], dd["v_cache"], dd["iq"], dd["ik_cache"],
+                       dd["iw"], dd["gate"], pooled, dd["kv_len"], out=o, sel=sel, nsel=nsel,
+                       workspace=ws)
+        step()
+        torch.cuda.synchronize()
+        kv_bytes = decode_selected_kv_bytes(w, sel.cpu().numpy(), nsel.cpu().numpy(),
+                                            inp["kv_len"])
+        esz = 2 if w.dtype == "bf16" else 4
+        io = w.batch * w.n_q * (2 * w.num_q_heads * w.head_dim * esz)   # q + out
+        io += w.batch * w.n_q * w.num_q_heads * w.head_dim * esz         # gate
+        alg = {"bound": "hbm", "work": kv_bytes + io, "peak_key": "hbm_gbs", "unit": "GB/s"}
+        in_names = ["q", "iq", "iw", "gate", "kv_len"]   # one decode step's new inputs
+
+    # warm-up
+    for _ in range(max(args.warmup, 0)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+
+    lib.qsa_set_stage_events(arr_t, 3)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    stage_attn = []
+    dev_id = ""
+    try:
+        dev_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid).replace("GPU-", "")
+    except Exception:
+        dev_id = str(local)
+    clocks = ClockSampler(dev_id)
+    clocks.start()
+    n0 = lib.qsa_kernel_launch_count()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+        torch.cuda.synchronize()       # read this step's stage events before reuse
+        stage_attn.append(ev_stage[1].elapsed_time(ev_stage[2]))
+    torch.cuda.synchronize()
+    launches = lib.qsa_kernel_launch_count() - n0
+    clk = clocks.stop()
+    lib.qsa_set_stage_events(None, 0)
+    step_ms = [starts[i].elapsed_time(ends[i]) for i in range(args.steps)]
+    total_ms = float(sum(step_ms))
+    if dist is not None:
+        import torch.distributed as tdist
+        t = torch.tensor([total_ms], device=dev)
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        dist.barrier()
+    value = units * args.steps * world / (total_ms / 1e3)
+
+    # roofline of the dominant kernel: attention (+ combine for decode)
+    attn_ms = float(np.mean(stage_attn))
+    peak = float(peaks.get(alg["peak_key"], FALLBACK_PEAKS[alg["peak_key"]]))
+    if alg["bound"] == "tensor":
+        achieved = alg["work"] / (attn_ms / 1e3) / 1e12
+    else:
+        achieved = alg["work"] / (attn_ms / 1e3) / 1e9
+    roof = {"bound": alg["bound"], "achieved": round(achieved, 3), "peak": peak,
+            "unit": alg["unit"], "frac": round(achieved / peak, 5), "traffic": None,
+            "kernel": "qsa attention" + (" + combine" if w.kind == "decode" else ""),
+            "kernel_ms": round(attn_ms, 5), "peak_source": f"{peak_kind} ({alg['peak_key']})",
+            "algorithmic_per_launch": alg["work"]}
+
+    # end to end: pinned host inputs -> device, the call, result -> host
+    e2e = None
+    if not args.no_e2e:
+        out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        h2d = sum(host[n].numel() * host[n].element_size() for n in in_names)
+        d2h = out_host.numel() * out_host.element_size()
+        e_st = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        e_en = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        for i in range(args.steps + 1):
+            flush.zero_()
+            if i > 0:
+                e_st[i - 1].record(stream)
+            for n in in_names:
+                d[n].copy_(host[n], non_blocking=True)
+            step()
+            out_host.copy_(out, non_blocking=True)
+            if i > 0:
+                e_en[i - 1].record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = float(sum(e_st[i].elapsed_time(e_en[i]) for i in range(args.steps)))
+        if dist is not None:
+            import torch.distributed as tdist
+            t = torch.tensor([e2e_ms], device=dev)
+            tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": units * args.steps * world / (e2e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": e2e_ms / args.steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        toks, secs, nq, cores = oracle_sample(w, inp, args.cpu_seconds)
+        cpu = {"value": toks / secs, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"{nq} query tokens drawn at random from this workload, fp64 numpy "
+                         f"oracle, {secs:.1f} s"}
+
+    extra = {"l2": "flushed before every timed step (256 MiB write, outside the events)",
+             "selected_kv_tokens_per_step": units, "input_gen_s": round(t_gen, 2)}
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic (seeded numpy draws, shapes of the workload)",
+            "config": config_of(w, extra), "parallelism": f"replicas{world}",
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": int(launches), "clocks": clk, "impl": "ours"}
+    if w.kind == "decode":
+        line["us_per_decode_step"] = total_ms / args.steps * 1e3
+    return line
+
+
+def ctypes_voidp_array(ptrs):
+    import ctypes
+    arr = (ctypes.c_void_p * len(ptrs))(*[ctypes.c_void_p(p) for p in ptrs])
+    return ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
+
+
+def decode_selected_kv_bytes(w, sel, nsel, kv_len):
+    """Distinct visible K/V bytes the step must read: per sequence, the union
+    over its new queries of their selected tokens, times Hkv heads, K and V."""
+    esz = 2 if w.dtype == "bf16" else 4
+    B = w.block_size
+    total = 0
+    for b in range(w.batch):
+        toks = set()
+        for i in range(w.n_q):
+            n = int(kv_len[b]) - w.n_q + 1 + i
+            nc = n // B
+            for e in range(int(nsel[b, i])):
+                blk = int(sel[b, i, e])
+                hi = min((blk + 1) * B, n) if blk == nc else (blk + 1) * B
+                toks.update(range(blk * B, hi))
+        total += len(toks)
+    return total * w.num_kv_heads * w.head_dim * 2 * esz
+
+
+# ------------------------------------------------------------- reference arm
+def run_reference(args, w):
+    """The fp64 oracle, as it stands, on the host cores: each step is a bounded
+    random sample of the workload's queries."""
+    inp = make_prefill_inputs(w) if w.kind == "prefill" else make_decode_inputs(w)
+    per_step_s = args.ref_step_seconds
+    tot_tok, tot_s, tot_q = 0, 0.0, 0
+    for i in range(args.warmup + args.steps):
+        toks, secs, nq, cores = oracle_sample(w, inp, per_step_s, seed=1000 + i)
+        if i >= args.warmup:
+            tot_tok += toks
+            tot_s += secs
+            tot_q += nq
+    value = tot_tok / tot_s
+    sample = (f"{tot_q} query tokens over {args.steps} steps (~{per_step_s:.1f} s each), drawn at "
+              f"random from this workload, fp64 numpy oracle, 1 thread")
+    return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": tot_s / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded numpy draws, shapes of the workload)",
+            "config": config_of(w), "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=2.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    w = WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, w)))
+        return 0
+
+    dist = None
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        dist = tdist
+    try:
+        line = run_ours(args, w, rank, world, dist)
+        if rank == 0:
+            print(json.dumps(line))
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

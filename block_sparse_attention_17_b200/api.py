@@ -1,0 +1,265 @@
+"""Python binding of the QSA C ABI (argument marshalling only).
+
+Every function takes CUDA torch tensors, allocates any output the caller did
+not pass (torch is used for device memory and streams only), and calls the
+matching entry point of libqsa.so on the current stream. Each step of the
+computation runs in the library's CUDA kernels; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+from . import _lib
+
+_DT = {torch.float32: _lib.QSA_F32, torch.bfloat16: _lib.QSA_BF16}
+
+
+@dataclass(frozen=True)
+class QSAConfig:
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    idx_heads: int
+    idx_dim: int
+    block_size: int
+    budget: int
+    softmax_scale: float = 0.0     # 0 => head_dim ** -0.5
+    index_scale: float = 0.0       # 0 => idx_dim ** -0.5
+    gate_headwise: bool = False
+    dtype: torch.dtype = torch.bfloat16
+
+    @property
+    def topk(self) -> int:
+        return self.budget // self.block_size
+
+    @classmethod
+    def from_workload(cls, w) -> "QSAConfig":
+        return cls(num_q_heads=w.num_q_heads, num_kv_heads=w.num_kv_heads,
+                   head_dim=w.head_dim, idx_heads=w.idx_heads, idx_dim=w.idx_dim,
+                   block_size=w.block_size, budget=w.budget,
+                   gate_headwise=bool(w.gate_headwise),
+                   dtype=torch.bfloat16 if w.dtype == "bf16" else torch.float32)
+
+    def c(self) -> _lib.QsaConfigC:
+        if self.dtype not in _DT:
+            raise TypeError(f"unsupported dtype {self.dtype}")
+        return _lib.QsaConfigC(self.num_q_heads, self.num_kv_heads, self.head_dim,
+                               self.idx_heads, self.idx_dim, self.block_size, self.budget,
+                               float(self.softmax_scale), float(self.index_scale),
+                               int(bool(self.gate_headwise)), _DT[self.dtype])
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]):
+    if workspace is not None:
+        if workspace.numel() * workspace.element_size() < nbytes:
+            raise ValueError(f"workspace smaller than {nbytes} bytes")
+        return workspace
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def prefill_workspace_size(cfg: QSAConfig, batch: int, total_tokens: int, max_seqlen: int) -> int:
+    c = cfg.c()
+    n = _lib.lib().qsa_prefill_workspace_size(ctypes.byref(c), batch, total_tokens, max_seqlen)
+    if n == 0 and total_tokens > 0:
+        _lib.check(_lib.QSA_ERR_INVALID_ARG, "qsa_prefill_workspace_size")
+    return int(n)
+
+
+def decode_workspace_size(cfg: QSAConfig, batch: int, n_q: int, cap: int) -> int:
+    c = cfg.c()
+    n = _lib.lib().qsa_decode_workspace_size(ctypes.byref(c), batch, n_q, cap)
+    if n == 0 and batch > 0:
+        _lib.check(_lib.QSA_ERR_INVALID_ARG, "qsa_decode_workspace_size")
+    return int(n)
+
+
+def _check_prefill(cfg, q, k, v, iq, ik, iw, gate, cu_seqlens):
+    T = q.shape[0]
+    dt = cfg.dtype
+    _need(q, "q", dt, (T, cfg.num_q_heads, cfg.head_dim))
+    _need(k, "k", dt, (T, cfg.num_kv_heads, cfg.head_dim))
+    _need(v, "v", dt, (T, cfg.num_kv_heads, cfg.head_dim))
+    _need(iq, "iq", dt, (T, cfg.idx_heads, cfg.idx_dim))
+    _need(ik, "ik", dt, (T, cfg.idx_dim))
+    _need(iw, "iw", torch.float32, (T, cfg.idx_heads))
+    if gate is not None:
+        _need(gate, "gate", dt, (T, cfg.num_q_heads) if cfg.gate_headwise
+              else (T, cfg.num_q_heads, cfg.head_dim))
+    _need(cu_seqlens, "cu_seqlens", torch.int32)
+    return T, cu_seqlens.shape[0] - 1
+
+
+def prefill(cfg: QSAConfig, q, k, v, iq, ik, iw, gate, cu_seqlens, max_seqlen: int, *,
+            out=None, lse=None, sel=None, nsel=None, pooled=None, workspace=None,
+            want_lse=False, want_sel=False, want_pooled=False, stream=None) -> dict:
+    """QSA prefill over packed sequences (qsa_prefill). Returns a dict with
+    "out" and, when requested or passed in, "lse", "sel", "nsel", "pooled"."""
+    T, batch = _check_prefill(cfg, q, k, v, iq, ik, iw, gate, cu_seqlens)
+    dev = q.device
+    K1 = cfg.topk + 1
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(T, cfg.num_q_heads, dtype=torch.float32, device=dev)
+    if sel is None and want_sel:
+        sel = torch.empty(T, K1, dtype=torch.int32, device=dev)
+    if nsel is None and want_sel:
+        nsel = torch.empty(T, dtype=torch.int32, device=dev)
+    if pooled is None and want_pooled:
+        nb = -(-max_seqlen // cfg.block_size)
+        pooled = torch.zeros(batch, nb, cfg.idx_dim, dtype=torch.float32, device=dev)
+    ws_bytes = prefill_workspace_size(cfg, batch, T, max_seqlen)
+    ws = _workspace(ws_bytes, dev, workspace)
+    c = cfg.c()
+    st = _lib.lib().qsa_prefill(ctypes.byref(c), batch, T, int(max_seqlen), _ptr(cu_seqlens),
+                                _ptr(q), _ptr(k), _ptr(v), _ptr(iq), _ptr(ik), _ptr(iw),
+                                _ptr(gate), _ptr(out), _ptr(lse), _ptr(sel), _ptr(nsel),
+                                _ptr(pooled), _ptr(ws), ws.numel(), _stream(stream))
+    _lib.check(st, "qsa_prefill")
+    return {"out": out, "lse": lse, "sel": sel, "nsel": nsel, "pooled": pooled}
+
+
+def select(cfg: QSAConfig, iq, ik, iw, cu_seqlens, max_seqlen: int, *, want_scores=False,
+           want_pooled=False, workspace=None, stream=None) -> dict:
+    """Selection only (qsa_select): sel [T, k+1], nsel [T], optional scores
+    [T, max_seqlen // B] and pooled keys."""
+    T = iq.shape[0]
+    dt = cfg.dtype
+    _need(iq, "iq", dt, (T, cfg.idx_heads, cfg.idx_dim))
+    _need(ik, "ik", dt, (T, cfg.idx_dim))
+    _need(iw, "iw", torch.float32, (T, cfg.idx_heads))
+    _need(cu_seqlens, "cu_seqlens", torch.int32)
+    batch = cu_seqlens.shape[0] - 1
+    dev = iq.device
+    sel = torch.empty(T, cfg.topk + 1, dtype=torch.int32, device=dev)
+    nsel = torch.empty(T, dtype=torch.int32, device=dev)
+    scores = (torch.empty(T, max(1, max_seqlen // cfg.block_size), dtype=torch.float32,
+                          device=dev) if want_scores else None)
+    pooled = None
+    if want_pooled:
+        nb = -(-max_seqlen // cfg.block_size)
+        pooled = torch.zeros(batch, nb, cfg.idx_dim, dtype=torch.float32, device=dev)
+    ws = _workspace(prefill_workspace_size(cfg, batch, T, max_seqlen), dev, workspace)
+    c = cfg.c()
+    st = _lib.lib().qsa_select(ctypes.byref(c), batch, T, int(max_seqlen), _ptr(cu_seqlens),
+                               _ptr(iq), _ptr(ik), _ptr(iw), _ptr(sel), _ptr(nsel),
+                               _ptr(scores), _ptr(pooled), _ptr(ws), ws.numel(),
+                               _stream(stream))
+    _lib.check(st, "qsa_select")
+    return {"sel": sel, "nsel": nsel, "scores": scores, "pooled": pooled}
+
+
+def _check_decode(cfg, q, k_cache, v_cache, iq, ik_cache, iw, gate, pooled_cache, kv_len):
+    dt = cfg.dtype
+    batch, n_q = q.shape[0], q.shape[1]
+    cap = k_cache.shape[1]
+    _need(q, "q", dt, (batch, n_q, cfg.num_q_heads, cfg.head_dim))
+    if k_cache is not None:
+        _need(k_cache, "k_cache", dt, (batch, cap, cfg.num_kv_heads, cfg.head_dim))
+        _need(v_cache, "v_cache", dt, (batch, cap, cfg.num_kv_heads, cfg.head_dim))
+    _need(iq, "iq", dt, (batch, n_q, cfg.idx_heads, cfg.idx_dim))
+    _need(ik_cache, "ik_cache", dt, (batch, cap, cfg.idx_dim))
+    _need(iw, "iw", torch.float32, (batch, n_q, cfg.idx_heads))
+    if gate is not None:
+        _need(gate, "gate", dt, (batch, n_q, cfg.num_q_heads) if cfg.gate_headwise
+              else (batch, n_q, cfg.num_q_heads, cfg.head_dim))
+    _need(pooled_cache, "pooled_cache", torch.float32,
+          (batch, cap // cfg.block_size, cfg.idx_dim))
+    _need(kv_len, "kv_len", torch.int32, (batch,))
+    return batch, n_q, cap
+
+
+def decode(cfg: QSAConfig, q, k_cache, v_cache, iq, ik_cache, iw, gate, pooled_cache, kv_len,
+           *, out=None, lse=None, sel=None, nsel=None, dev_err=None, workspace=None,
+           want_lse=False, want_sel=False, stream=None) -> dict:
+    """One QSA decode step (qsa_decode). pooled_cache is updated in place for
+    the blocks this step completes."""
+    batch, n_q, cap = _check_decode(cfg, q, k_cache, v_cache, iq, ik_cache, iw, gate,
+                                    pooled_cache, kv_len)
+    dev = q.device
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(batch, n_q, cfg.num_q_heads, dtype=torch.float32, device=dev)
+    if sel is None and want_sel:
+        sel = torch.empty(batch, n_q, cfg.topk + 1, dtype=torch.int32, device=dev)
+    if nsel is None and want_sel:
+        nsel = torch.empty(batch, n_q, dtype=torch.int32, device=dev)
+    ws = _workspace(decode_workspace_size(cfg, batch, n_q, cap), dev, workspace)
+    c = cfg.c()
+    st = _lib.lib().qsa_decode(ctypes.byref(c), batch, n_q, cap, _ptr(kv_len), _ptr(q),
+                               _ptr(k_cache), _ptr(v_cache), _ptr(iq), _ptr(ik_cache), _ptr(iw),
+                               _ptr(gate), _ptr(pooled_cache), _ptr(out), _ptr(lse), _ptr(sel),
+                               _ptr(nsel), _ptr(dev_err), _ptr(ws), ws.numel(), _stream(stream))
+    _lib.check(st, "qsa_decode")
+    return {"out": out, "lse": lse, "sel": sel, "nsel": nsel}
+
+
+def select_decode(cfg: QSAConfig, iq, ik_cache, iw, pooled_cache, kv_len, *, want_scores=False,
+                  dev_err=None, workspace=None, stream=None) -> dict:
+    """Decode selection only (qsa_select_decode); also finalises the pooled
+    rows completed by this step."""
+    dt = cfg.dtype
+    batch, n_q = iq.shape[0], iq.shape[1]
+    cap = ik_cache.shape[1]
+    _need(iq, "iq", dt, (batch, n_q, cfg.idx_heads, cfg.idx_dim))
+    _need(ik_cache, "ik_cache", dt, (batch, cap, cfg.idx_dim))
+    _need(iw, "iw", torch.float32, (batch, n_q, cfg.idx_heads))
+    _need(pooled_cache, "pooled_cache", torch.float32, (batch, cap // cfg.block_size, cfg.idx_dim))
+    _need(kv_len, "kv_len", torch.int32, (batch,))
+    dev = iq.device
+    sel = torch.empty(batch, n_q, cfg.topk + 1, dtype=torch.int32, device=dev)
+    nsel = torch.empty(batch, n_q, dtype=torch.int32, device=dev)
+    scores = (torch.empty(batch, n_q, cap // cfg.block_size, dtype=torch.float32, device=dev)
+              if want_scores else None)
+    ws = _workspace(decode_workspace_size(cfg, batch, n_q, cap), dev, workspace)
+    c = cfg.c()
+    st = _lib.lib().qsa_select_decode(ctypes.byref(c), batch, n_q, cap, _ptr(kv_len), _ptr(iq),
+                                      _ptr(ik_cache), _ptr(iw), _ptr(pooled_cache), _ptr(sel),
+                                      _ptr(nsel), _ptr(scores), _ptr(dev_err), _ptr(ws),
+                                      ws.numel(), _stream(stream))
+    _lib.check(st, "qsa_select_decode")
+    return {"sel": sel, "nsel": nsel, "scores": scores}
+
+
+def pool_build(cfg: QSAConfig, ik_cache, kv_len, pooled_cache=None, *, dev_err=None,
+               stream=None):
+    """Rebuild the pooled-key cache from the indexer-key cache (qsa_pool_build)."""
+    batch, cap = ik_cache.shape[0], ik_cache.shape[1]
+    _need(ik_cache, "ik_cache", cfg.dtype, (batch, cap, cfg.idx_dim))
+    _need(kv_len, "kv_len", torch.int32, (batch,))
+    if pooled_cache is None:
+        pooled_cache = torch.zeros(batch, cap // cfg.block_size, cfg.idx_dim,
+                                   dtype=torch.float32, device=ik_cache.device)
+    c = cfg.c()
+    st = _lib.lib().qsa_pool_build(ctypes.byref(c), batch, cap, _ptr(kv_len), _ptr(ik_cache),
+                                   _ptr(pooled_cache), _ptr(dev_err), _stream(stream))
+    _lib.check(st, "qsa_pool_build")
+    return pooled_cache

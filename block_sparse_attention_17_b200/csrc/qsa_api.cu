@@ -1,0 +1,411 @@
+// C ABI of the QSA library: argument validation, workspace carving and the
+// launch sequence of each entry point. Nothing here reads device memory or
+// synchronises the host; every kernel goes to the caller's stream.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <atomic>
+
+#include "qsa_common.cuh"
+#include "qsa_kernels.h"
+
+using namespace qsa;
+
+namespace {
+std::atomic<unsigned long long> g_launches{0};
+}  // namespace
+
+void qsa::note_launch(int n) { g_launches.fetch_add((unsigned long long)n); }
+
+namespace {
+
+// Optional profiling events (per host thread): recorded on the call's stream
+// at stage boundaries, see qsa_set_stage_events().
+thread_local cudaEvent_t g_stage_ev[4] = {nullptr, nullptr, nullptr, nullptr};
+thread_local int g_stage_n = 0;
+
+void stage_mark(int i, cudaStream_t st) {
+  if (i < g_stage_n && g_stage_ev[i]) cudaEventRecord(g_stage_ev[i], st);
+}
+
+thread_local char g_err[512] = "";
+
+qsa_status fail(qsa_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+qsa_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(QSA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+constexpr int kMaxDecodeBlocks = 16384;
+constexpr int kMaxDecodeQ = 4;
+constexpr int kMaxDecodeRows = 32;
+constexpr int kTargetCtas = 2 * 148;
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+qsa_status check_cfg(const qsa_config* c) {
+  if (!c) return fail(QSA_ERR_INVALID_ARG, "cfg is NULL");
+  if (c->num_q_heads <= 0 || c->num_kv_heads <= 0 || c->head_dim <= 0 || c->idx_heads <= 0 ||
+      c->idx_dim <= 0 || c->block_size <= 0 || c->budget <= 0)
+    return fail(QSA_ERR_INVALID_ARG, "geometry fields must be positive");
+  if (c->num_q_heads % c->num_kv_heads)
+    return fail(QSA_ERR_INVALID_ARG, "num_q_heads %% num_kv_heads != 0");
+  if (c->budget % c->block_size)
+    return fail(QSA_ERR_INVALID_ARG, "budget must be a multiple of block_size");
+  if (c->dtype != QSA_F32 && c->dtype != QSA_BF16)
+    return fail(QSA_ERR_INVALID_ARG, "unknown dtype %d", (int)c->dtype);
+  if (c->softmax_scale < 0.f || c->index_scale < 0.f || !isfinite(c->softmax_scale) ||
+      !isfinite(c->index_scale))
+    return fail(QSA_ERR_INVALID_ARG, "scales must be finite and >= 0 (0 = default)");
+  if (c->num_q_heads / c->num_kv_heads > 16)
+    return fail(QSA_ERR_UNSUPPORTED, "group size Hq/Hkv > 16");
+  if (c->head_dim != 64 && c->head_dim != 128)
+    return fail(QSA_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128)", c->head_dim);
+  if (c->block_size != 64 && c->block_size != 128)
+    return fail(QSA_ERR_UNSUPPORTED, "block_size %d (supported: 64, 128)", c->block_size);
+  if (c->budget / c->block_size > kMaxTopK)
+    return fail(QSA_ERR_UNSUPPORTED, "budget/block_size > %d", kMaxTopK);
+  if (c->idx_dim != 32 && c->idx_dim != 64)
+    return fail(QSA_ERR_UNSUPPORTED, "idx_dim %d (supported: 32, 64)", c->idx_dim);
+  if (c->idx_heads > 16) return fail(QSA_ERR_UNSUPPORTED, "idx_heads > 16");
+  return QSA_OK;
+}
+
+Geom make_geom(const qsa_config* c) {
+  Geom g;
+  g.Hq = c->num_q_heads;
+  g.Hkv = c->num_kv_heads;
+  g.G = g.Hq / g.Hkv;
+  g.D = c->head_dim;
+  g.Hi = c->idx_heads;
+  g.di = c->idx_dim;
+  g.B = c->block_size;
+  g.k = c->budget / c->block_size;
+  const float sm = c->softmax_scale > 0.f ? c->softmax_scale : 1.0f / sqrtf((float)g.D);
+  g.sm_scale_log2 = sm * kLog2e;
+  g.idx_scale = c->index_scale > 0.f ? c->index_scale : 1.0f / sqrtf((float)g.di);
+  g.gate_headwise = c->gate_headwise ? 1 : 0;
+  return g;
+}
+
+// Bump allocator over the caller's workspace; every region is 256-byte aligned.
+struct Carve {
+  char* base;
+  size_t off = 0;
+  explicit Carve(void* b) : base((char*)b) {}
+  template <typename T> T* take(size_t count) {
+    off = (off + 255) & ~(size_t)255;
+    T* p = base ? (T*)(base + off) : nullptr;
+    off += count * sizeof(T);
+    return p;
+  }
+};
+
+struct PrefillWs {
+  float* pooled;
+  int* sel;
+  int* nsel;
+  uint32_t* bitmask;
+  size_t bytes;
+};
+
+PrefillWs carve_prefill(const Geom& g, void* ws, int batch, int T, int max_seqlen) {
+  const int max_nblk = (max_seqlen + g.B - 1) / g.B;
+  const int words = (max_nblk + 31) / 32;
+  Carve c(ws);
+  PrefillWs w;
+  w.pooled = c.take<float>((size_t)batch * max_nblk * g.di);
+  w.sel = c.take<int>((size_t)T * (g.k + 1));
+  w.nsel = c.take<int>((size_t)T);
+  w.bitmask = c.take<uint32_t>((size_t)T * words);
+  w.bytes = (c.off + 255) & ~(size_t)255;
+  return w;
+}
+
+struct DecodeWs {
+  float* scores;
+  int* sel;
+  int* nsel;
+  float* part_ml;
+  float* part_o;
+  int nsplit, per_split;
+  size_t bytes;
+};
+
+DecodeWs carve_decode(const Geom& g, void* ws, int batch, int n_q, int cap) {
+  DecodeWs w;
+  const int max_union = n_q * (g.k + 1);
+  const int pairs = std::max(1, batch * g.Hkv);
+  int nsplit = std::min(max_union, std::max(1, (kTargetCtas + pairs - 1) / pairs));
+  w.per_split = (max_union + nsplit - 1) / nsplit;
+  w.nsplit = (max_union + w.per_split - 1) / w.per_split;
+  const int R = n_q * g.G;
+  Carve c(ws);
+  w.scores = c.take<float>((size_t)batch * n_q * (cap / g.B));
+  w.sel = c.take<int>((size_t)batch * n_q * (g.k + 1));
+  w.nsel = c.take<int>((size_t)batch * n_q);
+  w.part_ml = c.take<float>((size_t)batch * g.Hkv * w.nsplit * R * 2);
+  w.part_o = c.take<float>((size_t)batch * g.Hkv * w.nsplit * R * g.D);
+  w.bytes = (c.off + 255) & ~(size_t)255;
+  return w;
+}
+
+qsa_status check_prefill_dims(const qsa_config* cfg, int batch, int T, int max_seqlen) {
+  qsa_status s = check_cfg(cfg);
+  if (s != QSA_OK) return s;
+  if (batch < 0 || T < 0 || max_seqlen < 0)
+    return fail(QSA_ERR_INVALID_ARG, "batch, total_tokens and max_seqlen must be >= 0");
+  if (T > 0 && (batch == 0 || max_seqlen == 0))
+    return fail(QSA_ERR_INVALID_ARG, "total_tokens > 0 needs batch > 0 and max_seqlen > 0");
+  if ((long long)max_seqlen > (long long)T && batch == 1)
+    return fail(QSA_ERR_INVALID_ARG, "max_seqlen > total_tokens for a single sequence");
+  if ((max_seqlen + cfg->block_size - 1) / cfg->block_size > kMaxBlocksPerSeq)
+    return fail(QSA_ERR_UNSUPPORTED, "more than %d blocks per sequence", kMaxBlocksPerSeq);
+  return QSA_OK;
+}
+
+qsa_status check_decode_dims(const qsa_config* cfg, int batch, int n_q, int cap) {
+  qsa_status s = check_cfg(cfg);
+  if (s != QSA_OK) return s;
+  if (batch < 0 || n_q <= 0 || cap <= 0)
+    return fail(QSA_ERR_INVALID_ARG, "batch >= 0, n_q > 0 and cap > 0 are required");
+  if (cap % cfg->block_size) return fail(QSA_ERR_INVALID_ARG, "cap must be a multiple of B");
+  if (cap / cfg->block_size > kMaxDecodeBlocks)
+    return fail(QSA_ERR_UNSUPPORTED, "more than %d cache blocks", kMaxDecodeBlocks);
+  if (n_q > kMaxDecodeQ) return fail(QSA_ERR_UNSUPPORTED, "n_q > %d", kMaxDecodeQ);
+  if (n_q * (cfg->num_q_heads / cfg->num_kv_heads) > kMaxDecodeRows)
+    return fail(QSA_ERR_UNSUPPORTED, "n_q * group size > %d", kMaxDecodeRows);
+  return QSA_OK;
+}
+
+#define QSA_REQUIRE(p, name)                                                  \
+  do {                                                                        \
+    if (!(p)) return fail(QSA_ERR_INVALID_ARG, "%s is NULL", name);           \
+    if (!aligned16(p)) return fail(QSA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name); \
+  } while (0)
+
+#define QSA_CUDA(call, where)                          \
+  do {                                                 \
+    cudaError_t e_ = (call);                           \
+    if (e_ != cudaSuccess) return cuda_fail(e_, where); \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+const char* qsa_status_string(qsa_status s) {
+  switch (s) {
+    case QSA_OK: return "QSA_OK";
+    case QSA_ERR_INVALID_ARG: return "QSA_ERR_INVALID_ARG";
+    case QSA_ERR_UNSUPPORTED: return "QSA_ERR_UNSUPPORTED";
+    case QSA_ERR_WORKSPACE: return "QSA_ERR_WORKSPACE";
+    case QSA_ERR_CUDA: return "QSA_ERR_CUDA";
+  }
+  return "QSA_ERR_UNKNOWN";
+}
+
+const char* qsa_last_error(void) { return g_err; }
+
+int qsa_version(void) { return 100; }
+
+unsigned long long qsa_kernel_launch_count(void) { return g_launches.load(); }
+
+qsa_status qsa_set_stage_events(void* const* events, int count) {
+  if (count < 0 || count > 4 || (count > 0 && !events))
+    return fail(QSA_ERR_INVALID_ARG, "count must be in [0, 4] with non-NULL events");
+  for (int i = 0; i < 4; ++i) g_stage_ev[i] = i < count ? (cudaEvent_t)events[i] : nullptr;
+  g_stage_n = count;
+  return QSA_OK;
+}
+
+size_t qsa_prefill_workspace_size(const qsa_config* cfg, int batch, int total_tokens,
+                                  int max_seqlen) {
+  if (check_prefill_dims(cfg, batch, total_tokens, max_seqlen) != QSA_OK) return 0;
+  return carve_prefill(make_geom(cfg), nullptr, batch, total_tokens, max_seqlen).bytes;
+}
+
+static qsa_status prefill_select_common(const qsa_config* cfg, const Geom& g, int batch,
+                                        int T, int max_seqlen, const int32_t* cu,
+                                        const void* iq, const void* ik, const float* iw,
+                                        const PrefillWs& w, float* pooled, int32_t* sel,
+                                        int32_t* nsel, float* scores, cudaStream_t st) {
+  const int max_nblk = (max_seqlen + g.B - 1) / g.B;
+  const int words = (max_nblk + 31) / 32;
+  QSA_CUDA(launch_pool_prefill(cfg->dtype, ik, cu, batch, max_seqlen, g.B, g.di, pooled,
+                               max_nblk, st),
+           "pool");
+  QSA_CUDA(launch_select_prefill(cfg->dtype, g, cu, batch, max_seqlen, max_nblk, words, iq, iw,
+                                 pooled, sel, nsel, w.bitmask, scores,
+                                 std::max(1, max_seqlen / g.B), st),
+           "select");
+  return QSA_OK;
+}
+
+qsa_status qsa_prefill(const qsa_config* cfg, int batch, int total_tokens, int max_seqlen,
+                       const int32_t* cu_seqlens, const void* q, const void* k, const void* v,
+                       const void* iq, const void* ik, const float* iw, const void* gate,
+                       void* out, float* lse, int32_t* sel, int32_t* nsel, float* pooled_out,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  g_err[0] = 0;
+  qsa_status s = check_prefill_dims(cfg, batch, total_tokens, max_seqlen);
+  if (s != QSA_OK) return s;
+  if (total_tokens == 0) return QSA_OK;
+  QSA_REQUIRE(cu_seqlens, "cu_seqlens");
+  QSA_REQUIRE(q, "q"); QSA_REQUIRE(k, "k"); QSA_REQUIRE(v, "v");
+  QSA_REQUIRE(iq, "iq"); QSA_REQUIRE(ik, "ik"); QSA_REQUIRE(iw, "iw");
+  QSA_REQUIRE(gate, "gate"); QSA_REQUIRE(out, "out");
+  if (lse) QSA_REQUIRE(lse, "lse");
+  if (sel) QSA_REQUIRE(sel, "sel");
+  if (nsel) QSA_REQUIRE(nsel, "nsel");
+  if (pooled_out) QSA_REQUIRE(pooled_out, "pooled_out");
+  const Geom g = make_geom(cfg);
+  const PrefillWs need = carve_prefill(g, nullptr, batch, total_tokens, max_seqlen);
+  if (!workspace || workspace_bytes < need.bytes || ((uintptr_t)workspace & 255u))
+    return fail(QSA_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned", need.bytes);
+  const PrefillWs w = carve_prefill(g, workspace, batch, total_tokens, max_seqlen);
+  cudaStream_t st = (cudaStream_t)stream;
+  float* pooled = pooled_out ? pooled_out : w.pooled;
+  int* sel_p = sel ? sel : w.sel;
+  int* nsel_p = nsel ? nsel : w.nsel;
+  stage_mark(0, st);
+  s = prefill_select_common(cfg, g, batch, total_tokens, max_seqlen, cu_seqlens, iq, ik, iw, w,
+                            pooled, sel_p, nsel_p, nullptr, st);
+  if (s != QSA_OK) return s;
+  stage_mark(1, st);
+  QSA_CUDA(launch_attn_prefill_simt(cfg->dtype, g, cu_seqlens, batch, max_seqlen, q, k, v, gate,
+                                    sel_p, nsel_p, out, lse, st),
+           "attention");
+  stage_mark(2, st);
+  return QSA_OK;
+}
+
+qsa_status qsa_select(const qsa_config* cfg, int batch, int total_tokens, int max_seqlen,
+                      const int32_t* cu_seqlens, const void* iq, const void* ik, const float* iw,
+                      int32_t* sel, int32_t* nsel, float* scores, float* pooled_out,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+  g_err[0] = 0;
+  qsa_status s = check_prefill_dims(cfg, batch, total_tokens, max_seqlen);
+  if (s != QSA_OK) return s;
+  if (total_tokens == 0) return QSA_OK;
+  QSA_REQUIRE(cu_seqlens, "cu_seqlens");
+  QSA_REQUIRE(iq, "iq"); QSA_REQUIRE(ik, "ik"); QSA_REQUIRE(iw, "iw");
+  QSA_REQUIRE(sel, "sel"); QSA_REQUIRE(nsel, "nsel");
+  if (scores) QSA_REQUIRE(scores, "scores");
+  if (pooled_out) QSA_REQUIRE(pooled_out, "pooled_out");
+  const Geom g = make_geom(cfg);
+  const PrefillWs need = carve_prefill(g, nullptr, batch, total_tokens, max_seqlen);
+  if (!workspace || workspace_bytes < need.bytes || ((uintptr_t)workspace & 255u))
+    return fail(QSA_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned", need.bytes);
+  const PrefillWs w = carve_prefill(g, workspace, batch, total_tokens, max_seqlen);
+  return prefill_select_common(cfg, g, batch, total_tokens, max_seqlen, cu_seqlens, iq, ik, iw,
+                               w, pooled_out ? pooled_out : w.pooled, sel, nsel, scores,
+                               (cudaStream_t)stream);
+}
+
+size_t qsa_decode_workspace_size(const qsa_config* cfg, int batch, int n_q, int cap) {
+  if (check_decode_dims(cfg, batch, n_q, cap) != QSA_OK) return 0;
+  return carve_decode(make_geom(cfg), nullptr, batch, n_q, cap).bytes;
+}
+
+static qsa_status decode_select_common(const qsa_config* cfg, const Geom& g, int batch, int n_q,
+                                       int cap, const int32_t* kv_len, const void* iq,
+                                       const void* ik_cache, const float* iw,
+                                       float* pooled_cache, const DecodeWs& w, int32_t* sel,
+                                       int32_t* nsel, float* scores, int32_t* dev_err,
+                                       cudaStream_t st) {
+  QSA_CUDA(launch_pool_cache(cfg->dtype, ik_cache, kv_len, batch, cap, n_q, 1, g.B, g.di,
+                             pooled_cache, dev_err, st),
+           "pool finalize");
+  QSA_CUDA(launch_decode_select(cfg->dtype, g, batch, n_q, cap, kv_len, iq, iw, pooled_cache,
+                                w.scores, sel, nsel, scores, st),
+           "decode select");
+  return QSA_OK;
+}
+
+qsa_status qsa_decode(const qsa_config* cfg, int batch, int n_q, int cap, const int32_t* kv_len,
+                      const void* q, const void* k_cache, const void* v_cache, const void* iq,
+                      const void* ik_cache, const float* iw, const void* gate,
+                      float* pooled_cache, void* out, float* lse, int32_t* sel, int32_t* nsel,
+                      int32_t* dev_err, void* workspace, size_t workspace_bytes, void* stream) {
+  g_err[0] = 0;
+  qsa_status s = check_decode_dims(cfg, batch, n_q, cap);
+  if (s != QSA_OK) return s;
+  if (batch == 0) return QSA_OK;
+  QSA_REQUIRE(kv_len, "kv_len");
+  QSA_REQUIRE(q, "q"); QSA_REQUIRE(k_cache, "k_cache"); QSA_REQUIRE(v_cache, "v_cache");
+  QSA_REQUIRE(iq, "iq"); QSA_REQUIRE(ik_cache, "ik_cache"); QSA_REQUIRE(iw, "iw");
+  QSA_REQUIRE(gate, "gate"); QSA_REQUIRE(pooled_cache, "pooled_cache"); QSA_REQUIRE(out, "out");
+  if (lse) QSA_REQUIRE(lse, "lse");
+  if (sel) QSA_REQUIRE(sel, "sel");
+  if (nsel) QSA_REQUIRE(nsel, "nsel");
+  const Geom g = make_geom(cfg);
+  const DecodeWs need = carve_decode(g, nullptr, batch, n_q, cap);
+  if (!workspace || workspace_bytes < need.bytes || ((uintptr_t)workspace & 255u))
+    return fail(QSA_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned", need.bytes);
+  const DecodeWs w = carve_decode(g, workspace, batch, n_q, cap);
+  cudaStream_t st = (cudaStream_t)stream;
+  int* sel_p = sel ? sel : w.sel;
+  int* nsel_p = nsel ? nsel : w.nsel;
+  stage_mark(0, st);
+  s = decode_select_common(cfg, g, batch, n_q, cap, kv_len, iq, ik_cache, iw, pooled_cache, w,
+                           sel_p, nsel_p, nullptr, dev_err, st);
+  if (s != QSA_OK) return s;
+  stage_mark(1, st);
+  QSA_CUDA(launch_attn_decode_simt(cfg->dtype, g, batch, n_q, cap, w.nsplit, w.per_split, kv_len,
+                                   q, k_cache, v_cache, gate, sel_p, nsel_p, w.part_ml, w.part_o,
+                                   out, lse, st),
+           "decode attention");
+  stage_mark(2, st);
+  return QSA_OK;
+}
+
+qsa_status qsa_select_decode(const qsa_config* cfg, int batch, int n_q, int cap,
+                             const int32_t* kv_len, const void* iq, const void* ik_cache,
+                             const float* iw, float* pooled_cache, int32_t* sel, int32_t* nsel,
+                             float* scores, int32_t* dev_err, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  g_err[0] = 0;
+  qsa_status s = check_decode_dims(cfg, batch, n_q, cap);
+  if (s != QSA_OK) return s;
+  if (batch == 0) return QSA_OK;
+  QSA_REQUIRE(kv_len, "kv_len");
+  QSA_REQUIRE(iq, "iq"); QSA_REQUIRE(ik_cache, "ik_cache"); QSA_REQUIRE(iw, "iw");
+  QSA_REQUIRE(pooled_cache, "pooled_cache");
+  QSA_REQUIRE(sel, "sel"); QSA_REQUIRE(nsel, "nsel");
+  if (scores) QSA_REQUIRE(scores, "scores");
+  const Geom g = make_geom(cfg);
+  const DecodeWs need = carve_decode(g, nullptr, batch, n_q, cap);
+  if (!workspace || workspace_bytes < need.bytes || ((uintptr_t)workspace & 255u))
+    return fail(QSA_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned", need.bytes);
+  const DecodeWs w = carve_decode(g, workspace, batch, n_q, cap);
+  return decode_select_common(cfg, g, batch, n_q, cap, kv_len, iq, ik_cache, iw, pooled_cache,
+                              w, sel, nsel, scores, dev_err, (cudaStream_t)stream);
+}
+
+qsa_status qsa_pool_build(const qsa_config* cfg, int batch, int cap, const int32_t* kv_len,
+                          const void* ik_cache, float* pooled_cache, int32_t* dev_err,
+                          void* stream) {
+  g_err[0] = 0;
+  qsa_status s = check_decode_dims(cfg, batch, 1, cap);
+  if (s != QSA_OK) return s;
+  if (batch == 0) return QSA_OK;
+  QSA_REQUIRE(kv_len, "kv_len");
+  QSA_REQUIRE(ik_cache, "ik_cache");
+  QSA_REQUIRE(pooled_cache, "pooled_cache");
+  QSA_CUDA(launch_pool_cache(cfg->dtype, ik_cache, kv_len, batch, cap, 0, 0, cfg->block_size,
+                             cfg->idx_dim, pooled_cache, dev_err, (cudaStream_t)stream),
+           "pool build");
+  return QSA_OK;
+}
+
+}  // extern "C"

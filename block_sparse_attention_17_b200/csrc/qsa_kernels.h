@@ -1,0 +1,42 @@
+// Internal launcher declarations shared by the kernel files and the C ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/qsa.h"
+
+namespace qsa {
+
+struct Geom;
+
+// Counts kernel launches made by the library (all host threads).
+void note_launch(int n = 1);
+
+cudaError_t launch_pool_prefill(qsa_dtype dt, const void* ik, const int* cu, int batch,
+                                int max_seqlen, int B, int di, float* pooled, int max_nblk,
+                                cudaStream_t st);
+cudaError_t launch_pool_cache(qsa_dtype dt, const void* ik_cache, const int* kv_len, int batch,
+                              int cap, int n_q, int mode, int B, int di, float* pooled,
+                              int* dev_err, cudaStream_t st);
+size_t select_prefill_smem(const Geom& g, int nc_cap);
+cudaError_t launch_select_prefill(qsa_dtype dt, const Geom& g, const int* cu, int batch,
+                                  int max_seqlen, int max_nblk, int words, const void* iq,
+                                  const float* iw, const float* pooled, int* sel, int* nsel,
+                                  uint32_t* bitmask, float* scores, int scores_ld,
+                                  cudaStream_t st);
+cudaError_t launch_decode_select(qsa_dtype dt, const Geom& g, int batch, int n_q, int cap,
+                                 const int* kv_len, const void* iq, const float* iw,
+                                 const float* pooled, float* scores_ws, int* sel, int* nsel,
+                                 float* scores_out, cudaStream_t st);
+cudaError_t launch_attn_prefill_simt(qsa_dtype dt, const Geom& g, const int* cu, int batch,
+                                     int max_seqlen, const void* q, const void* k, const void* v,
+                                     const void* gate, const int* sel, const int* nsel,
+                                     void* out, float* lse, cudaStream_t st);
+cudaError_t launch_attn_decode_simt(qsa_dtype dt, const Geom& g, int batch, int n_q, int cap,
+                                    int nsplit, int per_split, const int* kv_len, const void* q,
+                                    const void* kc, const void* vc, const void* gate,
+                                    const int* sel, const int* nsel, float* part_ml,
+                                    float* part_o, void* out, float* lse, cudaStream_t st);
+
+}  // namespace qsa

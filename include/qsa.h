@@ -1,0 +1,190 @@
+/*
+ * qsa.h -- C ABI of the B200 (sm_100a) Qwen Sparse Attention (QSA) library.
+ *
+ * QSA is gated grouped-query attention whose causal mask is intersected with a
+ * per-query-token block selection (instagit "Native Backend Components for the
+ * Qwen4-Generation Preview Family in MTPLX", section "Qwen Sparse Attention
+ * (QSA)"; dev.to "Qwen4-Exp: How Per-Layer N-gram Embeddings and Sparse
+ * Attention ...", section "Qwen Sparse Attention: Block-Level Selection ...").
+ * For a query that sees n tokens of its sequence:
+ *
+ *   kbar[j]  = (1/B) * sum_{i<B} ik[j*B+i]                      complete blocks only
+ *   s[j]     = c * sum_h w[h] * relu(iq[h] . kbar[j]),  j < floor(n/B)
+ *   S        = top-(budget/B) blocks under (s desc, j asc)  U  tail [floor(n/B)*B, n)
+ *   out[h]   = sigmoid(gate[h]) * softmax_{s in S}(scale * q[h] . k[s, h/G]) v[s, h/G]
+ *
+ * The indexer settings (per-head weights, no n_head scale, c = idx_dim^-0.5,
+ * candidates = complete visible blocks) and the sigmoid output gate follow the
+ * QSA block-composition commit text on the llama.cpp PR #27739 page.
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ * - Every pointer argument is a DEVICE pointer unless stated otherwise; the
+ *   caller owns every buffer. The library never allocates device memory: the
+ *   caller passes a workspace of at least the size the matching
+ *   *_workspace_size() call returns (256-byte aligned).
+ * - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   All work is enqueued on it; no entry point synchronises the host, and no
+ *   entry point reads device memory (lengths, offsets) on the host.
+ * - Floating-point tensors are dense, row-major, in the config's dtype
+ *   (QSA_F32 or QSA_BF16) except `iw` (always fp32) and the pooled caches
+ *   (always fp32). Integer tensors are int32.
+ * - Arguments are validated before any launch; a bad argument returns
+ *   QSA_ERR_INVALID_ARG and a geometry outside the compiled kernels returns
+ *   QSA_ERR_UNSUPPORTED, in both cases with nothing enqueued. A launch failure
+ *   returns QSA_ERR_CUDA. qsa_last_error() gives a message for the calling
+ *   host thread. No entry point throws, exits or traps.
+ * - Supported on the GPU: head_dim in {64, 128}; block_size in {64, 128};
+ *   budget a positive multiple of block_size with budget/block_size <= 64;
+ *   num_q_heads % num_kv_heads == 0 with group size <= 16; idx_dim in {32, 64};
+ *   idx_heads <= 16; at most 4096 blocks per sequence.
+ */
+#ifndef QSA_H_
+#define QSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QSA_OK = 0,
+  QSA_ERR_INVALID_ARG = 1,
+  QSA_ERR_UNSUPPORTED = 2,
+  QSA_ERR_WORKSPACE = 3,
+  QSA_ERR_CUDA = 4
+} qsa_status;
+
+typedef enum { QSA_F32 = 0, QSA_BF16 = 1 } qsa_dtype;
+
+/* QSA geometry. This metadata decides which memory attention may read, so it
+ * is validated on every call (ramgpt "Porting Qwen4 to llama.cpp": QSA
+ * metadata is part of the execution contract). */
+typedef struct {
+  int num_q_heads;     /* Hq */
+  int num_kv_heads;    /* Hkv; query head h reads KV head h / (Hq/Hkv) */
+  int head_dim;        /* D */
+  int idx_heads;       /* Hi, indexer heads */
+  int idx_dim;         /* di, indexer head dim (one indexer key row per token) */
+  int block_size;      /* B, tokens per pooled block (the compression ratio) */
+  int budget;          /* tokens; k = budget / B complete blocks are kept */
+  float softmax_scale; /* attention logit scale; 0 => head_dim^-0.5 */
+  float index_scale;   /* indexer score scale c; 0 => idx_dim^-0.5 */
+  int gate_headwise;   /* 0: gate [.., Hq, D] elementwise; 1: gate [.., Hq] */
+  qsa_dtype dtype;     /* dtype of q, k, v, iq, ik, gate, out */
+} qsa_config;
+
+/* Human-readable name of a status code (static storage). */
+const char* qsa_status_string(qsa_status s);
+
+/* Message describing the last failed call on this host thread ("" if none). */
+const char* qsa_last_error(void);
+
+/* Library ABI version: 100 * major + minor. */
+int qsa_version(void);
+
+/* Number of kernels the library has launched since it was loaded (all host
+ * threads). Used to check that work really ran in the library's kernels. */
+unsigned long long qsa_kernel_launch_count(void);
+
+/* Profiling hook for the calling host thread: with count > 0, later calls of
+ * qsa_prefill / qsa_decode on this thread record events[0] when their first
+ * kernel is enqueued, events[1] before the attention kernel(s) and events[2]
+ * after the last kernel, all on the call's stream. `events` are cudaEvent_t
+ * handles created by the caller, passed as void*; count = 0 turns it off.
+ * Returns QSA_ERR_INVALID_ARG for count outside [0, 4]. */
+qsa_status qsa_set_stage_events(void* const* events, int count);
+
+/* ---------------------------------------------------------------- prefill --
+ * Packed variable-length prefill. Sequence b owns tokens
+ * [cu_seqlens[b], cu_seqlens[b+1]); query token t at position p of its
+ * sequence sees n = p + 1 tokens (causal).
+ *
+ *   cu_seqlens  [batch+1] int32 (device), non-decreasing, cu_seqlens[0] = 0,
+ *               cu_seqlens[batch] = total_tokens, every length <= max_seqlen.
+ *   q           [total_tokens, Hq, D]      k, v [total_tokens, Hkv, D]
+ *   iq          [total_tokens, Hi, di]     ik   [total_tokens, di]
+ *   iw          [total_tokens, Hi] fp32    gate [total_tokens, Hq, D] (or [.., Hq])
+ *   out         [total_tokens, Hq, D]      (written)
+ *   lse         optional [total_tokens, Hq] fp32: natural-log sum-exp of the
+ *               scaled logits over the selected tokens (written)
+ *   sel         optional [total_tokens, k+1] int32: the selected complete
+ *               blocks in ascending order, then the tail block id floor(n/B)
+ *               when n % B != 0, then -1 padding (written)
+ *   nsel        optional [total_tokens] int32: min(k, floor(n/B)) + (n%B != 0)
+ *   pooled_out  optional [batch, ceil(max_seqlen/B), di] fp32: pooled keys of
+ *               every complete block (rows past a sequence's last complete
+ *               block are left untouched)
+ * host_total_tokens and max_seqlen are host integers that must describe the
+ * device cu_seqlens; a device length above max_seqlen is not detected. */
+size_t qsa_prefill_workspace_size(const qsa_config* cfg, int batch, int total_tokens,
+                                  int max_seqlen);
+
+qsa_status qsa_prefill(const qsa_config* cfg, int batch, int total_tokens, int max_seqlen,
+                       const int32_t* cu_seqlens, const void* q, const void* k,
+                       const void* v, const void* iq, const void* ik, const float* iw,
+                       const void* gate, void* out, float* lse, int32_t* sel,
+                       int32_t* nsel, float* pooled_out, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/* Selection only, for packed prefill geometry (same arguments as qsa_prefill).
+ * scores: optional [total_tokens, max_seqlen/B] fp32; entry j of query t is
+ * the indexer score s[j] for j < floor(n/B) and -inf beyond. */
+qsa_status qsa_select(const qsa_config* cfg, int batch, int total_tokens, int max_seqlen,
+                      const int32_t* cu_seqlens, const void* iq, const void* ik,
+                      const float* iw, int32_t* sel, int32_t* nsel, float* scores,
+                      float* pooled_out, void* workspace, size_t workspace_bytes,
+                      void* stream);
+
+/* ----------------------------------------------------------------- decode --
+ * One decode step for `batch` sequences, each with n_q new query tokens
+ * (n_q = 1 plain decode, n_q = 2 MTP verification of one draft token).
+ * The caller has already appended this step's K, V and indexer-key rows to
+ * the caches; kv_len[b] counts the rows present after that append, and new
+ * query i of sequence b sees n = kv_len[b] - n_q + 1 + i tokens.
+ *
+ *   kv_len        [batch] int32 (device), n_q <= kv_len[b] <= cap
+ *   q             [batch, n_q, Hq, D]     gate [batch, n_q, Hq, D] (or [.., Hq])
+ *   k_cache/v_cache [batch, cap, Hkv, D]  ik_cache [batch, cap, di]
+ *   iq            [batch, n_q, Hi, di]    iw [batch, n_q, Hi] fp32
+ *   pooled_cache  [batch, cap/B, di] fp32, in/out: rows of blocks completed
+ *                 before this step must hold their pooled keys (qsa_prefill's
+ *                 pooled_out or qsa_pool_build give them); this call writes the
+ *                 rows of the blocks its n_q tokens complete.
+ *   out           [batch, n_q, Hq, D] (written); lse/sel/nsel as for prefill,
+ *                 with a leading [batch, n_q] instead of [total_tokens].
+ *   dev_err       optional int32 (device): set to a non-zero code when a
+ *                 kv_len entry is out of range; those sequences are skipped.
+ * cap must be a multiple of B. */
+size_t qsa_decode_workspace_size(const qsa_config* cfg, int batch, int n_q, int cap);
+
+qsa_status qsa_decode(const qsa_config* cfg, int batch, int n_q, int cap,
+                      const int32_t* kv_len, const void* q, const void* k_cache,
+                      const void* v_cache, const void* iq, const void* ik_cache,
+                      const float* iw, const void* gate, float* pooled_cache, void* out,
+                      float* lse, int32_t* sel, int32_t* nsel, int32_t* dev_err,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* Selection only, for decode geometry (same arguments as qsa_decode; it also
+ * finalises the pooled rows completed by this step). scores: optional
+ * [batch, n_q, cap/B] fp32, -inf past a query's candidates. */
+qsa_status qsa_select_decode(const qsa_config* cfg, int batch, int n_q, int cap,
+                             const int32_t* kv_len, const void* iq, const void* ik_cache,
+                             const float* iw, float* pooled_cache, int32_t* sel,
+                             int32_t* nsel, float* scores, int32_t* dev_err,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* Rebuild the pooled-key cache of every complete block j < kv_len[b]/B from
+ * the indexer-key cache (restore after a state reload). The rows it writes are
+ * bit-identical to the ones the incremental decode path writes. */
+qsa_status qsa_pool_build(const qsa_config* cfg, int batch, int cap, const int32_t* kv_len,
+                          const void* ik_cache, float* pooled_cache, int32_t* dev_err,
+                          void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QSA_H_ */

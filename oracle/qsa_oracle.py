@@ -149,16 +149,16 @@ def gated_attention(q_t: np.ndarray, K: np.ndarray, V: np.ndarray,
     lse = np.full(Hq, -np.inf, dtype=np.float64)
     if len(positions) == 0:
         return o, lse
-    for h in range(Hq):
-        kvh = h // G
-        Ks = np.asarray(K[positions, kvh, :], dtype=np.float64)
+    for kvh in range(Hkv):
+        Ks = np.asarray(K[positions, kvh, :], dtype=np.float64)    # [n, D]
         Vs = np.asarray(V[positions, kvh, :], dtype=np.float64)
-        logits = softmax_scale * (Ks @ q_t[h])
-        m = logits.max()
-        p = np.exp(logits - m)
-        l = p.sum()
-        o[h] = (p @ Vs) / l
-        lse[h] = m + math.log(l)
+        for h in range(kvh * G, (kvh + 1) * G):                     # heads reading this KV head
+            logits = softmax_scale * (Ks @ q_t[h])
+            m = logits.max()
+            p = np.exp(logits - m)
+            l = p.sum()
+            o[h] = (p @ Vs) / l
+            lse[h] = m + math.log(l)
     g = sigmoid(gate_t)
     if g.ndim == 1:
         g = g[:, None]
