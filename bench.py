@@ -206,7 +206,11 @@ def run_ours(args, w, rank, world, dist):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     ev_stage = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-    arr_t = (ctypes_voidp_array([e.cuda_event for e in ev_stage]))
+    for e in ev_stage:          # torch creates the CUDA event on its first record
+        e.record(stream)
+    torch.cuda.synchronize()
+    arr_t = ctypes_voidp_array([e.cuda_event for e in ev_stage])
+    assert all(e.cuda_event for e in ev_stage)
 
     if w.kind == "prefill":
         T = host["q"].shape[0]
