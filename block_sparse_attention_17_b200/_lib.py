@@ -26,7 +26,7 @@ EXPORTED = [
     "qsa_set_stage_events",
     "qsa_prefill_workspace_size", "qsa_prefill", "qsa_select",
     "qsa_decode_workspace_size", "qsa_decode", "qsa_select_decode",
-    "qsa_pool_build",
+    "qsa_pool_build", "qsa_decode_noalloc",
 ]
 
 
@@ -74,6 +74,7 @@ def _declare(lib):
         "qsa_decode": (I, [CFG, I, I, I, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]),
         "qsa_select_decode": (I, [CFG, I, I, I, P, P, P, P, P, P, P, P, P, P, SZ, P]),
         "qsa_pool_build": (I, [CFG, I, I, P, P, P, P, P]),
+        "qsa_decode_noalloc": (I, [CFG, I, I, I] + [P] * 15),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

@@ -222,6 +222,34 @@ def decode(cfg: QSAConfig, q, k_cache, v_cache, iq, ik_cache, iw, gate, pooled_c
     return {"out": out, "lse": lse, "sel": sel, "nsel": nsel}
 
 
+def decode_noalloc(cfg: QSAConfig, q, k_cache, v_cache, iq, ik_cache, iw, gate, pooled_cache,
+                   kv_len, *, out=None, lse=None, sel=None, nsel=None, dev_err=None,
+                   want_lse=False, want_sel=False, stream=None) -> dict:
+    """qsa_decode_noalloc: the decode step with the library's static 4 MiB
+    device scratch instead of a workspace, for callers that cannot allocate
+    scratch memory. Calls that overlap on the GPU share that scratch and race.
+    (Outputs the caller does not pass are still allocated here, by torch.)"""
+    batch, n_q, cap = _check_decode(cfg, q, k_cache, v_cache, iq, ik_cache, iw, gate,
+                                    pooled_cache, kv_len)
+    dev = q.device
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(batch, n_q, cfg.num_q_heads, dtype=torch.float32, device=dev)
+    if sel is None and want_sel:
+        sel = torch.empty(batch, n_q, cfg.topk + 1, dtype=torch.int32, device=dev)
+    if nsel is None and want_sel:
+        nsel = torch.empty(batch, n_q, dtype=torch.int32, device=dev)
+    c = cfg.c()
+    st = _lib.lib().qsa_decode_noalloc(ctypes.byref(c), batch, n_q, cap, _ptr(kv_len), _ptr(q),
+                                       _ptr(k_cache), _ptr(v_cache), _ptr(iq), _ptr(ik_cache),
+                                       _ptr(iw), _ptr(gate), _ptr(pooled_cache), _ptr(out),
+                                       _ptr(lse), _ptr(sel), _ptr(nsel), _ptr(dev_err),
+                                       _stream(stream))
+    _lib.check(st, "qsa_decode_noalloc")
+    return {"out": out, "lse": lse, "sel": sel, "nsel": nsel}
+
+
 def select_decode(cfg: QSAConfig, iq, ik_cache, iw, pooled_cache, kv_len, *, want_scores=False,
                   dev_err=None, workspace=None, stream=None) -> dict:
     """Decode selection only (qsa_select_decode); also finalises the pooled

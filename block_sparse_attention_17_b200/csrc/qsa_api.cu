@@ -41,6 +41,12 @@ qsa_status fail(qsa_status s, const char* fmt, ...) {
   return s;
 }
 
+}  // namespace
+
+void qsa::set_last_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+
+namespace {
+
 qsa_status cuda_fail(cudaError_t e, const char* where) {
   return fail(QSA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
 }

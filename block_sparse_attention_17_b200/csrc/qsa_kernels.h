@@ -13,6 +13,9 @@ struct Geom;
 // Counts kernel launches made by the library (all host threads).
 void note_launch(int n = 1);
 
+// Sets the message qsa_last_error() returns on this host thread.
+void set_last_error(const char* msg);
+
 cudaError_t launch_pool_prefill(qsa_dtype dt, const void* ik, const int* cu, int batch,
                                 int max_seqlen, int B, int di, float* pooled, int max_nblk,
                                 cudaStream_t st);

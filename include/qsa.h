@@ -176,6 +176,28 @@ qsa_status qsa_select_decode(const qsa_config* cfg, int batch, int n_q, int cap,
                              int32_t* nsel, float* scores, int32_t* dev_err,
                              void* workspace, size_t workspace_bytes, void* stream);
 
+/* qsa_decode without a workspace argument. The pages describe nothing like
+ * it; it exists for callers that cannot allocate device memory for scratch,
+ * such as a host program whose own allocator owns all of the GPU's memory, or
+ * a latency-critical loop that must never call cudaMalloc. The scratch comes
+ * from a 4 MiB array the library declares statically in device memory: every
+ * GPU that loads the library holds it until the process exits, and this call
+ * allocates nothing. Arguments are those of qsa_decode minus the workspace.
+ * - A geometry whose qsa_decode_workspace_size() exceeds 4 MiB returns
+ *   QSA_ERR_WORKSPACE (qsa_last_error() says how much it needs).
+ * - The first call on a device looks up the array's device address (once per
+ *   device, with that device current), so make the first call on each device
+ *   before any stream capture.
+ * - All calls on a device share the one array, which keeps the last call's
+ *   contents (no part of it needs to start at zero): calls that overlap on the
+ *   GPU, on different streams or host threads, race and corrupt each other. */
+qsa_status qsa_decode_noalloc(const qsa_config* cfg, int batch, int n_q, int cap,
+                              const int32_t* kv_len, const void* q, const void* k_cache,
+                              const void* v_cache, const void* iq, const void* ik_cache,
+                              const float* iw, const void* gate, float* pooled_cache,
+                              void* out, float* lse, int32_t* sel, int32_t* nsel,
+                              int32_t* dev_err, void* stream);
+
 /* Rebuild the pooled-key cache of every complete block j < kv_len[b]/B from
  * the indexer-key cache (restore after a state reload). The rows it writes are
  * bit-identical to the ones the incremental decode path writes. */
