@@ -143,7 +143,10 @@ def prefill(cfg: QSAConfig, q, k, v, iq, ik, iw, gate, cu_seqlens, max_seqlen: i
                                 _ptr(gate), _ptr(out), _ptr(lse), _ptr(sel), _ptr(nsel),
                                 _ptr(pooled), _ptr(ws), ws.numel(), _stream(stream))
     _lib.check(st, "qsa_prefill")
-    return {"out": out, "lse": lse, "sel": sel, "nsel": nsel, "pooled": pooled}
+    # int32 error word at the start of the workspace: non-zero once the call
+    # has run if a kernel gave up on a bounded wait
+    return {"out": out, "lse": lse, "sel": sel, "nsel": nsel, "pooled": pooled,
+            "error_word": ws[:4].view(torch.int32)}
 
 
 def select(cfg: QSAConfig, iq, ik, iw, cu_seqlens, max_seqlen: int, *, want_scores=False,

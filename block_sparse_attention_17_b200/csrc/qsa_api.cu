@@ -117,6 +117,7 @@ struct Carve {
 };
 
 struct PrefillWs {
+  int* err;
   float* pooled;
   int* sel;
   int* nsel;
@@ -129,6 +130,7 @@ PrefillWs carve_prefill(const Geom& g, void* ws, int batch, int T, int max_seqle
   const int words = (max_nblk + 31) / 32;
   Carve c(ws);
   PrefillWs w;
+  w.err = c.take<int>(1);
   w.pooled = c.take<float>((size_t)batch * max_nblk * g.di);
   w.sel = c.take<int>((size_t)T * (g.k + 1));
   w.nsel = c.take<int>((size_t)T);
@@ -283,14 +285,23 @@ qsa_status qsa_prefill(const qsa_config* cfg, int batch, int total_tokens, int m
   float* pooled = pooled_out ? pooled_out : w.pooled;
   int* sel_p = sel ? sel : w.sel;
   int* nsel_p = nsel ? nsel : w.nsel;
+  QSA_CUDA(cudaMemsetAsync(w.err, 0, sizeof(int), st), "clear error word");
   stage_mark(0, st);
   s = prefill_select_common(cfg, g, batch, total_tokens, max_seqlen, cu_seqlens, iq, ik, iw, w,
                             pooled, sel_p, nsel_p, nullptr, st);
   if (s != QSA_OK) return s;
   stage_mark(1, st);
-  QSA_CUDA(launch_attn_prefill_simt(cfg->dtype, g, cu_seqlens, batch, max_seqlen, q, k, v, gate,
-                                    sel_p, nsel_p, out, lse, st),
-           "attention");
+  if (cfg->dtype == QSA_BF16 && attn_prefill_tc_supported(g)) {
+    const int max_nblk = (max_seqlen + g.B - 1) / g.B;
+    QSA_CUDA(launch_attn_prefill_tc(g, cu_seqlens, batch, total_tokens, max_seqlen,
+                                    (max_nblk + 31) / 32, w.bitmask, q, k, v, gate, out, lse,
+                                    w.err, st),
+             "attention (tensor cores)");
+  } else {
+    QSA_CUDA(launch_attn_prefill_simt(cfg->dtype, g, cu_seqlens, batch, max_seqlen, q, k, v,
+                                      gate, sel_p, nsel_p, out, lse, st),
+             "attention");
+  }
   stage_mark(2, st);
   return QSA_OK;
 }

@@ -1,0 +1,480 @@
+// QSA prefill attention on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// One CTA owns a tile of 128 query rows: Qt = 128 / G consecutive query
+// tokens of one sequence times the G query heads that share one KV head
+// (standard GQA, instagit MTPLX page "Qwen Sparse Attention (QSA)"). It walks
+// the UNION of the selected blocks of its Qt queries (selected complete blocks
+// plus tail blocks), gathering each block's K and V rows with TMA, and masks
+// per row the blocks that row's query did not select and the keys after the
+// query inside its tail block. Rows never see a key outside their own
+// selection, so the result is exactly QSA; the only cost of sharing a tile is
+// the MMA work on masked entries.
+//
+// Warp roles (192 threads):
+//   warp 0      TMA producer: Q once, then K and V of each 128-key step
+//               (2 blocks of B = 64 or 1 block of B = 128) into rings of 3 K
+//               and 2 V stages.
+//   warp 1      allocates TMEM; one thread issues the MMAs:
+//               S[b] = Q K^T (SS, K-major, 128x128x128) into one of two TMEM
+//               buffers, then O += P V (A = P from TMEM, B = V MN-major).
+//   warps 2..5  softmax: thread i owns TMEM lane / row i; reads S, masks,
+//               online softmax in the log2 domain with lazy rescaling (O is
+//               rescaled only when the running max grows by more than 2^8),
+//               writes P as bf16 into the S buffer, and finally applies
+//               1/l and the sigmoid gate (llama.cpp PR #27739 page: sigmoid
+//               output gate) in the epilogue.
+// Every wait is bounded; a timeout sets the workspace error word and the CTA
+// unwinds (drains its TMA loads and MMAs, frees TMEM).
+#include "qsa_common.cuh"
+#include "qsa_kernels.h"
+#include "qsa_sm100.cuh"
+
+namespace qsa {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int kRows = 128;                  // M
+constexpr int kKeys = 128;                  // N of QK^T, K of PV
+constexpr int kHeadDim = 128;               // D
+constexpr int kNK = 3, kNV = 2;             // K / V ring depth
+constexpr int kChunkBytes = kRows * 128;    // 128 rows x 64 bf16
+constexpr int kTileBytes = 2 * kChunkBytes; // 128 rows x 128 bf16
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;   // log2 domain
+
+constexpr int kOffQ = 0;
+constexpr int kOffK = kOffQ + kTileBytes;
+constexpr int kOffV = kOffK + kNK * kTileBytes;
+constexpr int kOffBar = kOffV + kNV * kTileBytes;
+constexpr int kNumBars = 1 + 2 * kNK + 2 * kNV + 2 + 2 + 1 + 1;
+constexpr int kOffMisc = kOffBar + 8 * kNumBars;
+constexpr int kOffBits = kOffMisc + 64;
+constexpr int kMaxWords = kMaxBlocksPerSeq / 32;
+constexpr int kOffList = kOffBits + 4 * kMaxWords;
+constexpr int kSmemBytes = kOffList + 2 * kMaxBlocksPerSeq + 1024;   // + alignment slack
+
+struct TcParams {
+  Geom g;
+  const int* cu;
+  const uint32_t* bitmask;
+  int words;
+  int n_tiles;
+  int Qt;
+  int total_tokens;
+  const __nv_bfloat16* gate;
+  __nv_bfloat16* out;
+  float* lse;
+  int* err;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+template <int kB>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+                       const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const TcParams P) {
+  constexpr int kNh = kKeys / kB;   // blocks per 128-key step
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  const uint32_t sbase = smem_u32(smem);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.y, hk = blockIdx.z;
+  const int tile = P.n_tiles - 1 - static_cast<int>(blockIdx.x);   // longest tiles first
+  const int s0 = P.cu[b], L = P.cu[b + 1] - s0;
+  const int q0 = tile * P.Qt;
+  if (q0 >= L) return;
+  const int nq = min(P.Qt, L - q0);
+  const Geom& g = P.g;
+  const int G = g.G;
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = k_full + kNK;
+  uint64_t* v_full = k_empty + kNK;
+  uint64_t* v_empty = v_full + kNV;
+  uint64_t* s_full = v_empty + kNV;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_done = p_full + 2;
+  uint64_t* mma_done = o_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+  int* n_union_s = reinterpret_cast<int*>(smem + kOffMisc + 8);
+  uint32_t* ubits = reinterpret_cast<uint32_t*>(smem + kOffBits);
+  uint16_t* ulist = reinterpret_cast<uint16_t*>(smem + kOffList);
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < kNK; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
+    for (int i = 0; i < kNV; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&s_full[i], 1); mbar_init(&p_full[i], 128); }
+    mbar_init(o_done, 1);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async();
+  }
+  // union of the tile's selections (selected complete blocks + tail blocks)
+  for (int w = threadIdx.x; w < P.words; w += blockDim.x) {
+    uint32_t acc = 0;
+    for (int qi = 0; qi < nq; ++qi) acc |= P.bitmask[(size_t)(s0 + q0 + qi) * P.words + w];
+    ubits[w] = acc;
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+  __syncthreads();
+  if (warp == 0) {   // ascending list of the union's blocks
+    int base = 0;
+    for (int w0 = 0; w0 < P.words; w0 += 32) {
+      const int w = w0 + lane;
+      uint32_t bits = w < P.words ? ubits[w] : 0u;
+      const int c = __popc(bits);
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += v;
+      }
+      int off = base + incl - c;
+      while (bits) {
+        const int bp = __ffs(bits) - 1;
+        bits &= bits - 1;
+        ulist[off++] = static_cast<uint16_t>(w * 32 + bp);
+      }
+      base += __shfl_sync(kFull, incl, 31);
+    }
+    if (lane == 0) *n_union_s = base;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int n_union = *n_union_s;
+  const int n_iter = (n_union + kNh - 1) / kNh;
+
+  const uint32_t sQ = sbase + kOffQ;
+  const uint32_t sK = sbase + kOffK;
+  const uint32_t sV = sbase + kOffV;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && n_iter > 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      mbar_expect_tx(q_full, kTileBytes);
+      tma_load_3d(sQ, &tmQ, 0, hk * G, s0 + q0, q_full);
+      tma_load_3d(sQ + kChunkBytes, &tmQ, 64, hk * G, s0 + q0, q_full);
+      auto issue = [&](const CUtensorMap* tm, uint32_t dst, uint64_t* full, int j) {
+        mbar_expect_tx(full, kTileBytes);
+#pragma unroll
+        for (int h = 0; h < kNh; ++h) {
+          const int e = j * kNh + h;
+          // a missing second block reads rows past the tensor: TMA fills zeros
+          const int tok = e < n_union ? s0 + static_cast<int>(ulist[e]) * kB : P.total_tokens;
+#pragma unroll
+          for (int dc = 0; dc < 2; ++dc)
+            tma_load_3d(dst + dc * kChunkBytes + h * kB * 128, tm, dc * 64, hk, tok, full);
+        }
+      };
+      auto issue_k = [&](int j) -> bool {
+        const int s = j % kNK;
+        if (j >= kNK && !mbar_wait(&k_empty[s], ((j / kNK) - 1) & 1, abort_flag)) return false;
+        issue(&tmK, sK + s * kTileBytes, &k_full[s], j);
+        return true;
+      };
+      auto issue_v = [&](int j) -> bool {
+        const int s = j % kNV;
+        if (j >= kNV && !mbar_wait(&v_empty[s], ((j / kNV) - 1) & 1, abort_flag)) return false;
+        issue(&tmV, sV + s * kTileBytes, &v_full[s], j);
+        return true;
+      };
+      int nk = 0, nv = 0;   // loads issued
+      if (issue_k(0)) {
+        nk = 1;
+        for (int it = 0; it < n_iter; ++it) {
+          if (it + 1 < n_iter) {
+            if (!issue_k(it + 1)) break;
+            nk = it + 2;
+          }
+          if (!issue_v(it)) break;
+          nv = it + 1;
+        }
+      }
+      // drain: no TMA write may still be in flight when the CTA exits
+      mbar_wait(q_full, 0, abort_flag);
+      for (int j = max(0, nk - kNK); j < nk; ++j) mbar_wait(&k_full[j % kNK], (j / kNK) & 1, abort_flag);
+      for (int j = max(0, nv - kNV); j < nv; ++j) mbar_wait(&v_full[j % kNV], (j / kNV) & 1, abort_flag);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0 && n_iter > 0) {
+      constexpr uint32_t idq = idesc_bf16_f32(kRows, kKeys, false, false);
+      constexpr uint32_t idv = idesc_bf16_f32(kRows, kHeadDim, false, true);
+      const uint32_t tO = tmem + 256;
+      auto qk = [&](int it) -> bool {
+        const int s = it % kNK;
+        if (!mbar_wait(&k_full[s], (it / kNK) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t d = tmem + (it & 1) * 128;
+        const uint32_t kb = sK + s * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kHeadDim / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
+          umma_ss(d, desc_sw128(sQ + off, 16, 1024), desc_sw128(kb + off, 16, 1024), idq,
+                  kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&k_empty[s]);
+        umma_commit(&s_full[it & 1]);
+        return true;
+      };
+      auto pv = [&](int j) -> bool {
+        const int sb = j & 1, sv = j % kNV;
+        if (!mbar_wait(&p_full[sb], (j >> 1) & 1, abort_flag)) return false;
+        if (!mbar_wait(&v_full[sv], (j / kNV) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t vb = sV + sv * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kKeys / 16; ++kk) {
+          umma_ts(tO, tmem + sb * 128 + kk * 8, desc_sw128(vb + kk * 2048, kChunkBytes, 1024),
+                  idv, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&v_empty[sv]);
+        umma_commit(o_done);
+        return true;
+      };
+      bool ok = mbar_wait(q_full, 0, abort_flag);
+      if (ok) tc_fence_after();
+      for (int it = 0; ok && it < n_iter; ++it) {
+        ok = qk(it);
+        if (ok && it > 0) ok = pv(it - 1);
+      }
+      if (ok) pv(n_iter - 1);
+      umma_commit(mma_done);
+      mbar_wait(mma_done, 0, abort_flag);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int qi = r / G, gg = r - qi * G;
+    const bool valid = qi < nq;
+    const int pos = q0 + qi;
+    const size_t t = static_cast<size_t>(s0) + pos;
+    const int h = hk * G + gg;
+    const uint32_t* mrow = P.bitmask + (valid ? t : 0) * P.words;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const float sc = g.sm_scale_log2;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int it = 0; it < n_iter; ++it) {
+      const int sb = it & 1;
+      if (!__all_sync(kFull, mbar_wait(&s_full[sb], (it >> 1) & 1, abort_flag))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sv[kKeys];
+#pragma unroll
+      for (int c = 0; c < kKeys / 32; ++c) tmem_ld32(lane_base + sb * 128 + c * 32, sv + c * 32);
+      tmem_wait_ld();
+      int lim[kNh];
+#pragma unroll
+      for (int hh = 0; hh < kNh; ++hh) {
+        const int e = it * kNh + hh;
+        const int blk = e < n_union ? static_cast<int>(ulist[e]) : -1;
+        int v = 0;
+        if (valid && blk >= 0 && ((mrow[blk >> 5] >> (blk & 31)) & 1u))
+          v = min(kB, pos + 1 - blk * kB);   // the tail block stops at the query
+        lim[hh] = v;
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kKeys; ++c) {
+        const float x = __uint_as_float(sv[c]) * sc;
+        if ((c % kB) < lim[c / kB]) mx = fmaxf(mx, x);
+      }
+      float m_tgt = m_used, alpha = 1.f;
+      if (mx > m_used + kRescaleThreshold || (m_used == -INFINITY && mx != -INFINITY)) {
+        m_tgt = mx;
+        alpha = exp2f(m_used - mx);   // 0 when m_used is -inf
+      }
+      const float ref = m_tgt == -INFINITY ? 0.f : m_tgt;
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < kKeys; c += 2) {
+        const float x0 = __uint_as_float(sv[c]) * sc, x1 = __uint_as_float(sv[c + 1]) * sc;
+        const float p0 = ((c % kB) < lim[c / kB]) ? exp2f(x0 - ref) : 0.f;
+        const float p1 = (((c + 1) % kB) < lim[(c + 1) / kB]) ? exp2f(x1 - ref) : 0.f;
+        sum += p0 + p1;
+        sv[c >> 1] = pack_bf16(p0, p1);   // in place: index c/2 <= c
+      }
+      l = l * alpha + sum;
+      tmem_st32(lane_base + sb * 128, sv);
+      tmem_st32(lane_base + sb * 128 + 32, sv + 32);
+      if (it > 0 && __any_sync(kFull, alpha != 1.f)) {
+        if (!__all_sync(kFull, mbar_wait(o_done, (it - 1) & 1, abort_flag))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < kHeadDim / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(lane_base + 256 + c * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(lane_base + 256 + c * 32, o);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&p_full[sb]);
+      m_used = m_tgt;
+    }
+    // ------------------------------------------------------------ epilogue
+    if (ok && n_iter > 0 &&
+        __all_sync(kFull, mbar_wait(o_done, (n_iter - 1) & 1, abort_flag))) {
+      tc_fence_after();
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* orow = P.out + (t * g.Hq + h) * kHeadDim;
+      const __nv_bfloat16* grow = P.gate + (g.gate_headwise ? (t * g.Hq + h) : (t * g.Hq + h) * kHeadDim);
+      const float gh = (valid && g.gate_headwise) ? sigmoidf_(__bfloat162float(grow[0])) : 0.f;
+#pragma unroll
+      for (int c = 0; c < kHeadDim / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(lane_base + 256 + c * 32, o);
+        tmem_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int v8 = 0; v8 < 4; ++v8) {
+            const int d0 = c * 32 + v8 * 8;
+            float gv[8];
+            if (g.gate_headwise) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) gv[i] = gh;
+            } else {
+              const uint4 gu = *reinterpret_cast<const uint4*>(grow + d0);
+              const uint32_t gw[4] = {gu.x, gu.y, gu.z, gu.w};
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                gv[2 * i] = sigmoidf_(__uint_as_float(gw[i] << 16));
+                gv[2 * i + 1] = sigmoidf_(__uint_as_float(gw[i] & 0xffff0000u));
+              }
+            }
+            uint4 ou;
+            ou.x = pack_bf16(__uint_as_float(o[v8 * 8 + 0]) * inv_l * gv[0],
+                             __uint_as_float(o[v8 * 8 + 1]) * inv_l * gv[1]);
+            ou.y = pack_bf16(__uint_as_float(o[v8 * 8 + 2]) * inv_l * gv[2],
+                             __uint_as_float(o[v8 * 8 + 3]) * inv_l * gv[3]);
+            ou.z = pack_bf16(__uint_as_float(o[v8 * 8 + 4]) * inv_l * gv[4],
+                             __uint_as_float(o[v8 * 8 + 5]) * inv_l * gv[5]);
+            ou.w = pack_bf16(__uint_as_float(o[v8 * 8 + 6]) * inv_l * gv[6],
+                             __uint_as_float(o[v8 * 8 + 7]) * inv_l * gv[7]);
+            *reinterpret_cast<uint4*>(orow + d0) = ou;
+          }
+        }
+      }
+      if (valid && P.lse)
+        P.lse[t * g.Hq + h] = l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY;
+    }
+  }
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+  if (threadIdx.x == 0 && *abort_flag) atomicExch(P.err, 1);
+}
+
+// ------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 3-D bf16 map over a [rows, heads, D] tensor with a (64, box_h, box_rows) box.
+bool make_map_3d(CUtensorMap* m, const void* ptr, int D, int heads, int rows, int box_h,
+                 int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)heads * D * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_h, (cuuint32_t)box_rows};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool attn_prefill_tc_supported(const Geom& g) {
+  return g.D == kHeadDim && (g.B == 64 || g.B == 128) && g.G >= 1 && (kRows % g.G) == 0;
+}
+
+cudaError_t launch_attn_prefill_tc(const Geom& g, const int* cu, int batch, int total_tokens,
+                                   int max_seqlen, int words, const uint32_t* bitmask,
+                                   const void* q, const void* k, const void* v, const void* gate,
+                                   void* out, float* lse, int* err, cudaStream_t st) {
+  if (batch == 0 || max_seqlen == 0 || total_tokens == 0) return cudaSuccess;
+  const int Qt = kRows / g.G;
+  CUtensorMap mq, mk, mv;
+  if (!make_map_3d(&mq, q, kHeadDim, g.Hq, total_tokens, g.G, Qt) ||
+      !make_map_3d(&mk, k, kHeadDim, g.Hkv, total_tokens, 1, g.B) ||
+      !make_map_3d(&mv, v, kHeadDim, g.Hkv, total_tokens, 1, g.B))
+    return cudaErrorInvalidValue;
+  TcParams p;
+  p.g = g;
+  p.cu = cu;
+  p.bitmask = bitmask;
+  p.words = words;
+  p.n_tiles = (max_seqlen + Qt - 1) / Qt;
+  p.Qt = Qt;
+  p.total_tokens = total_tokens;
+  p.gate = static_cast<const __nv_bfloat16*>(gate);
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.err = err;
+  dim3 grid(p.n_tiles, batch, g.Hkv);
+  cudaError_t e;
+  if (g.B == 64) {
+    e = cudaFuncSetAttribute(attn_prefill_tc_kernel<64>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attn_prefill_tc_kernel<64><<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, p);
+  } else {
+    e = cudaFuncSetAttribute(attn_prefill_tc_kernel<128>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attn_prefill_tc_kernel<128><<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, p);
+  }
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace qsa

@@ -42,4 +42,10 @@ cudaError_t launch_attn_decode_simt(qsa_dtype dt, const Geom& g, int batch, int 
                                     const int* sel, const int* nsel, float* part_ml,
                                     float* part_o, void* out, float* lse, cudaStream_t st);
 
+bool attn_prefill_tc_supported(const Geom& g);
+cudaError_t launch_attn_prefill_tc(const Geom& g, const int* cu, int batch, int total_tokens,
+                                   int max_seqlen, int words, const uint32_t* bitmask,
+                                   const void* q, const void* k, const void* v, const void* gate,
+                                   void* out, float* lse, int* err, cudaStream_t st);
+
 }  // namespace qsa

@@ -117,8 +117,11 @@ qsa_status qsa_set_stage_events(void* const* events, int count);
  *   pooled_out  optional [batch, ceil(max_seqlen/B), di] fp32: pooled keys of
  *               every complete block (rows past a sequence's last complete
  *               block are left untouched)
- * host_total_tokens and max_seqlen are host integers that must describe the
- * device cu_seqlens; a device length above max_seqlen is not detected. */
+ * total_tokens and max_seqlen are host integers that must describe the
+ * device cu_seqlens; a device length above max_seqlen is not detected.
+ * The first 4 bytes of the workspace receive an int32 error word: 0 once the
+ * call has run, non-zero if a kernel gave up on one of its bounded waits
+ * (a pipeline that stopped making progress); the outputs are then invalid. */
 size_t qsa_prefill_workspace_size(const qsa_config* cfg, int batch, int total_tokens,
                                   int max_seqlen);
 

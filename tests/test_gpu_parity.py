@@ -46,6 +46,7 @@ def run_prefill(w, inp):
                     d["cu_seqlens"], inp["max_seqlen"], want_lse=True, want_sel=True,
                     want_pooled=True)
     torch.cuda.synchronize()
+    assert int(r["error_word"].item()) == 0, "a prefill kernel gave up on a bounded wait"
     return r
 
 
