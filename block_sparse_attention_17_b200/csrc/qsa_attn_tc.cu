@@ -1,28 +1,32 @@
 // QSA prefill attention on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
 //
-// One CTA owns a tile of 128 query rows: Qt = 128 / G consecutive query
-// tokens of one sequence times the G query heads that share one KV head
-// (standard GQA, instagit MTPLX page "Qwen Sparse Attention (QSA)"). It walks
-// the UNION of the selected blocks of its Qt queries (selected complete blocks
-// plus tail blocks), gathering each block's K and V rows with TMA, and masks
-// per row the blocks that row's query did not select and the keys after the
-// query inside its tail block. Rows never see a key outside their own
-// selection, so the result is exactly QSA; the only cost of sharing a tile is
-// the MMA work on masked entries.
+// One CTA owns two tiles of 128 query rows each. A tile is Qt = 128 / G
+// consecutive query tokens of one sequence times the G query heads that share
+// one KV head (standard GQA, instagit MTPLX page "Qwen Sparse Attention
+// (QSA)"). The CTA walks the UNION of the selected blocks of its 2 * Qt
+// queries (selected complete blocks plus tail blocks), gathering each block's
+// K and V rows with TMA, and masks per row the blocks that row's query did not
+// select and the keys after the query inside its tail block. Rows never see a
+// key outside their own selection, so the result is exactly QSA; the cost of
+// sharing a tile is MMA work on masked entries.
 //
-// Warp roles (192 threads):
-//   warp 0      TMA producer: Q once, then K and V of each 128-key step
-//               (2 blocks of B = 64 or 1 block of B = 128) into rings of 3 K
-//               and 2 V stages.
-//   warp 1      allocates TMEM; one thread issues the MMAs:
-//               S[b] = Q K^T (SS, K-major, 128x128x128) into one of two TMEM
-//               buffers, then O += P V (A = P from TMEM, B = V MN-major).
-//   warps 2..5  softmax: thread i owns TMEM lane / row i; reads S, masks,
-//               online softmax in the log2 domain with lazy rescaling (O is
-//               rescaled only when the running max grows by more than 2^8),
-//               writes P as bf16 into the S buffer, and finally applies
-//               1/l and the sigmoid gate (llama.cpp PR #27739 page: sigmoid
-//               output gate) in the epilogue.
+// Warp roles (320 threads):
+//   warp 0      TMA producer: Q of both tiles once, then K and V of each
+//               128-key step (2 blocks of B = 64 or 1 block of B = 128) into
+//               2-deep K and V rings.
+//   warp 1      allocates TMEM; one thread issues the MMAs. Per step j and
+//               tile t: O_t += P_t(j-1) V(j-1) (A = P from TMEM, V MN-major),
+//               then S_t = Q_t K(j)^T (SS, K-major). The two tiles alternate,
+//               so the tensor core works on one tile while the other tile's
+//               softmax runs.
+//   warps 2..5  softmax of tile 0, warps 6..9 softmax of tile 1: thread i of
+//               a tile owns TMEM lane / row i; it reads S twice (max, then
+//               exponentials), masks, keeps the online softmax in the log2
+//               domain with lazy rescaling (O is rescaled only when the running
+//               max grows by more than 2^8), writes P as bf16 over S, and in
+//               the epilogue applies 1/l and the sigmoid gate (llama.cpp PR
+//               #27739 page: sigmoid output gate). A quarter of the
+//               exponentials run on the FMA pipe (exp2_poly) to unload MUFU.
 // Every wait is bounded; a timeout sets the workspace error word and the CTA
 // unwinds (drains its TMA loads and MMAs, frees TMEM).
 #include "qsa_common.cuh"
@@ -35,21 +39,22 @@ using namespace sm100;
 
 namespace {
 
-constexpr int kRows = 128;                  // M
+constexpr int kRows = 128;                  // M per tile
+constexpr int kTiles = 2;                   // query tiles per CTA
 constexpr int kKeys = 128;                  // N of QK^T, K of PV
 constexpr int kHeadDim = 128;               // D
-constexpr int kNK = 3, kNV = 2;             // K / V ring depth
+constexpr int kNK = 2, kNV = 2;             // K / V ring depth
 constexpr int kChunkBytes = kRows * 128;    // 128 rows x 64 bf16
 constexpr int kTileBytes = 2 * kChunkBytes; // 128 rows x 128 bf16
-constexpr int kThreads = 192;
-constexpr uint32_t kTmemCols = 512;
+constexpr int kThreads = 64 + kTiles * 128;
+constexpr uint32_t kTmemCols = 512;         // S0 S1 O0 O1, 128 columns each
 constexpr float kRescaleThreshold = 8.0f;   // log2 domain
 
 constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kTileBytes;
+constexpr int kOffK = kOffQ + kTiles * kTileBytes;
 constexpr int kOffV = kOffK + kNK * kTileBytes;
 constexpr int kOffBar = kOffV + kNV * kTileBytes;
-constexpr int kNumBars = 1 + 2 * kNK + 2 * kNV + 2 + 2 + 1 + 1;
+constexpr int kNumBars = 1 + 2 * kNK + 2 * kNV + 3 * kTiles + 1;
 constexpr int kOffMisc = kOffBar + 8 * kNumBars;
 constexpr int kOffBits = kOffMisc + 64;
 constexpr int kMaxWords = kMaxBlocksPerSeq / 32;
@@ -61,8 +66,8 @@ struct TcParams {
   const int* cu;
   const uint32_t* bitmask;
   int words;
-  int n_tiles;
-  int Qt;
+  int n_ctas;        // CTAs per (sequence, KV head) along the query axis
+  int Qt;            // queries per tile
   int total_tokens;
   const __nv_bfloat16* gate;
   __nv_bfloat16* out;
@@ -88,11 +93,12 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.y, hk = blockIdx.z;
-  const int tile = P.n_tiles - 1 - static_cast<int>(blockIdx.x);   // longest tiles first
+  const int cta = P.n_ctas - 1 - static_cast<int>(blockIdx.x);   // longest first
   const int s0 = P.cu[b], L = P.cu[b + 1] - s0;
-  const int q0 = tile * P.Qt;
+  const int q0 = cta * kTiles * P.Qt;
   if (q0 >= L) return;
-  const int nq = min(P.Qt, L - q0);
+  const int nq = min(kTiles * P.Qt, L - q0);   // valid queries of the CTA
+  const int nt = nq > P.Qt ? 2 : 1;            // tiles with at least one valid query
   const Geom& g = P.g;
   const int G = g.G;
 
@@ -102,10 +108,10 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
   uint64_t* k_empty = k_full + kNK;
   uint64_t* v_full = k_empty + kNK;
   uint64_t* v_empty = v_full + kNV;
-  uint64_t* s_full = v_empty + kNV;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* o_done = p_full + 2;
-  uint64_t* mma_done = o_done + 1;
+  uint64_t* s_full = v_empty + kNV;     // [tile]
+  uint64_t* p_full = s_full + kTiles;   // [tile]
+  uint64_t* o_done = p_full + kTiles;   // [tile]
+  uint64_t* mma_done = o_done + kTiles;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
   int* n_union_s = reinterpret_cast<int*>(smem + kOffMisc + 8);
@@ -116,14 +122,17 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
     mbar_init(q_full, 1);
     for (int i = 0; i < kNK; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
     for (int i = 0; i < kNV; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(&s_full[i], 1); mbar_init(&p_full[i], 128); }
-    mbar_init(o_done, 1);
+    for (int t = 0; t < kTiles; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 128);
+      mbar_init(&o_done[t], 1);
+    }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async();
   }
-  // union of the tile's selections (selected complete blocks + tail blocks)
+  // union of the CTA's selections (selected complete blocks + tail blocks)
   for (int w = threadIdx.x; w < P.words; w += blockDim.x) {
     uint32_t acc = 0;
     for (int qi = 0; qi < nq; ++qi) acc |= P.bitmask[(size_t)(s0 + q0 + qi) * P.words + w];
@@ -170,9 +179,11 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      mbar_expect_tx(q_full, kTileBytes);
-      tma_load_3d(sQ, &tmQ, 0, hk * G, s0 + q0, q_full);
-      tma_load_3d(sQ + kChunkBytes, &tmQ, 64, hk * G, s0 + q0, q_full);
+      mbar_expect_tx(q_full, kTiles * kTileBytes);
+      for (int t = 0; t < kTiles; ++t)
+        for (int dc = 0; dc < 2; ++dc)
+          tma_load_3d(sQ + t * kTileBytes + dc * kChunkBytes, &tmQ, dc * 64, hk * G,
+                      s0 + q0 + t * P.Qt, q_full);
       auto issue = [&](const CUtensorMap* tm, uint32_t dst, uint64_t* full, int j) {
         mbar_expect_tx(full, kTileBytes);
 #pragma unroll
@@ -211,117 +222,165 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
       }
       // drain: no TMA write may still be in flight when the CTA exits
       mbar_wait(q_full, 0, abort_flag);
-      for (int j = max(0, nk - kNK); j < nk; ++j) mbar_wait(&k_full[j % kNK], (j / kNK) & 1, abort_flag);
-      for (int j = max(0, nv - kNV); j < nv; ++j) mbar_wait(&v_full[j % kNV], (j / kNV) & 1, abort_flag);
+      for (int j = max(0, nk - kNK); j < nk; ++j)
+        mbar_wait(&k_full[j % kNK], (j / kNK) & 1, abort_flag);
+      for (int j = max(0, nv - kNV); j < nv; ++j)
+        mbar_wait(&v_full[j % kNV], (j / kNV) & 1, abort_flag);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0 && n_iter > 0) {
       constexpr uint32_t idq = idesc_bf16_f32(kRows, kKeys, false, false);
       constexpr uint32_t idv = idesc_bf16_f32(kRows, kHeadDim, false, true);
-      const uint32_t tO = tmem + 256;
-      auto qk = [&](int it) -> bool {
-        const int s = it % kNK;
-        if (!mbar_wait(&k_full[s], (it / kNK) & 1, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t d = tmem + (it & 1) * 128;
-        const uint32_t kb = sK + s * kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < kHeadDim / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
-          umma_ss(d, desc_sw128(sQ + off, 16, 1024), desc_sw128(kb + off, 16, 1024), idq,
-                  kk > 0 ? 1u : 0u);
-        }
-        umma_commit(&k_empty[s]);
-        umma_commit(&s_full[it & 1]);
-        return true;
-      };
-      auto pv = [&](int j) -> bool {
-        const int sb = j & 1, sv = j % kNV;
-        if (!mbar_wait(&p_full[sb], (j >> 1) & 1, abort_flag)) return false;
-        if (!mbar_wait(&v_full[sv], (j / kNV) & 1, abort_flag)) return false;
+      // O_t += P_t(j) V(j)
+      auto pv = [&](int t, int j) -> bool {
+        const int sv = j % kNV;
+        if (!mbar_wait(&p_full[t], j & 1, abort_flag)) return false;
+        if (t == 0 && !mbar_wait(&v_full[sv], (j / kNV) & 1, abort_flag)) return false;
         tc_fence_after();
         const uint32_t vb = sV + sv * kTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < kKeys / 16; ++kk) {
-          umma_ts(tO, tmem + sb * 128 + kk * 8, desc_sw128(vb + kk * 2048, kChunkBytes, 1024),
-                  idv, (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(&v_empty[sv]);
-        umma_commit(o_done);
+        for (int kk = 0; kk < kKeys / 16; ++kk)
+          umma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
+                  desc_sw128(vb + kk * 2048, kChunkBytes, 1024), idv,
+                  (j > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&o_done[t]);
+        if (t == nt - 1) umma_commit(&v_empty[sv]);
         return true;
       };
+      // S_t = Q_t K(j)^T
+      auto qk = [&](int t, int j) {
+        const uint32_t kb = sK + (j % kNK) * kTileBytes;
+        const uint32_t qb = sQ + t * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kHeadDim / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
+          umma_ss(tmem + t * 128, desc_sw128(qb + off, 16, 1024), desc_sw128(kb + off, 16, 1024),
+                  idq, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[t]);
+      };
       bool ok = mbar_wait(q_full, 0, abort_flag);
-      if (ok) tc_fence_after();
-      for (int it = 0; ok && it < n_iter; ++it) {
-        ok = qk(it);
-        if (ok && it > 0) ok = pv(it - 1);
+      for (int j = 0; ok && j < n_iter; ++j) {
+        ok = mbar_wait(&k_full[j % kNK], (j / kNK) & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        for (int t = 0; t < nt; ++t) {
+          if (j > 0 && !(ok = pv(t, j - 1))) break;
+          qk(t, j);
+        }
+        umma_commit(&k_empty[j % kNK]);
       }
-      if (ok) pv(n_iter - 1);
+      for (int t = 0; ok && t < nt; ++t) ok = pv(t, n_iter - 1);
       umma_commit(mma_done);
       mbar_wait(mma_done, 0, abort_flag);
     }
   } else {
     // ------------------------------------------------------------ softmax
+    const int t = (warp - 2) >> 2;            // tile
     const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
-    const int qi = r / G, gg = r - qi * G;
+    const int r = quarter * 32 + lane;        // row within the tile = TMEM lane
+    const int qi = t * P.Qt + r / G, gg = r % G;
     const bool valid = qi < nq;
     const int pos = q0 + qi;
-    const size_t t = static_cast<size_t>(s0) + pos;
+    const size_t tok = static_cast<size_t>(s0) + pos;
     const int h = hk * G + gg;
-    const uint32_t* mrow = P.bitmask + (valid ? t : 0) * P.words;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const uint32_t* mrow = P.bitmask + (valid ? tok : 0) * P.words;
+    const uint32_t tS = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + t * 128;
+    const uint32_t tO = tS + 256;
     const float sc = g.sm_scale_log2;
     float m_used = -INFINITY, l = 0.f;
-    bool ok = true;
-    for (int it = 0; it < n_iter; ++it) {
-      const int sb = it & 1;
-      if (!__all_sync(kFull, mbar_wait(&s_full[sb], (it >> 1) & 1, abort_flag))) {
+    bool ok = t < nt;
+    for (int j = 0; ok && j < n_iter; ++j) {
+      if (!__all_sync(kFull, mbar_wait(&s_full[t], j & 1, abort_flag))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t sv[kKeys];
-#pragma unroll
-      for (int c = 0; c < kKeys / 32; ++c) tmem_ld32(lane_base + sb * 128 + c * 32, sv + c * 32);
-      tmem_wait_ld();
+      // visible keys per block of this step: lim = B for a selected complete
+      // block, pos + 1 - start for the tail block, 0 otherwise
       int lim[kNh];
+      bool any_vis[kNh], partial[kNh];
 #pragma unroll
       for (int hh = 0; hh < kNh; ++hh) {
-        const int e = it * kNh + hh;
+        const int e = j * kNh + hh;
         const int blk = e < n_union ? static_cast<int>(ulist[e]) : -1;
         int v = 0;
         if (valid && blk >= 0 && ((mrow[blk >> 5] >> (blk & 31)) & 1u))
-          v = min(kB, pos + 1 - blk * kB);   // the tail block stops at the query
+          v = min(kB, pos + 1 - blk * kB);
         lim[hh] = v;
+        any_vis[hh] = __any_sync(kFull, v > 0);
+        partial[hh] = __any_sync(kFull, v > 0 && v < kB);
       }
+      // pass 1: running max over the visible raw scores
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < kKeys; ++c) {
-        const float x = __uint_as_float(sv[c]) * sc;
-        if ((c % kB) < lim[c / kB]) mx = fmaxf(mx, x);
+      for (int c = 0; c < kKeys / 32; ++c) {
+        const int hh = (c * 32) / kB;
+        if (!any_vis[hh]) continue;
+        uint32_t v[32];
+        tmem_ld32(tS + c * 32, v);
+        tmem_wait_ld();
+        if (partial[hh]) {
+          const int base = (c * 32) % kB;
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (base + i < lim[hh]) mx = fmaxf(mx, __uint_as_float(v[i]));
+        } else {
+          float cm = __uint_as_float(v[0]);
+#pragma unroll
+          for (int i = 1; i < 32; ++i) cm = fmaxf(cm, __uint_as_float(v[i]));
+          if (lim[hh] > 0) mx = fmaxf(mx, cm);
+        }
       }
+      mx *= sc;   // sc > 0 keeps the order (and -inf)
       float m_tgt = m_used, alpha = 1.f;
       if (mx > m_used + kRescaleThreshold || (m_used == -INFINITY && mx != -INFINITY)) {
         m_tgt = mx;
         alpha = exp2f(m_used - mx);   // 0 when m_used is -inf
       }
       const float ref = m_tgt == -INFINITY ? 0.f : m_tgt;
+      // pass 2: probabilities, written as bf16 pairs over the first 64 columns
       float sum = 0.f;
 #pragma unroll
-      for (int c = 0; c < kKeys; c += 2) {
-        const float x0 = __uint_as_float(sv[c]) * sc, x1 = __uint_as_float(sv[c + 1]) * sc;
-        const float p0 = ((c % kB) < lim[c / kB]) ? exp2f(x0 - ref) : 0.f;
-        const float p1 = (((c + 1) % kB) < lim[(c + 1) / kB]) ? exp2f(x1 - ref) : 0.f;
-        sum += p0 + p1;
-        sv[c >> 1] = pack_bf16(p0, p1);   // in place: index c/2 <= c
+      for (int c = 0; c < kKeys / 32; ++c) {
+        const int hh = (c * 32) / kB;
+        uint32_t pk[16];
+        if (!any_vis[hh]) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pk[i] = 0u;
+        } else {
+          uint32_t v[32];
+          tmem_ld32(tS + c * 32, v);
+          tmem_wait_ld();
+          // rows that do not see this block subtract +inf: exp2(-inf) = 0
+          const float nref = lim[hh] > 0 ? -ref : -INFINITY;
+          const int base = (c * 32) % kB;
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            float x0 = fmaf(__uint_as_float(v[i]), sc, nref);
+            float x1 = fmaf(__uint_as_float(v[i + 1]), sc, nref);
+            if (partial[hh]) {
+              if (base + i >= lim[hh]) x0 = -INFINITY;
+              if (base + i + 1 >= lim[hh]) x1 = -INFINITY;
+            }
+            float p0, p1;
+            if ((i & 7) == 6) {   // a quarter of the elements on the FMA pipe
+              p0 = exp2_poly(x0);
+              p1 = exp2_poly(x1);
+            } else {
+              p0 = exp2f(x0);
+              p1 = exp2f(x1);
+            }
+            sum += p0 + p1;
+            pk[i >> 1] = pack_bf16(p0, p1);
+          }
+        }
+        tmem_st16(tS + c * 16, pk);
       }
       l = l * alpha + sum;
-      tmem_st32(lane_base + sb * 128, sv);
-      tmem_st32(lane_base + sb * 128 + 32, sv + 32);
-      if (it > 0 && __any_sync(kFull, alpha != 1.f)) {
-        if (!__all_sync(kFull, mbar_wait(o_done, (it - 1) & 1, abort_flag))) {
+      if (j > 0 && __any_sync(kFull, alpha != 1.f)) {
+        if (!__all_sync(kFull, mbar_wait(&o_done[t], (j - 1) & 1, abort_flag))) {
           ok = false;
           break;
         }
@@ -329,30 +388,31 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
 #pragma unroll
         for (int c = 0; c < kHeadDim / 32; ++c) {
           uint32_t o[32];
-          tmem_ld32(lane_base + 256 + c * 32, o);
+          tmem_ld32(tO + c * 32, o);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(lane_base + 256 + c * 32, o);
+          tmem_st32(tO + c * 32, o);
         }
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full[sb]);
+      mbar_arrive(&p_full[t]);
       m_used = m_tgt;
     }
     // ------------------------------------------------------------ epilogue
     if (ok && n_iter > 0 &&
-        __all_sync(kFull, mbar_wait(o_done, (n_iter - 1) & 1, abort_flag))) {
+        __all_sync(kFull, mbar_wait(&o_done[t], (n_iter - 1) & 1, abort_flag))) {
       tc_fence_after();
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
-      __nv_bfloat16* orow = P.out + (t * g.Hq + h) * kHeadDim;
-      const __nv_bfloat16* grow = P.gate + (g.gate_headwise ? (t * g.Hq + h) : (t * g.Hq + h) * kHeadDim);
+      __nv_bfloat16* orow = P.out + (tok * g.Hq + h) * kHeadDim;
+      const __nv_bfloat16* grow =
+          P.gate + (g.gate_headwise ? (tok * g.Hq + h) : (tok * g.Hq + h) * kHeadDim);
       const float gh = (valid && g.gate_headwise) ? sigmoidf_(__bfloat162float(grow[0])) : 0.f;
 #pragma unroll
       for (int c = 0; c < kHeadDim / 32; ++c) {
         uint32_t o[32];
-        tmem_ld32(lane_base + 256 + c * 32, o);
+        tmem_ld32(tO + c * 32, o);
         tmem_wait_ld();
         if (valid) {
 #pragma unroll
@@ -385,7 +445,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
         }
       }
       if (valid && P.lse)
-        P.lse[t * g.Hq + h] = l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY;
+        P.lse[tok * g.Hq + h] = l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY;
     }
   }
   // ------------------------------------------------------------ teardown
@@ -453,14 +513,14 @@ cudaError_t launch_attn_prefill_tc(const Geom& g, const int* cu, int batch, int 
   p.cu = cu;
   p.bitmask = bitmask;
   p.words = words;
-  p.n_tiles = (max_seqlen + Qt - 1) / Qt;
+  p.n_ctas = (max_seqlen + kTiles * Qt - 1) / (kTiles * Qt);
   p.Qt = Qt;
   p.total_tokens = total_tokens;
   p.gate = static_cast<const __nv_bfloat16*>(gate);
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
   p.err = err;
-  dim3 grid(p.n_tiles, batch, g.Hkv);
+  dim3 grid(p.n_ctas, batch, g.Hkv);
   cudaError_t e;
   if (g.B == 64) {
     e = cudaFuncSetAttribute(attn_prefill_tc_kernel<64>,

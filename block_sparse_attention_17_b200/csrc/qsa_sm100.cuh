@@ -157,6 +157,14 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
       QSA_W8(0), QSA_W8(8), QSA_W8(16), QSA_W8(24)
       : "memory");
 }
+// 16 consecutive 32-bit TMEM columns of this thread's lane (warp-collective).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      QSA_W8(0), QSA_W8(8)
+      : "memory");
+}
 #undef QSA_R8
 #undef QSA_W8
 
@@ -165,6 +173,25 @@ __device__ __forceinline__ void tmem_wait_ld() {
 }
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// ------------------------------------------------------------ exp2 on the FMA pipe
+// 2^x without the MUFU unit, for part of the softmax exponentials: range
+// reduction x = j + f with j = round(x), f in [-1/2, 1/2] (the rounding done by
+// adding 1.5 * 2^23), a cubic for 2^f, and 2^j added into the exponent bits.
+// The cubic's coefficients are a relative-error least-squares fit of 2^f on
+// [-1/2, 1/2] made for this library (max relative error 7.6e-5, far below the
+// 2^-9 rounding of the bf16 probabilities it feeds). Inputs below -126 give
+// about 2^-126 instead of 0.
+__device__ __forceinline__ float exp2_poly(float x) {
+  constexpr float kMagic = 12582912.0f;    // 1.5 * 2^23
+  x = fmaxf(x, -126.0f);
+  const float t = x + kMagic;
+  const float f = x - (t - kMagic);
+  float p = fmaf(0.055177733302116394f, f, 0.24262635409832f);
+  p = fmaf(p, f, 0.6932612061500549f);
+  p = fmaf(p, f, 0.9999268651008606f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 // ------------------------------------------------------------ descriptors
