@@ -25,8 +25,7 @@
 //               domain with lazy rescaling (O is rescaled only when the running
 //               max grows by more than 2^8), writes P as bf16 over S, and in
 //               the epilogue applies 1/l and the sigmoid gate (llama.cpp PR
-//               #27739 page: sigmoid output gate). A quarter of the
-//               exponentials run on the FMA pipe (exp2_poly) to unload MUFU.
+//               #27739 page: sigmoid output gate).
 // Every wait is bounded; a timeout sets the workspace error word and the CTA
 // unwinds (drains its TMA loads and MMAs, frees TMEM).
 #include "qsa_common.cuh"
@@ -291,27 +290,37 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
     const float sc = g.sm_scale_log2;
     float m_used = -INFINITY, l = 0.f;
     bool ok = t < nt;
+    // visible keys of this row in block e of the union: B for a selected
+    // complete block, pos + 1 - start for its tail block, 0 otherwise. The
+    // selection words are fetched one step ahead of their use.
+    auto fetch = [&](int j, uint32_t* w, int* blk) {
+#pragma unroll
+      for (int hh = 0; hh < kNh; ++hh) {
+        const int e = j * kNh + hh;
+        blk[hh] = e < n_union ? static_cast<int>(ulist[e]) : -1;
+        w[hh] = (valid && blk[hh] >= 0) ? __ldg(mrow + (blk[hh] >> 5)) : 0u;
+      }
+    };
+    uint32_t wnext[kNh];
+    int bnext[kNh];
+    if (ok) fetch(0, wnext, bnext);
     for (int j = 0; ok && j < n_iter; ++j) {
+      int lim[kNh];
+#pragma unroll
+      for (int hh = 0; hh < kNh; ++hh)
+        lim[hh] = ((wnext[hh] >> (bnext[hh] & 31)) & 1u) ? min(kB, pos + 1 - bnext[hh] * kB) : 0;
+      if (j + 1 < n_iter) fetch(j + 1, wnext, bnext);
+      bool any_vis[kNh], partial[kNh];
+#pragma unroll
+      for (int hh = 0; hh < kNh; ++hh) {
+        any_vis[hh] = __any_sync(kFull, lim[hh] > 0);
+        partial[hh] = __any_sync(kFull, lim[hh] > 0 && lim[hh] < kB);
+      }
       if (!__all_sync(kFull, mbar_wait(&s_full[t], j & 1, abort_flag))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      // visible keys per block of this step: lim = B for a selected complete
-      // block, pos + 1 - start for the tail block, 0 otherwise
-      int lim[kNh];
-      bool any_vis[kNh], partial[kNh];
-#pragma unroll
-      for (int hh = 0; hh < kNh; ++hh) {
-        const int e = j * kNh + hh;
-        const int blk = e < n_union ? static_cast<int>(ulist[e]) : -1;
-        int v = 0;
-        if (valid && blk >= 0 && ((mrow[blk >> 5] >> (blk & 31)) & 1u))
-          v = min(kB, pos + 1 - blk * kB);
-        lim[hh] = v;
-        any_vis[hh] = __any_sync(kFull, v > 0);
-        partial[hh] = __any_sync(kFull, v > 0 && v < kB);
-      }
       // pass 1: running max over the visible raw scores
       float mx = -INFINITY;
 #pragma unroll
@@ -325,7 +334,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
           const int base = (c * 32) % kB;
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            if (base + i < lim[hh]) mx = fmaxf(mx, __uint_as_float(v[i]));
+            mx = fmaxf(mx, base + i < lim[hh] ? __uint_as_float(v[i]) : -INFINITY);
         } else {
           float cm = __uint_as_float(v[0]);
 #pragma unroll
@@ -337,11 +346,11 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
       float m_tgt = m_used, alpha = 1.f;
       if (mx > m_used + kRescaleThreshold || (m_used == -INFINITY && mx != -INFINITY)) {
         m_tgt = mx;
-        alpha = exp2f(m_used - mx);   // 0 when m_used is -inf
+        alpha = ex2_approx(m_used - mx);   // 0 when m_used is -inf
       }
       const float ref = m_tgt == -INFINITY ? 0.f : m_tgt;
       // pass 2: probabilities, written as bf16 pairs over the first 64 columns
-      float sum = 0.f;
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < kKeys / 32; ++c) {
         const int hh = (c * 32) / kB;
@@ -355,29 +364,23 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
           tmem_wait_ld();
           // rows that do not see this block subtract +inf: exp2(-inf) = 0
           const float nref = lim[hh] > 0 ? -ref : -INFINITY;
-          const int base = (c * 32) % kB;
+          if (partial[hh]) {
+            const int base = (c * 32) % kB;
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (base + i >= lim[hh]) v[i] = __float_as_uint(-INFINITY);
+          }
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
-            float x0 = fmaf(__uint_as_float(v[i]), sc, nref);
-            float x1 = fmaf(__uint_as_float(v[i + 1]), sc, nref);
-            if (partial[hh]) {
-              if (base + i >= lim[hh]) x0 = -INFINITY;
-              if (base + i + 1 >= lim[hh]) x1 = -INFINITY;
-            }
-            float p0, p1;
-            if ((i & 7) == 6) {   // a quarter of the elements on the FMA pipe
-              p0 = exp2_poly(x0);
-              p1 = exp2_poly(x1);
-            } else {
-              p0 = exp2f(x0);
-              p1 = exp2f(x1);
-            }
-            sum += p0 + p1;
+            const float p0 = ex2_approx(fmaf(__uint_as_float(v[i]), sc, nref));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(v[i + 1]), sc, nref));
+            s4[(i >> 1) & 3] += p0 + p1;
             pk[i >> 1] = pack_bf16(p0, p1);
           }
         }
         tmem_st16(tS + c * 16, pk);
       }
+      const float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
       l = l * alpha + sum;
       if (j > 0 && __any_sync(kFull, alpha != 1.f)) {
         if (!__all_sync(kFull, mbar_wait(&o_done[t], (j - 1) & 1, abort_flag))) {

@@ -45,24 +45,46 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Suspends the calling thread until the phase completes or about `ns`
+// nanoseconds pass (the hardware resumes it as soon as the phase completes).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
 // About 2 s at the B200's top clock: far beyond any legitimate wait in these
 // kernels, short enough that a broken pipeline ends with an error, not a hang.
 constexpr long long kWaitCycles = 4000000000LL;
 
 // Waits for the phase of `bar` with the given parity. Gives up when another
 // thread of the CTA has already given up (*abort != 0) or after kWaitCycles,
-// in which case it sets *abort. Returns whether the phase completed.
+// in which case it sets *abort. Returns whether the phase completed. The
+// thread sleeps in the barrier between checks instead of spinning.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
     if (*abort) return false;
     if (clock64() - t0 > kWaitCycles) {
       *abort = 1;
       return false;
     }
   }
+}
+
+// 2^x on the MUFU unit (flushes denormal results to zero; exp2(-inf) = 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // ------------------------------------------------------------------ TMA
