@@ -4,7 +4,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/qsa.h"
+#include "qsa.h"
 
 namespace qsa {
 
