@@ -10,7 +10,7 @@
 // key outside their own selection, so the result is exactly QSA; the cost of
 // sharing a tile is MMA work on masked entries.
 //
-// Warp roles (320 threads):
+// Warp roles (576 threads):
 //   warp 0      TMA producer: Q of both tiles once, then K and V of each
 //               128-key step (2 blocks of B = 64 or 1 block of B = 128) into
 //               2-deep K and V rings.
@@ -19,13 +19,13 @@
 //               then S_t = Q_t K(j)^T (SS, K-major). The two tiles alternate,
 //               so the tensor core works on one tile while the other tile's
 //               softmax runs.
-//   warps 2..5  softmax of tile 0, warps 6..9 softmax of tile 1: thread i of
-//               a tile owns TMEM lane / row i; it reads S twice (max, then
-//               exponentials), masks, keeps the online softmax in the log2
-//               domain with lazy rescaling (O is rescaled only when the running
-//               max grows by more than 2^8), writes P as bf16 over S, and in
-//               the epilogue applies 1/l and the sigmoid gate (llama.cpp PR
-//               #27739 page: sigmoid output gate).
+//   warps 2..9  softmax of tile 0, warps 10..17 softmax of tile 1: two
+//               threads share each row (TMEM lane), one per 64-column half;
+//               they mask, exchange the partial row max, keep the online
+//               softmax in the log2 domain with lazy rescaling (O is rescaled
+//               only when the running max grows by more than 2^8), write P as
+//               bf16 over S, and in the epilogue apply 1/l and the sigmoid
+//               gate (llama.cpp PR #27739 page: sigmoid output gate).
 // Every wait is bounded; a timeout sets the workspace error word and the CTA
 // unwinds (drains its TMA loads and MMAs, frees TMEM).
 #include "qsa_common.cuh"
@@ -45,9 +45,14 @@ constexpr int kHeadDim = 128;               // D
 constexpr int kNK = 2, kNV = 2;             // K / V ring depth
 constexpr int kChunkBytes = kRows * 128;    // 128 rows x 64 bf16
 constexpr int kTileBytes = 2 * kChunkBytes; // 128 rows x 128 bf16
-constexpr int kThreads = 64 + kTiles * 128;
+constexpr int kSoftmaxThreads = 256;          // per tile: 128 rows x 2 column halves
+constexpr int kThreads = 64 + kTiles * kSoftmaxThreads;
 constexpr uint32_t kTmemCols = 512;         // S0 S1 O0 O1, 128 columns each
 constexpr float kRescaleThreshold = 8.0f;   // log2 domain
+// Of every 8 probability pairs, this many are exponentiated on the FMA pipe
+// (exp2_poly2) instead of MUFU, whose 16 results per clock and SM would
+// otherwise bound the softmax.
+constexpr int kPolyPairsOf8 = 2;
 
 constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + kTiles * kTileBytes;
@@ -58,7 +63,8 @@ constexpr int kOffMisc = kOffBar + 8 * kNumBars;
 constexpr int kOffBits = kOffMisc + 64;
 constexpr int kMaxWords = kMaxBlocksPerSeq / 32;
 constexpr int kOffList = kOffBits + 4 * kMaxWords;
-constexpr int kSmemBytes = kOffList + 2 * kMaxBlocksPerSeq + 1024;   // + alignment slack
+constexpr int kOffXch = kOffList + 2 * kMaxBlocksPerSeq;   // [tile][slot][half][row] floats
+constexpr int kSmemBytes = kOffXch + 4 * kTiles * 2 * 2 * kRows + 1024;   // + alignment slack
 
 struct TcParams {
   Geom g;
@@ -123,7 +129,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
     for (int i = 0; i < kNV; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
     for (int t = 0; t < kTiles; ++t) {
       mbar_init(&s_full[t], 1);
-      mbar_init(&p_full[t], 128);
+      mbar_init(&p_full[t], kSoftmaxThreads);
       mbar_init(&o_done[t], 1);
     }
     mbar_init(mma_done, 1);
@@ -240,7 +246,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
         const uint32_t vb = sV + sv * kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk)
-          umma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
+          umma_ts(tmem + 256 + t * 128, tmem + t * 128 + (kk >> 2) * 64 + (kk & 3) * 8,
                   desc_sw128(vb + kk * 2048, kChunkBytes, 1024), idv,
                   (j > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&o_done[t]);
@@ -276,7 +282,12 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int t = (warp - 2) >> 2;            // tile
+    // Tile t has 8 warps: each row (TMEM lane) is shared by two threads, one
+    // per 64-column half of S; they exchange their partial row max through
+    // shared memory behind a named barrier of the two warps.
+    const int wt = warp - 2;
+    const int t = wt >> 3;                    // tile
+    const int hf = (wt >> 2) & 1;             // column half
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;        // row within the tile = TMEM lane
     const int qi = t * P.Qt + r / G, gg = r % G;
@@ -287,101 +298,93 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
     const uint32_t* mrow = P.bitmask + (valid ? tok : 0) * P.words;
     const uint32_t tS = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + t * 128;
     const uint32_t tO = tS + 256;
+    float* xch = reinterpret_cast<float*>(smem + kOffXch);
+    auto xslot = [&](int slot, int half) { return xch + ((t * 2 + slot) * 2 + half) * kRows + r; };
+    const int bar_id = 1 + t * 4 + quarter;
     const float sc = g.sm_scale_log2;
     float m_used = -INFINITY, l = 0.f;
     bool ok = t < nt;
-    // visible keys of this row in block e of the union: B for a selected
-    // complete block, pos + 1 - start for its tail block, 0 otherwise. The
-    // selection words are fetched one step ahead of their use.
-    auto fetch = [&](int j, uint32_t* w, int* blk) {
-#pragma unroll
-      for (int hh = 0; hh < kNh; ++hh) {
-        const int e = j * kNh + hh;
-        blk[hh] = e < n_union ? static_cast<int>(ulist[e]) : -1;
-        w[hh] = (valid && blk[hh] >= 0) ? __ldg(mrow + (blk[hh] >> 5)) : 0u;
-      }
+    // the block under this thread's columns at step j, and its selection word
+    // (fetched one step ahead of its use)
+    auto fetch = [&](int j, uint32_t& w, int& blk) {
+      const int e = kB == 64 ? j * 2 + hf : j;
+      blk = e < n_union ? static_cast<int>(ulist[e]) : -1;
+      w = (valid && blk >= 0) ? __ldg(mrow + (blk >> 5)) : 0u;
     };
-    uint32_t wnext[kNh];
-    int bnext[kNh];
-    if (ok) fetch(0, wnext, bnext);
+    uint32_t wn = 0u;
+    int bn = -1;
+    if (ok) fetch(0, wn, bn);
     for (int j = 0; ok && j < n_iter; ++j) {
-      int lim[kNh];
-#pragma unroll
-      for (int hh = 0; hh < kNh; ++hh)
-        lim[hh] = ((wnext[hh] >> (bnext[hh] & 31)) & 1u) ? min(kB, pos + 1 - bnext[hh] * kB) : 0;
-      if (j + 1 < n_iter) fetch(j + 1, wnext, bnext);
-      bool any_vis[kNh], partial[kNh];
-#pragma unroll
-      for (int hh = 0; hh < kNh; ++hh) {
-        any_vis[hh] = __any_sync(kFull, lim[hh] > 0);
-        partial[hh] = __any_sync(kFull, lim[hh] > 0 && lim[hh] < kB);
+      // visible keys among this thread's 64 columns: all of a selected
+      // complete block, the keys up to the query in its tail block, or none
+      int lim = 0;
+      if (bn >= 0 && ((wn >> (bn & 31)) & 1u)) {
+        const int col0 = bn * kB + (kB == 128 ? 64 * hf : 0);   // position of column 0
+        lim = max(0, min(64, pos + 1 - col0));
       }
+      if (j + 1 < n_iter) fetch(j + 1, wn, bn);
+      const bool any_vis = __any_sync(kFull, lim > 0);
+      const bool partial = __any_sync(kFull, lim > 0 && lim < 64);
       if (!__all_sync(kFull, mbar_wait(&s_full[t], j & 1, abort_flag))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      // pass 1: running max over the visible raw scores
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < kKeys / 32; ++c) {
-        const int hh = (c * 32) / kB;
-        if (!any_vis[hh]) continue;
-        uint32_t v[32];
-        tmem_ld32(tS + c * 32, v);
+      float pm = -INFINITY;
+      {
+        uint32_t v[64];
+        tmem_ld32(tS + 64 * hf, v);
+        tmem_ld32(tS + 64 * hf + 32, v + 32);
         tmem_wait_ld();
-        if (partial[hh]) {
-          const int base = (c * 32) % kB;
+        if (any_vis) {
+          float cm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            mx = fmaxf(mx, base + i < lim[hh] ? __uint_as_float(v[i]) : -INFINITY);
-        } else {
-          float cm = __uint_as_float(v[0]);
-#pragma unroll
-          for (int i = 1; i < 32; ++i) cm = fmaxf(cm, __uint_as_float(v[i]));
-          if (lim[hh] > 0) mx = fmaxf(mx, cm);
+          for (int i = 0; i < 64; ++i)
+            cm[i & 3] = fmaxf(cm[i & 3], (!partial || i < lim) ? __uint_as_float(v[i]) : -INFINITY);
+          pm = lim > 0 ? fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3])) : -INFINITY;
         }
       }
-      mx *= sc;   // sc > 0 keeps the order (and -inf)
+      *xslot(j & 1, hf) = pm;
+      named_bar_sync(bar_id, 64);
+      const float mx = fmaxf(pm, *xslot(j & 1, hf ^ 1)) * sc;
       float m_tgt = m_used, alpha = 1.f;
       if (mx > m_used + kRescaleThreshold || (m_used == -INFINITY && mx != -INFINITY)) {
         m_tgt = mx;
         alpha = ex2_approx(m_used - mx);   // 0 when m_used is -inf
       }
       const float ref = m_tgt == -INFINITY ? 0.f : m_tgt;
-      // pass 2: probabilities, written as bf16 pairs over the first 64 columns
-      float s4[4] = {0.f, 0.f, 0.f, 0.f};
+      // P of this half is packed over the first 32 of its own 64 S columns,
+      // so the two halves never touch each other's S
+      float2 s2a = make_float2(0.f, 0.f), s2b = make_float2(0.f, 0.f);
+      uint32_t v[64];
+      if (!any_vis) {
 #pragma unroll
-      for (int c = 0; c < kKeys / 32; ++c) {
-        const int hh = (c * 32) / kB;
-        uint32_t pk[16];
-        if (!any_vis[hh]) {
+        for (int i = 0; i < 32; ++i) v[i] = 0u;
+      } else {
+        tmem_ld32(tS + 64 * hf, v);
+        tmem_ld32(tS + 64 * hf + 32, v + 32);
+        tmem_wait_ld();
+        if (partial) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) pk[i] = 0u;
-        } else {
-          uint32_t v[32];
-          tmem_ld32(tS + c * 32, v);
-          tmem_wait_ld();
-          // rows that do not see this block subtract +inf: exp2(-inf) = 0
-          const float nref = lim[hh] > 0 ? -ref : -INFINITY;
-          if (partial[hh]) {
-            const int base = (c * 32) % kB;
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (base + i >= lim[hh]) v[i] = __float_as_uint(-INFINITY);
-          }
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const float p0 = ex2_approx(fmaf(__uint_as_float(v[i]), sc, nref));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(v[i + 1]), sc, nref));
-            s4[(i >> 1) & 3] += p0 + p1;
-            pk[i >> 1] = pack_bf16(p0, p1);
-          }
+          for (int i = 0; i < 64; ++i)
+            if (i >= lim) v[i] = __float_as_uint(-INFINITY);
         }
-        tmem_st16(tS + c * 16, pk);
+        // rows that do not see these columns subtract +inf: exp2(-inf) = 0
+        const float nref = lim > 0 ? -ref : -INFINITY;
+        const float2 sc2 = make_float2(sc, sc), nref2 = make_float2(nref, nref);
+#pragma unroll
+        for (int i = 0; i < 64; i += 2) {
+          const float2 x = ffma2(make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])),
+                                 sc2, nref2);
+          const float2 pp = ((i >> 1) & 7) < kPolyPairsOf8
+                                ? exp2_poly2(x)
+                                : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          if ((i & 2) == 0) s2a = fadd2(s2a, pp); else s2b = fadd2(s2b, pp);
+          v[i >> 1] = pack_bf16(pp.x, pp.y);   // pair i/2 lands at index i/2 <= i
+        }
       }
-      const float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-      l = l * alpha + sum;
+      tmem_st32(tS + 64 * hf, v);
+      l = l * alpha + ((s2a.x + s2a.y) + (s2b.x + s2b.y));
       if (j > 0 && __any_sync(kFull, alpha != 1.f)) {
         if (!__all_sync(kFull, mbar_wait(&o_done[t], (j - 1) & 1, abort_flag))) {
           ok = false;
@@ -389,13 +392,13 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
         }
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < kHeadDim / 32; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t o[32];
-          tmem_ld32(tO + c * 32, o);
+          tmem_ld32(tO + 64 * hf + c * 32, o);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tO + c * 32, o);
+          tmem_st32(tO + 64 * hf + c * 32, o);
         }
       }
       tmem_wait_st();
@@ -404,23 +407,27 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
       m_used = m_tgt;
     }
     // ------------------------------------------------------------ epilogue
+    // each thread writes its 64 output dims; l is the sum of both halves
     if (ok && n_iter > 0 &&
         __all_sync(kFull, mbar_wait(&o_done[t], (n_iter - 1) & 1, abort_flag))) {
       tc_fence_after();
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      *xslot(n_iter & 1, hf) = l;
+      named_bar_sync(bar_id, 64);
+      const float lt = l + *xslot(n_iter & 1, hf ^ 1);
+      const float inv_l = lt > 0.f ? 1.f / lt : 0.f;
       __nv_bfloat16* orow = P.out + (tok * g.Hq + h) * kHeadDim;
       const __nv_bfloat16* grow =
           P.gate + (g.gate_headwise ? (tok * g.Hq + h) : (tok * g.Hq + h) * kHeadDim);
       const float gh = (valid && g.gate_headwise) ? sigmoidf_(__bfloat162float(grow[0])) : 0.f;
 #pragma unroll
-      for (int c = 0; c < kHeadDim / 32; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t o[32];
-        tmem_ld32(tO + c * 32, o);
+        tmem_ld32(tO + 64 * hf + c * 32, o);
         tmem_wait_ld();
         if (valid) {
 #pragma unroll
           for (int v8 = 0; v8 < 4; ++v8) {
-            const int d0 = c * 32 + v8 * 8;
+            const int d0 = 64 * hf + c * 32 + v8 * 8;
             float gv[8];
             if (g.gate_headwise) {
 #pragma unroll
@@ -447,8 +454,8 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
           }
         }
       }
-      if (valid && P.lse)
-        P.lse[tok * g.Hq + h] = l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY;
+      if (valid && hf == 0 && P.lse)
+        P.lse[tok * g.Hq + h] = lt > 0.f ? (m_used + log2f(lt)) * kLn2 : -INFINITY;
     }
   }
   // ------------------------------------------------------------ teardown

@@ -198,6 +198,28 @@ __device__ __forceinline__ void tmem_wait_st() {
 }
 
 // ------------------------------------------------------------ exp2 on the FMA pipe
+// Packed fp32 pairs (sm_100): d = a * b + c and d = a + b, lane by lane.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<uint64_t*>(&a)), "l"(*reinterpret_cast<uint64_t*>(&b)),
+        "l"(*reinterpret_cast<uint64_t*>(&c)));
+  return *reinterpret_cast<float2*>(&d);
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<uint64_t*>(&a)), "l"(*reinterpret_cast<uint64_t*>(&b)));
+  return *reinterpret_cast<float2*>(&d);
+}
+
+// Named barrier over `nthreads` threads (a multiple of 32) of the CTA.
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // 2^x without the MUFU unit, for part of the softmax exponentials: range
 // reduction x = j + f with j = round(x), f in [-1/2, 1/2] (the rounding done by
 // adding 1.5 * 2^23), a cubic for 2^f, and 2^j added into the exponent bits.
@@ -214,6 +236,22 @@ __device__ __forceinline__ float exp2_poly(float x) {
   p = fmaf(p, f, 0.6932612061500549f);
   p = fmaf(p, f, 0.9999268651008606f);
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// exp2_poly on a pair, with packed fp32x2 arithmetic.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  const float2 magic = make_float2(12582912.0f, 12582912.0f);
+  x.x = fmaxf(x.x, -126.0f);
+  x.y = fmaxf(x.y, -126.0f);
+  const float2 t = fadd2(x, magic);
+  const float2 j = fadd2(t, make_float2(-12582912.0f, -12582912.0f));
+  const float2 f = fadd2(x, make_float2(-j.x, -j.y));
+  float2 p = ffma2(make_float2(0.055177733302116394f, 0.055177733302116394f), f,
+                   make_float2(0.24262635409832f, 0.24262635409832f));
+  p = ffma2(p, f, make_float2(0.6932612061500549f, 0.6932612061500549f));
+  p = ffma2(p, f, make_float2(0.9999268651008606f, 0.9999268651008606f));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
 // ------------------------------------------------------------ descriptors
