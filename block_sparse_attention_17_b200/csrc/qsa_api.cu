@@ -140,6 +140,7 @@ PrefillWs carve_prefill(const Geom& g, void* ws, int batch, int T, int max_seqle
 }
 
 struct DecodeWs {
+  int* err;
   float* scores;
   int* sel;
   int* nsel;
@@ -149,15 +150,25 @@ struct DecodeWs {
   size_t bytes;
 };
 
-DecodeWs carve_decode(const Geom& g, void* ws, int batch, int n_q, int cap) {
+bool decode_uses_mma(const qsa_config* cfg, const Geom& g, int n_q) {
+  return cfg->dtype == QSA_BF16 && attn_decode_mma_supported(g, n_q);
+}
+
+DecodeWs carve_decode(const qsa_config* cfg, const Geom& g, void* ws, int batch, int n_q,
+                      int cap) {
   DecodeWs w;
-  const int max_union = n_q * (g.k + 1);
-  const int pairs = std::max(1, batch * g.Hkv);
-  int nsplit = std::min(max_union, std::max(1, (kTargetCtas + pairs - 1) / pairs));
-  w.per_split = (max_union + nsplit - 1) / nsplit;
-  w.nsplit = (max_union + w.per_split - 1) / w.per_split;
+  if (decode_uses_mma(cfg, g, n_q)) {
+    decode_mma_split(g, batch, n_q, &w.nsplit, &w.per_split);
+  } else {
+    const int max_union = n_q * (g.k + 1);
+    const int pairs = std::max(1, batch * g.Hkv);
+    int nsplit = std::min(max_union, std::max(1, (kTargetCtas + pairs - 1) / pairs));
+    w.per_split = (max_union + nsplit - 1) / nsplit;
+    w.nsplit = (max_union + w.per_split - 1) / w.per_split;
+  }
   const int R = n_q * g.G;
   Carve c(ws);
+  w.err = c.take<int>(1);
   w.scores = c.take<float>((size_t)batch * n_q * (cap / g.B));
   w.sel = c.take<int>((size_t)batch * n_q * (g.k + 1));
   w.nsel = c.take<int>((size_t)batch * n_q);
@@ -189,6 +200,8 @@ qsa_status check_decode_dims(const qsa_config* cfg, int batch, int n_q, int cap)
   if (cap % cfg->block_size) return fail(QSA_ERR_INVALID_ARG, "cap must be a multiple of B");
   if (cap / cfg->block_size > kMaxDecodeBlocks)
     return fail(QSA_ERR_UNSUPPORTED, "more than %d cache blocks", kMaxDecodeBlocks);
+  if ((long long)batch * cap > 2147483647LL)
+    return fail(QSA_ERR_UNSUPPORTED, "batch * cap must fit in 31 bits");
   if (n_q > kMaxDecodeQ) return fail(QSA_ERR_UNSUPPORTED, "n_q > %d", kMaxDecodeQ);
   if (n_q * (cfg->num_q_heads / cfg->num_kv_heads) > kMaxDecodeRows)
     return fail(QSA_ERR_UNSUPPORTED, "n_q * group size > %d", kMaxDecodeRows);
@@ -331,7 +344,7 @@ qsa_status qsa_select(const qsa_config* cfg, int batch, int total_tokens, int ma
 
 size_t qsa_decode_workspace_size(const qsa_config* cfg, int batch, int n_q, int cap) {
   if (check_decode_dims(cfg, batch, n_q, cap) != QSA_OK) return 0;
-  return carve_decode(make_geom(cfg), nullptr, batch, n_q, cap).bytes;
+  return carve_decode(cfg, make_geom(cfg), nullptr, batch, n_q, cap).bytes;
 }
 
 static qsa_status decode_select_common(const qsa_config* cfg, const Geom& g, int batch, int n_q,
@@ -366,10 +379,10 @@ qsa_status qsa_decode(const qsa_config* cfg, int batch, int n_q, int cap, const 
   if (sel) QSA_REQUIRE(sel, "sel");
   if (nsel) QSA_REQUIRE(nsel, "nsel");
   const Geom g = make_geom(cfg);
-  const DecodeWs need = carve_decode(g, nullptr, batch, n_q, cap);
+  const DecodeWs need = carve_decode(cfg, g, nullptr, batch, n_q, cap);
   if (!workspace || workspace_bytes < need.bytes || ((uintptr_t)workspace & 255u))
     return fail(QSA_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned", need.bytes);
-  const DecodeWs w = carve_decode(g, workspace, batch, n_q, cap);
+  const DecodeWs w = carve_decode(cfg, g, workspace, batch, n_q, cap);
   cudaStream_t st = (cudaStream_t)stream;
   int* sel_p = sel ? sel : w.sel;
   int* nsel_p = nsel ? nsel : w.nsel;
@@ -378,10 +391,20 @@ qsa_status qsa_decode(const qsa_config* cfg, int batch, int n_q, int cap, const 
                            sel_p, nsel_p, nullptr, dev_err, st);
   if (s != QSA_OK) return s;
   stage_mark(1, st);
-  QSA_CUDA(launch_attn_decode_simt(cfg->dtype, g, batch, n_q, cap, w.nsplit, w.per_split, kv_len,
-                                   q, k_cache, v_cache, gate, sel_p, nsel_p, w.part_ml, w.part_o,
-                                   out, lse, st),
-           "decode attention");
+  if (decode_uses_mma(cfg, g, n_q)) {
+    QSA_CUDA(launch_attn_decode_mma(g, batch, n_q, cap, w.nsplit, w.per_split, kv_len, q,
+                                    k_cache, v_cache, sel_p, nsel_p, w.part_ml, w.part_o,
+                                    dev_err ? dev_err : w.err, st),
+             "decode attention");
+    QSA_CUDA(launch_decode_combine(cfg->dtype, g, batch, n_q, cap, w.nsplit, kv_len, w.part_ml,
+                                   w.part_o, gate, out, lse, st),
+             "decode combine");
+  } else {
+    QSA_CUDA(launch_attn_decode_simt(cfg->dtype, g, batch, n_q, cap, w.nsplit, w.per_split,
+                                     kv_len, q, k_cache, v_cache, gate, sel_p, nsel_p, w.part_ml,
+                                     w.part_o, out, lse, st),
+             "decode attention");
+  }
   stage_mark(2, st);
   return QSA_OK;
 }
@@ -401,10 +424,10 @@ qsa_status qsa_select_decode(const qsa_config* cfg, int batch, int n_q, int cap,
   QSA_REQUIRE(sel, "sel"); QSA_REQUIRE(nsel, "nsel");
   if (scores) QSA_REQUIRE(scores, "scores");
   const Geom g = make_geom(cfg);
-  const DecodeWs need = carve_decode(g, nullptr, batch, n_q, cap);
+  const DecodeWs need = carve_decode(cfg, g, nullptr, batch, n_q, cap);
   if (!workspace || workspace_bytes < need.bytes || ((uintptr_t)workspace & 255u))
     return fail(QSA_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned", need.bytes);
-  const DecodeWs w = carve_decode(g, workspace, batch, n_q, cap);
+  const DecodeWs w = carve_decode(cfg, g, workspace, batch, n_q, cap);
   return decode_select_common(cfg, g, batch, n_q, cap, kv_len, iq, ik_cache, iw, pooled_cache,
                               w, sel, nsel, scores, dev_err, (cudaStream_t)stream);
 }

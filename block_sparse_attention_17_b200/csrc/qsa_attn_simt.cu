@@ -378,6 +378,25 @@ cudaError_t launch_attn_prefill_simt(qsa_dtype dt, const Geom& g, const int* cu,
   return cudaGetLastError();
 }
 
+cudaError_t launch_decode_combine(qsa_dtype dt, const Geom& g, int batch, int n_q, int cap,
+                                  int nsplit, const int* kv_len, const float* part_ml,
+                                  const float* part_o, const void* gate, void* out, float* lse,
+                                  cudaStream_t st) {
+  if (batch == 0) return cudaSuccess;
+  dim3 cgrid(n_q * g.Hq, batch);
+#define QSA_CB(T, DD)                                                                     \
+  decode_combine_kernel<T, DD><<<cgrid, DD, 0, st>>>(g, n_q, cap, nsplit, kv_len, part_ml,  \
+                                                     part_o, (const T*)gate, (T*)out, lse)
+  if (dt == QSA_BF16) {
+    if (g.D == 128) { QSA_CB(__nv_bfloat16, 128); } else { QSA_CB(__nv_bfloat16, 64); }
+  } else {
+    if (g.D == 128) { QSA_CB(float, 128); } else { QSA_CB(float, 64); }
+  }
+#undef QSA_CB
+  note_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t launch_attn_decode_simt(qsa_dtype dt, const Geom& g, int batch, int n_q, int cap,
                                     int nsplit, int per_split, const int* kv_len, const void* q,
                                     const void* kc, const void* vc, const void* gate,

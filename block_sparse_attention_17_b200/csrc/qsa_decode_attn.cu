@@ -1,0 +1,458 @@
+// QSA decode attention, split-KV over the selected blocks (sm_100a).
+//
+// One decode step reads, per (sequence, KV head), only the K/V rows of the
+// union of the step's n_q queries' selections (selected complete blocks plus
+// tail blocks): the gather consumer of the selection, never a mask over the
+// whole cache (ramgpt "Porting Qwen4 to llama.cpp", section "CUDA Optimization
+// Should Follow State Correctness"). The step is bound by HBM bandwidth, so
+// the kernel is built around streaming: the union is cut into 64-key chunks,
+// each CTA takes a contiguous range of chunks of one (sequence, KV head), and
+// a producer warp streams each chunk's K and V tiles with TMA through a
+// 3-stage ring (two CTAs per SM keep about 190 KB in flight per SM).
+//
+// The arithmetic per chunk is tiny (at most 16 query rows = n_q x group
+// heads), so the four consumer warps use warp-level bf16 MMAs (m16n8k16,
+// fp32 accumulation): warp w takes keys [16w, 16w + 16) of each chunk and
+// keeps its own online-softmax state (log2 domain); the four states are
+// merged at the end and written as one (m, l, O) partial per row, which
+// qsa_combine merges across CTAs before the sigmoid gate.
+#include "qsa_common.cuh"
+#include "qsa_kernels.h"
+#include "qsa_sm100.cuh"
+
+namespace qsa {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int kD = 128;
+constexpr int kChunk = 64;                      // keys per ring stage
+constexpr int kStages = 3;
+constexpr int kBoxBytes = kChunk * 128;         // 64 keys x 64 dims bf16 (one TMA box)
+constexpr int kTileBytes = 2 * kBoxBytes;       // 64 keys x 128 dims
+constexpr int kStageBytes = 2 * kTileBytes;     // K + V
+constexpr int kConsumers = 4;
+constexpr int kThreads = 32 * (kConsumers + 1);
+constexpr int kQStride = kD * 2 + 16;           // padded bf16 row of Q in shared memory
+constexpr int kMaxUnion = 4 * (kMaxTopK + 1);
+
+constexpr int kOffStages = 0;
+constexpr int kOffQ = kOffStages + kStages * kStageBytes;
+constexpr int kOffBar = kOffQ + 16 * kQStride;
+constexpr int kOffMisc = kOffBar + 8 * 2 * kStages;
+constexpr int kOffUnion = kOffMisc + 64;
+constexpr int kSmemBytes = kOffUnion + 8 * kMaxUnion + 1024;
+
+struct DecParams {
+  Geom g;
+  int n_q, cap, nsplit, per_split;   // per_split: chunks per CTA
+  const int* kv_len;
+  const __nv_bfloat16* q;
+  const int* sel;
+  const int* nsel;
+  float* part_ml;
+  float* part_o;
+  int* err;
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                          uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+// D = A (16x16 bf16, row) * B (16x8 bf16, col) + D, fp32
+__device__ __forceinline__ void mma_bf16(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Byte offset of (row, dim) in a 64-row K/V tile stored as two 128-byte-swizzled
+// TMA boxes (dims 0..63, then 64..127); dim must be a multiple of 8.
+__device__ __forceinline__ uint32_t tile_off(int row, int dim) {
+  const int box = dim >> 6;
+  const int chunk = (dim & 63) >> 3;
+  return box * kBoxBytes + row * 128 + ((chunk ^ (row & 7)) << 4);
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
+attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const DecParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  const uint32_t sbase = smem_u32(smem);
+  const Geom& g = P.g;
+  const int split = blockIdx.x, b = blockIdx.y, hk = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = g.G, n_q = P.n_q, R = n_q * G;
+  const int kv = P.kv_len[b];
+  const size_t row0 = (((size_t)b * g.Hkv + hk) * P.nsplit + split) * R;
+  if (kv < n_q || kv > P.cap) {   // reported by the pooling kernel; skip the sequence
+    for (int r = threadIdx.x; r < R; r += blockDim.x) {
+      P.part_ml[2 * (row0 + r)] = -INFINITY;
+      P.part_ml[2 * (row0 + r) + 1] = 0.f;
+    }
+    return;
+  }
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* empty = full + kStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc);
+  int* n_chunks_s = reinterpret_cast<int*>(smem + kOffMisc + 4);
+  int* u_blk = reinterpret_cast<int*>(smem + kOffUnion);
+  int* u_qm = u_blk + kMaxUnion;
+  const int cpb = g.B / kChunk;   // chunks per block
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumers);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async();
+    // union of the n_q selections, ascending, with a mask of the queries that
+    // selected each block (their tail blocks included)
+    const int kp1 = g.k + 1;
+    const int* sb = P.sel + (size_t)b * n_q * kp1;
+    const int* nb = P.nsel + (size_t)b * n_q;
+    int idx[4] = {0, 0, 0, 0}, cnt = 0;
+    while (true) {
+      int best = 0x7fffffff;
+      for (int i = 0; i < n_q; ++i)
+        if (idx[i] < nb[i]) best = min(best, sb[i * kp1 + idx[i]]);
+      if (best == 0x7fffffff) break;
+      int qm = 0;
+      for (int i = 0; i < n_q; ++i)
+        if (idx[i] < nb[i] && sb[i * kp1 + idx[i]] == best) {
+          qm |= 1 << i;
+          ++idx[i];
+        }
+      u_blk[cnt] = best;
+      u_qm[cnt] = qm;
+      ++cnt;
+    }
+    *n_chunks_s = cnt * cpb;
+  }
+  // Q rows r = i * G + gi (query i, head hk * G + gi), zero beyond R
+  for (int e = threadIdx.x; e < 16 * (kD / 8); e += blockDim.x) {
+    const int r = e / (kD / 8), c8 = e % (kD / 8);
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (r < R) {
+      const int i = r / G, gi = r % G;
+      v = *reinterpret_cast<const uint4*>(
+          P.q + (((size_t)b * n_q + i) * g.Hq + hk * G + gi) * kD + c8 * 8);
+    }
+    *reinterpret_cast<uint4*>(smem + kOffQ + r * kQStride + c8 * 16) = v;
+  }
+  __syncthreads();
+  const int n_chunks = *n_chunks_s;
+  const int c0 = split * P.per_split;
+  const int c1 = min(n_chunks, c0 + P.per_split);
+  const int my_chunks = max(0, c1 - c0);
+  const size_t krow_base = (size_t)b * P.cap;
+
+  if (warp == kConsumers) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && my_chunks > 0) {
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      int issued = 0;
+      for (int c = 0; c < my_chunks; ++c) {
+        const int s = c % kStages;
+        if (c >= kStages && !mbar_wait(&empty[s], ((c / kStages) - 1) & 1, abort_flag)) break;
+        const int uc = c0 + c;
+        const int key0 = u_blk[uc / cpb] * g.B + (uc % cpb) * kChunk;
+        const int rowk = (int)(krow_base + key0);
+        const uint32_t st = sbase + kOffStages + s * kStageBytes;
+        mbar_expect_tx(&full[s], kStageBytes);
+        tma_load_3d(st, &tmK, 0, hk, rowk, &full[s]);
+        tma_load_3d(st + kBoxBytes, &tmK, 64, hk, rowk, &full[s]);
+        tma_load_3d(st + kTileBytes, &tmV, 0, hk, rowk, &full[s]);
+        tma_load_3d(st + kTileBytes + kBoxBytes, &tmV, 64, hk, rowk, &full[s]);
+        issued = c + 1;
+      }
+      for (int c = max(0, issued - kStages); c < issued; ++c)
+        mbar_wait(&full[c % kStages], (c / kStages) & 1, abort_flag);
+    }
+  } else {
+    // ------------------------------------------------------------ consumers
+    const int gq = lane >> 2, tq = lane & 3;   // mma fragment row group / column pair
+    // Q as A fragments, all 8 k-slices of 16 dims
+    uint32_t qa[8][4];
+    {
+      const int mi = lane >> 3, ri = lane & 7;
+      const int row = (mi & 1) * 8 + ri;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const int col = kk * 16 + (mi >> 1) * 8;
+        ldsm_x4(sbase + kOffQ + row * kQStride + col * 2, qa[kk][0], qa[kk][1], qa[kk][2],
+                qa[kk][3]);
+      }
+    }
+    // the two rows this thread holds: gq and gq + 8
+    int qrow[2], qpos[2];
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      const int r = gq + 8 * h2;
+      qrow[h2] = r < R ? r / G : -1;                    // query index, -1 for padding
+      qpos[h2] = r < R ? kv - n_q + qrow[h2] : -1;      // last visible position
+    }
+    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+    float o[16][4];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    const float sc = g.sm_scale_log2;
+    const int mi = lane >> 3, ri = lane & 7;
+    for (int c = 0; c < my_chunks; ++c) {
+      const int s = c % kStages;
+      if (!mbar_wait(&full[s], (c / kStages) & 1, abort_flag)) break;
+      const uint32_t kt = sbase + kOffStages + s * kStageBytes;
+      const uint32_t vt = kt + kTileBytes;
+      const int uc = c0 + c;
+      const int ub = uc / cpb;
+      const int blk = u_blk[ub], qm = u_qm[ub];
+      const int key0 = blk * g.B + (uc % cpb) * kChunk;
+      // visible keys of this chunk per held row: keys key0 + j with j < lim
+      int lim[2];
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2)
+        lim[h2] = (qrow[h2] >= 0 && ((qm >> qrow[h2]) & 1))
+                      ? max(0, min(kChunk, qpos[h2] + 1 - key0))
+                      : 0;
+      // S = Q K^T for keys [16w, 16w + 16): two n-tiles of 8 keys
+      float sfr[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        uint32_t b0, b1, b2, b3;
+        const int key = warp * 16 + (mi >> 1) * 8 + ri;
+        ldsm_x4(kt + tile_off(key, kk * 16 + (mi & 1) * 8), b0, b1, b2, b3);
+        mma_bf16(sfr[0], qa[kk], b0, b1);
+        mma_bf16(sfr[1], qa[kk], b2, b3);
+      }
+      // mask, scale, online softmax (per row across the quad's 4 threads)
+      float x[2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int h2 = e >> 1;
+          const int j = warp * 16 + nt * 8 + 2 * tq + (e & 1);
+          x[nt][e] = j < lim[h2] ? sfr[nt][e] * sc : -INFINITY;
+        }
+      float alpha[2];
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        float mx = fmaxf(fmaxf(x[0][2 * h2], x[0][2 * h2 + 1]), fmaxf(x[1][2 * h2], x[1][2 * h2 + 1]));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+        const float m_new = fmaxf(m[h2], mx);
+        const float ref = m_new == -INFINITY ? 0.f : m_new;
+        alpha[h2] = ex2_approx(m[h2] - ref);
+        m[h2] = m_new;
+        float rs = 0.f;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 2 * h2; e < 2 * h2 + 2; ++e) {
+            x[nt][e] = ex2_approx(x[nt][e] - ref);
+            rs += x[nt][e];
+          }
+        l[h2] = l[h2] * alpha[h2] + rs;
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        o[i][0] *= alpha[0];
+        o[i][1] *= alpha[0];
+        o[i][2] *= alpha[1];
+        o[i][3] *= alpha[1];
+      }
+      // Keys no row of this CTA may see are not part of any selection (the
+      // tail block's keys past the newest query): their V rows are zeroed so
+      // that P = 0 cannot meet a non-finite V in the MMA.
+      int lim_all = 0;
+      for (int i = 0; i < n_q; ++i)
+        if ((qm >> i) & 1) lim_all = max(lim_all, min(kChunk, max(0, kv - n_q + i + 1 - key0)));
+      if (lim_all < warp * 16 + 16) {
+        for (int e = lane; e < 16 * 16; e += 32) {   // 16 rows x 2 boxes x 8 chunks of 16 B
+          const int row = warp * 16 + (e >> 4);
+          const int box = (e >> 3) & 1, ch = e & 7;
+          if (row >= lim_all)
+            *reinterpret_cast<uint4*>(smem + (vt - sbase) + box * kBoxBytes + row * 128 + ch * 16) =
+                make_uint4(0, 0, 0, 0);
+        }
+        __syncwarp();
+      }
+      // P as the A fragment of a 16x16 (rows x keys) tile
+      uint32_t pa[4];
+      pa[0] = pack2(x[0][0], x[0][1]);
+      pa[1] = pack2(x[0][2], x[0][3]);
+      pa[2] = pack2(x[1][0], x[1][1]);
+      pa[3] = pack2(x[1][2], x[1][3]);
+      // O += P V over the warp's 16 keys, 16 n-tiles of 8 dims
+#pragma unroll
+      for (int dn = 0; dn < 16; dn += 2) {
+        uint32_t b0, b1, b2, b3;
+        const int key = warp * 16 + (mi & 1) * 8 + ri;
+        ldsm_x4_t(vt + tile_off(key, dn * 8 + (mi >> 1) * 8), b0, b1, b2, b3);
+        mma_bf16(o[dn], pa, b0, b1);
+        mma_bf16(o[dn + 1], pa, b2, b3);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+    // merge the four warps' states through shared memory (the ring is free)
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      l[h2] += __shfl_xor_sync(kFull, l[h2], 1);
+      l[h2] += __shfl_xor_sync(kFull, l[h2], 2);
+    }
+    named_bar_sync(1, 32 * kConsumers);   // every consumer is done with the ring
+    float* so = reinterpret_cast<float*>(smem + kOffStages);   // [warp][16 rows][128]
+    float* sm = so + kConsumers * 16 * kD;                     // [warp][16 rows][2]
+#pragma unroll
+    for (int dn = 0; dn < 16; ++dn) {
+      const int d = dn * 8 + 2 * tq;
+      *reinterpret_cast<float2*>(so + (warp * 16 + gq) * kD + d) = make_float2(o[dn][0], o[dn][1]);
+      *reinterpret_cast<float2*>(so + (warp * 16 + gq + 8) * kD + d) =
+          make_float2(o[dn][2], o[dn][3]);
+    }
+    if (tq == 0) {
+      sm[(warp * 16 + gq) * 2] = m[0];
+      sm[(warp * 16 + gq) * 2 + 1] = l[0];
+      sm[(warp * 16 + gq + 8) * 2] = m[1];
+      sm[(warp * 16 + gq + 8) * 2 + 1] = l[1];
+    }
+    named_bar_sync(1, 32 * kConsumers);
+    // thread t of the 128 consumers: row t / 8, dims [16 (t % 8), + 16)
+    const int t = threadIdx.x;
+    const int r = t >> 3, d0 = (t & 7) * 16;
+    if (r < R) {
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kConsumers; ++w) M = fmaxf(M, sm[(w * 16 + r) * 2]);
+      float wsc[kConsumers], L = 0.f;
+#pragma unroll
+      for (int w = 0; w < kConsumers; ++w) {
+        const float mw = sm[(w * 16 + r) * 2];
+        wsc[w] = mw == -INFINITY ? 0.f : ex2_approx(mw - M);
+        L += sm[(w * 16 + r) * 2 + 1] * wsc[w];
+      }
+      float* dst = P.part_o + (row0 + r) * kD + d0;
+#pragma unroll
+      for (int d = 0; d < 16; d += 4) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int w = 0; w < kConsumers; ++w) {
+          const float4 v = *reinterpret_cast<const float4*>(so + (w * 16 + r) * kD + d0 + d);
+          acc.x += v.x * wsc[w];
+          acc.y += v.y * wsc[w];
+          acc.z += v.z * wsc[w];
+          acc.w += v.w * wsc[w];
+        }
+        *reinterpret_cast<float4*>(dst + d) = acc;
+      }
+      if ((t & 7) == 0) {
+        P.part_ml[2 * (row0 + r)] = M;
+        P.part_ml[2 * (row0 + r) + 1] = L;
+      }
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag && P.err) atomicExch(P.err, 2);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// [batch * cap, Hkv, 128] bf16 cache viewed as 3-D with a (64 dims, 1 head, 64 rows) box.
+bool make_cache_map(CUtensorMap* m, const void* ptr, int Hkv, long long rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)Hkv, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)Hkv * kD * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)kChunk};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool attn_decode_mma_supported(const Geom& g, int n_q) {
+  return g.D == kD && g.B % kChunk == 0 && n_q * g.G <= 16 && n_q <= 4;
+}
+
+// Chunks per CTA for the split-KV grid: about two CTAs per SM in one wave.
+void decode_mma_split(const Geom& g, int batch, int n_q, int* nsplit, int* per_split) {
+  const int max_chunks = n_q * (g.k + 1) * (g.B / kChunk);
+  const int pairs = batch * g.Hkv > 0 ? batch * g.Hkv : 1;
+  int ns = (2 * 148) / pairs;
+  if (ns < 1) ns = 1;
+  if (ns > max_chunks) ns = max_chunks;
+  *per_split = (max_chunks + ns - 1) / ns;
+  *nsplit = (max_chunks + *per_split - 1) / *per_split;
+}
+
+cudaError_t launch_attn_decode_mma(const Geom& g, int batch, int n_q, int cap, int nsplit,
+                                   int per_split, const int* kv_len, const void* q,
+                                   const void* kc, const void* vc, const int* sel,
+                                   const int* nsel, float* part_ml, float* part_o, int* err,
+                                   cudaStream_t st) {
+  if (batch == 0) return cudaSuccess;
+  CUtensorMap mk, mv;
+  if (!make_cache_map(&mk, kc, g.Hkv, (long long)batch * cap) ||
+      !make_cache_map(&mv, vc, g.Hkv, (long long)batch * cap))
+    return cudaErrorInvalidValue;
+  DecParams p;
+  p.g = g;
+  p.n_q = n_q;
+  p.cap = cap;
+  p.nsplit = nsplit;
+  p.per_split = per_split;
+  p.kv_len = kv_len;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.sel = sel;
+  p.nsel = nsel;
+  p.part_ml = part_ml;
+  p.part_o = part_o;
+  p.err = err;
+  cudaError_t e = cudaFuncSetAttribute(attn_decode_mma_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  attn_decode_mma_kernel<<<dim3(nsplit, batch, g.Hkv), kThreads, kSmemBytes, st>>>(mk, mv, p);
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace qsa

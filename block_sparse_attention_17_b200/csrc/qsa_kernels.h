@@ -42,6 +42,17 @@ cudaError_t launch_attn_decode_simt(qsa_dtype dt, const Geom& g, int batch, int 
                                     const int* sel, const int* nsel, float* part_ml,
                                     float* part_o, void* out, float* lse, cudaStream_t st);
 
+cudaError_t launch_decode_combine(qsa_dtype dt, const Geom& g, int batch, int n_q, int cap,
+                                  int nsplit, const int* kv_len, const float* part_ml,
+                                  const float* part_o, const void* gate, void* out, float* lse,
+                                  cudaStream_t st);
+bool attn_decode_mma_supported(const Geom& g, int n_q);
+void decode_mma_split(const Geom& g, int batch, int n_q, int* nsplit, int* per_split);
+cudaError_t launch_attn_decode_mma(const Geom& g, int batch, int n_q, int cap, int nsplit,
+                                   int per_split, const int* kv_len, const void* q,
+                                   const void* kc, const void* vc, const int* sel,
+                                   const int* nsel, float* part_ml, float* part_o, int* err,
+                                   cudaStream_t st);
 bool attn_prefill_tc_supported(const Geom& g);
 cudaError_t launch_attn_prefill_tc(const Geom& g, const int* cu, int batch, int total_tokens,
                                    int max_seqlen, int words, const uint32_t* bitmask,

@@ -1,9 +1,7 @@
 // Block pooling, indexer scoring and top-k selection (sm_100a).
 //
 // Pooling: kbar[j] = (1/B) sum_{i<B} ik[jB+i] for complete blocks (instagit MTPLX
-// page, "Qwen Sparse Attention (QSA)": mean-pooled key blocks). One device
-// function sums the rows of a block in a fixed order, so the prefill, the
-// incremental decode finalisation and the cache rebuild write identical bits.
+// page, "Qwen Sparse Attention (QSA)": mean-pooled key blocks).
 //
 // Score: s[j] = c * sum_h w[h] * relu(iq[h] . kbar[j]) over complete visible
 // blocks (llama.cpp PR #27739 page, QSA composition commit: per-head weights,
@@ -19,55 +17,83 @@
 namespace qsa {
 
 // ----------------------------------------------------------------- pooling
-// One warp pools one block: lane owns dims {lane, lane + 32}; rows are summed
-// in ascending order in fp32, then scaled by 1/B (B is a power of two).
+// One CTA of 256 threads pools one block: warp w sums rows w, w + 8, ... of
+// the block (coalesced rows; lane l owns dims 2l and 2l + 1) in ascending
+// order, then the 8 partial sums are combined in a fixed tree
+// ((p0 + p1) + (p2 + p3)) + ((p4 + p5) + (p6 + p7)) and scaled by 1/B (B is a
+// power of two). The prefill pooling, the incremental decode finalisation and
+// the cache rebuild all call this one function, so they write identical bits.
+constexpr int kPoolThreads = 256;
+
 template <typename T>
-__device__ __forceinline__ void pool_block_warp(const T* __restrict__ rows, int B, int di,
-                                                float* __restrict__ dst, int lane) {
-  float a0 = 0.f, a1 = 0.f;
-  const bool h0 = lane < di, h1 = lane + 32 < di;
-  for (int i = 0; i < B; ++i) {
-    const T* r = rows + (size_t)i * di;
-    if (h0) a0 += to_f32(r[lane]);
-    if (h1) a1 += to_f32(r[lane + 32]);
-  }
-  const float inv = 1.0f / (float)B;
-  if (h0) dst[lane] = a0 * inv;
-  if (h1) dst[lane + 32] = a1 * inv;
+__device__ __forceinline__ float2 load_pair(const T* p);
+template <>
+__device__ __forceinline__ float2 load_pair<float>(const float* p) {
+  return *reinterpret_cast<const float2*>(p);
+}
+template <>
+__device__ __forceinline__ float2 load_pair<__nv_bfloat16>(const __nv_bfloat16* p) {
+  const uint32_t u = *reinterpret_cast<const uint32_t*>(p);
+  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
 }
 
 template <typename T>
-__global__ void pool_prefill_kernel(const T* __restrict__ ik, const int* __restrict__ cu,
-                                    int B, int di, float* __restrict__ pooled, int max_nblk) {
-  const int b = blockIdx.y;
+__device__ __forceinline__ void pool_block_cta(const T* __restrict__ rows, int B, int di,
+                                               float* __restrict__ dst) {
+  __shared__ float2 part[8][32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int j = blockIdx.x * (blockDim.x >> 5) + warp;
+  const bool active = 2 * lane < di;
+  float2 acc = make_float2(0.f, 0.f);
+  if (active) {
+#pragma unroll 4
+    for (int i = warp; i < B; i += 8) {
+      const float2 x = load_pair<T>(rows + (size_t)i * di + 2 * lane);
+      acc.x += x.x;
+      acc.y += x.y;
+    }
+  }
+  part[warp][lane] = acc;
+  __syncthreads();
+  if (warp == 0 && active) {
+    float2 q[8];
+#pragma unroll
+    for (int w = 0; w < 8; ++w) q[w] = part[w][lane];
+    const float inv = 1.0f / (float)B;
+    const float sx = ((q[0].x + q[1].x) + (q[2].x + q[3].x)) + ((q[4].x + q[5].x) + (q[6].x + q[7].x));
+    const float sy = ((q[0].y + q[1].y) + (q[2].y + q[3].y)) + ((q[4].y + q[5].y) + (q[6].y + q[7].y));
+    *reinterpret_cast<float2*>(dst + 2 * lane) = make_float2(sx * inv, sy * inv);
+  }
+}
+
+// Grid (blocks of the longest sequence, batch).
+template <typename T>
+__global__ void __launch_bounds__(kPoolThreads)
+pool_prefill_kernel(const T* __restrict__ ik, const int* __restrict__ cu, int B, int di,
+                    float* __restrict__ pooled, int max_nblk) {
+  const int b = blockIdx.y, j = blockIdx.x;
   const int s0 = cu[b], L = cu[b + 1] - s0;
   if (j >= L / B) return;
-  pool_block_warp(ik + ((size_t)s0 + (size_t)j * B) * di, B, di,
-                  pooled + ((size_t)b * max_nblk + j) * di, lane);
+  pool_block_cta(ik + ((size_t)s0 + (size_t)j * B) * di, B, di,
+                 pooled + ((size_t)b * max_nblk + j) * di);
 }
 
 // mode 0: rebuild every complete block; mode 1: only the blocks completed by
-// the last n_q appended rows.
+// the last n_q appended rows. Grid (blocks in range, batch).
 template <typename T>
-__global__ void pool_cache_kernel(const T* __restrict__ ik_cache, const int* __restrict__ kv_len,
-                                  int cap, int n_q, int mode, int B, int di,
-                                  float* __restrict__ pooled, int* dev_err) {
+__global__ void __launch_bounds__(kPoolThreads)
+pool_cache_kernel(const T* __restrict__ ik_cache, const int* __restrict__ kv_len, int cap,
+                  int n_q, int mode, int B, int di, float* __restrict__ pooled, int* dev_err) {
   const int b = blockIdx.y;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kv = kv_len[b];
   if (kv < (mode ? n_q : 0) || kv > cap) {
     if (dev_err && threadIdx.x == 0 && blockIdx.x == 0) atomicExch(dev_err, 1);
     return;
   }
   const int jlo = mode ? (kv - n_q) / B : 0;
-  const int jhi = kv / B;
-  const int j = jlo + blockIdx.x * (blockDim.x >> 5) + warp;
-  if (j >= jhi) return;
-  const int nblk_cap = cap / B;
-  pool_block_warp(ik_cache + ((size_t)b * cap + (size_t)j * B) * di, B, di,
-                  pooled + ((size_t)b * nblk_cap + j) * di, lane);
+  const int j = jlo + blockIdx.x;
+  if (j >= kv / B) return;
+  pool_block_cta(ik_cache + ((size_t)b * cap + (size_t)j * B) * di, B, di,
+                 pooled + ((size_t)b * (cap / B) + j) * di);
 }
 
 // ----------------------------------------------------------------- scoring
@@ -345,8 +371,8 @@ static cudaError_t launch_pool_prefill_t(const void* ik, const int* cu, int batc
                                          cudaStream_t st) {
   const int nblk = max_seqlen / B;
   if (nblk == 0 || batch == 0) return cudaSuccess;
-  dim3 grid((nblk + 3) / 4, batch);
-  pool_prefill_kernel<T><<<grid, 128, 0, st>>>((const T*)ik, cu, B, di, pooled, max_nblk);
+  pool_prefill_kernel<T><<<dim3(nblk, batch), kPoolThreads, 0, st>>>((const T*)ik, cu, B, di,
+                                                                     pooled, max_nblk);
   note_launch();
   return cudaGetLastError();
 }
@@ -365,13 +391,13 @@ cudaError_t launch_pool_cache(qsa_dtype dt, const void* ik_cache, const int* kv_
                               int* dev_err, cudaStream_t st) {
   const int span = mode ? (n_q + B - 1) / B + 1 : cap / B;
   if (batch == 0 || span == 0) return cudaSuccess;
-  dim3 grid((span + 3) / 4, batch);
+  dim3 grid(span, batch);
   if (dt == QSA_BF16)
-    pool_cache_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(
+    pool_cache_kernel<__nv_bfloat16><<<grid, kPoolThreads, 0, st>>>(
         (const __nv_bfloat16*)ik_cache, kv_len, cap, n_q, mode, B, di, pooled, dev_err);
   else
-    pool_cache_kernel<float><<<grid, 128, 0, st>>>((const float*)ik_cache, kv_len, cap, n_q,
-                                                   mode, B, di, pooled, dev_err);
+    pool_cache_kernel<float><<<grid, kPoolThreads, 0, st>>>((const float*)ik_cache, kv_len, cap,
+                                                            n_q, mode, B, di, pooled, dev_err);
   note_launch();
   return cudaGetLastError();
 }
