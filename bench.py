@@ -248,18 +248,49 @@ def run_ours(args, w, rank, world, dist):
         alg = {"bound": "hbm", "work": kv_bytes + io, "peak_key": "hbm_gbs", "unit": "GB/s"}
         in_names = ["q", "iq", "iw", "gate", "kv_len"]   # one decode step's new inputs
 
-    # warm-up
+    # warm-up (eager)
     for _ in range(max(args.warmup, 0)):
         flush.zero_()
         step()
     torch.cuda.synchronize()
+    lib.qsa_set_stage_events(arr_t, 3)
+
+    def timed(run_once):
+        """Time K steps, each bracketed by CUDA events on the launching stream,
+        with the L2 flush outside the events; returns per-step ms and the
+        attention-stage ms read from the library's stage events."""
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        attn = []
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            run_once()
+            ends[i].record(stream)
+            torch.cuda.synchronize()       # read this step's stage events before reuse
+            attn.append(ev_stage[1].elapsed_time(ev_stage[2]))
+        return [starts[i].elapsed_time(ends[i]) for i in range(args.steps)], attn
+
+    # one step captured as a CUDA graph (the library makes no host sync, reads
+    # no device memory on the host and allocates nothing, so it captures whole)
+    graph = None
+    if not args.eager:
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            step()
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        torch.cuda.synchronize()
+        for _ in range(2):
+            flush.zero_()
+            graph.replay()
+        torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
-
-    lib.qsa_set_stage_events(arr_t, 3)
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    stage_attn = []
     dev_id = ""
     try:
         dev_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid).replace("GPU-", "")
@@ -269,18 +300,15 @@ def run_ours(args, w, rank, world, dist):
     clocks.start()
     n0 = lib.qsa_kernel_launch_count()
     torch.cuda.synchronize()
-    for i in range(args.steps):
-        flush.zero_()
-        starts[i].record(stream)
-        step()
-        ends[i].record(stream)
-        torch.cuda.synchronize()       # read this step's stage events before reuse
-        stage_attn.append(ev_stage[1].elapsed_time(ev_stage[2]))
-    torch.cuda.synchronize()
+    eager_ms, eager_attn = timed(step)
     launches = lib.qsa_kernel_launch_count() - n0
+    if graph is not None:
+        step_ms, stage_attn = timed(graph.replay)
+    else:
+        step_ms, stage_attn = eager_ms, eager_attn
+    torch.cuda.synchronize()
     clk = clocks.stop()
     lib.qsa_set_stage_events(None, 0)
-    step_ms = [starts[i].elapsed_time(ends[i]) for i in range(args.steps)]
     total_ms = float(sum(step_ms))
     if dist is not None:
         import torch.distributed as tdist
@@ -340,6 +368,9 @@ def run_ours(args, w, rank, world, dist):
                          f"oracle, {secs:.1f} s"}
 
     extra = {"l2": "flushed before every timed step (256 MiB write, outside the events)",
+             "timing": ("CUDA-graph replay of one library call per step" if graph is not None
+                        else "eager library call per step"),
+             "eager_ms_per_step": float(np.mean(eager_ms)),
              "selected_kv_tokens_per_step": units, "input_gen_s": round(t_gen, 2)}
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
@@ -347,7 +378,8 @@ def run_ours(args, w, rank, world, dist):
             "dtype": w.dtype, "data": "synthetic (seeded numpy draws, shapes of the workload)",
             "config": config_of(w, extra), "parallelism": f"replicas{world}",
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": int(launches), "clocks": clk, "impl": "ours"}
+            "gpu_launches": int(launches), "clocks": clk,
+            "impl": "ours"}
     if w.kind == "decode":
         line["us_per_decode_step"] = total_ms / args.steps * 1e3
     return line
@@ -413,6 +445,7 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--eager", action="store_true", help="time eager calls only (no CUDA graph)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-step-seconds", type=float, default=2.0)

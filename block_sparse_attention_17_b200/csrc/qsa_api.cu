@@ -8,6 +8,9 @@
 
 #include <algorithm>
 #include <atomic>
+#include <map>
+#include <mutex>
+#include <utility>
 
 #include "qsa_common.cuh"
 #include "qsa_kernels.h"
@@ -19,6 +22,21 @@ std::atomic<unsigned long long> g_launches{0};
 }  // namespace
 
 void qsa::note_launch(int n) { g_launches.fetch_add((unsigned long long)n); }
+
+cudaError_t qsa::set_max_dynamic_smem(const void* func, int bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, int> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  auto key = std::make_pair(func, dev);
+  auto it = done.find(key);
+  if (it != done.end() && it->second >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done[key] = bytes;
+  return e;
+}
 
 namespace {
 
@@ -51,7 +69,6 @@ qsa_status cuda_fail(cudaError_t e, const char* where) {
   return fail(QSA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
 }
 
-constexpr int kMaxDecodeBlocks = 16384;
 constexpr int kMaxDecodeQ = 4;
 constexpr int kMaxDecodeRows = 32;
 constexpr int kTargetCtas = 2 * 148;
@@ -141,7 +158,8 @@ PrefillWs carve_prefill(const Geom& g, void* ws, int batch, int T, int max_seqle
 
 struct DecodeWs {
   int* err;
-  float* scores;
+  int* counters;        // [batch] selection + [batch * Hkv] attention, zeroed per call
+  uint32_t* keys;       // [batch, n_q, cap / B] score keys
   int* sel;
   int* nsel;
   float* part_ml;
@@ -169,7 +187,8 @@ DecodeWs carve_decode(const qsa_config* cfg, const Geom& g, void* ws, int batch,
   const int R = n_q * g.G;
   Carve c(ws);
   w.err = c.take<int>(1);
-  w.scores = c.take<float>((size_t)batch * n_q * (cap / g.B));
+  w.counters = c.take<int>((size_t)batch * (1 + g.Hkv));
+  w.keys = c.take<uint32_t>((size_t)batch * n_q * (cap / g.B));
   w.sel = c.take<int>((size_t)batch * n_q * (g.k + 1));
   w.nsel = c.take<int>((size_t)batch * n_q);
   w.part_ml = c.take<float>((size_t)batch * g.Hkv * w.nsplit * R * 2);
@@ -198,8 +217,8 @@ qsa_status check_decode_dims(const qsa_config* cfg, int batch, int n_q, int cap)
   if (batch < 0 || n_q <= 0 || cap <= 0)
     return fail(QSA_ERR_INVALID_ARG, "batch >= 0, n_q > 0 and cap > 0 are required");
   if (cap % cfg->block_size) return fail(QSA_ERR_INVALID_ARG, "cap must be a multiple of B");
-  if (cap / cfg->block_size > kMaxDecodeBlocks)
-    return fail(QSA_ERR_UNSUPPORTED, "more than %d cache blocks", kMaxDecodeBlocks);
+  if (cap / cfg->block_size > kMaxDecodeBlocksPerSeq)
+    return fail(QSA_ERR_UNSUPPORTED, "more than %d cache blocks", kMaxDecodeBlocksPerSeq);
   if ((long long)batch * cap > 2147483647LL)
     return fail(QSA_ERR_UNSUPPORTED, "batch * cap must fit in 31 bits");
   if (n_q > kMaxDecodeQ) return fail(QSA_ERR_UNSUPPORTED, "n_q > %d", kMaxDecodeQ);
@@ -353,11 +372,10 @@ static qsa_status decode_select_common(const qsa_config* cfg, const Geom& g, int
                                        float* pooled_cache, const DecodeWs& w, int32_t* sel,
                                        int32_t* nsel, float* scores, int32_t* dev_err,
                                        cudaStream_t st) {
-  QSA_CUDA(launch_pool_cache(cfg->dtype, ik_cache, kv_len, batch, cap, n_q, 1, g.B, g.di,
-                             pooled_cache, dev_err, st),
-           "pool finalize");
-  QSA_CUDA(launch_decode_select(cfg->dtype, g, batch, n_q, cap, kv_len, iq, iw, pooled_cache,
-                                w.scores, sel, nsel, scores, st),
+  QSA_CUDA(cudaMemsetAsync(w.counters, 0, sizeof(int) * (size_t)batch * (1 + g.Hkv), st),
+           "clear counters");
+  QSA_CUDA(launch_decode_select(cfg->dtype, g, batch, n_q, cap, kv_len, iq, ik_cache, iw,
+                                pooled_cache, scores, w.keys, w.counters, sel, nsel, dev_err, st),
            "decode select");
   return QSA_OK;
 }
@@ -393,12 +411,9 @@ qsa_status qsa_decode(const qsa_config* cfg, int batch, int n_q, int cap, const 
   stage_mark(1, st);
   if (decode_uses_mma(cfg, g, n_q)) {
     QSA_CUDA(launch_attn_decode_mma(g, batch, n_q, cap, w.nsplit, w.per_split, kv_len, q,
-                                    k_cache, v_cache, sel_p, nsel_p, w.part_ml, w.part_o,
-                                    dev_err ? dev_err : w.err, st),
+                                    k_cache, v_cache, gate, sel_p, nsel_p, w.part_ml, w.part_o,
+                                    w.counters + batch, out, lse, dev_err ? dev_err : w.err, st),
              "decode attention");
-    QSA_CUDA(launch_decode_combine(cfg->dtype, g, batch, n_q, cap, w.nsplit, kv_len, w.part_ml,
-                                   w.part_o, gate, out, lse, st),
-             "decode combine");
   } else {
     QSA_CUDA(launch_attn_decode_simt(cfg->dtype, g, batch, n_q, cap, w.nsplit, w.per_split,
                                      kv_len, q, k_cache, v_cache, gate, sel_p, nsel_p, w.part_ml,

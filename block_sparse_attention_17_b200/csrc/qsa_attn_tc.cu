@@ -533,13 +533,11 @@ cudaError_t launch_attn_prefill_tc(const Geom& g, const int* cu, int batch, int 
   dim3 grid(p.n_ctas, batch, g.Hkv);
   cudaError_t e;
   if (g.B == 64) {
-    e = cudaFuncSetAttribute(attn_prefill_tc_kernel<64>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    e = set_max_dynamic_smem(reinterpret_cast<const void*>(attn_prefill_tc_kernel<64>), kSmemBytes);
     if (e != cudaSuccess) return e;
     attn_prefill_tc_kernel<64><<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, p);
   } else {
-    e = cudaFuncSetAttribute(attn_prefill_tc_kernel<128>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    e = set_max_dynamic_smem(reinterpret_cast<const void*>(attn_prefill_tc_kernel<128>), kSmemBytes);
     if (e != cudaSuccess) return e;
     attn_prefill_tc_kernel<128><<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, p);
   }

@@ -13,7 +13,8 @@ constexpr unsigned kFull = 0xffffffffu;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kMaxTopK = 64;          // budget / block_size
-constexpr int kMaxBlocksPerSeq = 4096;
+constexpr int kMaxBlocksPerSeq = 4096;        // prefill
+constexpr int kMaxDecodeBlocksPerSeq = 16384; // decode cache blocks (cap / B)
 
 // Geometry passed by value to every kernel.
 struct Geom {

@@ -14,8 +14,9 @@
 // heads), so the four consumer warps use warp-level bf16 MMAs (m16n8k16,
 // fp32 accumulation): warp w takes keys [16w, 16w + 16) of each chunk and
 // keeps its own online-softmax state (log2 domain); the four states are
-// merged at the end and written as one (m, l, O) partial per row, which
-// qsa_combine merges across CTAs before the sigmoid gate.
+// merged at the end and written as one (m, l, O) partial per row; the last
+// CTA of each (sequence, KV head) merges the partials by log-sum-exp and
+// applies the sigmoid output gate.
 #include "qsa_common.cuh"
 #include "qsa_kernels.h"
 #include "qsa_sm100.cuh"
@@ -42,17 +43,22 @@ constexpr int kOffQ = kOffStages + kStages * kStageBytes;
 constexpr int kOffBar = kOffQ + 16 * kQStride;
 constexpr int kOffMisc = kOffBar + 8 * 2 * kStages;
 constexpr int kOffUnion = kOffMisc + 64;
-constexpr int kSmemBytes = kOffUnion + 8 * kMaxUnion + 1024;
+constexpr int kOffBits = kOffUnion + 8 * kMaxUnion;   // [n_q][cap / B / 32] words
+// dynamic shared memory: kOffBits + 4 * n_q * words + 1024 (alignment slack)
 
 struct DecParams {
   Geom g;
   int n_q, cap, nsplit, per_split;   // per_split: chunks per CTA
   const int* kv_len;
   const __nv_bfloat16* q;
+  const __nv_bfloat16* gate;
   const int* sel;
   const int* nsel;
   float* part_ml;
   float* part_o;
+  int* counter;                      // [batch * Hkv], zero before the launch
+  __nv_bfloat16* out;
+  float* lse;
   int* err;
 };
 
@@ -102,11 +108,14 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
   const int G = g.G, n_q = P.n_q, R = n_q * G;
   const int kv = P.kv_len[b];
   const size_t row0 = (((size_t)b * g.Hkv + hk) * P.nsplit + split) * R;
-  if (kv < n_q || kv > P.cap) {   // reported by the pooling kernel; skip the sequence
-    for (int r = threadIdx.x; r < R; r += blockDim.x) {
-      P.part_ml[2 * (row0 + r)] = -INFINITY;
-      P.part_ml[2 * (row0 + r) + 1] = 0.f;
-    }
+  if (kv < n_q || kv > P.cap) {   // reported by the selection kernel; outputs are zero
+    if (split == 0)
+      for (int e = threadIdx.x; e < R * kD; e += blockDim.x) {
+        const int r = e / kD, d = e - r * kD;
+        const size_t orow = ((size_t)b * n_q + r / G) * g.Hq + hk * G + r % G;
+        P.out[orow * kD + d] = __float2bfloat16_rn(0.f);
+        if (P.lse && d == 0) P.lse[orow] = -INFINITY;
+      }
     return;
   }
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOffBar);
@@ -117,6 +126,12 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
   int* u_qm = u_blk + kMaxUnion;
   const int cpb = g.B / kChunk;   // chunks per block
 
+  // union of the n_q selections (selected blocks and tail blocks), ascending,
+  // with a mask of the queries that selected each block: per-query bitmaps in
+  // shared memory, then one ordered scan by warp 0
+  const int words = (P.cap / g.B + 31) / 32;
+  uint32_t* qbits = reinterpret_cast<uint32_t*>(smem + kOffBits);   // [n_q][words]
+  for (int e = threadIdx.x; e < n_q * words; e += blockDim.x) qbits[e] = 0u;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
@@ -125,28 +140,49 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async();
-    // union of the n_q selections, ascending, with a mask of the queries that
-    // selected each block (their tail blocks included)
+  }
+  __syncthreads();
+  {
     const int kp1 = g.k + 1;
-    const int* sb = P.sel + (size_t)b * n_q * kp1;
-    const int* nb = P.nsel + (size_t)b * n_q;
-    int idx[4] = {0, 0, 0, 0}, cnt = 0;
-    while (true) {
-      int best = 0x7fffffff;
-      for (int i = 0; i < n_q; ++i)
-        if (idx[i] < nb[i]) best = min(best, sb[i * kp1 + idx[i]]);
-      if (best == 0x7fffffff) break;
-      int qm = 0;
-      for (int i = 0; i < n_q; ++i)
-        if (idx[i] < nb[i] && sb[i * kp1 + idx[i]] == best) {
-          qm |= 1 << i;
-          ++idx[i];
-        }
-      u_blk[cnt] = best;
-      u_qm[cnt] = qm;
-      ++cnt;
+    for (int e = threadIdx.x; e < n_q * kp1; e += blockDim.x) {
+      const int i = e / kp1, j = e - i * kp1;
+      if (j < P.nsel[(size_t)b * n_q + i]) {
+        const int blk = P.sel[((size_t)b * n_q + i) * kp1 + j];
+        atomicOr(&qbits[i * words + (blk >> 5)], 1u << (blk & 31));
+      }
     }
-    *n_chunks_s = cnt * cpb;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int base = 0;
+    for (int w0 = 0; w0 < words; w0 += 32) {
+      const int w = w0 + lane;
+      uint32_t qw[4] = {0u, 0u, 0u, 0u}, bits = 0u;
+      if (w < words)
+        for (int i = 0; i < n_q; ++i) {
+          qw[i] = qbits[i * words + w];
+          bits |= qw[i];
+        }
+      const int c = __popc(bits);
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += v;
+      }
+      int off = base + incl - c;
+      while (bits) {
+        const int bp = __ffs(bits) - 1;
+        bits &= bits - 1;
+        int qm = 0;
+        for (int i = 0; i < n_q; ++i) qm |= ((qw[i] >> bp) & 1u) << i;
+        u_blk[off] = w * 32 + bp;
+        u_qm[off] = qm;
+        ++off;
+      }
+      base += __shfl_sync(kFull, incl, 31);
+    }
+    if (lane == 0) *n_chunks_s = base * cpb;
   }
   // Q rows r = i * G + gi (query i, head hk * G + gi), zero beyond R
   for (int e = threadIdx.x; e < 16 * (kD / 8); e += blockDim.x) {
@@ -372,7 +408,102 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
       }
     }
   }
+  // the last CTA of this (sequence, KV head) merges the splits' partials by
+  // log-sum-exp and applies the sigmoid output gate
+  __threadfence();
   __syncthreads();
+  __shared__ int last_s;
+  if (threadIdx.x == 0) last_s = atomicAdd(&P.counter[(size_t)b * g.Hkv + hk], 1) == P.nsplit - 1;
+  __syncthreads();
+  if (last_s) {
+    __threadfence();
+    const size_t rowb = ((size_t)b * g.Hkv + hk) * P.nsplit * R;
+    // per-row max over the splits, then each split's weight, in parallel
+    float* wgt = reinterpret_cast<float*>(smem + kOffStages);   // [nsplit][R] (ring is free)
+    float* rowM = wgt + P.nsplit * R;                            // [R]
+    float* rowL = rowM + 16;                                     // [R]
+    for (int e = threadIdx.x; e < P.nsplit * R; e += blockDim.x)
+      wgt[e] = __ldcg(P.part_ml + 2 * (rowb + e));
+    __syncthreads();
+    if (threadIdx.x < R) {
+      float M = -INFINITY;
+      for (int sp = 0; sp < P.nsplit; ++sp) M = fmaxf(M, wgt[sp * R + threadIdx.x]);
+      rowM[threadIdx.x] = M;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < P.nsplit * R; e += blockDim.x) {
+      const float ms = wgt[e], M = rowM[e % R];
+      wgt[e] = (ms == -INFINITY) ? 0.f : ex2_approx(ms - M);
+    }
+    __syncthreads();
+    float* lw = rowL + 16;                                        // [nsplit][R]
+    for (int e = threadIdx.x; e < P.nsplit * R; e += blockDim.x)
+      lw[e] = __ldcg(P.part_ml + 2 * (rowb + e) + 1) * wgt[e];
+    __syncthreads();
+    if (threadIdx.x < R) {
+      float L = 0.f;
+      for (int sp = 0; sp < P.nsplit; ++sp) L += lw[sp * R + threadIdx.x];
+      rowL[threadIdx.x] = L;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < R * (kD / 16); e += blockDim.x) {
+      const int r = e / (kD / 16), d0 = (e % (kD / 16)) * 16;
+      float acc[16];
+#pragma unroll
+      for (int d = 0; d < 16; ++d) acc[d] = 0.f;
+      // eight splits' loads in flight before they are used
+      for (int sp0 = 0; sp0 < P.nsplit; sp0 += 8) {
+        float4 v[8][4];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int sp = min(sp0 + u, P.nsplit - 1);
+          const float4* src =
+              reinterpret_cast<const float4*>(P.part_o + (rowb + sp * R + r) * kD + d0);
+#pragma unroll
+          for (int d = 0; d < 4; ++d) v[u][d] = __ldcg(src + d);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float wsp = sp0 + u < P.nsplit ? wgt[(sp0 + u) * R + r] : 0.f;
+#pragma unroll
+          for (int d = 0; d < 4; ++d) {
+            acc[4 * d] = fmaf(v[u][d].x, wsp, acc[4 * d]);
+            acc[4 * d + 1] = fmaf(v[u][d].y, wsp, acc[4 * d + 1]);
+            acc[4 * d + 2] = fmaf(v[u][d].z, wsp, acc[4 * d + 2]);
+            acc[4 * d + 3] = fmaf(v[u][d].w, wsp, acc[4 * d + 3]);
+          }
+        }
+      }
+      const float L = rowL[r], M = rowM[r];
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+      const int i = r / G, gi = r % G;
+      const size_t orow = ((size_t)b * n_q + i) * g.Hq + hk * G + gi;
+      float gsig[16];
+      if (g.gate_headwise) {
+        const float gs = sigmoidf_(__bfloat162float(P.gate[orow]));
+#pragma unroll
+        for (int d = 0; d < 16; ++d) gsig[d] = gs;
+      } else {
+        const uint4* gp = reinterpret_cast<const uint4*>(P.gate + orow * kD + d0);
+        const uint4 g0 = gp[0], g1 = gp[1];
+        const uint32_t gw[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+        for (int d = 0; d < 8; ++d) {
+          gsig[2 * d] = sigmoidf_(__uint_as_float(gw[d] << 16));
+          gsig[2 * d + 1] = sigmoidf_(__uint_as_float(gw[d] & 0xffff0000u));
+        }
+      }
+      uint32_t packed[8];
+#pragma unroll
+      for (int d = 0; d < 16; d += 2)
+        packed[d / 2] = pack2(acc[d] * inv * gsig[d], acc[d + 1] * inv * gsig[d + 1]);
+      uint4* dst = reinterpret_cast<uint4*>(P.out + orow * kD + d0);
+      dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+      if (P.lse && d0 == 0) P.lse[orow] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+    }
+    if (threadIdx.x == 0) P.counter[(size_t)b * g.Hkv + hk] = 0;
+  }
   if (threadIdx.x == 0 && *abort_flag && P.err) atomicExch(P.err, 2);
 }
 
@@ -419,15 +550,16 @@ void decode_mma_split(const Geom& g, int batch, int n_q, int* nsplit, int* per_s
   const int pairs = batch * g.Hkv > 0 ? batch * g.Hkv : 1;
   int ns = (2 * 148) / pairs;
   if (ns < 1) ns = 1;
-  if (ns > max_chunks) ns = max_chunks;
+  if (ns > (max_chunks + 7) / 8) ns = (max_chunks + 7) / 8;   // at least 8 chunks per CTA
   *per_split = (max_chunks + ns - 1) / ns;
   *nsplit = (max_chunks + *per_split - 1) / *per_split;
 }
 
 cudaError_t launch_attn_decode_mma(const Geom& g, int batch, int n_q, int cap, int nsplit,
                                    int per_split, const int* kv_len, const void* q,
-                                   const void* kc, const void* vc, const int* sel,
-                                   const int* nsel, float* part_ml, float* part_o, int* err,
+                                   const void* kc, const void* vc, const void* gate,
+                                   const int* sel, const int* nsel, float* part_ml,
+                                   float* part_o, int* counter, void* out, float* lse, int* err,
                                    cudaStream_t st) {
   if (batch == 0) return cudaSuccess;
   CUtensorMap mk, mv;
@@ -442,15 +574,20 @@ cudaError_t launch_attn_decode_mma(const Geom& g, int batch, int n_q, int cap, i
   p.per_split = per_split;
   p.kv_len = kv_len;
   p.q = static_cast<const __nv_bfloat16*>(q);
+  p.gate = static_cast<const __nv_bfloat16*>(gate);
+  p.counter = counter;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
   p.sel = sel;
   p.nsel = nsel;
   p.part_ml = part_ml;
   p.part_o = part_o;
   p.err = err;
-  cudaError_t e = cudaFuncSetAttribute(attn_decode_mma_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  const int words = (cap / g.B + 31) / 32;
+  const int smem = kOffBits + 4 * n_q * words + 1024;
+  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(attn_decode_mma_kernel), smem);
   if (e != cudaSuccess) return e;
-  attn_decode_mma_kernel<<<dim3(nsplit, batch, g.Hkv), kThreads, kSmemBytes, st>>>(mk, mv, p);
+  attn_decode_mma_kernel<<<dim3(nsplit, batch, g.Hkv), kThreads, smem, st>>>(mk, mv, p);
   note_launch();
   return cudaGetLastError();
 }

@@ -13,6 +13,10 @@ struct Geom;
 // Counts kernel launches made by the library (all host threads).
 void note_launch(int n = 1);
 
+// Raises a kernel's dynamic shared memory limit on the current device, once per
+// (kernel, device, size) instead of on every launch.
+cudaError_t set_max_dynamic_smem(const void* func, int bytes);
+
 // Sets the message qsa_last_error() returns on this host thread.
 void set_last_error(const char* msg);
 
@@ -28,10 +32,12 @@ cudaError_t launch_select_prefill(qsa_dtype dt, const Geom& g, const int* cu, in
                                   const float* iw, const float* pooled, int* sel, int* nsel,
                                   uint32_t* bitmask, float* scores, int scores_ld,
                                   cudaStream_t st);
+int decode_select_parts(const Geom& g, int cap);
 cudaError_t launch_decode_select(qsa_dtype dt, const Geom& g, int batch, int n_q, int cap,
-                                 const int* kv_len, const void* iq, const float* iw,
-                                 const float* pooled, float* scores_ws, int* sel, int* nsel,
-                                 float* scores_out, cudaStream_t st);
+                                 const int* kv_len, const void* iq, const void* ik_cache,
+                                 const float* iw, float* pooled, float* scores_out,
+                                 uint32_t* keys_ws, int* counter, int* sel, int* nsel,
+                                 int* dev_err, cudaStream_t st);
 cudaError_t launch_attn_prefill_simt(qsa_dtype dt, const Geom& g, const int* cu, int batch,
                                      int max_seqlen, const void* q, const void* k, const void* v,
                                      const void* gate, const int* sel, const int* nsel,
@@ -50,8 +56,9 @@ bool attn_decode_mma_supported(const Geom& g, int n_q);
 void decode_mma_split(const Geom& g, int batch, int n_q, int* nsplit, int* per_split);
 cudaError_t launch_attn_decode_mma(const Geom& g, int batch, int n_q, int cap, int nsplit,
                                    int per_split, const int* kv_len, const void* q,
-                                   const void* kc, const void* vc, const int* sel,
-                                   const int* nsel, float* part_ml, float* part_o, int* err,
+                                   const void* kc, const void* vc, const void* gate,
+                                   const int* sel, const int* nsel, float* part_ml,
+                                   float* part_o, int* counter, void* out, float* lse, int* err,
                                    cudaStream_t st);
 bool attn_prefill_tc_supported(const Geom& g);
 cudaError_t launch_attn_prefill_tc(const Geom& g, const int* cu, int batch, int total_tokens,

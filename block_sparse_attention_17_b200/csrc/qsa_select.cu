@@ -137,12 +137,51 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 // lower position wins a tie. Writes the chosen positions, ascending, to out[]
 // and returns how many (min(k, n)). The k-th largest key is found by an
 // MSB-first bit search on the 32-bit key; ties at that key are taken in
-// ascending position order.
+// ascending position order. Up to 256 keys are held in registers (8 per
+// lane) for the whole search; longer lists are re-read from memory.
 __device__ int warp_topk_positions(const uint32_t* keys, int n, int k, int* out, int lane) {
   if (n <= k) {
     for (int j = lane; j < n; j += 32) out[j] = j;
     __syncwarp();
     return n;
+  }
+  const unsigned lt = lanemask_lt();
+  if (n <= 256) {
+    uint32_t kr[8];
+    bool ok[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int j = lane + 32 * i;
+      ok[i] = j < n;
+      kr[i] = ok[i] ? keys[j] : 0u;
+    }
+    uint32_t tau = 0;
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = tau | (1u << bit);
+      int c = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) c += (ok[i] && kr[i] >= cand) ? 1 : 0;
+      c = __reduce_add_sync(kFull, c);
+      if (c >= k) tau = cand;
+    }
+    int gt = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) gt += (ok[i] && kr[i] > tau) ? 1 : 0;
+    gt = __reduce_add_sync(kFull, gt);
+    const int need = k - gt;
+    int m = 0, ties = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const bool tie = ok[i] && kr[i] == tau;
+      const unsigned tb = __ballot_sync(kFull, tie);
+      const bool pick = ok[i] && (kr[i] > tau || (tie && ties + __popc(tb & lt) < need));
+      const unsigned pb = __ballot_sync(kFull, pick);
+      if (pick) out[m + __popc(pb & lt)] = lane + 32 * i;
+      m += __popc(pb);
+      ties += __popc(tb);
+    }
+    __syncwarp();
+    return m;
   }
   uint32_t tau = 0;
   for (int bit = 31; bit >= 0; --bit) {
@@ -156,7 +195,6 @@ __device__ int warp_topk_positions(const uint32_t* keys, int n, int k, int* out,
   for (int j = lane; j < n; j += 32) gt += keys[j] > tau;
   gt = __reduce_add_sync(kFull, gt);
   const int need = k - gt;
-  const unsigned lt = lanemask_lt();
   int m = 0, ties = 0;
   for (int base = 0; base < n; base += 32) {
     const int j = base + lane;
@@ -258,110 +296,278 @@ select_prefill_kernel(Geom g, const int* __restrict__ cu, int max_nblk, int word
   }
 }
 
-// -------------------------------------------------------- decode: scoring
-// Grid (ceil(cap/B / 64), batch); 128 threads. Each CTA stages 64 pooled rows
-// once and scores them for every new query of its sequence.
-template <typename T, int kDI>
-__global__ void __launch_bounds__(128)
-decode_score_kernel(Geom g, int n_q, int cap, const int* __restrict__ kv_len,
-                    const T* __restrict__ iq, const float* __restrict__ iw,
-                    const float* __restrict__ pooled, float* __restrict__ scores) {
-  extern __shared__ __align__(16) float smem[];
-  constexpr int kStride = kDI + 1;
-  float* kbar_s = smem;
-  float* iq_s = kbar_s + kChunk * kStride;            // n_q * Hi * kDI
-  float* iw_s = iq_s + n_q * g.Hi * kDI;              // n_q * Hi
-  const int b = blockIdx.y;
-  const int kv = kv_len[b];
-  const int nblk_cap = cap / g.B;
-  if (kv < n_q || kv > cap) return;
-  const int nc_max = kv / g.B;                        // candidates of the last query
-  const int c0 = blockIdx.x * kChunk;
-  if (c0 >= nblk_cap) return;
-  float* srow_b = scores + (size_t)b * n_q * nblk_cap;
-  for (int e = threadIdx.x; e < n_q * g.Hi * kDI; e += blockDim.x)
-    iq_s[e] = to_f32(iq[(size_t)b * n_q * g.Hi * kDI + e]);
-  for (int e = threadIdx.x; e < n_q * g.Hi; e += blockDim.x)
-    iw_s[e] = iw[(size_t)b * n_q * g.Hi + e];
-  const int rows = max(0, min(kChunk, nc_max - c0));
-  const float* src = pooled + ((size_t)b * nblk_cap + c0) * kDI;
-  for (int e = threadIdx.x; e < rows * kDI; e += blockDim.x) {
-    const int r = e / kDI, d = e - r * kDI;
-    kbar_s[r * kStride + d] = src[(size_t)r * kDI + d];
+// ------------------------------------------------------- CTA top-k
+// The k largest of keys[0..n) (shared memory) where a lower position wins a
+// tie, chosen by a whole CTA of 256 threads with few dependent steps: four
+// 8-bit radix passes find the k-th largest key tau (a shared histogram per
+// pass, lanes with equal digits adding once), then each thread counts the
+// keys > tau and == tau in its contiguous run of positions, one block scan
+// turns the counts into output offsets, and the chosen positions are written
+// in ascending order. Returns min(k, n).
+constexpr int kTopkThreads = 256;
+
+__device__ int cta_topk_radix(const uint32_t* keys, int n, int k, int* out) {
+  __shared__ int hist[256];
+  __shared__ int scan_s[2][kTopkThreads / 32];
+  __shared__ uint32_t s_prefix, s_mask;
+  __shared__ int s_need;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (n <= k) {
+    for (int j = tid; j < n; j += kTopkThreads) out[j] = j;
+    __syncthreads();
+    return n;
+  }
+  if (tid == 0) { s_prefix = 0u; s_mask = 0u; s_need = k; }
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    hist[tid] = 0;
+    __syncthreads();
+    const uint32_t prefix = s_prefix, mask = s_mask;
+    for (int base = 0; base < n; base += kTopkThreads) {
+      const int j = base + tid;
+      const uint32_t key = j < n ? keys[j] : 0u;
+      const bool live = j < n && (key & mask) == prefix;
+      const uint32_t digit = live ? (key >> shift) & 255u : 256u;
+      const unsigned same = __match_any_sync(kFull, digit);
+      if (live && (__ffs(same) - 1) == lane) atomicAdd(&hist[digit], __popc(same));
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // lane l owns digits 255 - 8l down to 248 - 8l
+      int cnt[8], local = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        cnt[e] = hist[255 - 8 * lane - e];
+        local += cnt[e];
+      }
+      int incl = local;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const int need = s_need;
+      const int before = incl - local;
+      if (before < need && incl >= need) {
+        int run = before;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if (run + cnt[e] >= need) {
+            s_prefix = prefix | ((uint32_t)(255 - 8 * lane - e) << shift);
+            s_mask = mask | (255u << shift);
+            s_need = need - run;
+            break;
+          }
+          run += cnt[e];
+        }
+      }
+    }
+    __syncthreads();
+  }
+  const uint32_t tau = s_prefix;
+  const int need = s_need;   // keys equal to tau to take, lowest positions first
+  // each thread owns the contiguous run [lo, hi)
+  const int per = (n + kTopkThreads - 1) / kTopkThreads;
+  const int lo = min(n, tid * per), hi = min(n, lo + per);
+  int n_gt = 0, n_eq = 0;
+  for (int j = lo; j < hi; ++j) {
+    const uint32_t key = keys[j];
+    n_gt += key > tau;
+    n_eq += key == tau;
+  }
+  // exclusive scans of the tie counts and of the greater counts
+  int ie = n_eq, ig = n_gt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int a = __shfl_up_sync(kFull, ie, o), b = __shfl_up_sync(kFull, ig, o);
+    if (lane >= o) { ie += a; ig += b; }
+  }
+  if (lane == 31) { scan_s[0][warp] = ie; scan_s[1][warp] = ig; }
+  __syncthreads();
+  int eq_before = ie - n_eq, gt_before = ig - n_gt;
+  for (int w = 0; w < warp; ++w) { eq_before += scan_s[0][w]; gt_before += scan_s[1][w]; }
+  // ties before this run that are taken, plus greater keys before this run
+  int o_idx = gt_before + min(eq_before, need);
+  int t_rank = eq_before;
+  for (int j = lo; j < hi; ++j) {
+    const uint32_t key = keys[j];
+    if (key > tau) {
+      out[o_idx++] = j;
+    } else if (key == tau) {
+      if (t_rank < need) out[o_idx++] = j;
+      ++t_rank;
+    }
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < n_q * kChunk; e += blockDim.x) {
-    const int i = e / kChunk, r = e - i * kChunk;
-    const int j = c0 + r;
-    if (j >= nblk_cap) continue;
-    const int n = kv - n_q + 1 + i;
-    float s = -INFINITY;
-    if (j < n / g.B)
-      s = score_row<kDI>(kbar_s + r * kStride, iq_s + i * g.Hi * kDI, iw_s + i * g.Hi,
-                         g.Hi, g.idx_scale);
-    srow_b[(size_t)i * nblk_cap + j] = s;
-  }
+  return k;
 }
 
-// --------------------------------------------------------- decode: top-k
-// Grid (n_q, batch); 256 threads. Each warp takes the top-k of a contiguous
-// slice of candidates (positions come out ascending, so concatenating the
-// warps' picks keeps ascending block order); warp 0 then takes the top-k of
-// the concatenation, where a lower position is a lower block index.
-__global__ void __launch_bounds__(256)
-decode_topk_kernel(Geom g, int n_q, int cap, const int* __restrict__ kv_len,
-                   const float* __restrict__ scores, int* __restrict__ sel,
-                   int* __restrict__ nsel, float* __restrict__ scores_out) {
-  extern __shared__ __align__(16) uint32_t usmem[];
+// ------------------------------------------------ decode: fused selection
+// Grid (ceil(cap/B / 64), batch); 256 threads (8 warps). CTA c owns candidate blocks
+// [64c, 64c + 64) of sequence b and
+//  1. pools the blocks of its range that this step's tokens complete (the
+//     incremental pooled-key cache) and writes them to the cache,
+//  2. scores its blocks for every new query of the sequence (one thread per
+//     (block, indexer head), summed over the heads by shuffles) and publishes
+//     the score keys,
+//  3. the last CTA of the sequence to finish (an atomic counter that the
+//     caller zeroes before the launch) selects each query's top-k from all
+//     of them (cta_topk_radix), then appends the tail block.
+constexpr int kSelThreads = 256;
+constexpr int kPart = 64;                 // candidate blocks per CTA
+
+template <typename T, int kDI>
+__global__ void __launch_bounds__(kSelThreads)
+decode_select_kernel(Geom g, int n_q, int cap, const int* __restrict__ kv_len,
+                     const T* __restrict__ iq, const T* __restrict__ ik_cache,
+                     const float* __restrict__ iw, float* __restrict__ pooled,
+                     float* __restrict__ scores_out, uint32_t* __restrict__ keys_ws,
+                     int* __restrict__ counter, int* __restrict__ sel, int* __restrict__ nsel,
+                     int* dev_err) {
+  extern __shared__ __align__(16) float smem[];
+  constexpr int kStride = kDI + 1;
+  const int k = g.k;
   const int nblk_cap = cap / g.B;
-  uint32_t* keys = usmem;                                  // nblk_cap
-  uint32_t* ckeys = keys + nblk_cap;                       // 8 * k
-  int* cidx = reinterpret_cast<int*>(ckeys + 8 * g.k);     // 8 * k
-  int* cpos = cidx + 8 * g.k;                              // 8 * k (per-warp scratch)
-  __shared__ int cnt_w[8];
-  const int i = blockIdx.x, b = blockIdx.y;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* kbar_s = smem;                                       // kPart * kStride
+  float* iq_s = kbar_s + kPart * kStride;                     // n_q * Hi * kDI
+  float* iw_s = iq_s + n_q * g.Hi * kDI;                      // n_q * Hi
+  uint32_t* keys_s = reinterpret_cast<uint32_t*>(iw_s + n_q * g.Hi);   // nblk_cap (merge)
+  int* pos_s = reinterpret_cast<int*>(keys_s + nblk_cap);             // k
+  __shared__ int last_s;
+
+  const int c = blockIdx.x, b = blockIdx.y;
   const int kv = kv_len[b];
-  int* srow = sel + ((size_t)b * n_q + i) * (g.k + 1);
+  const int kp1 = k + 1;
   if (kv < n_q || kv > cap) {
-    for (int e = threadIdx.x; e < g.k + 1; e += blockDim.x) srow[e] = -1;
-    if (threadIdx.x == 0) nsel[(size_t)b * n_q + i] = 0;
+    if (c == 0) {
+      for (int e = threadIdx.x; e < n_q * kp1; e += blockDim.x) sel[(size_t)b * n_q * kp1 + e] = -1;
+      for (int e = threadIdx.x; e < n_q; e += blockDim.x) nsel[(size_t)b * n_q + e] = 0;
+      if (dev_err && threadIdx.x == 0) atomicExch(dev_err, 1);
+    }
     return;
   }
-  const int n = kv - n_q + 1 + i;
-  const int nc = n / g.B;
-  const float* s = scores + ((size_t)b * n_q + i) * nblk_cap;
-  for (int j = threadIdx.x; j < nc; j += blockDim.x) keys[j] = score_key(s[j]);
-  if (scores_out)
-    for (int j = threadIdx.x; j < nblk_cap; j += blockDim.x)
-      scores_out[((size_t)b * n_q + i) * nblk_cap + j] = j < nc ? s[j] : -INFINITY;
-  __syncthreads();
-  const int per = (nc + 7) / 8;
-  const int lo = min(nc, warp * per), hi = min(nc, lo + per);
-  int* wpos = cpos + warp * g.k;
-  const int mw = warp_topk_positions(keys + lo, hi - lo, g.k, wpos, lane);
-  if (lane == 0) cnt_w[warp] = mw;
-  __syncthreads();
-  int off = 0;
-  for (int w = 0; w < warp; ++w) off += cnt_w[w];
-  for (int e = lane; e < mw; e += 32) {
-    ckeys[off + e] = keys[lo + wpos[e]];
-    cidx[off + e] = lo + wpos[e];
+  const int nc_last = kv / g.B;                    // candidates of the last query
+  const int nparts = max(1, (nc_last + kPart - 1) / kPart);
+  if (c >= nparts) return;
+  const int j0 = c * kPart;
+  const int rows = max(0, min(kPart, nc_last - j0));
+
+  // 1. blocks completed by this step's tokens (pool_block_cta needs the whole CTA)
+  const int jnew_lo = max((kv - n_q) / g.B, j0), jnew_hi = min(nc_last, j0 + kPart);
+  for (int j = jnew_lo; j < jnew_hi; ++j) {
+    pool_block_cta(ik_cache + ((size_t)b * cap + (size_t)j * g.B) * kDI, g.B, kDI,
+                   pooled + ((size_t)b * nblk_cap + j) * kDI);
+    __syncthreads();
+  }
+  // 2. stage the range's pooled rows and the queries' indexer q / weights
+  {   // every load of the stage is issued before the first store
+    const float* src = pooled + ((size_t)b * nblk_cap + j0) * kDI;
+    constexpr int kPerThr = kPart * (kDI / 4) / kSelThreads;   // float4 per thread
+    float4 v[kPerThr];
+#pragma unroll
+    for (int u = 0; u < kPerThr; ++u) {
+      const int e = u * kSelThreads + threadIdx.x;
+      const int r = e / (kDI / 4), d4 = e - r * (kDI / 4);
+      v[u] = r < rows ? *reinterpret_cast<const float4*>(src + (size_t)r * kDI + 4 * d4)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    const int nq_e = n_q * g.Hi * kDI;
+    const T* iqb = iq + (size_t)b * nq_e;
+    float qv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int e = u * kSelThreads + threadIdx.x;
+      qv[u] = e < nq_e ? to_f32(iqb[e]) : 0.f;
+    }
+    const float wv = threadIdx.x < n_q * g.Hi ? iw[(size_t)b * n_q * g.Hi + threadIdx.x] : 0.f;
+    for (int e = 4 * kSelThreads + threadIdx.x; e < nq_e; e += kSelThreads)
+      iq_s[e] = to_f32(iqb[e]);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int e = u * kSelThreads + threadIdx.x;
+      if (e < nq_e) iq_s[e] = qv[u];
+    }
+    if (threadIdx.x < n_q * g.Hi) iw_s[threadIdx.x] = wv;
+#pragma unroll
+    for (int u = 0; u < kPerThr; ++u) {
+      const int e = u * kSelThreads + threadIdx.x;
+      const int r = e / (kDI / 4), d4 = e - r * (kDI / 4);
+      float* dst = kbar_s + r * kStride + 4 * d4;
+      dst[0] = v[u].x; dst[1] = v[u].y; dst[2] = v[u].z; dst[3] = v[u].w;
+    }
   }
   __syncthreads();
-  if (warp != 0) return;
-  int total = 0;
-  for (int w = 0; w < 8; ++w) total += cnt_w[w];
-  int* fpos = cpos;   // reuse warp 0's slot (the first k entries)
-  const int m = warp_topk_positions(ckeys, total, g.k, fpos, lane);
-  const int tail = n - nc * g.B;
-  for (int e = lane; e < g.k + 1; e += 32) {
-    int v = -1;
-    if (e < m) v = cidx[fpos[e]];
-    else if (e == m && tail > 0) v = nc;
-    srow[e] = v;
+  // scores: one (query, block, head) triple per thread; heads are adjacent
+  // lanes (Hi divides 32), so the weighted relu terms are summed by shuffles
+  const int per_q = kPart * g.Hi;
+  for (int base = 0; base < n_q * per_q; base += blockDim.x) {
+    const int e = base + threadIdx.x;
+    const int i = e / per_q, rem = e - i * per_q;
+    const int r = rem / g.Hi, h = rem - r * g.Hi;
+    float term = 0.f;
+    const int j = j0 + r;
+    const int nc_i = i < n_q ? (kv - n_q + 1 + i) / g.B : 0;
+    const bool live = i < n_q && j < nc_i;
+    if (live) {
+      const float* krow = kbar_s + r * kStride;
+      const float4* qh = reinterpret_cast<const float4*>(iq_s + (i * g.Hi + h) * kDI);
+      float dot = 0.f;
+#pragma unroll
+      for (int d4 = 0; d4 < kDI / 4; ++d4) {
+        const float4 qv = qh[d4];
+        dot = fmaf(qv.x, krow[4 * d4 + 0], dot);
+        dot = fmaf(qv.y, krow[4 * d4 + 1], dot);
+        dot = fmaf(qv.z, krow[4 * d4 + 2], dot);
+        dot = fmaf(qv.w, krow[4 * d4 + 3], dot);
+      }
+      term = iw_s[i * g.Hi + h] * fmaxf(dot, 0.f);
+    }
+    for (int o = 1; o < g.Hi; o <<= 1) term += __shfl_xor_sync(kFull, term, o);
+    if (i < n_q && h == 0 && j < j0 + kPart && j < nblk_cap) {
+      const float sc = live ? term * g.idx_scale : -INFINITY;
+      if (live) keys_ws[((size_t)b * n_q + i) * nblk_cap + j] = score_key(sc);
+      if (scores_out) scores_out[((size_t)b * n_q + i) * nblk_cap + j] = sc;
+    }
   }
-  if (lane == 0) nsel[(size_t)b * n_q + i] = m + (tail > 0 ? 1 : 0);
+  // 3. the last range to finish selects
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last_s = atomicAdd(&counter[b], 1) == nparts - 1;
+  __syncthreads();
+  if (!last_s) return;
+  __threadfence();
+  for (int i = 0; i < n_q; ++i) {
+    const int n = kv - n_q + 1 + i;
+    const int nc_i = n / g.B;
+    {   // eight loads in flight per thread before any store
+      const uint32_t* kq = keys_ws + ((size_t)b * n_q + i) * nblk_cap;
+      for (int j0 = 0; j0 < nc_i; j0 += 8 * kSelThreads) {
+        uint32_t v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int j = j0 + u * kSelThreads + threadIdx.x;
+          v[u] = j < nc_i ? __ldcg(kq + j) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int j = j0 + u * kSelThreads + threadIdx.x;
+          if (j < nc_i) keys_s[j] = v[u];
+        }
+      }
+    }
+    __syncthreads();
+    const int m = cta_topk_radix(keys_s, nc_i, k, pos_s);
+    const int tail = n - nc_i * g.B;
+    int* srow = sel + ((size_t)b * n_q + i) * kp1;
+    for (int e = threadIdx.x; e < kp1; e += blockDim.x) {
+      int v = -1;
+      if (e < m) v = pos_s[e];
+      else if (e == m && tail > 0) v = nc_i;
+      srow[e] = v;
+    }
+    if (threadIdx.x == 0) nsel[(size_t)b * n_q + i] = m + (tail > 0 ? 1 : 0);
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) counter[b] = 0;
 }
 
 // ------------------------------------------------------------ launchers
@@ -416,8 +622,7 @@ static cudaError_t launch_select_prefill_t(const Geom& g, const int* cu, int bat
   const int nc_cap = max(1, max_seqlen / g.B);
   const size_t smem = select_prefill_smem(g, nc_cap);
   auto kern = select_prefill_kernel<T, kDI>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(kern), (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((max_seqlen + 7) / 8, batch);
   kern<<<grid, 256, smem, st>>>(g, cu, max_nblk, words, (const T*)iq, iw, pooled, nc_cap, sel,
@@ -445,47 +650,47 @@ cudaError_t launch_select_prefill(qsa_dtype dt, const Geom& g, const int* cu, in
 #undef QSA_SEL
 }
 
+size_t decode_select_smem(const Geom& g, int n_q, int cap) {
+  return sizeof(float) * ((size_t)kPart * (g.di + 1) + (size_t)n_q * g.Hi * g.di + n_q * g.Hi) +
+         sizeof(uint32_t) * (size_t)(cap / g.B) + sizeof(int) * (size_t)g.k;
+}
+
+int decode_select_parts(const Geom& g, int cap) { return (cap / g.B + kPart - 1) / kPart; }
+
 template <typename T, int kDI>
-static cudaError_t launch_decode_score_t(const Geom& g, int batch, int n_q, int cap,
-                                         const int* kv_len, const void* iq, const float* iw,
-                                         const float* pooled, float* scores, cudaStream_t st) {
-  const int nblk_cap = cap / g.B;
-  const size_t smem =
-      sizeof(float) * ((size_t)kChunk * (kDI + 1) + (size_t)n_q * g.Hi * kDI + n_q * g.Hi);
-  auto kern = decode_score_kernel<T, kDI>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+static cudaError_t launch_decode_select_t(const Geom& g, int batch, int n_q, int cap,
+                                          const int* kv_len, const void* iq, const void* ik_cache,
+                                          const float* iw, float* pooled, float* scores_out,
+                                          uint32_t* keys_ws, int* counter, int* sel, int* nsel,
+                                          int* dev_err, cudaStream_t st) {
+  const size_t smem = decode_select_smem(g, n_q, cap);
+  auto kern = decode_select_kernel<T, kDI>;
+  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(kern), (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((nblk_cap + kChunk - 1) / kChunk, batch);
-  kern<<<grid, 128, smem, st>>>(g, n_q, cap, kv_len, (const T*)iq, iw, pooled, scores);
+  kern<<<dim3(decode_select_parts(g, cap), batch), kSelThreads, smem, st>>>(
+      g, n_q, cap, kv_len, (const T*)iq, (const T*)ik_cache, iw, pooled, scores_out, keys_ws,
+      counter, sel, nsel, dev_err);
   note_launch();
   return cudaGetLastError();
 }
 
 cudaError_t launch_decode_select(qsa_dtype dt, const Geom& g, int batch, int n_q, int cap,
-                                 const int* kv_len, const void* iq, const float* iw,
-                                 const float* pooled, float* scores_ws, int* sel, int* nsel,
-                                 float* scores_out, cudaStream_t st) {
+                                 const int* kv_len, const void* iq, const void* ik_cache,
+                                 const float* iw, float* pooled, float* scores_out,
+                                 uint32_t* keys_ws, int* counter, int* sel, int* nsel,
+                                 int* dev_err, cudaStream_t st) {
   if (batch == 0) return cudaSuccess;
-  cudaError_t e;
-#define QSA_DS(T, DI) \
-  e = launch_decode_score_t<T, DI>(g, batch, n_q, cap, kv_len, iq, iw, pooled, scores_ws, st)
+#define QSA_DS(T, DI)                                                                       \
+  return launch_decode_select_t<T, DI>(g, batch, n_q, cap, kv_len, iq, ik_cache, iw, pooled, \
+                                       scores_out, keys_ws, counter, sel, nsel, dev_err, st)
   if (dt == QSA_BF16) {
-    if (g.di == 64) QSA_DS(__nv_bfloat16, 64); else QSA_DS(__nv_bfloat16, 32);
+    if (g.di == 64) QSA_DS(__nv_bfloat16, 64);
+    QSA_DS(__nv_bfloat16, 32);
   } else {
-    if (g.di == 64) QSA_DS(float, 64); else QSA_DS(float, 32);
+    if (g.di == 64) QSA_DS(float, 64);
+    QSA_DS(float, 32);
   }
 #undef QSA_DS
-  if (e != cudaSuccess) return e;
-  const int nblk_cap = cap / g.B;
-  const size_t smem = sizeof(uint32_t) * ((size_t)nblk_cap + 3 * 8 * g.k);
-  e = cudaFuncSetAttribute(decode_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem);
-  if (e != cudaSuccess) return e;
-  decode_topk_kernel<<<dim3(n_q, batch), 256, smem, st>>>(g, n_q, cap, kv_len, scores_ws, sel,
-                                                          nsel, scores_out);
-  note_launch();
-  return cudaGetLastError();
 }
 
 }  // namespace qsa
