@@ -10,9 +10,9 @@ of keys each query attends, |S(t)| = min(k, floor(n/B)) * B + n mod B.
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                   [--impl ours|reference]
 
-Under torchrun every rank runs its own copy of the workload (independent
-problems, no collective on the data path: weak scaling); the reported value is
-all ranks' tokens over the slowest rank's device time.
+Under torchrun every rank runs its own shard: the workload's shapes with its own
+seed (independent problems, no collective on the data path: weak scaling); the
+reported value is all ranks' tokens over the slowest rank's device time.
 """
 from __future__ import annotations
 
@@ -55,6 +55,48 @@ def workload_units(w):
     else:
         ns = [w.kv_len - w.n_q + 1 + i for _ in range(w.batch) for i in range(w.n_q)]
     return sum(selected_tokens(n, w.block_size, w.topk) for n in ns), ns
+
+
+def recorded_traffic(kernel_file: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the kernel source as it is now (sha256 prefix match); else None."""
+    import hashlib
+    src = os.path.join(ROOT, "block_sparse_attention_17_b200", "csrc", kernel_file)
+    table = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not (os.path.exists(src) and os.path.exists(table)):
+        return None
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    for line in open(table):
+        parts = line.split()
+        if len(parts) == 4 and not line.startswith("#") and parts[0] == kernel_file \
+                and sha.startswith(parts[1]) and parts[2] == workload:
+            return int(parts[3])
+    return None
+
+
+def rank_workload(w, rank: int):
+    """The shard rank ``rank`` processes: the workload's shapes, its own seed.
+
+    Rank 0 keeps the workload's seed, so a 1-GPU run and rank 0 of an N-GPU run
+    draw the same inputs; ragged workloads draw their lengths per rank too.
+    """
+    return w if rank == 0 else w.with_(seed=w.seed + 7919 * rank)
+
+
+def reduce_over_ranks(dist, units: float, ms: float, device):
+    """(sum of ``units`` over ranks, max of ``ms`` over ranks).
+
+    Two collectives, taken in the same order by every rank; ``device`` is the
+    device the process group's backend reduces on (cuda for NCCL, cpu for gloo).
+    """
+    if dist is None:
+        return units, ms
+    import torch
+    u = torch.tensor([float(units)], dtype=torch.float64, device=device)
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(u.item()), float(t.item())
 
 
 def load_peaks():
@@ -310,13 +352,10 @@ def run_ours(args, w, rank, world, dist):
     clk = clocks.stop()
     lib.qsa_set_stage_events(None, 0)
     total_ms = float(sum(step_ms))
+    job_units, total_ms = reduce_over_ranks(dist, units, total_ms, dev)
     if dist is not None:
-        import torch.distributed as tdist
-        t = torch.tensor([total_ms], device=dev)
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        total_ms = float(t.item())
         dist.barrier()
-    value = units * args.steps * world / (total_ms / 1e3)
+    value = job_units * args.steps / (total_ms / 1e3)
 
     # roofline of the dominant kernel: attention (+ combine for decode)
     attn_ms = float(np.mean(stage_attn))
@@ -325,8 +364,11 @@ def run_ours(args, w, rank, world, dist):
         achieved = alg["work"] / (attn_ms / 1e3) / 1e12
     else:
         achieved = alg["work"] / (attn_ms / 1e3) / 1e9
+    kfile = ("qsa_decode_attn.cu" if w.kind == "decode" else
+             "qsa_attn_tc.cu" if (w.dtype == "bf16" and w.head_dim == 128) else "qsa_attn_simt.cu")
     roof = {"bound": alg["bound"], "achieved": round(achieved, 3), "peak": peak,
-            "unit": alg["unit"], "frac": round(achieved / peak, 5), "traffic": None,
+            "unit": alg["unit"], "frac": round(achieved / peak, 5),
+            "traffic": recorded_traffic(kfile, w.name),
             "kernel": "qsa attention" + (" + combine" if w.kind == "decode" else ""),
             "kernel_ms": round(attn_ms, 5), "peak_source": f"{peak_kind} ({alg['peak_key']})",
             "algorithmic_per_launch": alg["work"]}
@@ -351,12 +393,8 @@ def run_ours(args, w, rank, world, dist):
                 e_en[i - 1].record(stream)
         torch.cuda.synchronize()
         e2e_ms = float(sum(e_st[i].elapsed_time(e_en[i]) for i in range(args.steps)))
-        if dist is not None:
-            import torch.distributed as tdist
-            t = torch.tensor([e2e_ms], device=dev)
-            tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": units * args.steps * world / (e2e_ms / 1e3), "unit": UNIT,
+        _, e2e_ms = reduce_over_ranks(dist, units, e2e_ms, dev)
+        e2e = {"value": job_units * args.steps / (e2e_ms / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e2e_ms / args.steps}
 
@@ -371,12 +409,14 @@ def run_ours(args, w, rank, world, dist):
              "timing": ("CUDA-graph replay of one library call per step" if graph is not None
                         else "eager library call per step"),
              "eager_ms_per_step": float(np.mean(eager_ms)),
-             "selected_kv_tokens_per_step": units, "input_gen_s": round(t_gen, 2)}
+             "selected_kv_tokens_per_step": units, "job_selected_kv_tokens_per_step": job_units,
+             "shards": "one per rank: the workload's shapes, seed + 7919 * rank",
+             "input_gen_s": round(t_gen, 2)}
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": w.dtype, "data": "synthetic (seeded numpy draws, shapes of the workload)",
-            "config": config_of(w, extra), "parallelism": f"replicas{world}",
+            "config": config_of(w, extra), "parallelism": f"dp{world}",
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": int(launches), "clocks": clk,
             "impl": "ours"}
@@ -452,9 +492,9 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
-    w = WORKLOADS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+    w = rank_workload(WORKLOADS[args.workload], rank)
 
     if args.impl == "reference":
         if rank != 0:
