@@ -10,6 +10,7 @@
 #include <atomic>
 #include <map>
 #include <mutex>
+#include <tuple>
 #include <utility>
 
 #include "qsa_common.cuh"
@@ -36,6 +37,29 @@ cudaError_t qsa::set_max_dynamic_smem(const void* func, int bytes) {
   e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e == cudaSuccess) done[key] = bytes;
   return e;
+}
+
+cudaError_t qsa::resident_ctas(const void* func, int threads, size_t smem, int* per_sm,
+                               int* sms) {
+  static std::mutex mu;
+  static std::map<std::tuple<const void*, int, int, size_t>, std::pair<int, int>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_tuple(func, dev, threads, smem);
+  auto it = done.find(key);
+  if (it != done.end()) {
+    *per_sm = it->second.first;
+    *sms = it->second.second;
+    return cudaSuccess;
+  }
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, func, threads, smem);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  done[key] = std::make_pair(*per_sm, *sms);
+  return cudaSuccess;
 }
 
 namespace {
@@ -134,7 +158,8 @@ struct Carve {
 };
 
 struct PrefillWs {
-  int* err;
+  int* err;             // error word, then the selection kernel's work counter
+  int* sched;
   float* pooled;
   int* sel;
   int* nsel;
@@ -147,7 +172,8 @@ PrefillWs carve_prefill(const Geom& g, void* ws, int batch, int T, int max_seqle
   const int words = (max_nblk + 31) / 32;
   Carve c(ws);
   PrefillWs w;
-  w.err = c.take<int>(1);
+  w.err = c.take<int>(2);
+  w.sched = w.err + 1;
   w.pooled = c.take<float>((size_t)batch * max_nblk * g.di);
   w.sel = c.take<int>((size_t)T * (g.k + 1));
   w.nsel = c.take<int>((size_t)T);
@@ -281,11 +307,13 @@ static qsa_status prefill_select_common(const qsa_config* cfg, const Geom& g, in
                                         int32_t* nsel, float* scores, cudaStream_t st) {
   const int max_nblk = (max_seqlen + g.B - 1) / g.B;
   const int words = (max_nblk + 31) / 32;
+  // the error word and the selection's work counter start at zero
+  QSA_CUDA(cudaMemsetAsync(w.err, 0, 2 * sizeof(int), st), "clear error word");
   QSA_CUDA(launch_pool_prefill(cfg->dtype, ik, cu, batch, max_seqlen, g.B, g.di, pooled,
                                max_nblk, st),
            "pool");
   QSA_CUDA(launch_select_prefill(cfg->dtype, g, cu, batch, max_seqlen, max_nblk, words, iq, iw,
-                                 pooled, sel, nsel, w.bitmask, scores,
+                                 pooled, w.sched, sel, nsel, w.bitmask, scores,
                                  std::max(1, max_seqlen / g.B), st),
            "select");
   return QSA_OK;
@@ -317,7 +345,6 @@ qsa_status qsa_prefill(const qsa_config* cfg, int batch, int total_tokens, int m
   float* pooled = pooled_out ? pooled_out : w.pooled;
   int* sel_p = sel ? sel : w.sel;
   int* nsel_p = nsel ? nsel : w.nsel;
-  QSA_CUDA(cudaMemsetAsync(w.err, 0, sizeof(int), st), "clear error word");
   stage_mark(0, st);
   s = prefill_select_common(cfg, g, batch, total_tokens, max_seqlen, cu_seqlens, iq, ik, iw, w,
                             pooled, sel_p, nsel_p, nullptr, st);

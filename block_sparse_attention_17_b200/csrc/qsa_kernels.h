@@ -17,6 +17,10 @@ void note_launch(int n = 1);
 // (kernel, device, size) instead of on every launch.
 cudaError_t set_max_dynamic_smem(const void* func, int bytes);
 
+// CTAs of `func` (threads, dynamic shared memory) resident per SM, and the
+// SM count of the current device (cached per function, device and shape).
+cudaError_t resident_ctas(const void* func, int threads, size_t smem, int* per_sm, int* sms);
+
 // Sets the message qsa_last_error() returns on this host thread.
 void set_last_error(const char* msg);
 
@@ -27,10 +31,12 @@ cudaError_t launch_pool_cache(qsa_dtype dt, const void* ik_cache, const int* kv_
                               int cap, int n_q, int mode, int B, int di, float* pooled,
                               int* dev_err, cudaStream_t st);
 size_t select_prefill_smem(const Geom& g, int nc_cap);
+// sched: one int the caller zeroed on the stream before the launch (the
+// kernel's work counter).
 cudaError_t launch_select_prefill(qsa_dtype dt, const Geom& g, const int* cu, int batch,
                                   int max_seqlen, int max_nblk, int words, const void* iq,
-                                  const float* iw, const float* pooled, int* sel, int* nsel,
-                                  uint32_t* bitmask, float* scores, int scores_ld,
+                                  const float* iw, const float* pooled, int* sched, int* sel,
+                                  int* nsel, uint32_t* bitmask, float* scores, int scores_ld,
                                   cudaStream_t st);
 int decode_select_parts(const Geom& g, int cap);
 cudaError_t launch_decode_select(qsa_dtype dt, const Geom& g, int batch, int n_q, int cap,

@@ -11,6 +11,8 @@
 // written in ascending block order, followed by the tail block when the
 // query's visible length is not a multiple of B (dev.to page, "Qwen Sparse
 // Attention": the trailing incomplete block is always kept).
+#include <algorithm>
+
 #include "qsa_common.cuh"
 #include "qsa_kernels.h"
 
@@ -96,36 +98,6 @@ pool_cache_kernel(const T* __restrict__ ik_cache, const int* __restrict__ kv_len
                  pooled + ((size_t)b * (cap / B) + j) * di);
 }
 
-// ----------------------------------------------------------------- scoring
-constexpr int kChunk = 64;   // pooled rows staged in shared memory at a time
-
-// Score of pooled row `row` (kDI floats, padded stride) for one query whose
-// indexer q (Hi x kDI, fp32) and weights sit in shared memory.
-template <int kDI>
-__device__ __forceinline__ float score_row(const float* __restrict__ krow,
-                                           const float* __restrict__ iq_s,
-                                           const float* __restrict__ iw_s, int Hi,
-                                           float c) {
-  float kv[kDI];
-#pragma unroll
-  for (int d = 0; d < kDI; ++d) kv[d] = krow[d];
-  float s = 0.f;
-  for (int h = 0; h < Hi; ++h) {
-    const float4* qh = reinterpret_cast<const float4*>(iq_s + h * kDI);
-    float dot = 0.f;
-#pragma unroll
-    for (int d4 = 0; d4 < kDI / 4; ++d4) {
-      const float4 qv = qh[d4];
-      dot = fmaf(qv.x, kv[4 * d4 + 0], dot);
-      dot = fmaf(qv.y, kv[4 * d4 + 1], dot);
-      dot = fmaf(qv.z, kv[4 * d4 + 2], dot);
-      dot = fmaf(qv.w, kv[4 * d4 + 3], dot);
-    }
-    s = fmaf(iw_s[h], fmaxf(dot, 0.f), s);
-  }
-  return s * c;
-}
-
 // ----------------------------------------------------------------- top-k
 __device__ __forceinline__ unsigned lanemask_lt() {
   unsigned m;
@@ -135,66 +107,111 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 
 // Warp-cooperative selection of the k largest keys among keys[0..n) where a
 // lower position wins a tie. Writes the chosen positions, ascending, to out[]
-// and returns how many (min(k, n)). The k-th largest key is found by an
-// MSB-first bit search on the 32-bit key; ties at that key are taken in
-// ascending position order. Up to 256 keys are held in registers (8 per
-// lane) for the whole search; longer lists are re-read from memory.
-__device__ int warp_topk_positions(const uint32_t* keys, int n, int k, int* out, int lane) {
+// and their bitmap (bit j % 32 of word j / 32 for position j) to
+// words[0..nw), and returns how many were chosen (min(k, n)).
+//
+// The selection threshold tau is found by an MSB-first bit search that keeps
+// count(keys >= tau) >= k. It starts below the bits all keys share (those of
+// the warp's max and min key agree above their highest differing bit) and
+// stops as soon as a candidate threshold has exactly k keys at or above it;
+// otherwise it ends on the k-th largest key, whose ties are then taken in
+// ascending position order. Up to 32 * kR keys are held in registers; longer
+// lists are re-read from shared memory.
+template <int kR>
+__device__ __forceinline__ uint32_t topk_threshold_regs(const uint32_t (&kr)[kR],
+                                                        const bool (&ok)[kR], int k) {
+  uint32_t hi = 0u, lo = 0xffffffffu;
+#pragma unroll
+  for (int i = 0; i < kR; ++i) {
+    if (ok[i]) { hi = max(hi, kr[i]); lo = min(lo, kr[i]); }
+  }
+  hi = __reduce_max_sync(kFull, hi);
+  lo = __reduce_min_sync(kFull, lo);
+  if (hi == lo) return hi;
+  const int top = 31 - __clz(hi ^ lo);                  // highest differing bit
+  uint32_t tau = top == 31 ? 0u : (hi & ~((2u << top) - 1u));
+#pragma unroll 1
+  for (int bit = top; bit >= 0; --bit) {
+    const uint32_t cand = tau | (1u << bit);
+    int c = 0;
+#pragma unroll
+    for (int i = 0; i < kR; ++i) c += (ok[i] && kr[i] >= cand) ? 1 : 0;
+    c = __reduce_add_sync(kFull, c);
+    if (c >= k) tau = cand;
+    if (c == k) break;
+  }
+  return tau;
+}
+
+template <int kR>
+__device__ int warp_topk_regs(const uint32_t* keys, int n, int k, int* out, uint32_t* words,
+                              int nw, int lane) {
+  const unsigned lt = lanemask_lt();
+  uint32_t kr[kR];
+  bool ok[kR];
+#pragma unroll
+  for (int i = 0; i < kR; ++i) {
+    const int j = lane + 32 * i;
+    ok[i] = j < n;
+    kr[i] = ok[i] ? keys[j] : 0u;
+  }
+  const uint32_t tau = topk_threshold_regs<kR>(kr, ok, k);
+  int gt = 0;
+#pragma unroll
+  for (int i = 0; i < kR; ++i) gt += (ok[i] && kr[i] > tau) ? 1 : 0;
+  const int need = k - __reduce_add_sync(kFull, gt);
+  int m = 0, ties = 0;
+  uint32_t mine = 0u;   // lane w keeps word w
+#pragma unroll
+  for (int i = 0; i < kR; ++i) {
+    const bool tie = ok[i] && kr[i] == tau;
+    const unsigned tb = __ballot_sync(kFull, tie);
+    const bool pick = ok[i] && (kr[i] > tau || (tie && ties + __popc(tb & lt) < need));
+    const unsigned pb = __ballot_sync(kFull, pick);
+    if (pick) out[m + __popc(pb & lt)] = lane + 32 * i;
+    if (lane == i) mine = pb;
+    m += __popc(pb);
+    ties += __popc(tb);
+  }
+  for (int w = lane; w < nw; w += 32) words[w] = w < kR ? mine : 0u;
+  __syncwarp();
+  return m;
+}
+
+__device__ int warp_topk(const uint32_t* keys, int n, int k, int* out, uint32_t* words, int nw,
+                         int lane) {
   if (n <= k) {
     for (int j = lane; j < n; j += 32) out[j] = j;
+    for (int w = lane; w < nw; w += 32) {
+      const int lo = 32 * w;
+      words[w] = lo >= n ? 0u : (n - lo >= 32 ? kFull : ((1u << (n - lo)) - 1u));
+    }
     __syncwarp();
     return n;
   }
+  if (n <= 128) return warp_topk_regs<4>(keys, n, k, out, words, nw, lane);
+  if (n <= 256) return warp_topk_regs<8>(keys, n, k, out, words, nw, lane);
   const unsigned lt = lanemask_lt();
-  if (n <= 256) {
-    uint32_t kr[8];
-    bool ok[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int j = lane + 32 * i;
-      ok[i] = j < n;
-      kr[i] = ok[i] ? keys[j] : 0u;
-    }
-    uint32_t tau = 0;
-    for (int bit = 31; bit >= 0; --bit) {
+  uint32_t hi = 0u, lo = 0xffffffffu;
+  for (int j = lane; j < n; j += 32) { hi = max(hi, keys[j]); lo = min(lo, keys[j]); }
+  hi = __reduce_max_sync(kFull, hi);
+  lo = __reduce_min_sync(kFull, lo);
+  uint32_t tau = hi;
+  if (hi != lo) {
+    const int top = 31 - __clz(hi ^ lo);
+    tau = top == 31 ? 0u : (hi & ~((2u << top) - 1u));
+    for (int bit = top; bit >= 0; --bit) {
       const uint32_t cand = tau | (1u << bit);
       int c = 0;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) c += (ok[i] && kr[i] >= cand) ? 1 : 0;
+      for (int j = lane; j < n; j += 32) c += keys[j] >= cand;
       c = __reduce_add_sync(kFull, c);
       if (c >= k) tau = cand;
+      if (c == k) break;
     }
-    int gt = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) gt += (ok[i] && kr[i] > tau) ? 1 : 0;
-    gt = __reduce_add_sync(kFull, gt);
-    const int need = k - gt;
-    int m = 0, ties = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const bool tie = ok[i] && kr[i] == tau;
-      const unsigned tb = __ballot_sync(kFull, tie);
-      const bool pick = ok[i] && (kr[i] > tau || (tie && ties + __popc(tb & lt) < need));
-      const unsigned pb = __ballot_sync(kFull, pick);
-      if (pick) out[m + __popc(pb & lt)] = lane + 32 * i;
-      m += __popc(pb);
-      ties += __popc(tb);
-    }
-    __syncwarp();
-    return m;
-  }
-  uint32_t tau = 0;
-  for (int bit = 31; bit >= 0; --bit) {
-    const uint32_t cand = tau | (1u << bit);
-    int c = 0;
-    for (int j = lane; j < n; j += 32) c += keys[j] >= cand;
-    c = __reduce_add_sync(kFull, c);
-    if (c >= k) tau = cand;
   }
   int gt = 0;
   for (int j = lane; j < n; j += 32) gt += keys[j] > tau;
-  gt = __reduce_add_sync(kFull, gt);
-  const int need = k - gt;
+  const int need = k - __reduce_add_sync(kFull, gt);
   int m = 0, ties = 0;
   for (int base = 0; base < n; base += 32) {
     const int j = base + lane;
@@ -204,95 +221,203 @@ __device__ int warp_topk_positions(const uint32_t* keys, int n, int k, int* out,
     const bool pick = j < n && (key > tau || (tie && ties + __popc(tb & lt) < need));
     const unsigned pb = __ballot_sync(kFull, pick);
     if (pick) out[m + __popc(pb & lt)] = j;
+    if (lane == 0 && (base >> 5) < nw) words[base >> 5] = pb;
     m += __popc(pb);
     ties += __popc(tb);
   }
+  for (int w = (n + 31) / 32 + lane; w < nw; w += 32) words[w] = 0u;
   __syncwarp();
   return m;
 }
 
 // ------------------------------------------------- prefill: score + top-k
-// Grid (ceil(max_seqlen / 8), batch); 8 warps, one query token per warp.
-// Dynamic shared memory: kbar chunk [64][kDI+1], iq [8][Hi][kDI], iw [8][Hi],
-// keys [8][nc_cap], positions [8][k].
+// Work item = a group of kQc = 8 consecutive query tokens of one sequence.
+// A CTA of 128 threads takes items from a counter in the workspace (zeroed
+// before the launch), the groups with the most candidates first, so the SMs
+// finish together. For an item it scores the group's queries against the
+// pooled rows of the blocks its last query sees, 64 rows at a time staged in
+// shared memory: thread (q, u) owns query q and rows u, u + 16, ... of the
+// chunk and accumulates the dot products of four indexer heads at once; per
+// head the dot runs over d in ascending order and the heads are folded in
+// ascending order, s = c * sum_h w[h] * relu(dot_h). Then warp w selects the
+// top-k of queries w and w + 4 from their score keys in shared memory.
+// Dynamic shared memory: iq [kQc][Hi][kDI], iw [kQc][Hi], pooled chunk
+// [64][kDI + 4], keys [kQc][nc_cap], positions [4][k].
+constexpr int kChunk = 64;           // pooled rows staged in shared memory at a time
+constexpr int kSelQc = 8;            // query tokens per work item
+constexpr int kSelThreadsPrefill = 128;
+constexpr int kSelCtasPerSm = 6;
+
 template <typename T, int kDI>
-__global__ void __launch_bounds__(256)
-select_prefill_kernel(Geom g, const int* __restrict__ cu, int max_nblk, int words,
-                      const T* __restrict__ iq, const float* __restrict__ iw,
-                      const float* __restrict__ pooled, int nc_cap,
-                      int* __restrict__ sel, int* __restrict__ nsel,
+__global__ void __launch_bounds__(kSelThreadsPrefill, 8)
+select_prefill_kernel(Geom g, const int* __restrict__ cu, int batch, int n_groups,
+                      int max_nblk, int words, const T* __restrict__ iq,
+                      const float* __restrict__ iw, const float* __restrict__ pooled, int nc_cap,
+                      int* __restrict__ sched, int* __restrict__ sel, int* __restrict__ nsel,
                       uint32_t* __restrict__ bitmask, float* __restrict__ scores,
                       int scores_ld) {
+  constexpr int kQc = kSelQc;
+  constexpr int kTpq = kSelThreadsPrefill / kQc;   // scoring threads per query (16)
+  constexpr int kRpt = kChunk / kTpq;              // rows per thread per chunk (4)
+  constexpr int kWarps = kSelThreadsPrefill / 32;
+  constexpr int kStride = kDI + 4;                 // 16-byte rows, banks spread
   extern __shared__ __align__(16) float smem[];
-  constexpr int kStride = kDI + 1;
-  float* kbar_s = smem;                               // kChunk * kStride
-  float* iq_s = kbar_s + kChunk * kStride;            // 8 * Hi * kDI
-  float* iw_s = iq_s + 8 * g.Hi * kDI;                // 8 * Hi
-  uint32_t* keys_s = reinterpret_cast<uint32_t*>(iw_s + 8 * g.Hi);   // 8 * nc_cap
-  int* pos_s = reinterpret_cast<int*>(keys_s + 8 * nc_cap);          // 8 * k
+  __shared__ int s_item;
+  const int Hi = g.Hi;
+  float* iq_s = smem;                                             // kQc * Hi * kDI
+  float* iw_s = iq_s + kQc * Hi * kDI;                            // kQc * Hi (padded to 4)
+  float* kb_s = iw_s + ((kQc * Hi + 3) & ~3);                     // kChunk * kStride
+  uint32_t* keys_s = reinterpret_cast<uint32_t*>(kb_s + kChunk * kStride);   // kQc * nc_cap
+  int* pos_s = reinterpret_cast<int*>(keys_s + kQc * nc_cap);     // kWarps * k
 
-  const int b = blockIdx.y;
-  const int s0 = cu[b], L = cu[b + 1] - s0;
-  const int p0 = blockIdx.x * 8;
-  if (p0 >= L) return;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int p = p0 + warp;
-  const bool valid = p < L;
-  const int n = p + 1;
-  const int nc = valid ? n / g.B : 0;
-  const size_t t = (size_t)s0 + p;
-
-  float* my_iq = iq_s + warp * g.Hi * kDI;
-  float* my_iw = iw_s + warp * g.Hi;
-  for (int e = lane; e < g.Hi * kDI; e += 32)
-    my_iq[e] = valid ? to_f32(iq[t * g.Hi * kDI + e]) : 0.f;
-  for (int e = lane; e < g.Hi; e += 32) my_iw[e] = valid ? iw[t * g.Hi + e] : 0.f;
-
-  uint32_t* my_keys = keys_s + warp * nc_cap;
-  const int last = min(p0 + 8, L);          // one past the CTA's last valid position
-  const int nc_cta = last / g.B;            // candidates of the CTA's last query
-  const float* pooled_b = pooled + (size_t)b * max_nblk * kDI;
-
-  for (int c0 = 0; c0 < nc_cta; c0 += kChunk) {
-    const int rows = min(kChunk, nc_cta - c0);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int q = tid / kTpq, u = tid % kTpq;
+  const int n_items = n_groups * batch;
+  for (;;) {
+    if (tid == 0) s_item = atomicAdd(sched, 1);
     __syncthreads();
-    for (int e = threadIdx.x; e < rows * kDI; e += blockDim.x) {
-      const int r = e / kDI, d = e - r * kDI;
-      kbar_s[r * kStride + d] = pooled_b[(size_t)(c0 + r) * kDI + d];
-    }
-    __syncthreads();
-    for (int r = lane; r < rows; r += 32) {
-      const int j = c0 + r;
-      if (j < nc) {
-        const float s = score_row<kDI>(kbar_s + r * kStride, my_iq, my_iw, g.Hi, g.idx_scale);
-        my_keys[j] = score_key(s);
-        if (scores) scores[t * scores_ld + j] = s;
+    const int item = s_item;
+    if (item >= n_items) break;
+    const int b = item % batch;
+    const int p0 = (n_groups - 1 - item / batch) * kQc;
+    const int s0 = cu[b], L = cu[b + 1] - s0;
+    if (p0 < L) {
+      const int nq = min(kQc, L - p0);
+      const int nc_cta = (p0 + nq) / g.B;          // candidates of the group's last query
+
+      // stage iq and iw of the group's queries (zeros past the sequence)
+      {
+        constexpr int kVec = 16 / sizeof(T);
+        const int per_q = Hi * kDI;
+        const T* src = iq + ((size_t)s0 + p0) * per_q;
+        for (int e = tid * kVec; e < kQc * per_q; e += kSelThreadsPrefill * kVec) {
+          const bool in = e < nq * per_q;
+          const uint4 v = in ? *reinterpret_cast<const uint4*>(src + e) : make_uint4(0, 0, 0, 0);
+          if constexpr (sizeof(T) == 2) {
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              iq_s[e + 2 * i] = __uint_as_float(w4[i] << 16);
+              iq_s[e + 2 * i + 1] = __uint_as_float(w4[i] & 0xffff0000u);
+            }
+          } else {
+            *reinterpret_cast<float4*>(iq_s + e) =
+                make_float4(__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z),
+                            __uint_as_float(v.w));
+          }
+        }
+        for (int e = tid; e < kQc * Hi; e += kSelThreadsPrefill)
+          iw_s[e] = e < nq * Hi ? iw[((size_t)s0 + p0) * Hi + e] : 0.f;
+      }
+
+      const int nc_q = q < nq ? (p0 + q + 1) / g.B : 0;
+      const size_t tq = (size_t)s0 + p0 + q;
+      const float* pooled_b = pooled + (size_t)b * max_nblk * kDI;
+      const float* myq = iq_s + q * Hi * kDI;
+      const float* myw = iw_s + q * Hi;
+
+      for (int c0 = 0; c0 < nc_cta; c0 += kChunk) {
+        const int rows = min(kChunk, nc_cta - c0);
+        const int nrpt = (rows + kTpq - 1) / kTpq;   // row slots in use (uniform)
+        __syncthreads();
+        {
+          constexpr int kF4 = kChunk * kDI / 4 / kSelThreadsPrefill;   // float4 per thread
+          float4 buf[kF4];
+#pragma unroll
+          for (int i = 0; i < kF4; ++i) {
+            const int e = (tid + i * kSelThreadsPrefill) * 4;
+            const int r = e / kDI;
+            buf[i] = r < rows ? *reinterpret_cast<const float4*>(
+                                    pooled_b + (size_t)(c0 + r) * kDI + (e - r * kDI))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int i = 0; i < kF4; ++i) {
+            const int e = (tid + i * kSelThreadsPrefill) * 4;
+            const int r = e / kDI;
+            *reinterpret_cast<float4*>(kb_s + r * kStride + (e - r * kDI)) = buf[i];
+          }
+        }
+        __syncthreads();
+        float s[kRpt];
+#pragma unroll
+        for (int i = 0; i < kRpt; ++i) s[i] = 0.f;
+        for (int hg = 0; hg < Hi; hg += 4) {
+          float acc[kRpt][4];
+#pragma unroll
+          for (int i = 0; i < kRpt; ++i)
+#pragma unroll
+            for (int hh = 0; hh < 4; ++hh) acc[i][hh] = 0.f;
+#pragma unroll 1
+          for (int d = 0; d < kDI; d += 4) {
+            float4 qv[4];
+#pragma unroll
+            for (int hh = 0; hh < 4; ++hh)
+              qv[hh] = hg + hh < Hi ? *reinterpret_cast<const float4*>(myq + (hg + hh) * kDI + d)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int i = 0; i < kRpt; ++i) {
+              if (i < nrpt) {
+                const float4 kv =
+                    *reinterpret_cast<const float4*>(kb_s + (u + i * kTpq) * kStride + d);
+#pragma unroll
+                for (int hh = 0; hh < 4; ++hh) {
+                  float a = acc[i][hh];
+                  a = fmaf(qv[hh].x, kv.x, a);
+                  a = fmaf(qv[hh].y, kv.y, a);
+                  a = fmaf(qv[hh].z, kv.z, a);
+                  a = fmaf(qv[hh].w, kv.w, a);
+                  acc[i][hh] = a;
+                }
+              }
+            }
+          }
+#pragma unroll
+          for (int hh = 0; hh < 4; ++hh) {
+            if (hg + hh < Hi) {
+              const float wh = myw[hg + hh];
+#pragma unroll
+              for (int i = 0; i < kRpt; ++i) s[i] = fmaf(wh, fmaxf(acc[i][hh], 0.f), s[i]);
+            }
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < kRpt; ++i) {
+          const int j = c0 + u + i * kTpq;
+          if (j < nc_q) {
+            const float sc = s[i] * g.idx_scale;
+            keys_s[q * nc_cap + j] = score_key(sc);
+            if (scores) scores[tq * scores_ld + j] = sc;
+          }
+        }
+      }
+      if (scores && q < nq)
+        for (int j = nc_q + u; j < scores_ld; j += kTpq) scores[tq * scores_ld + j] = -INFINITY;
+      __syncthreads();
+
+      int* my_pos = pos_s + warp * g.k;
+      for (int qq = warp; qq < nq; qq += kWarps) {
+        const int n = p0 + qq + 1;
+        const int nc = n / g.B;
+        const size_t t = (size_t)s0 + p0 + qq;
+        uint32_t* brow = bitmask + t * words;
+        const int m = warp_topk(keys_s + qq * nc_cap, nc, g.k, my_pos, brow, words, lane);
+        const int tail = n - nc * g.B;
+        int* srow = sel + t * (g.k + 1);
+        for (int e = lane; e < g.k + 1; e += 32) {
+          int v = -1;
+          if (e < m) v = my_pos[e];
+          else if (e == m && tail > 0) v = nc;
+          srow[e] = v;
+        }
+        if (lane == 0) {
+          nsel[t] = m + (tail > 0 ? 1 : 0);
+          if (tail > 0 && words > 0) brow[nc >> 5] |= 1u << (nc & 31);   // after the word writes
+        }
+        __syncwarp();
       }
     }
-  }
-  __syncwarp();
-  if (!valid) return;
-  if (scores)
-    for (int j = nc + lane; j < scores_ld; j += 32) scores[t * scores_ld + j] = -INFINITY;
-
-  int* my_pos = pos_s + warp * g.k;
-  const int m = warp_topk_positions(my_keys, nc, g.k, my_pos, lane);
-  const int tail = n - nc * g.B;
-  const int cnt = m + (tail > 0 ? 1 : 0);
-  int* srow = sel + t * (g.k + 1);
-  for (int e = lane; e < g.k + 1; e += 32) {
-    int v = -1;
-    if (e < m) v = my_pos[e];
-    else if (e == m && tail > 0) v = nc;
-    srow[e] = v;
-  }
-  if (lane == 0) nsel[t] = cnt;
-  if (bitmask) {
-    uint32_t* brow = bitmask + t * words;
-    for (int w = lane; w < words; w += 32) brow[w] = 0u;
-    __syncwarp();
-    for (int e = lane; e < m; e += 32) atomicOr(&brow[my_pos[e] >> 5], 1u << (my_pos[e] & 31));
-    if (lane == 0 && tail > 0) atomicOr(&brow[nc >> 5], 1u << (nc & 31));
+    __syncthreads();   // every thread has read s_item and finished with shared memory
   }
 }
 
@@ -609,37 +734,49 @@ cudaError_t launch_pool_cache(qsa_dtype dt, const void* ik_cache, const int* kv_
 }
 
 size_t select_prefill_smem(const Geom& g, int nc_cap) {
-  return sizeof(float) * ((size_t)kChunk * (g.di + 1) + 8 * g.Hi * g.di + 8 * g.Hi) +
-         sizeof(uint32_t) * 8 * (size_t)nc_cap + sizeof(int) * 8 * (size_t)g.k;
+  return sizeof(float) * ((size_t)kSelQc * g.Hi * g.di +
+                          (((size_t)kSelQc * g.Hi + 3) & ~(size_t)3) +
+                          (size_t)kChunk * (g.di + 4)) +
+         sizeof(uint32_t) * (size_t)kSelQc * nc_cap +
+         sizeof(int) * (kSelThreadsPrefill / 32) * (size_t)g.k;
 }
 
 template <typename T, int kDI>
 static cudaError_t launch_select_prefill_t(const Geom& g, const int* cu, int batch,
                                            int max_seqlen, int max_nblk, int words,
                                            const void* iq, const float* iw, const float* pooled,
-                                           int* sel, int* nsel, uint32_t* bitmask,
+                                           int* sched, int* sel, int* nsel, uint32_t* bitmask,
                                            float* scores, int scores_ld, cudaStream_t st) {
   const int nc_cap = max(1, max_seqlen / g.B);
   const size_t smem = select_prefill_smem(g, nc_cap);
   auto kern = select_prefill_kernel<T, kDI>;
   cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(kern), (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((max_seqlen + 7) / 8, batch);
-  kern<<<grid, 256, smem, st>>>(g, cu, max_nblk, words, (const T*)iq, iw, pooled, nc_cap, sel,
-                                nsel, bitmask, scores, scores_ld);
+  int per_sm = 0, sms = 0;
+  e = resident_ctas(reinterpret_cast<const void*>(kern), kSelThreadsPrefill, smem, &per_sm, &sms);
+  if (e != cudaSuccess) return e;
+  const int n_groups = (max_seqlen + kSelQc - 1) / kSelQc;
+  const long long items = (long long)n_groups * batch;
+  // fewer CTAs than items, so that the SMs that finish early take more items
+  const int ctas = std::max(1, std::min(per_sm, kSelCtasPerSm) * sms);
+  const int grid = (int)std::min<long long>(items, ctas);
+  kern<<<grid, kSelThreadsPrefill, smem, st>>>(g, cu, batch, n_groups, max_nblk,
+                                               bitmask ? words : 0, (const T*)iq, iw, pooled,
+                                               nc_cap, sched, sel, nsel, bitmask, scores,
+                                               scores_ld);
   note_launch();
   return cudaGetLastError();
 }
 
 cudaError_t launch_select_prefill(qsa_dtype dt, const Geom& g, const int* cu, int batch,
                                   int max_seqlen, int max_nblk, int words, const void* iq,
-                                  const float* iw, const float* pooled, int* sel, int* nsel,
-                                  uint32_t* bitmask, float* scores, int scores_ld,
+                                  const float* iw, const float* pooled, int* sched, int* sel,
+                                  int* nsel, uint32_t* bitmask, float* scores, int scores_ld,
                                   cudaStream_t st) {
   if (batch == 0 || max_seqlen == 0) return cudaSuccess;
 #define QSA_SEL(T, DI)                                                                      \
   return launch_select_prefill_t<T, DI>(g, cu, batch, max_seqlen, max_nblk, words, iq, iw,  \
-                                        pooled, sel, nsel, bitmask, scores, scores_ld, st)
+                                        pooled, sched, sel, nsel, bitmask, scores, scores_ld, st)
   if (dt == QSA_BF16) {
     if (g.di == 64) QSA_SEL(__nv_bfloat16, 64);
     QSA_SEL(__nv_bfloat16, 32);
