@@ -52,7 +52,7 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 domain
 // Of every 8 probability pairs, this many are exponentiated on the FMA pipe
 // (exp2_poly2) instead of MUFU, whose 16 results per clock and SM would
 // otherwise bound the softmax.
-constexpr int kPolyPairsOf8 = 2;
+constexpr int kPolyPairsOf8 = 1;
 
 constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + kTiles * kTileBytes;
@@ -337,11 +337,17 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
         tmem_ld32(tS + 64 * hf + 32, v + 32);
         tmem_wait_ld();
         if (any_vis) {
+          if (partial) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i)
+              if (i >= lim) v[i] = __float_as_uint(-INFINITY);
+          }
           float cm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-          for (int i = 0; i < 64; ++i)
-            cm[i & 3] = fmaxf(cm[i & 3], (!partial || i < lim) ? __uint_as_float(v[i]) : -INFINITY);
-          pm = lim > 0 ? fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3])) : -INFINITY;
+          for (int i = 0; i < 64; i += 2)
+            cm[(i >> 1) & 3] =
+                fmax3(cm[(i >> 1) & 3], __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
+          pm = lim > 0 ? fmax3(cm[0], cm[1], fmaxf(cm[2], cm[3])) : -INFINITY;
         }
       }
       *xslot(j & 1, hf) = pm;
