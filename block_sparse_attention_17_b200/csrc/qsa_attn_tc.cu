@@ -136,14 +136,25 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async();
+    // Q does not depend on the selections: start its load now
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+    mbar_expect_tx(q_full, kTiles * kTileBytes);
+    for (int t = 0; t < kTiles; ++t)
+      for (int dc = 0; dc < 2; ++dc)
+        tma_load_3d(smem_u32(smem + kOffQ + t * kTileBytes + dc * kChunkBytes), &tmQ, dc * 64,
+                    hk * G, s0 + q0 + t * P.Qt, q_full);
   }
-  // union of the CTA's selections (selected complete blocks + tail blocks)
-  for (int w = threadIdx.x; w < P.words; w += blockDim.x) {
-    uint32_t acc = 0;
-    for (int qi = 0; qi < nq; ++qi) acc |= P.bitmask[(size_t)(s0 + q0 + qi) * P.words + w];
-    ubits[w] = acc;
-  }
+  // union of the CTA's selections (selected complete blocks + tail blocks):
+  // one selection word per thread, OR-ed into shared memory
+  for (int w = threadIdx.x; w < P.words; w += blockDim.x) ubits[w] = 0u;
   if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+  __syncthreads();
+  for (int e = threadIdx.x; e < nq * P.words; e += blockDim.x) {
+    const uint32_t bits = P.bitmask[(size_t)(s0 + q0) * P.words + e];
+    if (bits) atomicOr(&ubits[e % P.words], bits);
+  }
   __syncthreads();
   if (warp == 0) {   // ascending list of the union's blocks
     int base = 0;
@@ -180,15 +191,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0 && n_iter > 0) {
-      prefetch_tmap(&tmQ);
-      prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
-      mbar_expect_tx(q_full, kTiles * kTileBytes);
-      for (int t = 0; t < kTiles; ++t)
-        for (int dc = 0; dc < 2; ++dc)
-          tma_load_3d(sQ + t * kTileBytes + dc * kChunkBytes, &tmQ, dc * 64, hk * G,
-                      s0 + q0 + t * P.Qt, q_full);
+    if (lane == 0) {
       auto issue = [&](const CUtensorMap* tm, uint32_t dst, uint64_t* full, int j) {
         mbar_expect_tx(full, kTileBytes);
 #pragma unroll
@@ -214,7 +217,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
         return true;
       };
       int nk = 0, nv = 0;   // loads issued
-      if (issue_k(0)) {
+      if (n_iter > 0 && issue_k(0)) {
         nk = 1;
         for (int it = 0; it < n_iter; ++it) {
           if (it + 1 < n_iter) {
@@ -296,6 +299,9 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
     const size_t tok = static_cast<size_t>(s0) + pos;
     const int h = hk * G + gg;
     const uint32_t* mrow = P.bitmask + (valid ? tok : 0) * P.words;
+    // the epilogue's gate row: fetch it into L2 now
+    if (valid && t < nt && !g.gate_headwise)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(P.gate + (tok * g.Hq + h) * kHeadDim + 64 * hf));
     const uint32_t tS = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + t * 128;
     const uint32_t tO = tS + 256;
     float* xch = reinterpret_cast<float*>(smem + kOffXch);

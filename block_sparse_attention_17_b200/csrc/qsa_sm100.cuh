@@ -252,7 +252,7 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   x.y = fmaxf(x.y, -126.0f);
   const float2 t = fadd2(x, magic);
   const float2 j = fadd2(t, make_float2(-12582912.0f, -12582912.0f));
-  const float2 f = fadd2(x, make_float2(-j.x, -j.y));
+  const float2 f = ffma2(j, make_float2(-1.0f, -1.0f), x);   // x - j, exactly
   float2 p = ffma2(make_float2(0.055177733302116394f, 0.055177733302116394f), f,
                    make_float2(0.24262635409832f, 0.24262635409832f));
   p = ffma2(p, f, make_float2(0.6932612061500549f, 0.6932612061500549f));
