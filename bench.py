@@ -295,12 +295,11 @@ def run_ours(args, w, rank, world, dist):
         flush.zero_()
         step()
     torch.cuda.synchronize()
-    lib.qsa_set_stage_events(arr_t, 3)
 
-    def timed(run_once):
+    def timed(run_once, stages):
         """Time K steps, each bracketed by CUDA events on the launching stream,
-        with the L2 flush outside the events; returns per-step ms and the
-        attention-stage ms read from the library's stage events."""
+        with the L2 flush outside the events; returns per-step ms and, with
+        stages, the attention-stage ms read from the library's stage events."""
         starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
         ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
         attn = []
@@ -310,11 +309,14 @@ def run_ours(args, w, rank, world, dist):
             run_once()
             ends[i].record(stream)
             torch.cuda.synchronize()       # read this step's stage events before reuse
-            attn.append(ev_stage[1].elapsed_time(ev_stage[2]))
+            if stages:
+                attn.append(ev_stage[1].elapsed_time(ev_stage[2]))
         return [starts[i].elapsed_time(ends[i]) for i in range(args.steps)], attn
 
     # one step captured as a CUDA graph (the library makes no host sync, reads
-    # no device memory on the host and allocates nothing, so it captures whole)
+    # no device memory on the host and allocates nothing, so it captures whole);
+    # captured without stage events, so the kernels chain by programmatic
+    # dependent launch as in a user's graph
     graph = None
     if not args.eager:
         side = torch.cuda.Stream()
@@ -342,15 +344,17 @@ def run_ours(args, w, rank, world, dist):
     clocks.start()
     n0 = lib.qsa_kernel_launch_count()
     torch.cuda.synchronize()
-    eager_ms, eager_attn = timed(step)
+    # eager steps with stage events: the attention kernel's own duration
+    lib.qsa_set_stage_events(arr_t, 3)
+    eager_ms, stage_attn = timed(step, True)
+    lib.qsa_set_stage_events(None, 0)
     launches = lib.qsa_kernel_launch_count() - n0
     if graph is not None:
-        step_ms, stage_attn = timed(graph.replay)
+        step_ms, _ = timed(graph.replay, False)
     else:
-        step_ms, stage_attn = eager_ms, eager_attn
+        step_ms = eager_ms
     torch.cuda.synchronize()
     clk = clocks.stop()
-    lib.qsa_set_stage_events(None, 0)
     total_ms = float(sum(step_ms))
     job_units, total_ms = reduce_over_ranks(dist, units, total_ms, dev)
     if dist is not None:

@@ -150,6 +150,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
   // one selection word per thread, OR-ed into shared memory
   for (int w = threadIdx.x; w < P.words; w += blockDim.x) ubits[w] = 0u;
   if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+  grid_dependency_wait();   // the selection bitmaps come from the selection kernel
   __syncthreads();
   for (int e = threadIdx.x; e < nq * P.words; e += blockDim.x) {
     const uint32_t bits = P.bitmask[(size_t)(s0 + q0) * P.words + e];
@@ -544,17 +545,12 @@ cudaError_t launch_attn_prefill_tc(const Geom& g, const int* cu, int batch, int 
   p.err = err;
   dim3 grid(p.n_ctas, batch, g.Hkv);
   cudaError_t e;
-  if (g.B == 64) {
-    e = set_max_dynamic_smem(reinterpret_cast<const void*>(attn_prefill_tc_kernel<64>), kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attn_prefill_tc_kernel<64><<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, p);
-  } else {
-    e = set_max_dynamic_smem(reinterpret_cast<const void*>(attn_prefill_tc_kernel<128>), kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attn_prefill_tc_kernel<128><<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, p);
-  }
+  auto kern = g.B == 64 ? attn_prefill_tc_kernel<64> : attn_prefill_tc_kernel<128>;
+  e = set_max_dynamic_smem(reinterpret_cast<const void*>(kern), kSmemBytes);
+  if (e != cudaSuccess) return e;
+  e = launch_dependent(kern, grid, dim3(kThreads), kSmemBytes, st, mq, mk, mv, p);
   note_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace qsa

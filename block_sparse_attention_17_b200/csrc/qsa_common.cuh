@@ -57,6 +57,17 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// Programmatic dependent launch: a kernel launched with launch_dependent()
+// may start while the kernel before it on the stream still runs; it calls
+// grid_dependency_wait() before reading anything that kernel wrote. A kernel
+// calls grid_dependents_launch() once the next kernel may start.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // 1 / (1 + e^-x) with the fast exponential and division (a few ulp; 0 for
 // very negative x).
 __device__ __forceinline__ float sigmoidf_(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }

@@ -141,14 +141,16 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
     fence_barrier_init();
     fence_proxy_async();
   }
+  grid_dependency_wait();   // the selections come from the selection kernel
   __syncthreads();
   {
     const int kp1 = g.k + 1;
+    const int nblk = P.cap / g.B;
     for (int e = threadIdx.x; e < n_q * kp1; e += blockDim.x) {
       const int i = e / kp1, j = e - i * kp1;
       if (j < P.nsel[(size_t)b * n_q + i]) {
         const int blk = P.sel[((size_t)b * n_q + i) * kp1 + j];
-        atomicOr(&qbits[i * words + (blk >> 5)], 1u << (blk & 31));
+        if (blk >= 0 && blk < nblk) atomicOr(&qbits[i * words + (blk >> 5)], 1u << (blk & 31));
       }
     }
   }
@@ -587,9 +589,10 @@ cudaError_t launch_attn_decode_mma(const Geom& g, int batch, int n_q, int cap, i
   const int smem = kOffBits + 4 * n_q * words + 1024;
   cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(attn_decode_mma_kernel), smem);
   if (e != cudaSuccess) return e;
-  attn_decode_mma_kernel<<<dim3(nsplit, batch, g.Hkv), kThreads, smem, st>>>(mk, mv, p);
+  e = launch_dependent(attn_decode_mma_kernel, dim3(nsplit, batch, g.Hkv), dim3(kThreads), smem, st,
+                       mk, mv, p);
   note_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace qsa

@@ -1,6 +1,8 @@
 // Internal launcher declarations shared by the kernel files and the C ABI.
 #pragma once
 
+#include <utility>
+
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -20,6 +22,25 @@ cudaError_t set_max_dynamic_smem(const void* func, int bytes);
 // CTAs of `func` (threads, dynamic shared memory) resident per SM, and the
 // SM count of the current device (cached per function, device and shape).
 cudaError_t resident_ctas(const void* func, int threads, size_t smem, int* per_sm, int* sms);
+
+// Launches `kernel` on `st` with programmatic stream serialization: it may
+// start before the previous kernel on the stream finishes, and must call
+// grid_dependency_wait() before reading that kernel's outputs.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Sets the message qsa_last_error() returns on this host thread.
 void set_last_error(const char* msg);

@@ -72,6 +72,7 @@ template <typename T>
 __global__ void __launch_bounds__(kPoolThreads)
 pool_prefill_kernel(const T* __restrict__ ik, const int* __restrict__ cu, int B, int di,
                     float* __restrict__ pooled, int max_nblk) {
+  grid_dependents_launch();   // the selection kernel may start its prologue
   const int b = blockIdx.y, j = blockIdx.x;
   const int s0 = cu[b], L = cu[b + 1] - s0;
   if (j >= L / B) return;
@@ -273,6 +274,7 @@ select_prefill_kernel(Geom g, const int* __restrict__ cu, int batch, int n_group
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int q = tid / kTpq, u = tid % kTpq;
   const int n_items = n_groups * batch;
+  grid_dependents_launch();   // the attention kernel may start its prologue
   for (;;) {
     if (tid == 0) s_item = atomicAdd(sched, 1);
     __syncthreads();
@@ -310,6 +312,7 @@ select_prefill_kernel(Geom g, const int* __restrict__ cu, int batch, int n_group
           iw_s[e] = e < nq * Hi ? iw[((size_t)s0 + p0) * Hi + e] : 0.f;
       }
 
+      grid_dependency_wait();   // pooled rows come from the pooling kernel
       const int nc_q = q < nq ? (p0 + q + 1) / g.B : 0;
       const size_t tq = (size_t)s0 + p0 + q;
       const float* pooled_b = pooled + (size_t)b * max_nblk * kDI;
@@ -548,6 +551,7 @@ decode_select_kernel(Geom g, int n_q, int cap, const int* __restrict__ kv_len,
                      float* __restrict__ scores_out, uint32_t* __restrict__ keys_ws,
                      int* __restrict__ counter, int* __restrict__ sel, int* __restrict__ nsel,
                      int* dev_err) {
+  grid_dependents_launch();   // the attention kernel may start its prologue
   extern __shared__ __align__(16) float smem[];
   constexpr int kStride = kDI + 1;
   const int k = g.k;
@@ -760,12 +764,11 @@ static cudaError_t launch_select_prefill_t(const Geom& g, const int* cu, int bat
   // fewer CTAs than items, so that the SMs that finish early take more items
   const int ctas = std::max(1, std::min(per_sm, kSelCtasPerSm) * sms);
   const int grid = (int)std::min<long long>(items, ctas);
-  kern<<<grid, kSelThreadsPrefill, smem, st>>>(g, cu, batch, n_groups, max_nblk,
-                                               bitmask ? words : 0, (const T*)iq, iw, pooled,
-                                               nc_cap, sched, sel, nsel, bitmask, scores,
-                                               scores_ld);
+  e = launch_dependent(kern, dim3(grid), dim3(kSelThreadsPrefill), smem, st, g, cu, batch,
+                       n_groups, max_nblk, bitmask ? words : 0, (const T*)iq, iw, pooled, nc_cap,
+                       sched, sel, nsel, bitmask, scores, scores_ld);
   note_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_select_prefill(qsa_dtype dt, const Geom& g, const int* cu, int batch,
