@@ -141,6 +141,24 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
     fence_barrier_init();
     fence_proxy_async();
   }
+  // Q rows r = i * G + gi (query i, head hk * G + gi), zero beyond R: Q is an
+  // input, so it is loaded before waiting for the selection kernel
+  for (int e = threadIdx.x; e < 16 * (kD / 8); e += blockDim.x) {
+    const int r = e / (kD / 8), c8 = e % (kD / 8);
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (r < R) {
+      const int i = r / G, gi = r % G;
+      v = *reinterpret_cast<const uint4*>(
+          P.q + (((size_t)b * n_q + i) * g.Hq + hk * G + gi) * kD + c8 * 8);
+    }
+    *reinterpret_cast<uint4*>(smem + kOffQ + r * kQStride + c8 * 16) = v;
+  }
+  // the merging CTA's gate rows: fetch them into L2 now
+  if (split == 0 && !g.gate_headwise && threadIdx.x < R * (kD * 2 / 128)) {
+    const int r = threadIdx.x / (kD * 2 / 128), part = threadIdx.x % (kD * 2 / 128);
+    const size_t orow = ((size_t)b * n_q + r / G) * g.Hq + hk * G + r % G;
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(P.gate + orow * kD + part * 64));
+  }
   grid_dependency_wait();   // the selections come from the selection kernel
   __syncthreads();
   {
@@ -185,17 +203,6 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
       base += __shfl_sync(kFull, incl, 31);
     }
     if (lane == 0) *n_chunks_s = base * cpb;
-  }
-  // Q rows r = i * G + gi (query i, head hk * G + gi), zero beyond R
-  for (int e = threadIdx.x; e < 16 * (kD / 8); e += blockDim.x) {
-    const int r = e / (kD / 8), c8 = e % (kD / 8);
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (r < R) {
-      const int i = r / G, gi = r % G;
-      v = *reinterpret_cast<const uint4*>(
-          P.q + (((size_t)b * n_q + i) * g.Hq + hk * G + gi) * kD + c8 * 8);
-    }
-    *reinterpret_cast<uint4*>(smem + kOffQ + r * kQStride + c8 * 16) = v;
   }
   __syncthreads();
   const int n_chunks = *n_chunks_s;

@@ -426,78 +426,96 @@ select_prefill_kernel(Geom g, const int* __restrict__ cu, int batch, int n_group
 
 // ------------------------------------------------------- CTA top-k
 // The k largest of keys[0..n) (shared memory) where a lower position wins a
-// tie, chosen by a whole CTA of 256 threads with few dependent steps: four
-// 8-bit radix passes find the k-th largest key tau (a shared histogram per
-// pass, lanes with equal digits adding once), then each thread counts the
-// keys > tau and == tau in its contiguous run of positions, one block scan
-// turns the counts into output offsets, and the chosen positions are written
-// in ascending order. Returns min(k, n).
+// tie, chosen by a whole CTA of 256 threads. The threshold tau comes from an
+// MSB-first bit search that keeps count(keys >= tau) >= k: it starts below
+// the bits all keys share (those of the CTA's max and min key agree above
+// their highest differing bit), counts with one block reduction per bit, and
+// stops as soon as a candidate has exactly k keys at or above it (else it
+// ends on the k-th largest key). Then each thread counts the keys > tau and
+// == tau in its contiguous run of positions, one block scan turns the counts
+// into output offsets, and the chosen positions are written in ascending
+// order, ties at tau lowest position first. Returns min(k, n).
 constexpr int kTopkThreads = 256;
 
-__device__ int cta_topk_radix(const uint32_t* keys, int n, int k, int* out) {
-  __shared__ int hist[256];
-  __shared__ int scan_s[2][kTopkThreads / 32];
-  __shared__ uint32_t s_prefix, s_mask;
-  __shared__ int s_need;
+__device__ int cta_topk_bits(const uint32_t* keys, int n, int k, int* out) {
+  constexpr int kW = kTopkThreads / 32;
+  constexpr int kR = 8;                         // keys per thread kept in registers
+  __shared__ uint32_t red_u[2][kW];
+  __shared__ int red_c[2][kW];
+  __shared__ int red_g[kW];
+  __shared__ int scan_s[2][kW];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (n <= k) {
     for (int j = tid; j < n; j += kTopkThreads) out[j] = j;
     __syncthreads();
     return n;
   }
-  if (tid == 0) { s_prefix = 0u; s_mask = 0u; s_need = k; }
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    hist[tid] = 0;
-    __syncthreads();
-    const uint32_t prefix = s_prefix, mask = s_mask;
-    for (int base = 0; base < n; base += kTopkThreads) {
-      const int j = base + tid;
-      const uint32_t key = j < n ? keys[j] : 0u;
-      const bool live = j < n && (key & mask) == prefix;
-      const uint32_t digit = live ? (key >> shift) & 255u : 256u;
-      const unsigned same = __match_any_sync(kFull, digit);
-      if (live && (__ffs(same) - 1) == lane) atomicAdd(&hist[digit], __popc(same));
-    }
-    __syncthreads();
-    if (warp == 0) {
-      // lane l owns digits 255 - 8l down to 248 - 8l
-      int cnt[8], local = 0;
+  const bool in_regs = n <= kR * kTopkThreads;
+  uint32_t kr[kR];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        cnt[e] = hist[255 - 8 * lane - e];
-        local += cnt[e];
-      }
-      int incl = local;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(kFull, incl, o);
-        if (lane >= o) incl += v;
-      }
-      const int need = s_need;
-      const int before = incl - local;
-      if (before < need && incl >= need) {
-        int run = before;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          if (run + cnt[e] >= need) {
-            s_prefix = prefix | ((uint32_t)(255 - 8 * lane - e) << shift);
-            s_mask = mask | (255u << shift);
-            s_need = need - run;
-            break;
-          }
-          run += cnt[e];
-        }
-      }
-    }
-    __syncthreads();
+  for (int u = 0; u < kR; ++u) {
+    const int j = tid + u * kTopkThreads;
+    kr[u] = (in_regs && j < n) ? keys[j] : 0u;
   }
-  const uint32_t tau = s_prefix;
-  const int need = s_need;   // keys equal to tau to take, lowest positions first
-  // each thread owns the contiguous run [lo, hi)
+  uint32_t hi = 0u, lo = 0xffffffffu;
+  if (in_regs) {
+#pragma unroll
+    for (int u = 0; u < kR; ++u)
+      if (tid + u * kTopkThreads < n) { hi = max(hi, kr[u]); lo = min(lo, kr[u]); }
+  } else {
+    for (int j = tid; j < n; j += kTopkThreads) { hi = max(hi, keys[j]); lo = min(lo, keys[j]); }
+  }
+  hi = __reduce_max_sync(kFull, hi);
+  lo = __reduce_min_sync(kFull, lo);
+  if (lane == 0) { red_u[0][warp] = hi; red_u[1][warp] = lo; }
+  __syncthreads();
+#pragma unroll
+  for (int w = 0; w < kW; ++w) { hi = max(hi, red_u[0][w]); lo = min(lo, red_u[1][w]); }
+  uint32_t tau = hi;
+  if (hi != lo) {
+    const int top = 31 - __clz(hi ^ lo);                  // highest differing bit
+    tau = top == 31 ? 0u : (hi & ~((2u << top) - 1u));
+    int slot = 0;
+    for (int bit = top; bit >= 0; --bit) {
+      const uint32_t cand = tau | (1u << bit);
+      int c = 0;
+      if (in_regs) {
+#pragma unroll
+        for (int u = 0; u < kR; ++u) c += (tid + u * kTopkThreads < n && kr[u] >= cand) ? 1 : 0;
+      } else {
+        for (int j = tid; j < n; j += kTopkThreads) c += keys[j] >= cand ? 1 : 0;
+      }
+      c = __reduce_add_sync(kFull, c);
+      if (lane == 0) red_c[slot][warp] = c;
+      __syncthreads();
+      int tot = 0;
+#pragma unroll
+      for (int w = 0; w < kW; ++w) tot += red_c[slot][w];
+      slot ^= 1;                                           // the next step writes the other slot
+      if (tot >= k) tau = cand;
+      if (tot == k) break;                                 // uniform: every thread read tot
+    }
+  }
+  // keys > tau are all taken; of the keys == tau, the first `need` positions
+  int gt = 0;
+  if (in_regs) {
+#pragma unroll
+    for (int u = 0; u < kR; ++u) gt += (tid + u * kTopkThreads < n && kr[u] > tau) ? 1 : 0;
+  } else {
+    for (int j = tid; j < n; j += kTopkThreads) gt += keys[j] > tau ? 1 : 0;
+  }
+  gt = __reduce_add_sync(kFull, gt);
+  if (lane == 0) red_g[warp] = gt;
+  __syncthreads();
+  int n_gt_all = 0;
+#pragma unroll
+  for (int w = 0; w < kW; ++w) n_gt_all += red_g[w];
+  const int need = k - n_gt_all;   // keys equal to tau to take, lowest positions first
+  // each thread owns the contiguous run [r_lo, r_hi)
   const int per = (n + kTopkThreads - 1) / kTopkThreads;
-  const int lo = min(n, tid * per), hi = min(n, lo + per);
+  const int r_lo = min(n, tid * per), r_hi = min(n, r_lo + per);
   int n_gt = 0, n_eq = 0;
-  for (int j = lo; j < hi; ++j) {
+  for (int j = r_lo; j < r_hi; ++j) {
     const uint32_t key = keys[j];
     n_gt += key > tau;
     n_eq += key == tau;
@@ -516,7 +534,7 @@ __device__ int cta_topk_radix(const uint32_t* keys, int n, int k, int* out) {
   // ties before this run that are taken, plus greater keys before this run
   int o_idx = gt_before + min(eq_before, need);
   int t_rank = eq_before;
-  for (int j = lo; j < hi; ++j) {
+  for (int j = r_lo; j < r_hi; ++j) {
     const uint32_t key = keys[j];
     if (key > tau) {
       out[o_idx++] = j;
@@ -539,7 +557,7 @@ __device__ int cta_topk_radix(const uint32_t* keys, int n, int k, int* out) {
 //     the score keys,
 //  3. the last CTA of the sequence to finish (an atomic counter that the
 //     caller zeroes before the launch) selects each query's top-k from all
-//     of them (cta_topk_radix), then appends the tail block.
+//     of them (cta_topk_bits), then appends the tail block.
 constexpr int kSelThreads = 256;
 constexpr int kPart = 64;                 // candidate blocks per CTA
 
@@ -684,7 +702,7 @@ decode_select_kernel(Geom g, int n_q, int cap, const int* __restrict__ kv_len,
       }
     }
     __syncthreads();
-    const int m = cta_topk_radix(keys_s, nc_i, k, pos_s);
+    const int m = cta_topk_bits(keys_s, nc_i, k, pos_s);
     const int tail = n - nc_i * g.B;
     int* srow = sel + ((size_t)b * n_q + i) * kp1;
     for (int e = threadIdx.x; e < kp1; e += blockDim.x) {
