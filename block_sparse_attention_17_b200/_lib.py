@@ -26,7 +26,7 @@ EXPORTED = [
     "qsa_set_stage_events",
     "qsa_prefill_workspace_size", "qsa_prefill", "qsa_select",
     "qsa_decode_workspace_size", "qsa_decode", "qsa_select_decode",
-    "qsa_pool_build", "qsa_decode_noalloc",
+    "qsa_pool_build", "qsa_decode_noalloc", "qsa_decode_paged", "qsa_pool_build_paged",
 ]
 
 
@@ -75,6 +75,11 @@ def _declare(lib):
         "qsa_select_decode": (I, [CFG, I, I, I, P, P, P, P, P, P, P, P, P, P, SZ, P]),
         "qsa_pool_build": (I, [CFG, I, I, P, P, P, P, P]),
         "qsa_decode_noalloc": (I, [CFG, I, I, I] + [P] * 15),
+        # cfg, batch, n_q, max_blocks, block_table, num_pages, kv_len, q, k, v, iq, ik, iw,
+        # gate, pooled, out, lse, sel, nsel, dev_err, ws, ws_bytes, stream (15 pointers)
+        "qsa_decode_paged": (I, [CFG, I, I, I, P, I] + [P] * 15 + [SZ, P]),
+        # cfg, batch, max_blocks, block_table, num_pages, kv_len, ik, pooled, dev_err, stream
+        "qsa_pool_build_paged": (I, [CFG, I, I, P, I, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

@@ -294,3 +294,65 @@ def pool_build(cfg: QSAConfig, ik_cache, kv_len, pooled_cache=None, *, dev_err=N
                                    _ptr(pooled_cache), _ptr(dev_err), _stream(stream))
     _lib.check(st, "qsa_pool_build")
     return pooled_cache
+
+
+def decode_paged(cfg: QSAConfig, q, k_pages, v_pages, iq, ik_pages, iw, gate, pooled_cache,
+                 kv_len, block_table, *, out=None, lse=None, sel=None, nsel=None, dev_err=None,
+                 workspace=None, want_lse=False, want_sel=False, stream=None) -> dict:
+    """One QSA decode step over a paged cache (qsa_decode_paged): page p holds
+    B rows, k_pages/v_pages [num_pages, B, Hkv, D], ik_pages [num_pages, B, di];
+    block_table [batch, max_blocks] int32 maps a sequence's block to its page."""
+    dt = cfg.dtype
+    batch, n_q = q.shape[0], q.shape[1]
+    num_pages, B = k_pages.shape[0], cfg.block_size
+    max_blocks = block_table.shape[1]
+    _need(q, "q", dt, (batch, n_q, cfg.num_q_heads, cfg.head_dim))
+    _need(k_pages, "k_pages", dt, (num_pages, B, cfg.num_kv_heads, cfg.head_dim))
+    _need(v_pages, "v_pages", dt, (num_pages, B, cfg.num_kv_heads, cfg.head_dim))
+    _need(iq, "iq", dt, (batch, n_q, cfg.idx_heads, cfg.idx_dim))
+    _need(ik_pages, "ik_pages", dt, (num_pages, B, cfg.idx_dim))
+    _need(iw, "iw", torch.float32, (batch, n_q, cfg.idx_heads))
+    gshape = ((batch, n_q, cfg.num_q_heads) if cfg.gate_headwise
+              else (batch, n_q, cfg.num_q_heads, cfg.head_dim))
+    _need(gate, "gate", dt, gshape)
+    _need(pooled_cache, "pooled_cache", torch.float32, (batch, max_blocks, cfg.idx_dim))
+    _need(kv_len, "kv_len", torch.int32, (batch,))
+    _need(block_table, "block_table", torch.int32, (batch, max_blocks))
+    dev = q.device
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(batch, n_q, cfg.num_q_heads, dtype=torch.float32, device=dev)
+    if sel is None and want_sel:
+        sel = torch.empty(batch, n_q, cfg.topk + 1, dtype=torch.int32, device=dev)
+    if nsel is None and want_sel:
+        nsel = torch.empty(batch, n_q, dtype=torch.int32, device=dev)
+    ws = _workspace(decode_workspace_size(cfg, batch, n_q, max_blocks * B), dev, workspace)
+    c = cfg.c()
+    st = _lib.lib().qsa_decode_paged(ctypes.byref(c), batch, n_q, max_blocks, _ptr(block_table),
+                                     num_pages, _ptr(kv_len), _ptr(q), _ptr(k_pages),
+                                     _ptr(v_pages), _ptr(iq), _ptr(ik_pages), _ptr(iw),
+                                     _ptr(gate), _ptr(pooled_cache), _ptr(out), _ptr(lse),
+                                     _ptr(sel), _ptr(nsel), _ptr(dev_err), _ptr(ws), ws.numel(),
+                                     _stream(stream))
+    _lib.check(st, "qsa_decode_paged")
+    return {"out": out, "lse": lse, "sel": sel, "nsel": nsel}
+
+
+def pool_build_paged(cfg: QSAConfig, ik_pages, kv_len, block_table, pooled_cache=None, *,
+                     dev_err=None, stream=None):
+    """qsa_pool_build over a paged indexer-key cache (qsa_pool_build_paged)."""
+    num_pages = ik_pages.shape[0]
+    batch, max_blocks = block_table.shape
+    _need(ik_pages, "ik_pages", cfg.dtype, (num_pages, cfg.block_size, cfg.idx_dim))
+    _need(kv_len, "kv_len", torch.int32, (batch,))
+    _need(block_table, "block_table", torch.int32, (batch, max_blocks))
+    if pooled_cache is None:
+        pooled_cache = torch.zeros(batch, max_blocks, cfg.idx_dim, dtype=torch.float32,
+                                   device=ik_pages.device)
+    c = cfg.c()
+    st = _lib.lib().qsa_pool_build_paged(ctypes.byref(c), batch, max_blocks, _ptr(block_table),
+                                         num_pages, _ptr(kv_len), _ptr(ik_pages),
+                                         _ptr(pooled_cache), _ptr(dev_err), _stream(stream))
+    _lib.check(st, "qsa_pool_build_paged")
+    return pooled_cache

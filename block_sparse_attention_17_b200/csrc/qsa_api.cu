@@ -398,21 +398,22 @@ static qsa_status decode_select_common(const qsa_config* cfg, const Geom& g, int
                                        const void* ik_cache, const float* iw,
                                        float* pooled_cache, const DecodeWs& w, int32_t* sel,
                                        int32_t* nsel, float* scores, int32_t* dev_err,
-                                       cudaStream_t st) {
+                                       cudaStream_t st, Pages pg = Pages()) {
   QSA_CUDA(cudaMemsetAsync(w.counters, 0, sizeof(int) * (size_t)batch * (1 + g.Hkv), st),
            "clear counters");
   QSA_CUDA(launch_decode_select(cfg->dtype, g, batch, n_q, cap, kv_len, iq, ik_cache, iw,
-                                pooled_cache, scores, w.keys, w.counters, sel, nsel, dev_err, st),
+                                pooled_cache, scores, w.keys, w.counters, sel, nsel, dev_err, st,
+                                pg),
            "decode select");
   return QSA_OK;
 }
 
-qsa_status qsa_decode(const qsa_config* cfg, int batch, int n_q, int cap, const int32_t* kv_len,
+static qsa_status decode_impl(const qsa_config* cfg, int batch, int n_q, int cap, const int32_t* kv_len,
                       const void* q, const void* k_cache, const void* v_cache, const void* iq,
                       const void* ik_cache, const float* iw, const void* gate,
                       float* pooled_cache, void* out, float* lse, int32_t* sel, int32_t* nsel,
-                      int32_t* dev_err, void* workspace, size_t workspace_bytes, void* stream) {
-  g_err[0] = 0;
+                      int32_t* dev_err, void* workspace, size_t workspace_bytes, void* stream,
+                      Pages pg) {
   qsa_status s = check_decode_dims(cfg, batch, n_q, cap);
   if (s != QSA_OK) return s;
   if (batch == 0) return QSA_OK;
@@ -433,13 +434,14 @@ qsa_status qsa_decode(const qsa_config* cfg, int batch, int n_q, int cap, const 
   int* nsel_p = nsel ? nsel : w.nsel;
   stage_mark(0, st);
   s = decode_select_common(cfg, g, batch, n_q, cap, kv_len, iq, ik_cache, iw, pooled_cache, w,
-                           sel_p, nsel_p, nullptr, dev_err, st);
+                           sel_p, nsel_p, nullptr, dev_err, st, pg);
   if (s != QSA_OK) return s;
   stage_mark(1, st);
   if (decode_uses_mma(cfg, g, n_q)) {
     QSA_CUDA(launch_attn_decode_mma(g, batch, n_q, cap, w.nsplit, w.per_split, kv_len, q,
                                     k_cache, v_cache, gate, sel_p, nsel_p, w.part_ml, w.part_o,
-                                    w.counters + batch, out, lse, dev_err ? dev_err : w.err, st),
+                                    w.counters + batch, out, lse, dev_err ? dev_err : w.err, st,
+                                    pg),
              "decode attention");
   } else {
     QSA_CUDA(launch_attn_decode_simt(cfg->dtype, g, batch, n_q, cap, w.nsplit, w.per_split,
@@ -449,6 +451,47 @@ qsa_status qsa_decode(const qsa_config* cfg, int batch, int n_q, int cap, const 
   }
   stage_mark(2, st);
   return QSA_OK;
+}
+
+qsa_status qsa_decode(const qsa_config* cfg, int batch, int n_q, int cap, const int32_t* kv_len,
+                      const void* q, const void* k_cache, const void* v_cache, const void* iq,
+                      const void* ik_cache, const float* iw, const void* gate,
+                      float* pooled_cache, void* out, float* lse, int32_t* sel, int32_t* nsel,
+                      int32_t* dev_err, void* workspace, size_t workspace_bytes, void* stream) {
+  g_err[0] = 0;
+  return decode_impl(cfg, batch, n_q, cap, kv_len, q, k_cache, v_cache, iq, ik_cache, iw, gate,
+                     pooled_cache, out, lse, sel, nsel, dev_err, workspace, workspace_bytes,
+                     stream, Pages());
+}
+
+static qsa_status check_pages(const qsa_config* cfg, int max_blocks, const int32_t* block_table,
+                              int num_pages) {
+  if (max_blocks <= 0 || num_pages <= 0)
+    return fail(QSA_ERR_INVALID_ARG, "max_blocks and num_pages must be > 0");
+  if ((long long)max_blocks * cfg->block_size > INT32_MAX ||
+      (long long)num_pages * cfg->block_size > INT32_MAX)
+    return fail(QSA_ERR_UNSUPPORTED, "more than 2^31 cache rows");
+  QSA_REQUIRE(block_table, "block_table");
+  return QSA_OK;
+}
+
+qsa_status qsa_decode_paged(const qsa_config* cfg, int batch, int n_q, int max_blocks,
+                            const int32_t* block_table, int num_pages, const int32_t* kv_len,
+                            const void* q, const void* k_pages, const void* v_pages,
+                            const void* iq, const void* ik_pages, const float* iw,
+                            const void* gate, float* pooled_cache, void* out, float* lse,
+                            int32_t* sel, int32_t* nsel, int32_t* dev_err, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  g_err[0] = 0;
+  qsa_status s = check_cfg(cfg);
+  if (s != QSA_OK) return s;
+  if ((s = check_pages(cfg, max_blocks, block_table, num_pages)) != QSA_OK) return s;
+  const Geom g = make_geom(cfg);
+  if (!decode_uses_mma(cfg, g, n_q))
+    return fail(QSA_ERR_UNSUPPORTED, "paged decode needs bf16 and n_q * group size <= 16");
+  return decode_impl(cfg, batch, n_q, max_blocks * cfg->block_size, kv_len, q, k_pages, v_pages,
+                     iq, ik_pages, iw, gate, pooled_cache, out, lse, sel, nsel, dev_err,
+                     workspace, workspace_bytes, stream, Pages{block_table, num_pages});
 }
 
 qsa_status qsa_select_decode(const qsa_config* cfg, int batch, int n_q, int cap,
@@ -486,6 +529,27 @@ qsa_status qsa_pool_build(const qsa_config* cfg, int batch, int cap, const int32
   QSA_REQUIRE(pooled_cache, "pooled_cache");
   QSA_CUDA(launch_pool_cache(cfg->dtype, ik_cache, kv_len, batch, cap, 0, 0, cfg->block_size,
                              cfg->idx_dim, pooled_cache, dev_err, (cudaStream_t)stream),
+           "pool build");
+  return QSA_OK;
+}
+
+qsa_status qsa_pool_build_paged(const qsa_config* cfg, int batch, int max_blocks,
+                                const int32_t* block_table, int num_pages,
+                                const int32_t* kv_len, const void* ik_pages,
+                                float* pooled_cache, int32_t* dev_err, void* stream) {
+  g_err[0] = 0;
+  qsa_status s = check_cfg(cfg);
+  if (s != QSA_OK) return s;
+  if ((s = check_pages(cfg, max_blocks, block_table, num_pages)) != QSA_OK) return s;
+  const int cap = max_blocks * cfg->block_size;
+  if ((s = check_decode_dims(cfg, batch, 1, cap)) != QSA_OK) return s;
+  if (batch == 0) return QSA_OK;
+  QSA_REQUIRE(kv_len, "kv_len");
+  QSA_REQUIRE(ik_pages, "ik_pages");
+  QSA_REQUIRE(pooled_cache, "pooled_cache");
+  QSA_CUDA(launch_pool_cache(cfg->dtype, ik_pages, kv_len, batch, cap, 0, 0, cfg->block_size,
+                             cfg->idx_dim, pooled_cache, dev_err, (cudaStream_t)stream,
+                             Pages{block_table, num_pages}),
            "pool build");
   return QSA_OK;
 }

@@ -60,6 +60,7 @@ struct DecParams {
   __nv_bfloat16* out;
   float* lse;
   int* err;
+  const int* table;                  // paged caches: [batch, cap / B] page ids, else null
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
@@ -221,8 +222,12 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
         const int s = c % kStages;
         if (c >= kStages && !mbar_wait(&empty[s], ((c / kStages) - 1) & 1, abort_flag)) break;
         const int uc = c0 + c;
-        const int key0 = u_blk[uc / cpb] * g.B + (uc % cpb) * kChunk;
-        const int rowk = (int)(krow_base + key0);
+        const int blk = u_blk[uc / cpb], off = (uc % cpb) * kChunk;
+        // the chunk's first cache row: in the sequence's slab, or in the block's
+        // page (an out-of-range page id reads zeros; the selection kernel has
+        // reported it)
+        const int rowk = P.table ? P.table[(size_t)b * (P.cap / g.B) + blk] * g.B + off
+                                 : (int)(krow_base + (size_t)blk * g.B + off);
         const uint32_t st = sbase + kOffStages + s * kStageBytes;
         mbar_expect_tx(&full[s], kStageBytes);
         tma_load_3d(st, &tmK, 0, hk, rowk, &full[s]);
@@ -569,11 +574,11 @@ cudaError_t launch_attn_decode_mma(const Geom& g, int batch, int n_q, int cap, i
                                    const void* kc, const void* vc, const void* gate,
                                    const int* sel, const int* nsel, float* part_ml,
                                    float* part_o, int* counter, void* out, float* lse, int* err,
-                                   cudaStream_t st) {
+                                   cudaStream_t st, Pages pg) {
   if (batch == 0) return cudaSuccess;
   CUtensorMap mk, mv;
-  if (!make_cache_map(&mk, kc, g.Hkv, (long long)batch * cap) ||
-      !make_cache_map(&mv, vc, g.Hkv, (long long)batch * cap))
+  const long long rows = pg.table ? (long long)pg.num_pages * g.B : (long long)batch * cap;
+  if (!make_cache_map(&mk, kc, g.Hkv, rows) || !make_cache_map(&mv, vc, g.Hkv, rows))
     return cudaErrorInvalidValue;
   DecParams p;
   p.g = g;
@@ -592,6 +597,7 @@ cudaError_t launch_attn_decode_mma(const Geom& g, int batch, int n_q, int cap, i
   p.part_ml = part_ml;
   p.part_o = part_o;
   p.err = err;
+  p.table = pg.table;
   const int words = (cap / g.B + 31) / 32;
   const int smem = kOffBits + 4 * n_q * words + 1024;
   cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(attn_decode_mma_kernel), smem);

@@ -12,6 +12,14 @@ namespace qsa {
 
 struct Geom;
 
+// Paged caches: block j of sequence b lives in page table[b * (cap / B) + j]
+// of a pool of num_pages pages of B rows each. table == nullptr: contiguous
+// [batch, cap] caches.
+struct Pages {
+  const int* table = nullptr;
+  int num_pages = 0;
+};
+
 // Counts kernel launches made by the library (all host threads).
 void note_launch(int n = 1);
 
@@ -50,7 +58,7 @@ cudaError_t launch_pool_prefill(qsa_dtype dt, const void* ik, const int* cu, int
                                 cudaStream_t st);
 cudaError_t launch_pool_cache(qsa_dtype dt, const void* ik_cache, const int* kv_len, int batch,
                               int cap, int n_q, int mode, int B, int di, float* pooled,
-                              int* dev_err, cudaStream_t st);
+                              int* dev_err, cudaStream_t st, Pages pg = Pages());
 size_t select_prefill_smem(const Geom& g, int nc_cap);
 // sched: one int the caller zeroed on the stream before the launch (the
 // kernel's work counter).
@@ -64,7 +72,7 @@ cudaError_t launch_decode_select(qsa_dtype dt, const Geom& g, int batch, int n_q
                                  const int* kv_len, const void* iq, const void* ik_cache,
                                  const float* iw, float* pooled, float* scores_out,
                                  uint32_t* keys_ws, int* counter, int* sel, int* nsel,
-                                 int* dev_err, cudaStream_t st);
+                                 int* dev_err, cudaStream_t st, Pages pg = Pages());
 cudaError_t launch_attn_prefill_simt(qsa_dtype dt, const Geom& g, const int* cu, int batch,
                                      int max_seqlen, const void* q, const void* k, const void* v,
                                      const void* gate, const int* sel, const int* nsel,
@@ -86,7 +94,7 @@ cudaError_t launch_attn_decode_mma(const Geom& g, int batch, int n_q, int cap, i
                                    const void* kc, const void* vc, const void* gate,
                                    const int* sel, const int* nsel, float* part_ml,
                                    float* part_o, int* counter, void* out, float* lse, int* err,
-                                   cudaStream_t st);
+                                   cudaStream_t st, Pages pg = Pages());
 bool attn_prefill_tc_supported(const Geom& g);
 cudaError_t launch_attn_prefill_tc(const Geom& g, const int* cu, int batch, int total_tokens,
                                    int max_seqlen, int words, const uint32_t* bitmask,

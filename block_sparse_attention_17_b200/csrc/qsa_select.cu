@@ -85,7 +85,8 @@ pool_prefill_kernel(const T* __restrict__ ik, const int* __restrict__ cu, int B,
 template <typename T>
 __global__ void __launch_bounds__(kPoolThreads)
 pool_cache_kernel(const T* __restrict__ ik_cache, const int* __restrict__ kv_len, int cap,
-                  int n_q, int mode, int B, int di, float* __restrict__ pooled, int* dev_err) {
+                  int n_q, int mode, int B, int di, float* __restrict__ pooled, int* dev_err,
+                  Pages pg) {
   const int b = blockIdx.y;
   const int kv = kv_len[b];
   if (kv < (mode ? n_q : 0) || kv > cap) {
@@ -95,8 +96,16 @@ pool_cache_kernel(const T* __restrict__ ik_cache, const int* __restrict__ kv_len
   const int jlo = mode ? (kv - n_q) / B : 0;
   const int j = jlo + blockIdx.x;
   if (j >= kv / B) return;
-  pool_block_cta(ik_cache + ((size_t)b * cap + (size_t)j * B) * di, B, di,
-                 pooled + ((size_t)b * (cap / B) + j) * di);
+  size_t row0 = ((size_t)b * cap + (size_t)j * B);
+  if (pg.table) {
+    const int page = pg.table[(size_t)b * (cap / B) + j];
+    if (page < 0 || page >= pg.num_pages) {
+      if (dev_err && threadIdx.x == 0) atomicExch(dev_err, 3);
+      return;
+    }
+    row0 = (size_t)page * B;
+  }
+  pool_block_cta(ik_cache + row0 * di, B, di, pooled + ((size_t)b * (cap / B) + j) * di);
 }
 
 // ----------------------------------------------------------------- top-k
@@ -568,7 +577,7 @@ decode_select_kernel(Geom g, int n_q, int cap, const int* __restrict__ kv_len,
                      const float* __restrict__ iw, float* __restrict__ pooled,
                      float* __restrict__ scores_out, uint32_t* __restrict__ keys_ws,
                      int* __restrict__ counter, int* __restrict__ sel, int* __restrict__ nsel,
-                     int* dev_err) {
+                     int* dev_err, Pages pg) {
   grid_dependents_launch();   // the attention kernel may start its prologue
   extern __shared__ __align__(16) float smem[];
   constexpr int kStride = kDI + 1;
@@ -598,11 +607,26 @@ decode_select_kernel(Geom g, int n_q, int cap, const int* __restrict__ kv_len,
   const int j0 = c * kPart;
   const int rows = max(0, min(kPart, nc_last - j0));
 
+  // 0. paged caches: every page id the attention may gather from this range
+  //    (and the tail block, by the last range) must name a page of the pool
+  if (pg.table) {
+    const int nb_used = (kv + g.B - 1) / g.B;
+    const int jend = c == nparts - 1 ? nb_used : min(nb_used, j0 + kPart);
+    for (int j = j0 + (int)threadIdx.x; j < jend; j += blockDim.x) {
+      const int page = pg.table[(size_t)b * nblk_cap + j];
+      if ((page < 0 || page >= pg.num_pages) && dev_err) atomicExch(dev_err, 3);
+    }
+  }
   // 1. blocks completed by this step's tokens (pool_block_cta needs the whole CTA)
   const int jnew_lo = max((kv - n_q) / g.B, j0), jnew_hi = min(nc_last, j0 + kPart);
   for (int j = jnew_lo; j < jnew_hi; ++j) {
-    pool_block_cta(ik_cache + ((size_t)b * cap + (size_t)j * g.B) * kDI, g.B, kDI,
-                   pooled + ((size_t)b * nblk_cap + j) * kDI);
+    size_t row0 = (size_t)b * cap + (size_t)j * g.B;
+    if (pg.table) {
+      const int page = pg.table[(size_t)b * nblk_cap + j];
+      row0 = (page >= 0 && page < pg.num_pages) ? (size_t)page * g.B : SIZE_MAX;
+    }
+    if (row0 != SIZE_MAX)   // uniform across the CTA
+      pool_block_cta(ik_cache + row0 * kDI, g.B, kDI, pooled + ((size_t)b * nblk_cap + j) * kDI);
     __syncthreads();
   }
   // 2. stage the range's pooled rows and the queries' indexer q / weights
@@ -741,16 +765,16 @@ cudaError_t launch_pool_prefill(qsa_dtype dt, const void* ik, const int* cu, int
 
 cudaError_t launch_pool_cache(qsa_dtype dt, const void* ik_cache, const int* kv_len, int batch,
                               int cap, int n_q, int mode, int B, int di, float* pooled,
-                              int* dev_err, cudaStream_t st) {
+                              int* dev_err, cudaStream_t st, Pages pg) {
   const int span = mode ? (n_q + B - 1) / B + 1 : cap / B;
   if (batch == 0 || span == 0) return cudaSuccess;
   dim3 grid(span, batch);
   if (dt == QSA_BF16)
     pool_cache_kernel<__nv_bfloat16><<<grid, kPoolThreads, 0, st>>>(
-        (const __nv_bfloat16*)ik_cache, kv_len, cap, n_q, mode, B, di, pooled, dev_err);
+        (const __nv_bfloat16*)ik_cache, kv_len, cap, n_q, mode, B, di, pooled, dev_err, pg);
   else
     pool_cache_kernel<float><<<grid, kPoolThreads, 0, st>>>((const float*)ik_cache, kv_len, cap,
-                                                            n_q, mode, B, di, pooled, dev_err);
+                                                            n_q, mode, B, di, pooled, dev_err, pg);
   note_launch();
   return cudaGetLastError();
 }
@@ -820,14 +844,14 @@ static cudaError_t launch_decode_select_t(const Geom& g, int batch, int n_q, int
                                           const int* kv_len, const void* iq, const void* ik_cache,
                                           const float* iw, float* pooled, float* scores_out,
                                           uint32_t* keys_ws, int* counter, int* sel, int* nsel,
-                                          int* dev_err, cudaStream_t st) {
+                                          int* dev_err, cudaStream_t st, Pages pg) {
   const size_t smem = decode_select_smem(g, n_q, cap);
   auto kern = decode_select_kernel<T, kDI>;
   cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(kern), (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<dim3(decode_select_parts(g, cap), batch), kSelThreads, smem, st>>>(
       g, n_q, cap, kv_len, (const T*)iq, (const T*)ik_cache, iw, pooled, scores_out, keys_ws,
-      counter, sel, nsel, dev_err);
+      counter, sel, nsel, dev_err, pg);
   note_launch();
   return cudaGetLastError();
 }
@@ -836,11 +860,11 @@ cudaError_t launch_decode_select(qsa_dtype dt, const Geom& g, int batch, int n_q
                                  const int* kv_len, const void* iq, const void* ik_cache,
                                  const float* iw, float* pooled, float* scores_out,
                                  uint32_t* keys_ws, int* counter, int* sel, int* nsel,
-                                 int* dev_err, cudaStream_t st) {
+                                 int* dev_err, cudaStream_t st, Pages pg) {
   if (batch == 0) return cudaSuccess;
 #define QSA_DS(T, DI)                                                                       \
   return launch_decode_select_t<T, DI>(g, batch, n_q, cap, kv_len, iq, ik_cache, iw, pooled, \
-                                       scores_out, keys_ws, counter, sel, nsel, dev_err, st)
+                                       scores_out, keys_ws, counter, sel, nsel, dev_err, st, pg)
   if (dt == QSA_BF16) {
     if (g.di == 64) QSA_DS(__nv_bfloat16, 64);
     QSA_DS(__nv_bfloat16, 32);

@@ -201,6 +201,39 @@ qsa_status qsa_decode_noalloc(const qsa_config* cfg, int batch, int n_q, int cap
                               void* out, float* lse, int32_t* sel, int32_t* nsel,
                               int32_t* dev_err, void* stream);
 
+/* --------------------------------------------------------- paged decode --
+ * qsa_decode over a paged KV cache (a speed lever the llama.cpp PR #27739
+ * page lists: "continuous batching and paged KV"; the QSA block is the page).
+ * A page holds the B consecutive rows of one block of one sequence:
+ *   k_pages/v_pages [num_pages, B, Hkv, D]   ik_pages [num_pages, B, di]
+ *   block_table     [batch, max_blocks] int32 (device): block j of sequence b
+ *                   lives in page block_table[b * max_blocks + j]. Entries of
+ *                   blocks past the sequence's last token are not read.
+ * Everything else is as for qsa_decode with cap = max_blocks * B (pooled_cache
+ * [batch, max_blocks, di]; the workspace size is
+ * qsa_decode_workspace_size(cfg, batch, n_q, max_blocks * B)). The results
+ * are bit-identical to qsa_decode on the same rows laid out contiguously.
+ * A page id outside [0, num_pages) among a sequence's blocks sets *dev_err
+ * to 3 (that sequence's outputs are then unspecified, and nothing outside the
+ * pools is read). Supported: bf16 with n_q * (Hq / Hkv) <= 16; otherwise
+ * QSA_ERR_UNSUPPORTED. */
+qsa_status qsa_decode_paged(const qsa_config* cfg, int batch, int n_q, int max_blocks,
+                            const int32_t* block_table, int num_pages, const int32_t* kv_len,
+                            const void* q, const void* k_pages, const void* v_pages,
+                            const void* iq, const void* ik_pages, const float* iw,
+                            const void* gate, float* pooled_cache, void* out, float* lse,
+                            int32_t* sel, int32_t* nsel, int32_t* dev_err, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/* qsa_pool_build for a paged indexer-key cache (arguments as for
+ * qsa_decode_paged); the rows it writes are bit-identical to qsa_pool_build's
+ * on the same rows laid out contiguously. A bad page id sets *dev_err to 3
+ * and leaves that block's pooled row untouched. */
+qsa_status qsa_pool_build_paged(const qsa_config* cfg, int batch, int max_blocks,
+                                const int32_t* block_table, int num_pages,
+                                const int32_t* kv_len, const void* ik_pages,
+                                float* pooled_cache, int32_t* dev_err, void* stream);
+
 /* Rebuild the pooled-key cache of every complete block j < kv_len[b]/B from
  * the indexer-key cache (restore after a state reload). The rows it writes are
  * bit-identical to the ones the incremental decode path writes. */

@@ -131,3 +131,27 @@ def test_workspace_sizes_grow_with_the_problem():
     assert 0 < a < b
     assert lib.qsa_decode_workspace_size(ctypes.byref(c), 4, 1, 4096) < \
         lib.qsa_decode_workspace_size(ctypes.byref(c), 8, 1, 4096)
+
+
+def test_paged_decode_rejects_bad_arguments():
+    lib = _lib.lib()
+    c = cfg()
+    max_blocks = 512
+    ws = lib.qsa_decode_workspace_size(ctypes.byref(c), 32, 1, max_blocks * c.block_size)
+    assert ws > 0
+
+    def call(n_q=1, max_blocks=max_blocks, table=FAKE, num_pages=32 * 512, ws_bytes=ws, c=c):
+        return lib.qsa_decode_paged(ctypes.byref(c), 32, n_q, max_blocks, table, num_pages, FAKE,
+                                    FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None,
+                                    None, None, None, ctypes.c_void_p(0x20000), ws_bytes, None)
+    assert call(table=None) == _lib.QSA_ERR_INVALID_ARG
+    assert call(table=MISALIGNED) == _lib.QSA_ERR_INVALID_ARG
+    assert call(max_blocks=0) == _lib.QSA_ERR_INVALID_ARG
+    assert call(num_pages=0) == _lib.QSA_ERR_INVALID_ARG
+    assert call(n_q=0) == _lib.QSA_ERR_INVALID_ARG
+    assert call(n_q=3) == _lib.QSA_ERR_UNSUPPORTED                    # 3 * 8 rows > 16
+    assert call(c=cfg(dtype=_lib.QSA_F32)) == _lib.QSA_ERR_UNSUPPORTED  # tensor-map gather: bf16
+    assert call(ws_bytes=ws - 256) == _lib.QSA_ERR_WORKSPACE
+    st = lib.qsa_pool_build_paged(ctypes.byref(c), 32, max_blocks, None, 16, FAKE, FAKE, FAKE,
+                                  None, None)
+    assert st == _lib.QSA_ERR_INVALID_ARG
