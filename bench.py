@@ -276,10 +276,33 @@ def run_ours(args, w, rank, world, dist):
         sel = torch.empty(w.batch, w.n_q, w.topk + 1, dtype=torch.int32, device=dev)
         nsel = torch.empty(w.batch, w.n_q, dtype=torch.int32, device=dev)
 
-        def step(dd=d, o=out):
-            qsa.decode(cfg, dd["q"], dd["k_cache"], dd["v_cache"], dd["iq"], dd["ik_cache"],
-                       dd["iw"], dd["gate"], pooled, dd["kv_len"], out=o, sel=sel, nsel=nsel,
-                       workspace=ws)
+        if args.paged:
+            # the same rows scattered into a page pool (page = one block) under a
+            # seeded random block table
+            B = w.block_size
+            max_blocks = inp["cap"] // B
+            perm = np.random.default_rng(w.seed + 1).permutation(w.batch * max_blocks)
+            table = torch.from_numpy(perm.reshape(w.batch, max_blocks).astype(np.int32)).to(dev)
+            idx = table.reshape(-1).long()
+
+            def scatter(cache):
+                pool = torch.empty((w.batch * max_blocks, B, *cache.shape[2:]), dtype=cache.dtype,
+                                   device=dev)
+                pool[idx] = cache.reshape(w.batch * max_blocks, B, *cache.shape[2:])
+                return pool
+            pages = {n: scatter(d[n]) for n in ("k_cache", "v_cache", "ik_cache")}
+            pooled = qsa.pool_build_paged(cfg, pages["ik_cache"], (kv - w.n_q).to(torch.int32),
+                                          table)
+
+            def step(dd=d, o=out):
+                qsa.decode_paged(cfg, dd["q"], pages["k_cache"], pages["v_cache"], dd["iq"],
+                                 pages["ik_cache"], dd["iw"], dd["gate"], pooled, dd["kv_len"],
+                                 table, out=o, sel=sel, nsel=nsel, workspace=ws)
+        else:
+            def step(dd=d, o=out):
+                qsa.decode(cfg, dd["q"], dd["k_cache"], dd["v_cache"], dd["iq"], dd["ik_cache"],
+                           dd["iw"], dd["gate"], pooled, dd["kv_len"], out=o, sel=sel, nsel=nsel,
+                           workspace=ws)
         step()
         torch.cuda.synchronize()
         kv_bytes = decode_selected_kv_bytes(w, sel.cpu().numpy(), nsel.cpu().numpy(),
@@ -413,6 +436,8 @@ def run_ours(args, w, rank, world, dist):
              "timing": ("CUDA-graph replay of one library call per step" if graph is not None
                         else "eager library call per step"),
              "eager_ms_per_step": float(np.mean(eager_ms)),
+             "kv_layout": "paged (one block per page)" if (args.paged and w.kind == "decode")
+             else "contiguous",
              "selected_kv_tokens_per_step": units, "job_selected_kv_tokens_per_step": job_units,
              "shards": "one per rank: the workload's shapes, seed + 7919 * rank",
              "input_gen_s": round(t_gen, 2)}
@@ -490,6 +515,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager calls only (no CUDA graph)")
+    ap.add_argument("--paged", action="store_true",
+                    help="decode workloads: run qsa_decode_paged over a page pool")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-step-seconds", type=float, default=2.0)
