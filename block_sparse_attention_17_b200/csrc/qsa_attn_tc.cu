@@ -58,7 +58,7 @@ constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + kTiles * kTileBytes;
 constexpr int kOffV = kOffK + kNK * kTileBytes;
 constexpr int kOffBar = kOffV + kNV * kTileBytes;
-constexpr int kNumBars = 1 + 2 * kNK + 2 * kNV + 3 * kTiles + 1;
+constexpr int kNumBars = 1 + 2 * kNK + 2 * kNV + 3 * kTiles + 1 + 4 * kTiles;
 constexpr int kOffMisc = kOffBar + 8 * kNumBars;
 constexpr int kOffBits = kOffMisc + 64;
 constexpr int kMaxWords = kMaxBlocksPerSeq / 32;
@@ -117,6 +117,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
   uint64_t* p_full = s_full + kTiles;   // [tile]
   uint64_t* o_done = p_full + kTiles;   // [tile]
   uint64_t* mma_done = o_done + kTiles;
+  uint64_t* xbar = mma_done + 1;        // [tile][lane quarter]: the row-max exchange of a warp pair
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
   int* n_union_s = reinterpret_cast<int*>(smem + kOffMisc + 8);
@@ -133,6 +134,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
       mbar_init(&o_done[t], 1);
     }
     mbar_init(mma_done, 1);
+    for (int i = 0; i < 4 * kTiles; ++i) mbar_init(&xbar[i], 64);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async();
@@ -288,7 +290,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
     // ------------------------------------------------------------ softmax
     // Tile t has 8 warps: each row (TMEM lane) is shared by two threads, one
     // per 64-column half of S; they exchange their partial row max through
-    // shared memory behind a named barrier of the two warps.
+    // shared memory, ordered by an mbarrier of the two warps (bounded waits).
     const int wt = warp - 2;
     const int t = wt >> 3;                    // tile
     const int hf = (wt >> 2) & 1;             // column half
@@ -307,7 +309,14 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
     const uint32_t tO = tS + 256;
     float* xch = reinterpret_cast<float*>(smem + kOffXch);
     auto xslot = [&](int slot, int half) { return xch + ((t * 2 + slot) * 2 + half) * kRows + r; };
-    const int bar_id = 1 + t * 4 + quarter;
+    // exchange number e (step j, then n_iter for the final sums) uses data slot
+    // e & 1 and phase e of the pair's mbarrier; the wait is bounded, so a warp
+    // whose partner gave up does not block
+    auto exchange = [&](int e, float x) -> bool {
+      *xslot(e & 1, hf) = x;
+      mbar_arrive(&xbar[t * 4 + quarter]);
+      return __all_sync(kFull, mbar_wait_spin(&xbar[t * 4 + quarter], e & 1, abort_flag));
+    };
     const float sc = g.sm_scale_log2;
     float m_used = -INFINITY, l = 0.f;
     bool ok = t < nt;
@@ -357,8 +366,10 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
           pm = lim > 0 ? fmax3(cm[0], cm[1], fmaxf(cm[2], cm[3])) : -INFINITY;
         }
       }
-      *xslot(j & 1, hf) = pm;
-      named_bar_sync(bar_id, 64);
+      if (!exchange(j, pm)) {
+        ok = false;
+        break;
+      }
       const float mx = fmaxf(pm, *xslot(j & 1, hf ^ 1)) * sc;
       float m_tgt = m_used, alpha = 1.f;
       if (mx > m_used + kRescaleThreshold || (m_used == -INFINITY && mx != -INFINITY)) {
@@ -424,9 +435,8 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
     if (ok && n_iter > 0 &&
         __all_sync(kFull, mbar_wait(&o_done[t], (n_iter - 1) & 1, abort_flag))) {
       tc_fence_after();
-      *xslot(n_iter & 1, hf) = l;
-      named_bar_sync(bar_id, 64);
-      const float lt = l + *xslot(n_iter & 1, hf ^ 1);
+      const bool have_l = exchange(n_iter, l);
+      const float lt = have_l ? l + *xslot(n_iter & 1, hf ^ 1) : 0.f;
       const float inv_l = lt > 0.f ? 1.f / lt : 0.f;
       __nv_bfloat16* orow = P.out + (tok * g.Hq + h) * kHeadDim;
       const __nv_bfloat16* grow =

@@ -80,6 +80,24 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// mbar_wait for a phase expected within a few hundred cycles: polls without
+// the suspend hint, with the same bound and abort protocol.
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity,
+                                               volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255u) == 0) {
+      if (*abort) return false;
+      if (clock64() - t0 > kWaitCycles) {
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
 // 2^x on the MUFU unit (flushes denormal results to zero; exp2(-inf) = 0).
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
