@@ -436,6 +436,8 @@ def run_ours(args, w, rank, world, dist):
              "timing": ("CUDA-graph replay of one library call per step" if graph is not None
                         else "eager library call per step"),
              "eager_ms_per_step": float(np.mean(eager_ms)),
+             "median_ms_per_step": float(np.median(step_ms)),
+             "eager_median_ms_per_step": float(np.median(eager_ms)),
              "kv_layout": "paged (one block per page)" if (args.paged and w.kind == "decode")
              else "contiguous",
              "selected_kv_tokens_per_step": units, "job_selected_kv_tokens_per_step": job_units,
@@ -509,8 +511,8 @@ def run_reference(args, w):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
