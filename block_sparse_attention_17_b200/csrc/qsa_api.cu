@@ -184,7 +184,8 @@ PrefillWs carve_prefill(const Geom& g, void* ws, int batch, int T, int max_seqle
 
 struct DecodeWs {
   int* err;
-  int* counters;        // [batch] selection + [batch * Hkv] attention, zeroed per call
+  int* counters;        // [batch] selection + [batch * Hkv] attention + [batch] ready
+                        // flags, zeroed per call
   uint32_t* keys;       // [batch, n_q, cap / B] score keys
   int* sel;
   int* nsel;
@@ -213,7 +214,7 @@ DecodeWs carve_decode(const qsa_config* cfg, const Geom& g, void* ws, int batch,
   const int R = n_q * g.G;
   Carve c(ws);
   w.err = c.take<int>(1);
-  w.counters = c.take<int>((size_t)batch * (1 + g.Hkv));
+  w.counters = c.take<int>((size_t)batch * (2 + g.Hkv));
   w.keys = c.take<uint32_t>((size_t)batch * n_q * (cap / g.B));
   w.sel = c.take<int>((size_t)batch * n_q * (g.k + 1));
   w.nsel = c.take<int>((size_t)batch * n_q);
@@ -399,11 +400,11 @@ static qsa_status decode_select_common(const qsa_config* cfg, const Geom& g, int
                                        float* pooled_cache, const DecodeWs& w, int32_t* sel,
                                        int32_t* nsel, float* scores, int32_t* dev_err,
                                        cudaStream_t st, Pages pg = Pages()) {
-  QSA_CUDA(cudaMemsetAsync(w.counters, 0, sizeof(int) * (size_t)batch * (1 + g.Hkv), st),
+  QSA_CUDA(cudaMemsetAsync(w.counters, 0, sizeof(int) * (size_t)batch * (2 + g.Hkv), st),
            "clear counters");
   QSA_CUDA(launch_decode_select(cfg->dtype, g, batch, n_q, cap, kv_len, iq, ik_cache, iw,
                                 pooled_cache, scores, w.keys, w.counters, sel, nsel, dev_err, st,
-                                pg),
+                                pg, w.counters + (size_t)batch * (1 + g.Hkv)),
            "decode select");
   return QSA_OK;
 }
@@ -441,7 +442,7 @@ static qsa_status decode_impl(const qsa_config* cfg, int batch, int n_q, int cap
     QSA_CUDA(launch_attn_decode_mma(g, batch, n_q, cap, w.nsplit, w.per_split, kv_len, q,
                                     k_cache, v_cache, gate, sel_p, nsel_p, w.part_ml, w.part_o,
                                     w.counters + batch, out, lse, dev_err ? dev_err : w.err, st,
-                                    pg),
+                                    pg, w.counters + (size_t)batch * (1 + g.Hkv)),
              "decode attention");
   } else {
     QSA_CUDA(launch_attn_decode_simt(cfg->dtype, g, batch, n_q, cap, w.nsplit, w.per_split,

@@ -61,6 +61,7 @@ struct DecParams {
   float* lse;
   int* err;
   const int* table;                  // paged caches: [batch, cap / B] page ids, else null
+  const int* ready;                  // [batch] selection-written flags, else null
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
@@ -160,8 +161,30 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
     const size_t orow = ((size_t)b * n_q + r / G) * g.Hq + hk * G + r % G;
     asm volatile("prefetch.global.L2 [%0];" ::"l"(P.gate + orow * kD + part * 64));
   }
-  grid_dependency_wait();   // the selections come from the selection kernel
+  // the selections come from the selection kernel: wait for this sequence's
+  // flag (bounded), or for the whole selection grid
+  if (P.ready) {
+    if (threadIdx.x == 0) {
+      const long long t0 = clock64();
+      while (true) {
+        int v;
+        asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(P.ready + b) : "memory");
+        if (v != 0) break;
+        if (clock64() - t0 > kWaitCycles) {
+          *abort_flag = 1;
+          break;
+        }
+        __nanosleep(128);
+      }
+    }
+  } else {
+    grid_dependency_wait();
+  }
   __syncthreads();
+  if (*abort_flag) {   // nothing issued yet: report and leave (no merge for this pair)
+    if (threadIdx.x == 0 && P.err) atomicExch(P.err, 2);
+    return;
+  }
   {
     const int kp1 = g.k + 1;
     const int nblk = P.cap / g.B;
@@ -574,7 +597,7 @@ cudaError_t launch_attn_decode_mma(const Geom& g, int batch, int n_q, int cap, i
                                    const void* kc, const void* vc, const void* gate,
                                    const int* sel, const int* nsel, float* part_ml,
                                    float* part_o, int* counter, void* out, float* lse, int* err,
-                                   cudaStream_t st, Pages pg) {
+                                   cudaStream_t st, Pages pg, const int* ready) {
   if (batch == 0) return cudaSuccess;
   CUtensorMap mk, mv;
   const long long rows = pg.table ? (long long)pg.num_pages * g.B : (long long)batch * cap;
@@ -598,6 +621,7 @@ cudaError_t launch_attn_decode_mma(const Geom& g, int batch, int n_q, int cap, i
   p.part_o = part_o;
   p.err = err;
   p.table = pg.table;
+  p.ready = ready;
   const int words = (cap / g.B + 31) / 32;
   const int smem = kOffBits + 4 * n_q * words + 1024;
   cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(attn_decode_mma_kernel), smem);

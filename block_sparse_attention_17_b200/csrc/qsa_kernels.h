@@ -31,6 +31,10 @@ cudaError_t set_max_dynamic_smem(const void* func, int bytes);
 // SM count of the current device (cached per function, device and shape).
 cudaError_t resident_ctas(const void* func, int threads, size_t smem, int* per_sm, int* sms);
 
+// ready: [batch] flags the selection kernel sets (release) once a sequence's
+// selections are written, zero before the launch; the decode attention kernel
+// waits on its sequence's flag instead of on the whole selection grid.
+
 // Launches `kernel` on `st` with programmatic stream serialization: it may
 // start before the previous kernel on the stream finishes, and must call
 // grid_dependency_wait() before reading that kernel's outputs.
@@ -72,7 +76,8 @@ cudaError_t launch_decode_select(qsa_dtype dt, const Geom& g, int batch, int n_q
                                  const int* kv_len, const void* iq, const void* ik_cache,
                                  const float* iw, float* pooled, float* scores_out,
                                  uint32_t* keys_ws, int* counter, int* sel, int* nsel,
-                                 int* dev_err, cudaStream_t st, Pages pg = Pages());
+                                 int* dev_err, cudaStream_t st, Pages pg = Pages(),
+                                 int* ready = nullptr);
 cudaError_t launch_attn_prefill_simt(qsa_dtype dt, const Geom& g, const int* cu, int batch,
                                      int max_seqlen, const void* q, const void* k, const void* v,
                                      const void* gate, const int* sel, const int* nsel,
@@ -94,7 +99,7 @@ cudaError_t launch_attn_decode_mma(const Geom& g, int batch, int n_q, int cap, i
                                    const void* kc, const void* vc, const void* gate,
                                    const int* sel, const int* nsel, float* part_ml,
                                    float* part_o, int* counter, void* out, float* lse, int* err,
-                                   cudaStream_t st, Pages pg = Pages());
+                                   cudaStream_t st, Pages pg = Pages(), const int* ready = nullptr);
 bool attn_prefill_tc_supported(const Geom& g);
 cudaError_t launch_attn_prefill_tc(const Geom& g, const int* cu, int batch, int total_tokens,
                                    int max_seqlen, int words, const uint32_t* bitmask,

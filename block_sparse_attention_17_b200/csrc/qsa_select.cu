@@ -577,7 +577,7 @@ decode_select_kernel(Geom g, int n_q, int cap, const int* __restrict__ kv_len,
                      const float* __restrict__ iw, float* __restrict__ pooled,
                      float* __restrict__ scores_out, uint32_t* __restrict__ keys_ws,
                      int* __restrict__ counter, int* __restrict__ sel, int* __restrict__ nsel,
-                     int* dev_err, Pages pg) {
+                     int* dev_err, Pages pg, int* ready) {
   grid_dependents_launch();   // the attention kernel may start its prologue
   extern __shared__ __align__(16) float smem[];
   constexpr int kStride = kDI + 1;
@@ -739,6 +739,12 @@ decode_select_kernel(Geom g, int n_q, int cap, const int* __restrict__ kv_len,
     __syncthreads();
   }
   if (threadIdx.x == 0) counter[b] = 0;
+  if (ready) {   // this sequence's selections are written: release its attention CTAs
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0)
+      asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(ready + b), "r"(1) : "memory");
+  }
 }
 
 // ------------------------------------------------------------ launchers
@@ -844,14 +850,14 @@ static cudaError_t launch_decode_select_t(const Geom& g, int batch, int n_q, int
                                           const int* kv_len, const void* iq, const void* ik_cache,
                                           const float* iw, float* pooled, float* scores_out,
                                           uint32_t* keys_ws, int* counter, int* sel, int* nsel,
-                                          int* dev_err, cudaStream_t st, Pages pg) {
+                                          int* dev_err, cudaStream_t st, Pages pg, int* ready) {
   const size_t smem = decode_select_smem(g, n_q, cap);
   auto kern = decode_select_kernel<T, kDI>;
   cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(kern), (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<dim3(decode_select_parts(g, cap), batch), kSelThreads, smem, st>>>(
       g, n_q, cap, kv_len, (const T*)iq, (const T*)ik_cache, iw, pooled, scores_out, keys_ws,
-      counter, sel, nsel, dev_err, pg);
+      counter, sel, nsel, dev_err, pg, ready);
   note_launch();
   return cudaGetLastError();
 }
@@ -860,11 +866,12 @@ cudaError_t launch_decode_select(qsa_dtype dt, const Geom& g, int batch, int n_q
                                  const int* kv_len, const void* iq, const void* ik_cache,
                                  const float* iw, float* pooled, float* scores_out,
                                  uint32_t* keys_ws, int* counter, int* sel, int* nsel,
-                                 int* dev_err, cudaStream_t st, Pages pg) {
+                                 int* dev_err, cudaStream_t st, Pages pg, int* ready) {
   if (batch == 0) return cudaSuccess;
 #define QSA_DS(T, DI)                                                                       \
   return launch_decode_select_t<T, DI>(g, batch, n_q, cap, kv_len, iq, ik_cache, iw, pooled, \
-                                       scores_out, keys_ws, counter, sel, nsel, dev_err, st, pg)
+                                       scores_out, keys_ws, counter, sel, nsel, dev_err, st, pg, \
+                                       ready)
   if (dt == QSA_BF16) {
     if (g.di == 64) QSA_DS(__nv_bfloat16, 64);
     QSA_DS(__nv_bfloat16, 32);
