@@ -276,7 +276,31 @@ def run_ours(args, w, rank, world, dist):
         sel = torch.empty(w.batch, w.n_q, w.topk + 1, dtype=torch.int32, device=dev)
         nsel = torch.empty(w.batch, w.n_q, dtype=torch.int32, device=dev)
 
-        if args.paged:
+        if args.kv != "bf16":
+            # the same rows as e4m3 with one fp32 scale per (token, KV head) row,
+            # optionally stored in the Walsh-Hadamard-rotated basis
+            rotated = args.kv == "fp8-rotated"
+            Dh = w.head_dim
+            Hm = torch.ones(1, 1, dtype=torch.float64)
+            while Hm.shape[0] < Dh:
+                Hm = torch.cat([torch.cat([Hm, Hm], 1), torch.cat([Hm, -Hm], 1)], 0)
+            Hm = (Hm / Dh ** 0.5).to(dev, torch.float32)
+            fp8 = {}
+            for n in ("k_cache", "v_cache"):
+                x = d[n].float()
+                if rotated:
+                    x = x @ Hm
+                scale = (x.abs().amax(-1) / 448.0).clamp_min(1e-30)
+                codes = (x / scale[..., None]).to(torch.float8_e4m3fn).view(torch.uint8)
+                fp8[n] = (codes.contiguous(), scale.contiguous())
+                del x
+
+            def step(dd=d, o=out):
+                qsa.decode_fp8(cfg, dd["q"], fp8["k_cache"][0], fp8["k_cache"][1],
+                               fp8["v_cache"][0], fp8["v_cache"][1], dd["iq"], dd["ik_cache"],
+                               dd["iw"], dd["gate"], pooled, dd["kv_len"], rotated=rotated, out=o,
+                               sel=sel, nsel=nsel, workspace=ws)
+        elif args.paged:
             # the same rows scattered into a page pool (page = one block) under a
             # seeded random block table
             B = w.block_size
@@ -306,7 +330,7 @@ def run_ours(args, w, rank, world, dist):
         step()
         torch.cuda.synchronize()
         kv_bytes = decode_selected_kv_bytes(w, sel.cpu().numpy(), nsel.cpu().numpy(),
-                                            inp["kv_len"])
+                                            inp["kv_len"], args.kv)
         esz = 2 if w.dtype == "bf16" else 4
         io = w.batch * w.n_q * (2 * w.num_q_heads * w.head_dim * esz)   # q + out
         io += w.batch * w.n_q * w.num_q_heads * w.head_dim * esz         # gate
@@ -440,6 +464,7 @@ def run_ours(args, w, rank, world, dist):
              "eager_median_ms_per_step": float(np.median(eager_ms)),
              "kv_layout": "paged (one block per page)" if (args.paged and w.kind == "decode")
              else "contiguous",
+             "kv_format": args.kv if w.kind == "decode" else "bf16",
              "selected_kv_tokens_per_step": units, "job_selected_kv_tokens_per_step": job_units,
              "shards": "one per rank: the workload's shapes, seed + 7919 * rank",
              "input_gen_s": round(t_gen, 2)}
@@ -462,9 +487,10 @@ def ctypes_voidp_array(ptrs):
     return ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
 
 
-def decode_selected_kv_bytes(w, sel, nsel, kv_len):
+def decode_selected_kv_bytes(w, sel, nsel, kv_len, kv_format="bf16"):
     """Distinct visible K/V bytes the step must read: per sequence, the union
-    over its new queries of their selected tokens, times Hkv heads, K and V."""
+    over its new queries of their selected tokens, times Hkv heads, K and V
+    (fp8 caches: one byte per element plus a 4-byte scale per row)."""
     esz = 2 if w.dtype == "bf16" else 4
     B = w.block_size
     total = 0
@@ -478,6 +504,8 @@ def decode_selected_kv_bytes(w, sel, nsel, kv_len):
                 hi = min((blk + 1) * B, n) if blk == nc else (blk + 1) * B
                 toks.update(range(blk * B, hi))
         total += len(toks)
+    if kv_format != "bf16":
+        return total * w.num_kv_heads * (w.head_dim + 4) * 2
     return total * w.num_kv_heads * w.head_dim * 2 * esz
 
 
@@ -519,6 +547,8 @@ def main():
     ap.add_argument("--eager", action="store_true", help="time eager calls only (no CUDA graph)")
     ap.add_argument("--paged", action="store_true",
                     help="decode workloads: run qsa_decode_paged over a page pool")
+    ap.add_argument("--kv", default="bf16", choices=["bf16", "fp8", "fp8-rotated"],
+                    help="decode workloads: K/V cache format (fp8: qsa_decode_fp8)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-step-seconds", type=float, default=2.0)

@@ -356,3 +356,49 @@ def pool_build_paged(cfg: QSAConfig, ik_pages, kv_len, block_table, pooled_cache
                                          _ptr(pooled_cache), _ptr(dev_err), _stream(stream))
     _lib.check(st, "qsa_pool_build_paged")
     return pooled_cache
+
+
+def decode_fp8(cfg: QSAConfig, q, k_cache, k_scale, v_cache, v_scale, iq, ik_cache, iw, gate,
+               pooled_cache, kv_len, *, rotated=False, out=None, lse=None, sel=None, nsel=None,
+               dev_err=None, workspace=None, want_lse=False, want_sel=False, stream=None) -> dict:
+    """One QSA decode step over fp8 (e4m3) K/V caches (qsa_decode_fp8):
+    k_cache/v_cache [batch, cap, Hkv, D] uint8 codes (or torch.float8_e4m3fn),
+    k_scale/v_scale [batch, cap, Hkv] fp32 row scales; rotated: the caches hold
+    the Walsh-Hadamard-rotated rows."""
+    batch, n_q = q.shape[0], q.shape[1]
+    cap = k_cache.shape[1]
+    if k_cache.dtype != torch.uint8:
+        k_cache, v_cache = k_cache.view(torch.uint8), v_cache.view(torch.uint8)
+    shp = (batch, cap, cfg.num_kv_heads, cfg.head_dim)
+    _need(q, "q", cfg.dtype, (batch, n_q, cfg.num_q_heads, cfg.head_dim))
+    _need(k_cache, "k_cache", torch.uint8, shp)
+    _need(v_cache, "v_cache", torch.uint8, shp)
+    _need(k_scale, "k_scale", torch.float32, shp[:3])
+    _need(v_scale, "v_scale", torch.float32, shp[:3])
+    _need(iq, "iq", cfg.dtype, (batch, n_q, cfg.idx_heads, cfg.idx_dim))
+    _need(ik_cache, "ik_cache", cfg.dtype, (batch, cap, cfg.idx_dim))
+    _need(iw, "iw", torch.float32, (batch, n_q, cfg.idx_heads))
+    gshape = ((batch, n_q, cfg.num_q_heads) if cfg.gate_headwise
+              else (batch, n_q, cfg.num_q_heads, cfg.head_dim))
+    _need(gate, "gate", cfg.dtype, gshape)
+    _need(pooled_cache, "pooled_cache", torch.float32, (batch, cap // cfg.block_size, cfg.idx_dim))
+    _need(kv_len, "kv_len", torch.int32, (batch,))
+    dev = q.device
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(batch, n_q, cfg.num_q_heads, dtype=torch.float32, device=dev)
+    if sel is None and want_sel:
+        sel = torch.empty(batch, n_q, cfg.topk + 1, dtype=torch.int32, device=dev)
+    if nsel is None and want_sel:
+        nsel = torch.empty(batch, n_q, dtype=torch.int32, device=dev)
+    ws = _workspace(decode_workspace_size(cfg, batch, n_q, cap), dev, workspace)
+    c = cfg.c()
+    st = _lib.lib().qsa_decode_fp8(ctypes.byref(c), batch, n_q, cap, _ptr(kv_len), _ptr(q),
+                                   _ptr(k_cache), _ptr(k_scale), _ptr(v_cache), _ptr(v_scale),
+                                   1 if rotated else 0, _ptr(iq), _ptr(ik_cache), _ptr(iw),
+                                   _ptr(gate), _ptr(pooled_cache), _ptr(out), _ptr(lse),
+                                   _ptr(sel), _ptr(nsel), _ptr(dev_err), _ptr(ws), ws.numel(),
+                                   _stream(stream))
+    _lib.check(st, "qsa_decode_fp8")
+    return {"out": out, "lse": lse, "sel": sel, "nsel": nsel}

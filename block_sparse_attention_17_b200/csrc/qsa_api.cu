@@ -414,7 +414,7 @@ static qsa_status decode_impl(const qsa_config* cfg, int batch, int n_q, int cap
                       const void* ik_cache, const float* iw, const void* gate,
                       float* pooled_cache, void* out, float* lse, int32_t* sel, int32_t* nsel,
                       int32_t* dev_err, void* workspace, size_t workspace_bytes, void* stream,
-                      Pages pg) {
+                      Pages pg, Fp8Kv f8 = Fp8Kv()) {
   qsa_status s = check_decode_dims(cfg, batch, n_q, cap);
   if (s != QSA_OK) return s;
   if (batch == 0) return QSA_OK;
@@ -442,7 +442,7 @@ static qsa_status decode_impl(const qsa_config* cfg, int batch, int n_q, int cap
     QSA_CUDA(launch_attn_decode_mma(g, batch, n_q, cap, w.nsplit, w.per_split, kv_len, q,
                                     k_cache, v_cache, gate, sel_p, nsel_p, w.part_ml, w.part_o,
                                     w.counters + batch, out, lse, dev_err ? dev_err : w.err, st,
-                                    pg, w.counters + (size_t)batch * (1 + g.Hkv)),
+                                    pg, w.counters + (size_t)batch * (1 + g.Hkv), f8),
              "decode attention");
   } else {
     QSA_CUDA(launch_attn_decode_simt(cfg->dtype, g, batch, n_q, cap, w.nsplit, w.per_split,
@@ -463,6 +463,33 @@ qsa_status qsa_decode(const qsa_config* cfg, int batch, int n_q, int cap, const 
   return decode_impl(cfg, batch, n_q, cap, kv_len, q, k_cache, v_cache, iq, ik_cache, iw, gate,
                      pooled_cache, out, lse, sel, nsel, dev_err, workspace, workspace_bytes,
                      stream, Pages());
+}
+
+qsa_status qsa_decode_fp8(const qsa_config* cfg, int batch, int n_q, int cap,
+                          const int32_t* kv_len, const void* q, const void* k_cache,
+                          const float* k_scale, const void* v_cache, const float* v_scale,
+                          int rotated, const void* iq, const void* ik_cache, const float* iw,
+                          const void* gate, float* pooled_cache, void* out, float* lse,
+                          int32_t* sel, int32_t* nsel, int32_t* dev_err, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  g_err[0] = 0;
+  qsa_status s = check_cfg(cfg);
+  if (s != QSA_OK) return s;
+  const Geom g = make_geom(cfg);
+  if (cfg->dtype != QSA_BF16 || !attn_decode_fp8_supported(g, n_q))
+    return fail(QSA_ERR_UNSUPPORTED,
+                "fp8 decode needs bf16 activations, head_dim 128, Hkv <= 8 and n_q * group <= 16");
+  if (batch == 0) return QSA_OK;
+  QSA_REQUIRE(k_scale, "k_scale");
+  QSA_REQUIRE(v_scale, "v_scale");
+  Fp8Kv f8;
+  f8.on = true;
+  f8.k_scale = k_scale;
+  f8.v_scale = v_scale;
+  f8.rotated = rotated ? 1 : 0;
+  return decode_impl(cfg, batch, n_q, cap, kv_len, q, k_cache, v_cache, iq, ik_cache, iw, gate,
+                     pooled_cache, out, lse, sel, nsel, dev_err, workspace, workspace_bytes,
+                     stream, Pages(), f8);
 }
 
 static qsa_status check_pages(const qsa_config* cfg, int max_blocks, const int32_t* block_table,

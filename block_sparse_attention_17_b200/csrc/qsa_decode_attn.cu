@@ -38,6 +38,20 @@ constexpr int kThreads = 32 * (kConsumers + 1);
 constexpr int kQStride = kD * 2 + 16;           // padded bf16 row of Q in shared memory
 constexpr int kMaxUnion = 4 * (kMaxTopK + 1);
 
+// fp8 caches: a stage holds the K and V rows as e4m3 bytes (one 128-byte box
+// each) and the 64 rows' scales for every KV head (K, then V); each consumer
+// warp widens its 16 keys into its own fp16 K and V tiles before its MMAs.
+constexpr int kMaxHkvFp8 = 8;
+constexpr int kF8BoxBytes = kChunk * kD;                      // 64 keys x 128 e4m3
+constexpr int kF8ScaleBytes = kChunk * kMaxHkvFp8 * 4;       // 64 rows x Hkv fp32
+constexpr int kF8StageBytes = 2 * kF8BoxBytes + 2 * kF8ScaleBytes;
+constexpr int kWarpTileBytes = 16 * 128 * 2;                  // 16 keys x 128 fp16: two 2 KB boxes
+constexpr int kF8ConvBytes = kConsumers * 2 * kWarpTileBytes; // [warp][K, V]
+static_assert(kStages * kF8StageBytes + kF8ConvBytes >= kConsumers * 16 * kD * 4 + 512,
+              "the fp8 layout must hold the partial-merge scratch");
+static_assert(kStages * kF8StageBytes + kF8ConvBytes <= kStages * kStageBytes,
+              "the fp8 layout fits in the bf16 ring's space");
+
 constexpr int kOffStages = 0;
 constexpr int kOffQ = kOffStages + kStages * kStageBytes;
 constexpr int kOffBar = kOffQ + 16 * kQStride;
@@ -62,6 +76,9 @@ struct DecParams {
   int* err;
   const int* table;                  // paged caches: [batch, cap / B] page ids, else null
   const int* ready;                  // [batch] selection-written flags, else null
+  const float* k_scale;              // fp8 caches: [batch, cap, Hkv] fp32 row scales
+  const float* v_scale;
+  int rotated;                       // fp8 caches hold H k and H v (Walsh-Hadamard, order D)
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
@@ -89,6 +106,56 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+__device__ __forceinline__ void mma_f16(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack2h(float a, float b) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+  return r;
+}
+// two e4m3 codes (low byte first) -> fp16x2 times an fp16x2 scale
+__device__ __forceinline__ uint32_t e4m3x2_scaled(uint32_t two_bytes, uint32_t scale2) {
+  uint32_t h, r;
+  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}"
+      : "=r"(h) : "r"(two_bytes));
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(h), "r"(scale2));
+  return r;
+}
+
+// Byte offset of (row, dim) in a warp's 16-row fp16 tile (two 128-byte-swizzled
+// boxes of 64 dims, as tile_off); dim must be a multiple of 8.
+__device__ __forceinline__ uint32_t tile16_off(int row, int dim) {
+  const int box = dim >> 6;
+  const int chunk = (dim & 63) >> 3;
+  return box * 2048 + row * 128 + ((chunk ^ (row & 7)) << 4);
+}
+
+// In-place orthonormal Walsh-Hadamard transform of nrows rows of 128 floats
+// (row stride 128) by nthr threads that synchronise with `sync` between the
+// 7 butterfly stages; the result is scaled by 128^-1/2.
+template <typename Sync>
+__device__ __forceinline__ void fwht128_rows(float* rows, int nrows, int tid, int nthr, Sync sync) {
+  for (int h = 1; h < kD; h <<= 1) {
+    for (int e = tid; e < nrows * (kD / 2); e += nthr) {
+      const int r = e / (kD / 2), p = e % (kD / 2);
+      const int i = (p / h) * 2 * h + (p % h);
+      float* row = rows + r * kD;
+      const float a = row[i], c = row[i + h];
+      row[i] = a + c;
+      row[i + h] = a - c;
+    }
+    sync();
+  }
+  const float norm = 0.08838834764831845f;   // 128^-1/2
+  for (int e = tid; e < nrows * kD; e += nthr) rows[e] *= norm;
+  sync();
+}
+
 // Byte offset of (row, dim) in a 64-row K/V tile stored as two 128-byte-swizzled
 // TMA boxes (dims 0..63, then 64..127); dim must be a multiple of 8.
 __device__ __forceinline__ uint32_t tile_off(int row, int dim) {
@@ -97,6 +164,7 @@ __device__ __forceinline__ uint32_t tile_off(int row, int dim) {
   return box * kBoxBytes + row * 128 + ((chunk ^ (row & 7)) << 4);
 }
 
+template <bool kFp8>
 __global__ void __launch_bounds__(kThreads, 2)
 attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const DecParams P) {
@@ -145,15 +213,39 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
   }
   // Q rows r = i * G + gi (query i, head hk * G + gi), zero beyond R: Q is an
   // input, so it is loaded before waiting for the selection kernel
-  for (int e = threadIdx.x; e < 16 * (kD / 8); e += blockDim.x) {
-    const int r = e / (kD / 8), c8 = e % (kD / 8);
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (r < R) {
-      const int i = r / G, gi = r % G;
-      v = *reinterpret_cast<const uint4*>(
-          P.q + (((size_t)b * n_q + i) * g.Hq + hk * G + gi) * kD + c8 * 8);
+  if constexpr (!kFp8) {
+    for (int e = threadIdx.x; e < 16 * (kD / 8); e += blockDim.x) {
+      const int r = e / (kD / 8), c8 = e % (kD / 8);
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (r < R) {
+        const int i = r / G, gi = r % G;
+        v = *reinterpret_cast<const uint4*>(
+            P.q + (((size_t)b * n_q + i) * g.Hq + hk * G + gi) * kD + c8 * 8);
+      }
+      *reinterpret_cast<uint4*>(smem + kOffQ + r * kQStride + c8 * 16) = v;
     }
-    *reinterpret_cast<uint4*>(smem + kOffQ + r * kQStride + c8 * 16) = v;
+  } else {
+    // fp32 rows in the (still unused) fp16 tile area, rotated into the cache's
+    // basis (q' = H q) when the cache holds H k, then stored as fp16
+    float* qf = reinterpret_cast<float*>(smem + kOffStages + kStages * kF8StageBytes);
+    for (int e = threadIdx.x; e < 16 * kD; e += blockDim.x) {
+      const int r = e / kD, d = e - r * kD;
+      float v = 0.f;
+      if (r < R) {
+        const int i = r / G, gi = r % G;
+        v = __bfloat162float(P.q[(((size_t)b * n_q + i) * g.Hq + hk * G + gi) * kD + d]);
+      }
+      qf[e] = v;
+    }
+    __syncthreads();
+    if (P.rotated) fwht128_rows(qf, 16, (int)threadIdx.x, (int)blockDim.x, [] { __syncthreads(); });
+    for (int e = threadIdx.x; e < 16 * (kD / 8); e += blockDim.x) {
+      const int r = e / (kD / 8), c8 = e % (kD / 8);
+      const float* src = qf + r * kD + c8 * 8;
+      const uint4 v = make_uint4(pack2h(src[0], src[1]), pack2h(src[2], src[3]),
+                                 pack2h(src[4], src[5]), pack2h(src[6], src[7]));
+      *reinterpret_cast<uint4*>(smem + kOffQ + r * kQStride + c8 * 16) = v;
+    }
   }
   // the merging CTA's gate rows: fetch them into L2 now
   if (split == 0 && !g.gate_headwise && threadIdx.x < R * (kD * 2 / 128)) {
@@ -251,12 +343,25 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
         // reported it)
         const int rowk = P.table ? P.table[(size_t)b * (P.cap / g.B) + blk] * g.B + off
                                  : (int)(krow_base + (size_t)blk * g.B + off);
-        const uint32_t st = sbase + kOffStages + s * kStageBytes;
-        mbar_expect_tx(&full[s], kStageBytes);
-        tma_load_3d(st, &tmK, 0, hk, rowk, &full[s]);
-        tma_load_3d(st + kBoxBytes, &tmK, 64, hk, rowk, &full[s]);
-        tma_load_3d(st + kTileBytes, &tmV, 0, hk, rowk, &full[s]);
-        tma_load_3d(st + kTileBytes + kBoxBytes, &tmV, 64, hk, rowk, &full[s]);
+        if constexpr (!kFp8) {
+          const uint32_t st = sbase + kOffStages + s * kStageBytes;
+          mbar_expect_tx(&full[s], kStageBytes);
+          tma_load_3d(st, &tmK, 0, hk, rowk, &full[s]);
+          tma_load_3d(st + kBoxBytes, &tmK, 64, hk, rowk, &full[s]);
+          tma_load_3d(st + kTileBytes, &tmV, 0, hk, rowk, &full[s]);
+          tma_load_3d(st + kTileBytes + kBoxBytes, &tmV, 64, hk, rowk, &full[s]);
+        } else {
+          // e4m3 rows (one 128-byte box each) and the chunk's row scales of all
+          // KV heads (64 * Hkv contiguous floats: rowk is a multiple of 64)
+          const uint32_t st = sbase + kOffStages + s * kF8StageBytes;
+          const uint32_t sb = 64u * g.Hkv * 4u;
+          mbar_expect_tx(&full[s], 2 * kF8BoxBytes + 2 * sb);
+          tma_load_3d(st, &tmK, 0, hk, rowk, &full[s]);
+          tma_load_3d(st + kF8BoxBytes, &tmV, 0, hk, rowk, &full[s]);
+          bulk_load(st + 2 * kF8BoxBytes, P.k_scale + (size_t)rowk * g.Hkv, sb, &full[s]);
+          bulk_load(st + 2 * kF8BoxBytes + kF8ScaleBytes, P.v_scale + (size_t)rowk * g.Hkv, sb,
+                    &full[s]);
+        }
         issued = c + 1;
       }
       for (int c = max(0, issued - kStages); c < issued; ++c)
@@ -294,12 +399,52 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
     for (int c = 0; c < my_chunks; ++c) {
       const int s = c % kStages;
       if (!mbar_wait(&full[s], (c / kStages) & 1, abort_flag)) break;
-      const uint32_t kt = sbase + kOffStages + s * kStageBytes;
-      const uint32_t vt = kt + kTileBytes;
       const int uc = c0 + c;
       const int ub = uc / cpb;
       const int blk = u_blk[ub], qm = u_qm[ub];
       const int key0 = blk * g.B + (uc % cpb) * kChunk;
+      // Keys no row of this CTA may see are not part of any selection (the
+      // tail block's keys past the newest query): their V rows are zeroed so
+      // that P = 0 cannot meet a non-finite V in the MMA.
+      int lim_all = 0;
+      for (int i = 0; i < n_q; ++i)
+        if ((qm >> i) & 1) lim_all = max(lim_all, min(kChunk, max(0, kv - n_q + i + 1 - key0)));
+      uint32_t kt, vt;   // this warp's K and V tiles (64-key bf16 tiles, or 16-key fp16 tiles)
+      if constexpr (!kFp8) {
+        kt = sbase + kOffStages + s * kStageBytes;
+        vt = kt + kTileBytes;
+      } else {
+        // widen this warp's 16 keys (rows 16w .. 16w + 15 of the chunk) from
+        // e4m3 times the row scale into fp16, then release the stage
+        const uint32_t st8 = kOffStages + s * kF8StageBytes;
+        const float* ks = reinterpret_cast<const float*>(smem + st8 + 2 * kF8BoxBytes);
+        const float* vs = reinterpret_cast<const float*>(smem + st8 + 2 * kF8BoxBytes + kF8ScaleBytes);
+        const uint32_t tiles = kOffStages + kStages * kF8StageBytes + warp * 2 * kWarpTileBytes;
+        kt = sbase + tiles;
+        vt = kt + kWarpTileBytes;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int u = lane + 32 * i;
+          const int which = u >> 7, rr = (u >> 3) & 15, ch = u & 7;   // K/V, row, 16-dim chunk
+          const int row = warp * 16 + rr;                               // row in the chunk
+          uint4 out0 = make_uint4(0, 0, 0, 0), out1 = make_uint4(0, 0, 0, 0);
+          if (!(which == 1 && row >= lim_all)) {
+            const uint4 in = *reinterpret_cast<const uint4*>(
+                smem + st8 + which * kF8BoxBytes + row * 128 + ((ch ^ (row & 7)) << 4));
+            const float scl = (which ? vs : ks)[row * g.Hkv + hk];
+            const uint32_t s2 = pack2h(scl, scl);
+            out0 = make_uint4(e4m3x2_scaled(in.x & 0xffffu, s2), e4m3x2_scaled(in.x >> 16, s2),
+                              e4m3x2_scaled(in.y & 0xffffu, s2), e4m3x2_scaled(in.y >> 16, s2));
+            out1 = make_uint4(e4m3x2_scaled(in.z & 0xffffu, s2), e4m3x2_scaled(in.z >> 16, s2),
+                              e4m3x2_scaled(in.w & 0xffffu, s2), e4m3x2_scaled(in.w >> 16, s2));
+          }
+          uint8_t* dst = smem + tiles + which * kWarpTileBytes;
+          *reinterpret_cast<uint4*>(dst + tile16_off(rr, 16 * ch)) = out0;
+          *reinterpret_cast<uint4*>(dst + tile16_off(rr, 16 * ch + 8)) = out1;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+      }
       // visible keys of this chunk per held row: keys key0 + j with j < lim
       int lim[2];
 #pragma unroll
@@ -312,10 +457,17 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         uint32_t b0, b1, b2, b3;
-        const int key = warp * 16 + (mi >> 1) * 8 + ri;
-        ldsm_x4(kt + tile_off(key, kk * 16 + (mi & 1) * 8), b0, b1, b2, b3);
-        mma_bf16(sfr[0], qa[kk], b0, b1);
-        mma_bf16(sfr[1], qa[kk], b2, b3);
+        if constexpr (!kFp8) {
+          const int key = warp * 16 + (mi >> 1) * 8 + ri;
+          ldsm_x4(kt + tile_off(key, kk * 16 + (mi & 1) * 8), b0, b1, b2, b3);
+          mma_bf16(sfr[0], qa[kk], b0, b1);
+          mma_bf16(sfr[1], qa[kk], b2, b3);
+        } else {
+          const int key = (mi >> 1) * 8 + ri;
+          ldsm_x4(kt + tile16_off(key, kk * 16 + (mi & 1) * 8), b0, b1, b2, b3);
+          mma_f16(sfr[0], qa[kk], b0, b1);
+          mma_f16(sfr[1], qa[kk], b2, b3);
+        }
       }
       // mask, scale, online softmax (per row across the quad's 4 threads)
       float x[2][4];
@@ -354,13 +506,7 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
         o[i][2] *= alpha[1];
         o[i][3] *= alpha[1];
       }
-      // Keys no row of this CTA may see are not part of any selection (the
-      // tail block's keys past the newest query): their V rows are zeroed so
-      // that P = 0 cannot meet a non-finite V in the MMA.
-      int lim_all = 0;
-      for (int i = 0; i < n_q; ++i)
-        if ((qm >> i) & 1) lim_all = max(lim_all, min(kChunk, max(0, kv - n_q + i + 1 - key0)));
-      if (lim_all < warp * 16 + 16) {
+      if (!kFp8 && lim_all < warp * 16 + 16) {
         for (int e = lane; e < 16 * 16; e += 32) {   // 16 rows x 2 boxes x 8 chunks of 16 B
           const int row = warp * 16 + (e >> 4);
           const int box = (e >> 3) & 1, ch = e & 7;
@@ -372,21 +518,35 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
       }
       // P as the A fragment of a 16x16 (rows x keys) tile
       uint32_t pa[4];
-      pa[0] = pack2(x[0][0], x[0][1]);
-      pa[1] = pack2(x[0][2], x[0][3]);
-      pa[2] = pack2(x[1][0], x[1][1]);
-      pa[3] = pack2(x[1][2], x[1][3]);
+      if constexpr (!kFp8) {
+        pa[0] = pack2(x[0][0], x[0][1]);
+        pa[1] = pack2(x[0][2], x[0][3]);
+        pa[2] = pack2(x[1][0], x[1][1]);
+        pa[3] = pack2(x[1][2], x[1][3]);
+      } else {
+        pa[0] = pack2h(x[0][0], x[0][1]);
+        pa[1] = pack2h(x[0][2], x[0][3]);
+        pa[2] = pack2h(x[1][0], x[1][1]);
+        pa[3] = pack2h(x[1][2], x[1][3]);
+      }
       // O += P V over the warp's 16 keys, 16 n-tiles of 8 dims
 #pragma unroll
       for (int dn = 0; dn < 16; dn += 2) {
         uint32_t b0, b1, b2, b3;
-        const int key = warp * 16 + (mi & 1) * 8 + ri;
-        ldsm_x4_t(vt + tile_off(key, dn * 8 + (mi >> 1) * 8), b0, b1, b2, b3);
-        mma_bf16(o[dn], pa, b0, b1);
-        mma_bf16(o[dn + 1], pa, b2, b3);
+        if constexpr (!kFp8) {
+          const int key = warp * 16 + (mi & 1) * 8 + ri;
+          ldsm_x4_t(vt + tile_off(key, dn * 8 + (mi >> 1) * 8), b0, b1, b2, b3);
+          mma_bf16(o[dn], pa, b0, b1);
+          mma_bf16(o[dn + 1], pa, b2, b3);
+        } else {
+          const int key = (mi & 1) * 8 + ri;
+          ldsm_x4_t(vt + tile16_off(key, dn * 8 + (mi >> 1) * 8), b0, b1, b2, b3);
+          mma_f16(o[dn], pa, b0, b1);
+          mma_f16(o[dn + 1], pa, b2, b3);
+        }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
+      if (!kFp8 && lane == 0) mbar_arrive(&empty[s]);
     }
     // merge the four warps' states through shared memory (the ring is free)
 #pragma unroll
@@ -414,6 +574,10 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
     // thread t of the 128 consumers: row t / 8, dims [16 (t % 8), + 16)
     const int t = threadIdx.x;
     const int r = t >> 3, d0 = (t & 7) * 16;
+    // a rotated fp8 cache gives O' = H O: the merged rows are rotated back
+    // (H is symmetric and orthonormal) before they leave as the partial
+    float* urow = sm + kConsumers * 16 * 2;                    // [16 rows][128]
+    const bool unrotate = kFp8 && P.rotated;
     if (r < R) {
       float M = -INFINITY;
 #pragma unroll
@@ -425,7 +589,7 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
         wsc[w] = mw == -INFINITY ? 0.f : ex2_approx(mw - M);
         L += sm[(w * 16 + r) * 2 + 1] * wsc[w];
       }
-      float* dst = P.part_o + (row0 + r) * kD + d0;
+      float* dst = unrotate ? urow + r * kD + d0 : P.part_o + (row0 + r) * kD + d0;
 #pragma unroll
       for (int d = 0; d < 16; d += 4) {
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -442,6 +606,16 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
       if ((t & 7) == 0) {
         P.part_ml[2 * (row0 + r)] = M;
         P.part_ml[2 * (row0 + r) + 1] = L;
+      }
+    }
+    if (unrotate) {
+      named_bar_sync(1, 32 * kConsumers);
+      fwht128_rows(urow, R, t, 32 * kConsumers, [] { named_bar_sync(1, 32 * kConsumers); });
+      if (r < R) {
+        float* gdst = P.part_o + (row0 + r) * kD + d0;
+#pragma unroll
+        for (int d = 0; d < 16; d += 4)
+          *reinterpret_cast<float4*>(gdst + d) = *reinterpret_cast<const float4*>(urow + r * kD + d0 + d);
       }
     }
   }
@@ -575,7 +749,25 @@ bool make_cache_map(CUtensorMap* m, const void* ptr, int Hkv, long long rows) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D uint8 map over [rows, Hkv, D] e4m3 codes with a (128, 1, 64) box: one
+// 128-byte row per key.
+bool make_cache_map_u8(CUtensorMap* m, const void* ptr, int Hkv, long long rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)Hkv, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)kD, (cuuint64_t)Hkv * kD};
+  cuuint32_t box[3] = {(cuuint32_t)kD, 1, (cuuint32_t)kChunk};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
+
+bool attn_decode_fp8_supported(const Geom& g, int n_q) {
+  return attn_decode_mma_supported(g, n_q) && g.Hkv <= kMaxHkvFp8;
+}
 
 bool attn_decode_mma_supported(const Geom& g, int n_q) {
   return g.D == kD && g.B % kChunk == 0 && n_q * g.G <= 16 && n_q <= 4;
@@ -597,12 +789,13 @@ cudaError_t launch_attn_decode_mma(const Geom& g, int batch, int n_q, int cap, i
                                    const void* kc, const void* vc, const void* gate,
                                    const int* sel, const int* nsel, float* part_ml,
                                    float* part_o, int* counter, void* out, float* lse, int* err,
-                                   cudaStream_t st, Pages pg, const int* ready) {
+                                   cudaStream_t st, Pages pg, const int* ready, Fp8Kv f8) {
   if (batch == 0) return cudaSuccess;
   CUtensorMap mk, mv;
   const long long rows = pg.table ? (long long)pg.num_pages * g.B : (long long)batch * cap;
-  if (!make_cache_map(&mk, kc, g.Hkv, rows) || !make_cache_map(&mv, vc, g.Hkv, rows))
-    return cudaErrorInvalidValue;
+  const bool ok = f8.on ? make_cache_map_u8(&mk, kc, g.Hkv, rows) && make_cache_map_u8(&mv, vc, g.Hkv, rows)
+                        : make_cache_map(&mk, kc, g.Hkv, rows) && make_cache_map(&mv, vc, g.Hkv, rows);
+  if (!ok) return cudaErrorInvalidValue;
   DecParams p;
   p.g = g;
   p.n_q = n_q;
@@ -622,12 +815,15 @@ cudaError_t launch_attn_decode_mma(const Geom& g, int batch, int n_q, int cap, i
   p.err = err;
   p.table = pg.table;
   p.ready = ready;
+  p.k_scale = f8.k_scale;
+  p.v_scale = f8.v_scale;
+  p.rotated = f8.rotated;
   const int words = (cap / g.B + 31) / 32;
   const int smem = kOffBits + 4 * n_q * words + 1024;
-  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(attn_decode_mma_kernel), smem);
+  auto kern = f8.on ? attn_decode_mma_kernel<true> : attn_decode_mma_kernel<false>;
+  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
-  e = launch_dependent(attn_decode_mma_kernel, dim3(nsplit, batch, g.Hkv), dim3(kThreads), smem, st,
-                       mk, mv, p);
+  e = launch_dependent(kern, dim3(nsplit, batch, g.Hkv), dim3(kThreads), smem, st, mk, mv, p);
   note_launch();
   return e;
 }

@@ -31,6 +31,16 @@ cudaError_t set_max_dynamic_smem(const void* func, int bytes);
 // SM count of the current device (cached per function, device and shape).
 cudaError_t resident_ctas(const void* func, int threads, size_t smem, int* per_sm, int* sms);
 
+// fp8 (e4m3) K/V caches for the decode attention: one fp32 scale per
+// (token, KV head) row, [batch, cap, Hkv]; rotated != 0 when the caches hold
+// H k and H v for the orthonormal Walsh-Hadamard matrix H of order D.
+struct Fp8Kv {
+  bool on = false;
+  const float* k_scale = nullptr;
+  const float* v_scale = nullptr;
+  int rotated = 0;
+};
+
 // ready: [batch] flags the selection kernel sets (release) once a sequence's
 // selections are written, zero before the launch; the decode attention kernel
 // waits on its sequence's flag instead of on the whole selection grid.
@@ -99,7 +109,9 @@ cudaError_t launch_attn_decode_mma(const Geom& g, int batch, int n_q, int cap, i
                                    const void* kc, const void* vc, const void* gate,
                                    const int* sel, const int* nsel, float* part_ml,
                                    float* part_o, int* counter, void* out, float* lse, int* err,
-                                   cudaStream_t st, Pages pg = Pages(), const int* ready = nullptr);
+                                   cudaStream_t st, Pages pg = Pages(), const int* ready = nullptr,
+                                   Fp8Kv f8 = Fp8Kv());
+bool attn_decode_fp8_supported(const Geom& g, int n_q);
 bool attn_prefill_tc_supported(const Geom& g);
 cudaError_t launch_attn_prefill_tc(const Geom& g, const int* cu, int batch, int total_tokens,
                                    int max_seqlen, int words, const uint32_t* bitmask,

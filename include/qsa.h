@@ -225,6 +225,33 @@ qsa_status qsa_decode_paged(const qsa_config* cfg, int batch, int n_q, int max_b
                             int32_t* sel, int32_t* nsel, int32_t* dev_err, void* workspace,
                             size_t workspace_bytes, void* stream);
 
+/* ------------------------------------------------------------ fp8 decode --
+ * qsa_decode over fp8 K/V caches (ramgpt "Porting Qwen4 to llama.cpp",
+ * section "Quantized KV Is a Representation Contract": quantized K/V may be
+ * stored in a Hadamard-rotated basis, and a fast attention path must honour
+ * that storage contract).
+ *   k_cache/v_cache [batch, cap, Hkv, D] uint8: e4m3 codes (OCP FP8 E4M3,
+ *                   no infinities; code 0x7F/0xFF is NaN)
+ *   k_scale/v_scale [batch, cap, Hkv] fp32: the row (token, KV head) stands
+ *                   for scale * decode(code), elementwise over D
+ *   rotated         0: the rows are k and v; non-zero: they are H k and H v
+ *                   for the orthonormal Walsh-Hadamard matrix of order D
+ *                   (Sylvester order, scaled by D^-1/2). The query is
+ *                   rotated and the output rotated back inside the kernel, so
+ *                   out is the attention over k and v either way.
+ * q, gate, iq, ik_cache and the rest are as for qsa_decode (bf16; the indexer
+ * path is unchanged); the workspace is qsa_decode_workspace_size's. K/V are
+ * widened to fp16 times the scale before the MMAs; accumulation is fp32.
+ * Supported: bf16 config, head_dim 128, Hkv <= 8, n_q * (Hq / Hkv) <= 16;
+ * otherwise QSA_ERR_UNSUPPORTED. */
+qsa_status qsa_decode_fp8(const qsa_config* cfg, int batch, int n_q, int cap,
+                          const int32_t* kv_len, const void* q, const void* k_cache,
+                          const float* k_scale, const void* v_cache, const float* v_scale,
+                          int rotated, const void* iq, const void* ik_cache, const float* iw,
+                          const void* gate, float* pooled_cache, void* out, float* lse,
+                          int32_t* sel, int32_t* nsel, int32_t* dev_err, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
 /* qsa_pool_build for a paged indexer-key cache (arguments as for
  * qsa_decode_paged); the rows it writes are bit-identical to qsa_pool_build's
  * on the same rows laid out contiguously. A bad page id sets *dev_err to 3
