@@ -434,6 +434,26 @@ static qsa_status decode_impl(const qsa_config* cfg, int batch, int n_q, int cap
   int* sel_p = sel ? sel : w.sel;
   int* nsel_p = nsel ? nsel : w.nsel;
   stage_mark(0, st);
+  const bool vec_ok = (((uintptr_t)iq | (uintptr_t)ik_cache | (uintptr_t)pooled_cache) & 15u) == 0;
+  if (decode_uses_mma(cfg, g, n_q) && vec_ok &&
+      decode_fused_supported(g, n_q, cap, w.nsplit, f8.on)) {
+    // one launch: each (sequence, KV head) cluster pools, scores and selects,
+    // then gathers K/V and merges its partials
+    stage_mark(1, st);
+    DecodeSelIn si;
+    si.iq = iq;
+    si.ik_cache = ik_cache;
+    si.iw = iw;
+    si.pooled = pooled_cache;
+    si.sel = sel_p;
+    si.nsel = nsel_p;
+    QSA_CUDA(launch_decode_fused(g, batch, n_q, cap, w.nsplit, w.per_split, kv_len, q, k_cache,
+                                 v_cache, gate, si, out, lse, dev_err ? dev_err : w.err, st, pg,
+                                 f8),
+             "decode");
+    stage_mark(2, st);
+    return QSA_OK;
+  }
   s = decode_select_common(cfg, g, batch, n_q, cap, kv_len, iq, ik_cache, iw, pooled_cache, w,
                            sel_p, nsel_p, nullptr, dev_err, st, pg);
   if (s != QSA_OK) return s;

@@ -14,11 +14,18 @@
 // heads), so the four consumer warps use warp-level bf16 MMAs (m16n8k16,
 // fp32 accumulation): warp w takes keys [16w, 16w + 16) of each chunk and
 // keeps its own online-softmax state (log2 domain); the four states are
-// merged at the end and written as one (m, l, O) partial per row; the last
-// CTA of each (sequence, KV head) merges the partials by log-sum-exp and
-// applies the sigmoid output gate.
+// merged at the end into one (m, l, O) partial per row. The CTAs of one
+// (sequence, KV head) form a thread-block cluster and merge their partials by
+// log-sum-exp through distributed shared memory (each CTA takes some rows),
+// applying the sigmoid output gate; where such a cluster cannot be resident,
+// the partials go through global memory and the last CTA merges them.
+#include <map>
+#include <mutex>
+#include <tuple>
+
 #include "qsa_common.cuh"
 #include "qsa_kernels.h"
+#include "qsa_pool.cuh"
 #include "qsa_sm100.cuh"
 
 namespace qsa {
@@ -37,6 +44,8 @@ constexpr int kConsumers = 4;
 constexpr int kThreads = 32 * (kConsumers + 1);
 constexpr int kQStride = kD * 2 + 16;           // padded bf16 row of Q in shared memory
 constexpr int kMaxUnion = 4 * (kMaxTopK + 1);
+constexpr int kMaxClusterSplits = 16;           // CTAs of one cluster-merged (sequence, KV head)
+constexpr int kSelRows = 128;                   // in-kernel selection: blocks per scoring pass
 
 // fp8 caches: a stage holds the K and V rows as e4m3 bytes (one 128-byte box
 // each) and the 64 rows' scales for every KV head (K, then V); each consumer
@@ -57,7 +66,8 @@ constexpr int kOffQ = kOffStages + kStages * kStageBytes;
 constexpr int kOffBar = kOffQ + 16 * kQStride;
 constexpr int kOffMisc = kOffBar + 8 * 2 * kStages;
 constexpr int kOffUnion = kOffMisc + 64;
-constexpr int kOffBits = kOffUnion + 8 * kMaxUnion;   // [n_q][cap / B / 32] words
+constexpr int kOffGate = kOffUnion + 8 * kMaxUnion;   // cluster merge: [16 rows][128] gate bf16
+constexpr int kOffBits = kOffGate + 16 * kD * 2;      // [n_q][cap / B / 32] words
 // dynamic shared memory: kOffBits + 4 * n_q * words + 1024 (alignment slack)
 
 struct DecParams {
@@ -79,6 +89,17 @@ struct DecParams {
   const float* k_scale;              // fp8 caches: [batch, cap, Hkv] fp32 row scales
   const float* v_scale;
   int rotated;                       // fp8 caches hold H k and H v (Walsh-Hadamard, order D)
+  int cluster;                       // the nsplit CTAs of a (sequence, KV head) form one
+                                     // cluster and merge through distributed shared memory
+  // selection inside the kernel (the cluster scores, pools and selects itself)
+  const __nv_bfloat16* iq;           // [batch, n_q, Hi, di]
+  const __nv_bfloat16* ik_cache;     // [batch * cap, di] (or pages)
+  const float* iw;                   // [batch, n_q, Hi]
+  float* pooled;                     // [batch, cap / B, di] pooled-key cache
+  int num_pages;                     // paged caches: pages in the pool
+  int* sel_w;                        // [batch, n_q, k + 1] selections out
+  int* nsel_w;                       // [batch, n_q]
+  int fo_keys, fo_kbar, fo_iq, fo_iw, fo_new, fo_hist;   // byte offsets in the ring's space
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
@@ -164,7 +185,373 @@ __device__ __forceinline__ uint32_t tile_off(int row, int dim) {
   return box * kBoxBytes + row * 128 + ((chunk ^ (row & 7)) << 4);
 }
 
-template <bool kFp8>
+// ------------------------------------------------- selection in the cluster
+// The k largest of keys[0 .. n) (shared memory), a lower position winning a
+// tie, written as a bitmap: bits[w] for w < ceil(n / 32), bit j % 32 of word
+// j / 32 set for a chosen position j. Radix select over the 32-bit keys: the
+// bits above the highest bit where the largest and smallest key differ are
+// common to all keys; below them, 8-bit digits, most significant first. Each
+// pass histograms the digit of the keys that still match the chosen prefix
+// (shared-memory atomics), warp 0 finds the digit value holding the k-th
+// largest key by a suffix scan, and the passes stop as soon as every key with
+// that digit value is taken. Otherwise the last pass ends on the k-th largest
+// key itself, and of the keys equal to it the lowest positions are taken.
+// hist: 256 ints, ctl: 16 ints of shared memory. All threads call it.
+__device__ __forceinline__ void cta_topk_radix(const uint32_t* keys, int n, int k, uint32_t* bits, int* hist,
+                               int* ctl) {
+  const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31, warp = tid >> 5;
+  const int nwarps = nthr >> 5;
+  const int nwords = (n + 31) >> 5;
+  if (n <= k) {
+    for (int w = tid; w < nwords; w += nthr)
+      bits[w] = (w == nwords - 1 && (n & 31)) ? ((1u << (n & 31)) - 1u) : 0xffffffffu;
+    __syncthreads();
+    return;
+  }
+  uint32_t hi = 0u, lo = 0xffffffffu;
+  for (int j = tid; j < n; j += nthr) {
+    const uint32_t key = keys[j];
+    hi = max(hi, key);
+    lo = min(lo, key);
+  }
+  hi = __reduce_max_sync(kFull, hi);
+  lo = __reduce_min_sync(kFull, lo);
+  if (lane == 0) {
+    ctl[4 + warp] = (int)hi;
+    ctl[10 + warp] = (int)lo;
+  }
+  for (int e = tid; e < 256; e += nthr) hist[e] = 0;
+  __syncthreads();
+  for (int w = 0; w < nwarps; ++w) {
+    hi = max(hi, (uint32_t)ctl[4 + w]);
+    lo = min(lo, (uint32_t)ctl[10 + w]);
+  }
+  const int top = hi == lo ? -1 : 31 - __clz(hi ^ lo);   // highest differing bit
+  uint32_t pmask = top < 0 ? 0xffffffffu : top == 31 ? 0u : ~((2u << top) - 1u);   // common bits
+  uint32_t prefix = hi & pmask;
+  int krem = k;
+  bool exact = false;
+  for (int shift = top - 7 > 0 ? top - 7 : 0; top >= 0; shift = shift - 8 > 0 ? shift - 8 : 0) {
+    const bool last = shift == 0;
+    if (shift != (top - 7 > 0 ? top - 7 : 0)) {
+      for (int e = tid; e < 256; e += nthr) hist[e] = 0;
+      __syncthreads();
+    }
+    for (int j = tid; j < n; j += nthr) {
+      const uint32_t key = keys[j];
+      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // lane l holds byte values 255 - 8l down to 248 - 8l
+      int c[8], sum = 0;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        c[t] = hist[255 - 8 * lane - t];
+        sum += c[t];
+      }
+      int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const int excl = incl - sum;
+      if (excl < krem && krem <= incl) {
+        int run = excl;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          if (run + c[t] >= krem) {
+            ctl[0] = 255 - 8 * lane - t;   // the byte value
+            ctl[1] = run;                  // keys above it
+            ctl[2] = c[t];                 // keys with it
+            break;
+          }
+          run += c[t];
+        }
+      }
+    }
+    __syncthreads();
+    const int dv = ctl[0], above = ctl[1], with = ctl[2];
+    krem -= above;
+    prefix |= (uint32_t)dv << shift;
+    pmask |= 0xffu << shift;
+    if (with == krem) {
+      exact = true;
+      break;
+    }
+    if (last) break;
+  }
+  // exact: the keys whose prefix bits are >= prefix (k of them); else the keys
+  // above the k-th largest, then its ties below
+  for (int w = warp; w < nwords; w += nwarps) {
+    const int j = w * 32 + lane;
+    bool take = false;
+    if (j < n) {
+      const uint32_t key = keys[j];
+      take = exact ? (key & pmask) >= prefix : key > prefix;
+    }
+    const uint32_t m = __ballot_sync(kFull, take);
+    if (lane == 0) bits[w] = m;
+  }
+  if (!exact) {
+    __syncthreads();
+    if (warp == 0) {
+      int left = krem;
+      for (int w = 0; w < nwords && left > 0; ++w) {
+        const int j = w * 32 + lane;
+        uint32_t m = __ballot_sync(kFull, j < n && keys[j] == prefix);
+        while (__popc(m) > left) m &= ~(1u << (31 - __clz(m)));   // keep the lowest `left`
+        if (lane == 0) bits[w] |= m;
+        left -= __popc(m);
+      }
+    }
+  }
+  __syncthreads();
+}
+
+__device__ __forceinline__ void cluster_arrive_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_all() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint4 ld_cluster_u32x4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr) : "memory");
+  return v;
+}
+
+// Chunk of candidate blocks one CTA of the cluster scores: a multiple of 4, so
+// that the gather below moves 16-byte groups owned by one CTA.
+__host__ __device__ __forceinline__ int select_range(int nc_last, int nsplit) {
+  const int per = ((nc_last > 1 ? nc_last : 1) + nsplit - 1) / nsplit;
+  return (per + 3) & ~3;
+}
+
+// The selection step of one decode step, done by the cluster of one (sequence,
+// KV head) before it gathers K and V (the indexer of the llama.cpp PR #27739
+// page, QSA composition commit; the pooled keys of the instagit MTPLX page).
+// CTA `split` owns candidate blocks [split * per, (split + 1) * per): it pools
+// the blocks of its range that this step's tokens complete (writing them to the
+// pooled-key cache once, from the KV head 0 cluster), scores its blocks for
+// every query, s = c * sum_h w_h relu(q_h . kbar) (one thread per (query,
+// block, head), the heads summed by shuffles; the same arithmetic as the
+// selection kernel), and keeps the score keys in its shared memory. After a
+// cluster barrier every CTA gathers each query's keys from all CTAs, selects
+// the top k (cta_topk_radix) into the query's bitmap and adds the tail block;
+// CTA (0, b, 0) also writes the selection lists. Ends with this CTA's arrival
+// on the cluster barrier that the caller waits on before reusing the space.
+// Starts moving what select_in_cluster reads into L2 (bulk prefetches by one
+// thread): the CTA's range of pooled rows, the indexer rows of the blocks this
+// step completes, and the queries' indexer q.
+template <int kDI>
+__device__ __forceinline__ void select_prefetch(const DecParams& P, int kv, int split, int b) {
+  const Geom& g = P.g;
+  const int nblk_cap = P.cap / g.B, nc_last = kv / g.B;
+  const int per = select_range(nc_last, P.nsplit);
+  const int j0 = split * per, j1 = min(nc_last, j0 + per);
+  if (j1 > j0)
+    bulk_prefetch_l2(P.pooled + ((size_t)b * nblk_cap + j0) * kDI, (uint32_t)(j1 - j0) * kDI * 4u);
+  const int jn_lo = max((kv - P.n_q) / g.B, j0), jn_hi = min(nc_last, j1);
+  for (int j = jn_lo; j < jn_hi; ++j) {
+    size_t r0 = (size_t)b * P.cap + (size_t)j * g.B;
+    if (P.table) {
+      const int page = P.table[(size_t)b * nblk_cap + j];
+      if (page < 0 || page >= P.num_pages) continue;
+      r0 = (size_t)page * g.B;
+    }
+    bulk_prefetch_l2(P.ik_cache + r0 * kDI, (uint32_t)g.B * kDI * 2u);
+  }
+  if (split == 0 || j1 > j0)
+    bulk_prefetch_l2(P.iq + (size_t)b * P.n_q * g.Hi * kDI, (uint32_t)(P.n_q * g.Hi * kDI * 2));
+}
+
+template <int kDI>
+__device__ __forceinline__ void select_in_cluster(const DecParams& P, uint8_t* smem, int kv, int split, int b,
+                                  int hk, uint32_t* qbits, int words) {
+  constexpr int kStride = kDI + 4;                 // 16-byte rows; 8 rows of a warp hit distinct banks
+  constexpr int kQStrideI = kDI + 4;
+  constexpr int kRows = kSelRows;                 // candidate blocks per scoring pass
+  const Geom& g = P.g;
+  const int n_q = P.n_q, Hi = g.Hi, k = g.k, kp1 = k + 1;
+  const int tid = threadIdx.x, nthr = blockDim.x, warp = tid >> 5, lane = tid & 31;
+  const int nblk_cap = P.cap / g.B;
+  const int nc_last = kv / g.B;
+  const int per = select_range(nc_last, P.nsplit);
+  const int j0 = split * per, j1 = min(nc_last, j0 + per);
+  uint8_t* ring = smem + kOffStages;
+  uint32_t* keys_mine = reinterpret_cast<uint32_t*>(ring);                  // [n_q][per]
+  uint32_t* keys_all = reinterpret_cast<uint32_t*>(ring + P.fo_keys);       // [nblk_cap]
+  float* kbar_s = reinterpret_cast<float*>(ring + P.fo_kbar);               // [kRows][kStride]
+  float* iq_s = reinterpret_cast<float*>(ring + P.fo_iq);                   // [n_q][Hi][kDI]
+  float* iw_s = reinterpret_cast<float*>(ring + P.fo_iw);                   // [n_q][Hi]
+  float* new_s = reinterpret_cast<float*>(ring + P.fo_new);                 // [2][kDI]
+  int* hist = reinterpret_cast<int*>(ring + P.fo_hist);                     // [256] + ctl [16]
+  float2(*part)[32] = reinterpret_cast<float2(*)[32]>(hist + 272);           // [8][32]
+
+  // paged caches: every page the step may gather must be in the pool
+  if (P.table && hk == 0) {
+    const int nb_used = (kv + g.B - 1) / g.B;
+    for (int j = split + P.nsplit * tid; j < nb_used; j += P.nsplit * nthr) {
+      const int page = P.table[(size_t)b * nblk_cap + j];
+      if ((page < 0 || page >= P.num_pages) && P.err) atomicExch(P.err, 3);
+    }
+  }
+  __syncthreads();   // the caller staged iq_s and iw_s
+  // blocks completed by this step's tokens (at most two: n_q <= 4 < B)
+  const int jn_lo = max((kv - n_q) / g.B, j0), jn_hi = min(nc_last, j1);
+  for (int j = jn_lo; j < jn_hi; ++j) {
+    size_t r0 = (size_t)b * P.cap + (size_t)j * g.B;
+    bool ok = true;
+    if (P.table) {
+      const int page = P.table[(size_t)b * nblk_cap + j];
+      ok = page >= 0 && page < P.num_pages;
+      r0 = (size_t)page * g.B;
+    }
+    float* dst = new_s + (j - jn_lo) * kDI;
+    if (ok) {   // uniform across the CTA
+      pool_block<__nv_bfloat16>(P.ik_cache + (ok ? r0 : 0) * kDI, g.B, kDI, dst, part, nthr >> 5);
+    } else {    // a page outside the pool (reported): the cached row stands
+      for (int d = tid; d < kDI; d += nthr) dst[d] = P.pooled[((size_t)b * nblk_cap + j) * kDI + d];
+    }
+    __syncthreads();
+    if (hk == 0 && ok)
+      for (int d = tid; d < kDI; d += nthr) P.pooled[((size_t)b * nblk_cap + j) * kDI + d] = dst[d];
+  }
+  // score the range, kRows blocks at a time
+  for (int r0 = j0; r0 < j1; r0 += kRows) {
+    const int rows = min(kRows, j1 - r0);
+    {   // every load of the pass is issued before the first store
+      constexpr int kLd = (kRows * (kDI / 4) + kThreads - 1) / kThreads;   // float4 per thread
+      float4 v[kLd];
+#pragma unroll
+      for (int u = 0; u < kLd; ++u) {
+        const int e = tid + u * kThreads;
+        const int r = e / (kDI / 4), d4 = e - r * (kDI / 4);
+        const int j = r0 + r;
+        v[u] = r >= rows ? make_float4(0.f, 0.f, 0.f, 0.f)
+               : (j >= jn_lo && j < jn_hi)
+                   ? *reinterpret_cast<const float4*>(new_s + (j - jn_lo) * kDI + 4 * d4)
+                   : __ldg(reinterpret_cast<const float4*>(P.pooled + ((size_t)b * nblk_cap + j) * kDI) + d4);
+      }
+#pragma unroll
+      for (int u = 0; u < kLd; ++u) {
+        const int e = tid + u * kThreads;
+        const int r = e / (kDI / 4), d4 = e - r * (kDI / 4);
+        if (r < rows) *reinterpret_cast<float4*>(kbar_s + r * kStride + 4 * d4) = v[u];
+      }
+    }
+    __syncthreads();
+    // Thread t takes head t % Hi of the (query, block) slots t / Hi + m * hpr
+    // (hpr = nthr / Hi; nthr is a multiple of Hi, so a slot's heads are adjacent
+    // lanes of one warp), two slots per pass. Each dot product is one fma chain
+    // over the dims in ascending order, as in the selection kernel; the heads'
+    // terms are summed by shuffles. iq rows are padded to kQStride floats so
+    // that the heads of a warp read distinct banks.
+    const int hpr = nthr / Hi, h = tid % Hi, slot = tid / Hi;
+    for (int base = 0; base < n_q * kRows; base += 2 * hpr) {
+      int ii[2], rr[2];
+      bool live[2];
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const int sl = base + slot + t * hpr;
+        ii[t] = sl / kRows;
+        rr[t] = sl % kRows;
+        // block r0 + rr is complete for query ii: (r0 + rr + 1) B <= kv - n_q + 1 + ii
+        live[t] = ii[t] < n_q && rr[t] < rows && (r0 + rr[t] + 1) * g.B <= kv - n_q + 1 + ii[t];
+      }
+      const float4* kr0 = reinterpret_cast<const float4*>(kbar_s + (live[0] ? rr[0] : 0) * kStride);
+      const float4* kr1 = reinterpret_cast<const float4*>(kbar_s + (live[1] ? rr[1] : 0) * kStride);
+      const float4* q0 = reinterpret_cast<const float4*>(iq_s + ((live[0] ? ii[0] : 0) * Hi + h) * kQStrideI);
+      const float4* q1 = reinterpret_cast<const float4*>(iq_s + ((live[1] ? ii[1] : 0) * Hi + h) * kQStrideI);
+      float d0 = 0.f, d1 = 0.f;
+#pragma unroll
+      for (int d4 = 0; d4 < kDI / 4; ++d4) {
+        const float4 ka = kr0[d4], qa = q0[d4], kb = kr1[d4], qb = q1[d4];
+        d0 = fmaf(qa.x, ka.x, d0);
+        d1 = fmaf(qb.x, kb.x, d1);
+        d0 = fmaf(qa.y, ka.y, d0);
+        d1 = fmaf(qb.y, kb.y, d1);
+        d0 = fmaf(qa.z, ka.z, d0);
+        d1 = fmaf(qb.z, kb.z, d1);
+        d0 = fmaf(qa.w, ka.w, d0);
+        d1 = fmaf(qb.w, kb.w, d1);
+      }
+      float t0 = live[0] ? iw_s[ii[0] * Hi + h] * fmaxf(d0, 0.f) : 0.f;
+      float t1 = live[1] ? iw_s[ii[1] * Hi + h] * fmaxf(d1, 0.f) : 0.f;
+      for (int o = 1; o < Hi; o <<= 1) {
+        t0 += __shfl_xor_sync(kFull, t0, o);
+        t1 += __shfl_xor_sync(kFull, t1, o);
+      }
+      if (h == 0) {
+        if (live[0]) keys_mine[ii[0] * per + (r0 + rr[0] - j0)] = score_key(t0 * g.idx_scale);
+        if (live[1]) keys_mine[ii[1] * per + (r0 + rr[1] - j0)] = score_key(t1 * g.idx_scale);
+      }
+    }
+    __syncthreads();
+  }
+  cluster_sync_all();   // every CTA's keys are in place
+  const uint32_t mine_s = smem_u32(keys_mine);
+  for (int i = 0; i < n_q; ++i) {
+    const int n = kv - n_q + 1 + i;
+    const int nc_i = n / g.B;
+    // gather: 16-byte groups of four positions, each owned by one CTA; four
+    // groups per thread in flight
+    for (int jb = 4 * tid; jb < nc_i; jb += 16 * nthr) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = jb + 4 * u * nthr;
+        if (j < nc_i) {
+          const int c = j / per;
+          v[u] = ld_cluster_u32x4(cluster_map(mine_s + 4u * (uint32_t)(i * per + j - c * per), c));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = jb + 4 * u * nthr;
+        if (j < nc_i) *reinterpret_cast<uint4*>(keys_all + j) = v[u];
+      }
+    }
+    __syncthreads();
+    uint32_t* qb = qbits + i * words;
+    cta_topk_radix(keys_all, nc_i, k, qb, hist, hist + 256);
+    const int tail = n - nc_i * g.B;
+    if (tid == 0 && tail > 0) qb[nc_i >> 5] |= 1u << (nc_i & 31);
+    __syncthreads();
+    if (split == 0 && hk == 0 && warp == 0) {   // the selection list: ascending, tail last
+      int* srow = P.sel_w + ((size_t)b * n_q + i) * kp1;
+      const int nw = min(words, (nc_i + 1 + 31) >> 5);
+      int base = 0;
+      for (int w0 = 0; w0 < nw; w0 += 32) {
+        const int w = w0 + lane;
+        uint32_t m = w < nw ? qb[w] : 0u;
+        const int c = __popc(m);
+        int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(kFull, incl, o);
+          if (lane >= o) incl += v;
+        }
+        int off = base + incl - c;
+        while (m) {
+          const int bp = __ffs(m) - 1;
+          m &= m - 1;
+          if (off < kp1) srow[off] = w * 32 + bp;
+          ++off;
+        }
+        base += __shfl_sync(kFull, incl, 31);
+      }
+      for (int e = base + lane; e < kp1; e += 32) srow[e] = -1;
+      if (lane == 0) P.nsel_w[(size_t)b * n_q + i] = min(base, kp1);
+    }
+  }
+  cluster_arrive_all();   // this CTA has read the other CTAs' keys
+}
+
+template <bool kFp8, int kSelDI>
 __global__ void __launch_bounds__(kThreads, 2)
 attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const DecParams P) {
@@ -176,9 +563,59 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
   const int split = blockIdx.x, b = blockIdx.y, hk = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = g.G, n_q = P.n_q, R = n_q * G;
+  if constexpr (kSelDI > 0) grid_dependency_wait();   // every input may come from the previous kernel
+  // Inputs that do not depend on the sequence's length are loaded together
+  // with it, into registers: Q rows r = i * G + gi (query i, head hk * G + gi;
+  // zero beyond R), the gate rows this CTA merges (cluster merge: rows split,
+  // split + nsplit, ...), and for the in-kernel selection the queries' indexer
+  // q and weights.
+  constexpr int kQLd = (16 * (kD / 8) + kThreads - 1) / kThreads;
+  uint4 qreg[kQLd];
+#pragma unroll
+  for (int u = 0; u < kQLd; ++u) {
+    const int e = threadIdx.x + u * kThreads, r = e / (kD / 8), c8 = e % (kD / 8);
+    qreg[u] = make_uint4(0, 0, 0, 0);
+    if (e < 16 * (kD / 8) && r < R)
+      qreg[u] = *reinterpret_cast<const uint4*>(
+          P.q + (((size_t)b * n_q + r / G) * g.Hq + hk * G + r % G) * kD + c8 * 8);
+  }
+  const int g_per_row = g.gate_headwise ? 1 : kD / 8;   // uint4 per gate row (or one value)
+  const int g_rows = P.cluster && split < R ? (R - split + P.nsplit - 1) / P.nsplit : 0;
+  uint4 greg[2];   // g_rows * g_per_row <= 16 * 16 <= 2 * kThreads
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int e = threadIdx.x + u * kThreads;
+    greg[u] = make_uint4(0, 0, 0, 0);
+    if (e < g_rows * g_per_row) {
+      const int lr = e / g_per_row, c8 = e - lr * g_per_row, r = split + lr * P.nsplit;
+      const size_t orow = ((size_t)b * n_q + r / G) * g.Hq + hk * G + r % G;
+      if (g.gate_headwise)
+        greg[u].x = *reinterpret_cast<const unsigned short*>(P.gate + orow);
+      else
+        greg[u] = *reinterpret_cast<const uint4*>(P.gate + orow * kD + c8 * 8);
+    }
+  }
+  uint4 iqreg[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+  float iwreg = 0.f;
+  if constexpr (kSelDI > 0) {
+    const int nq8 = n_q * g.Hi * kSelDI / 8;
+    const uint4* iqb = reinterpret_cast<const uint4*>(P.iq + (size_t)b * nq8 * 8);
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+      if (threadIdx.x + u * kThreads < nq8) iqreg[u] = iqb[threadIdx.x + u * kThreads];
+    if (threadIdx.x < n_q * g.Hi) iwreg = P.iw[(size_t)b * n_q * g.Hi + threadIdx.x];
+  }
   const int kv = P.kv_len[b];
   const size_t row0 = (((size_t)b * g.Hkv + hk) * P.nsplit + split) * R;
-  if (kv < n_q || kv > P.cap) {   // reported by the selection kernel; outputs are zero
+  if (kv < n_q || kv > P.cap) {   // reported by the selection; outputs are zero
+    if constexpr (kSelDI > 0) {
+      if (split == 0 && hk == 0) {
+        const int kp1 = g.k + 1;
+        for (int e = threadIdx.x; e < n_q * kp1; e += blockDim.x) P.sel_w[(size_t)b * n_q * kp1 + e] = -1;
+        for (int e = threadIdx.x; e < n_q; e += blockDim.x) P.nsel_w[(size_t)b * n_q + e] = 0;
+        if (P.err && threadIdx.x == 0) atomicExch(P.err, 1);
+      }
+    }
     if (split == 0)
       for (int e = threadIdx.x; e < R * kD; e += blockDim.x) {
         const int r = e / kD, d = e - r * kD;
@@ -188,6 +625,8 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
       }
     return;
   }
+  if constexpr (kSelDI > 0)
+    if (threadIdx.x == 0) select_prefetch<kSelDI>(P, kv, split, b);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* empty = full + kStages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc);
@@ -211,31 +650,28 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
     fence_barrier_init();
     fence_proxy_async();
   }
-  // Q rows r = i * G + gi (query i, head hk * G + gi), zero beyond R: Q is an
-  // input, so it is loaded before waiting for the selection kernel
+  // Q to shared memory (before the selection exists)
   if constexpr (!kFp8) {
-    for (int e = threadIdx.x; e < 16 * (kD / 8); e += blockDim.x) {
-      const int r = e / (kD / 8), c8 = e % (kD / 8);
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (r < R) {
-        const int i = r / G, gi = r % G;
-        v = *reinterpret_cast<const uint4*>(
-            P.q + (((size_t)b * n_q + i) * g.Hq + hk * G + gi) * kD + c8 * 8);
-      }
-      *reinterpret_cast<uint4*>(smem + kOffQ + r * kQStride + c8 * 16) = v;
+#pragma unroll
+    for (int u = 0; u < kQLd; ++u) {
+      const int e = threadIdx.x + u * kThreads, r = e / (kD / 8), c8 = e % (kD / 8);
+      if (e < 16 * (kD / 8)) *reinterpret_cast<uint4*>(smem + kOffQ + r * kQStride + c8 * 16) = qreg[u];
     }
   } else {
     // fp32 rows in the (still unused) fp16 tile area, rotated into the cache's
     // basis (q' = H q) when the cache holds H k, then stored as fp16
     float* qf = reinterpret_cast<float*>(smem + kOffStages + kStages * kF8StageBytes);
-    for (int e = threadIdx.x; e < 16 * kD; e += blockDim.x) {
-      const int r = e / kD, d = e - r * kD;
-      float v = 0.f;
-      if (r < R) {
-        const int i = r / G, gi = r % G;
-        v = __bfloat162float(P.q[(((size_t)b * n_q + i) * g.Hq + hk * G + gi) * kD + d]);
+#pragma unroll
+    for (int u = 0; u < kQLd; ++u) {
+      const int e = threadIdx.x + u * kThreads;
+      if (e < 16 * (kD / 8)) {
+        const uint32_t w[4] = {qreg[u].x, qreg[u].y, qreg[u].z, qreg[u].w};
+        float4* dst = reinterpret_cast<float4*>(qf + 8 * e);
+        dst[0] = make_float4(__uint_as_float(w[0] << 16), __uint_as_float(w[0] & 0xffff0000u),
+                             __uint_as_float(w[1] << 16), __uint_as_float(w[1] & 0xffff0000u));
+        dst[1] = make_float4(__uint_as_float(w[2] << 16), __uint_as_float(w[2] & 0xffff0000u),
+                             __uint_as_float(w[3] << 16), __uint_as_float(w[3] & 0xffff0000u));
       }
-      qf[e] = v;
     }
     __syncthreads();
     if (P.rotated) fwht128_rows(qf, 16, (int)threadIdx.x, (int)blockDim.x, [] { __syncthreads(); });
@@ -247,48 +683,99 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
       *reinterpret_cast<uint4*>(smem + kOffQ + r * kQStride + c8 * 16) = v;
     }
   }
-  // the merging CTA's gate rows: fetch them into L2 now
-  if (split == 0 && !g.gate_headwise && threadIdx.x < R * (kD * 2 / 128)) {
+  // the gate rows this CTA merges (cluster merge), or the merging CTA's rows
+  // into L2
+  __nv_bfloat16* gate_s = reinterpret_cast<__nv_bfloat16*>(smem + kOffGate);
+  if (P.cluster) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int e = threadIdx.x + u * kThreads;
+      if (e < g_rows * g_per_row) {
+        const int lr = e / g_per_row, c8 = e - lr * g_per_row;
+        if (g.gate_headwise)
+          *reinterpret_cast<unsigned short*>(gate_s + lr * kD) = (unsigned short)greg[u].x;
+        else
+          *reinterpret_cast<uint4*>(gate_s + lr * kD + c8 * 8) = greg[u];
+      }
+    }
+  } else if (split == 0 && !g.gate_headwise && threadIdx.x < R * (kD * 2 / 128)) {
     const int r = threadIdx.x / (kD * 2 / 128), part = threadIdx.x % (kD * 2 / 128);
     const size_t orow = ((size_t)b * n_q + r / G) * g.Hq + hk * G + r % G;
     asm volatile("prefetch.global.L2 [%0];" ::"l"(P.gate + orow * kD + part * 64));
   }
-  // the selections come from the selection kernel: wait for this sequence's
-  // flag (bounded), or for the whole selection grid
-  if (P.ready) {
-    if (threadIdx.x == 0) {
-      const long long t0 = clock64();
-      while (true) {
-        int v;
-        asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(P.ready + b) : "memory");
-        if (v != 0) break;
-        if (clock64() - t0 > kWaitCycles) {
-          *abort_flag = 1;
-          break;
+  bool gave_up = false;
+  if constexpr (kSelDI > 0) {
+    __syncthreads();   // Q staging may have used the ring's space
+    {   // the queries' indexer q (fp32, rows padded to di + 4 floats) and weights
+      float* iq_s = reinterpret_cast<float*>(smem + kOffStages + P.fo_iq);
+      const int nq8 = n_q * g.Hi * kSelDI / 8;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int e = threadIdx.x + u * kThreads;
+        if (e < nq8) {
+          const uint32_t w[4] = {iqreg[u].x, iqreg[u].y, iqreg[u].z, iqreg[u].w};
+          float4* dst = reinterpret_cast<float4*>(iq_s + (8 * e / kSelDI) * (kSelDI + 4) + 8 * e % kSelDI);
+          dst[0] = make_float4(__uint_as_float(w[0] << 16), __uint_as_float(w[0] & 0xffff0000u),
+                               __uint_as_float(w[1] << 16), __uint_as_float(w[1] & 0xffff0000u));
+          dst[1] = make_float4(__uint_as_float(w[2] << 16), __uint_as_float(w[2] & 0xffff0000u),
+                               __uint_as_float(w[3] << 16), __uint_as_float(w[3] & 0xffff0000u));
         }
-        __nanosleep(128);
       }
+      const uint4* iqb = reinterpret_cast<const uint4*>(P.iq + (size_t)b * nq8 * 8);
+      for (int e = threadIdx.x + 2 * kThreads; e < nq8; e += kThreads) {   // beyond 2 per thread
+        const uint4 v = iqb[e];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        float4* dst = reinterpret_cast<float4*>(iq_s + (8 * e / kSelDI) * (kSelDI + 4) + 8 * e % kSelDI);
+        dst[0] = make_float4(__uint_as_float(w[0] << 16), __uint_as_float(w[0] & 0xffff0000u),
+                             __uint_as_float(w[1] << 16), __uint_as_float(w[1] & 0xffff0000u));
+        dst[1] = make_float4(__uint_as_float(w[2] << 16), __uint_as_float(w[2] & 0xffff0000u),
+                             __uint_as_float(w[3] << 16), __uint_as_float(w[3] & 0xffff0000u));
+      }
+      float* iw_s = reinterpret_cast<float*>(smem + kOffStages + P.fo_iw);
+      if (threadIdx.x < n_q * g.Hi) iw_s[threadIdx.x] = iwreg;
     }
+    select_in_cluster<kSelDI>(P, smem, kv, split, b, hk, qbits, words);
   } else {
-    grid_dependency_wait();
-  }
-  __syncthreads();
-  if (*abort_flag) {   // nothing issued yet: report and leave (no merge for this pair)
-    if (threadIdx.x == 0 && P.err) atomicExch(P.err, 2);
-    return;
-  }
-  {
-    const int kp1 = g.k + 1;
-    const int nblk = P.cap / g.B;
-    for (int e = threadIdx.x; e < n_q * kp1; e += blockDim.x) {
-      const int i = e / kp1, j = e - i * kp1;
-      if (j < P.nsel[(size_t)b * n_q + i]) {
-        const int blk = P.sel[((size_t)b * n_q + i) * kp1 + j];
-        if (blk >= 0 && blk < nblk) atomicOr(&qbits[i * words + (blk >> 5)], 1u << (blk & 31));
+    // the selections come from the selection kernel: wait for this sequence's
+    // flag (bounded), or for the whole selection grid
+    if (P.ready) {
+      if (threadIdx.x == 0) {
+        const long long t0 = clock64();
+        while (true) {
+          int v;
+          asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(P.ready + b) : "memory");
+          if (v != 0) break;
+          if (clock64() - t0 > kWaitCycles) {
+            *abort_flag = 1;
+            break;
+          }
+          __nanosleep(128);
+        }
+      }
+    } else {
+      grid_dependency_wait();
+    }
+    __syncthreads();
+    gave_up = *abort_flag != 0;
+    if (gave_up && !P.cluster) {   // nothing issued yet: report and leave (no merge for this pair)
+      if (threadIdx.x == 0 && P.err) atomicExch(P.err, 2);
+      return;
+    }
+    // (a cluster CTA that gave up still takes part in the cluster's barriers, with
+    // an empty partial)
+    if (!gave_up) {
+      const int kp1 = g.k + 1;
+      const int nblk = P.cap / g.B;
+      for (int e = threadIdx.x; e < n_q * kp1; e += blockDim.x) {
+        const int i = e / kp1, j = e - i * kp1;
+        if (j < P.nsel[(size_t)b * n_q + i]) {
+          const int blk = P.sel[((size_t)b * n_q + i) * kp1 + j];
+          if (blk >= 0 && blk < nblk) atomicOr(&qbits[i * words + (blk >> 5)], 1u << (blk & 31));
+        }
       }
     }
+    __syncthreads();
   }
-  __syncthreads();
   if (warp == 0) {
     int base = 0;
     for (int w0 = 0; w0 < words; w0 += 32) {
@@ -318,9 +805,12 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
       }
       base += __shfl_sync(kFull, incl, 31);
     }
-    if (lane == 0) *n_chunks_s = base * cpb;
+    if (lane == 0) *n_chunks_s = gave_up ? 0 : base * cpb;
   }
   __syncthreads();
+  // (in-kernel selection: the other CTAs of the cluster have finished reading
+  // this CTA's score keys, so the ring may be filled)
+  if constexpr (kSelDI > 0) cluster_wait_all();
   const int n_chunks = *n_chunks_s;
   const int c0 = split * P.per_split;
   const int c1 = min(n_chunks, c0 + P.per_split);
@@ -576,8 +1066,12 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
     const int r = t >> 3, d0 = (t & 7) * 16;
     // a rotated fp8 cache gives O' = H O: the merged rows are rotated back
     // (H is symmetric and orthonormal) before they leave as the partial
+    // (cluster merge: every CTA's partial stays in its own shared memory, O in
+    // urow and (m, l) in pml, for the cluster's CTAs to read)
     float* urow = sm + kConsumers * 16 * 2;                    // [16 rows][128]
+    float* pml = urow + 16 * kD;                               // [16 rows][2]
     const bool unrotate = kFp8 && P.rotated;
+    const bool local = unrotate || P.cluster;
     if (r < R) {
       float M = -INFINITY;
 #pragma unroll
@@ -589,7 +1083,7 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
         wsc[w] = mw == -INFINITY ? 0.f : ex2_approx(mw - M);
         L += sm[(w * 16 + r) * 2 + 1] * wsc[w];
       }
-      float* dst = unrotate ? urow + r * kD + d0 : P.part_o + (row0 + r) * kD + d0;
+      float* dst = local ? urow + r * kD + d0 : P.part_o + (row0 + r) * kD + d0;
 #pragma unroll
       for (int d = 0; d < 16; d += 4) {
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -604,20 +1098,76 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
         *reinterpret_cast<float4*>(dst + d) = acc;
       }
       if ((t & 7) == 0) {
-        P.part_ml[2 * (row0 + r)] = M;
-        P.part_ml[2 * (row0 + r) + 1] = L;
+        float* ml = P.cluster ? pml + 2 * r : P.part_ml + 2 * (row0 + r);
+        ml[0] = M;
+        ml[1] = L;
       }
     }
     if (unrotate) {
       named_bar_sync(1, 32 * kConsumers);
       fwht128_rows(urow, R, t, 32 * kConsumers, [] { named_bar_sync(1, 32 * kConsumers); });
-      if (r < R) {
+      if (r < R && !P.cluster) {
         float* gdst = P.part_o + (row0 + r) * kD + d0;
 #pragma unroll
         for (int d = 0; d < 16; d += 4)
           *reinterpret_cast<float4*>(gdst + d) = *reinterpret_cast<const float4*>(urow + r * kD + d0 + d);
       }
     }
+  }
+  if (P.cluster) {
+    // The cluster's CTAs merge the partials by log-sum-exp straight from each
+    // other's shared memory: CTA `split` takes rows split, split + nsplit, ...,
+    // and each of its threads four dims of one row (all partials' loads in
+    // flight at once), then applies the sigmoid output gate staged at the start.
+    cluster_sync_all();
+    const int ns = P.nsplit;
+    const uint32_t pml_s = sbase + kOffStages + (uint32_t)(kConsumers * 16 * kD + kConsumers * 16 * 2 + 16 * kD) * 4u;
+    const uint32_t po_s = sbase + kOffStages + (uint32_t)(kConsumers * 16 * kD + kConsumers * 16 * 2) * 4u;
+    const int mr = split < R ? (R - split + ns - 1) / ns : 0;
+    for (int e = threadIdx.x; e < mr * (kD / 4); e += blockDim.x) {
+      const int lr = e / (kD / 4), f = e - lr * (kD / 4), r = split + lr * ns;
+      float2 ml[kMaxClusterSplits];
+#pragma unroll
+      for (int j = 0; j < kMaxClusterSplits; ++j)
+        if (j < ns) ml[j] = ld_cluster_f32x2(cluster_map(pml_s + 8u * r, j));
+      float4 ov[kMaxClusterSplits];
+#pragma unroll
+      for (int j = 0; j < kMaxClusterSplits; ++j)
+        if (j < ns) ov[j] = ld_cluster_f32x4(cluster_map(po_s + 4u * (r * kD + 4 * f), j));
+      float M = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < kMaxClusterSplits; ++j)
+        if (j < ns) M = fmaxf(M, ml[j].x);
+      float L = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int j = 0; j < kMaxClusterSplits; ++j)
+        if (j < ns) {
+          const float wj = ml[j].x == -INFINITY ? 0.f : ex2_approx(ml[j].x - M);
+          L = fmaf(ml[j].y, wj, L);
+          acc.x = fmaf(ov[j].x, wj, acc.x);
+          acc.y = fmaf(ov[j].y, wj, acc.y);
+          acc.z = fmaf(ov[j].z, wj, acc.z);
+          acc.w = fmaf(ov[j].w, wj, acc.w);
+        }
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+      float gs[4];
+      if (g.gate_headwise) {
+        gs[0] = gs[1] = gs[2] = gs[3] = sigmoidf_(__bfloat162float(gate_s[lr * kD]));
+      } else {
+#pragma unroll
+        for (int d = 0; d < 4; ++d) gs[d] = sigmoidf_(__bfloat162float(gate_s[lr * kD + 4 * f + d]));
+      }
+      const int i = r / G, gi = r % G;
+      const size_t orow = ((size_t)b * n_q + i) * g.Hq + hk * G + gi;
+      *reinterpret_cast<uint2*>(P.out + orow * kD + 4 * f) =
+          make_uint2(pack2(acc.x * inv * gs[0], acc.y * inv * gs[1]),
+                     pack2(acc.z * inv * gs[2], acc.w * inv * gs[3]));
+      if (P.lse && f == 0) P.lse[orow] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+    }
+    cluster_sync_relaxed();   // no CTA leaves while another may still read its partial
+    if (threadIdx.x == 0 && *abort_flag && P.err) atomicExch(P.err, 2);
+    return;
   }
   // the last CTA of this (sequence, KV head) merges the splits' partials by
   // log-sum-exp and applies the sigmoid output gate
@@ -763,6 +1313,42 @@ bool make_cache_map_u8(CUtensorMap* m, const void* ptr, int Hkv, long long rows)
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Whether clusters of `size` CTAs of `kern` (with `smem` bytes of dynamic shared
+// memory) can be resident at once; answers are cached per (kernel, size, smem).
+bool cluster_fits(const void* kern, int size, int smem) {
+  static std::mutex mu;
+  static std::map<std::tuple<const void*, int, int>, bool> done;
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_tuple(kern, size, smem);
+  auto it = done.find(key);
+  if (it != done.end()) return it->second;
+  bool ok = size <= kMaxClusterSplits, refused = false;
+  if (ok && size > 8) {
+    ok = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+    refused = !ok;
+  }
+  if (ok) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(size, 1, 1);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = size;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    const cudaError_t q = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+    refused = q != cudaSuccess;
+    ok = !refused && n >= 1;
+  }
+  if (refused) cudaGetLastError();   // a refused query leaves no error behind
+  done[key] = ok;
+  return ok;
+}
+
 }  // namespace
 
 bool attn_decode_fp8_supported(const Geom& g, int n_q) {
@@ -773,16 +1359,110 @@ bool attn_decode_mma_supported(const Geom& g, int n_q) {
   return g.D == kD && g.B % kChunk == 0 && n_q * g.G <= 16 && n_q <= 4;
 }
 
-// Chunks per CTA for the split-KV grid: about two CTAs per SM in one wave.
+// Chunks per CTA for the split-KV grid: about two CTAs per SM in one wave, and
+// at most kMaxClusterSplits CTAs per (sequence, KV head) so that they can form
+// one cluster.
 void decode_mma_split(const Geom& g, int batch, int n_q, int* nsplit, int* per_split) {
   const int max_chunks = n_q * (g.k + 1) * (g.B / kChunk);
   const int pairs = batch * g.Hkv > 0 ? batch * g.Hkv : 1;
   int ns = (2 * 148) / pairs;
   if (ns < 1) ns = 1;
+  if (ns > kMaxClusterSplits) ns = kMaxClusterSplits;
   if (ns > (max_chunks + 7) / 8) ns = (max_chunks + 7) / 8;   // at least 8 chunks per CTA
   *per_split = (max_chunks + ns - 1) / ns;
   *nsplit = (max_chunks + *per_split - 1) / *per_split;
 }
+
+namespace {
+
+// The fused selection's shared-memory layout inside the ring's space (byte
+// offsets; the CTA's own score keys first); false when it does not fit.
+bool fused_layout(const Geom& g, int n_q, int cap, int nsplit, DecParams* p) {
+  auto a16 = [](long long x) { return (x + 15) & ~15LL; };
+  const int nblk_cap = cap / g.B;
+  const long long per = select_range(nblk_cap, nsplit);
+  long long off = a16(4LL * n_q * per);
+  p->fo_keys = (int)off;
+  off += a16(4LL * (nblk_cap + 4));
+  p->fo_kbar = (int)off;
+  off += a16(4LL * kSelRows * (g.di + 4));
+  p->fo_iq = (int)off;
+  off += a16(4LL * n_q * g.Hi * (g.di + 4));
+  p->fo_iw = (int)off;
+  off += a16(4LL * n_q * g.Hi);
+  p->fo_new = (int)off;
+  off += a16(4LL * 2 * g.di);
+  p->fo_hist = (int)off;
+  off += 4LL * 272 + 8LL * 8 * 32;
+  return off <= (long long)kStages * kStageBytes;
+}
+
+template <bool kFp8>
+const void* fused_kernel(int di) {
+  return di == 64 ? reinterpret_cast<const void*>(attn_decode_mma_kernel<kFp8, 64>)
+                  : reinterpret_cast<const void*>(attn_decode_mma_kernel<kFp8, 32>);
+}
+
+int decode_smem(const Geom& g, int n_q, int cap) {
+  const int words = (cap / g.B + 31) / 32;
+  return kOffBits + 4 * n_q * words + 1024;
+}
+
+DecParams base_params(const Geom& g, int n_q, int cap, int nsplit, int per_split,
+                      const int* kv_len, const void* q, const void* gate, void* out, float* lse,
+                      int* err, Pages pg, Fp8Kv f8) {
+  DecParams p = {};
+  p.g = g;
+  p.n_q = n_q;
+  p.cap = cap;
+  p.nsplit = nsplit;
+  p.per_split = per_split;
+  p.kv_len = kv_len;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.gate = static_cast<const __nv_bfloat16*>(gate);
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.err = err;
+  p.table = pg.table;
+  p.num_pages = pg.num_pages;
+  p.k_scale = f8.k_scale;
+  p.v_scale = f8.v_scale;
+  p.rotated = f8.rotated;
+  return p;
+}
+
+bool make_maps(const Geom& g, int batch, int cap, const void* kc, const void* vc, Pages pg,
+               bool fp8, CUtensorMap* mk, CUtensorMap* mv) {
+  const long long rows = pg.table ? (long long)pg.num_pages * g.B : (long long)batch * cap;
+  return fp8 ? make_cache_map_u8(mk, kc, g.Hkv, rows) && make_cache_map_u8(mv, vc, g.Hkv, rows)
+             : make_cache_map(mk, kc, g.Hkv, rows) && make_cache_map(mv, vc, g.Hkv, rows);
+}
+
+cudaError_t launch_decode_kernel(const void* kern, dim3 grid, int smem, int cluster,
+                                 cudaStream_t st, const CUtensorMap& mk, const CUtensorMap& mv,
+                                 const DecParams& p) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cluster;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = cluster > 0 ? 2 : 1;
+  void* args[3] = {const_cast<CUtensorMap*>(&mk), const_cast<CUtensorMap*>(&mv),
+                   const_cast<DecParams*>(&p)};
+  const cudaError_t e = cudaLaunchKernelExC(&cfg, kern, args);
+  note_launch();
+  return e;
+}
+
+}  // namespace
 
 cudaError_t launch_attn_decode_mma(const Geom& g, int batch, int n_q, int cap, int nsplit,
                                    int per_split, const int* kv_len, const void* q,
@@ -792,40 +1472,61 @@ cudaError_t launch_attn_decode_mma(const Geom& g, int batch, int n_q, int cap, i
                                    cudaStream_t st, Pages pg, const int* ready, Fp8Kv f8) {
   if (batch == 0) return cudaSuccess;
   CUtensorMap mk, mv;
-  const long long rows = pg.table ? (long long)pg.num_pages * g.B : (long long)batch * cap;
-  const bool ok = f8.on ? make_cache_map_u8(&mk, kc, g.Hkv, rows) && make_cache_map_u8(&mv, vc, g.Hkv, rows)
-                        : make_cache_map(&mk, kc, g.Hkv, rows) && make_cache_map(&mv, vc, g.Hkv, rows);
-  if (!ok) return cudaErrorInvalidValue;
-  DecParams p;
-  p.g = g;
-  p.n_q = n_q;
-  p.cap = cap;
-  p.nsplit = nsplit;
-  p.per_split = per_split;
-  p.kv_len = kv_len;
-  p.q = static_cast<const __nv_bfloat16*>(q);
-  p.gate = static_cast<const __nv_bfloat16*>(gate);
-  p.counter = counter;
-  p.out = static_cast<__nv_bfloat16*>(out);
-  p.lse = lse;
+  if (!make_maps(g, batch, cap, kc, vc, pg, f8.on, &mk, &mv)) return cudaErrorInvalidValue;
+  DecParams p = base_params(g, n_q, cap, nsplit, per_split, kv_len, q, gate, out, lse, err, pg, f8);
   p.sel = sel;
   p.nsel = nsel;
   p.part_ml = part_ml;
   p.part_o = part_o;
-  p.err = err;
-  p.table = pg.table;
+  p.counter = counter;
   p.ready = ready;
-  p.k_scale = f8.k_scale;
-  p.v_scale = f8.v_scale;
-  p.rotated = f8.rotated;
-  const int words = (cap / g.B + 31) / 32;
-  const int smem = kOffBits + 4 * n_q * words + 1024;
-  auto kern = f8.on ? attn_decode_mma_kernel<true> : attn_decode_mma_kernel<false>;
-  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(kern), smem);
+  const int smem = decode_smem(g, n_q, cap);
+  const void* kern = f8.on ? reinterpret_cast<const void*>(attn_decode_mma_kernel<true, 0>)
+                           : reinterpret_cast<const void*>(attn_decode_mma_kernel<false, 0>);
+  cudaError_t e = set_max_dynamic_smem(kern, smem);
   if (e != cudaSuccess) return e;
-  e = launch_dependent(kern, dim3(nsplit, batch, g.Hkv), dim3(kThreads), smem, st, mk, mv, p);
-  note_launch();
-  return e;
+  p.cluster = nsplit > 1 && cluster_fits(kern, nsplit, smem) ? 1 : 0;
+  return launch_decode_kernel(kern, dim3(nsplit, batch, g.Hkv), smem, p.cluster ? nsplit : 0, st,
+                              mk, mv, p);
+}
+
+bool decode_fused_supported(const Geom& g, int n_q, int cap, int nsplit, bool fp8) {
+  if (!(fp8 ? attn_decode_fp8_supported(g, n_q) : attn_decode_mma_supported(g, n_q))) return false;
+  if (g.di != 32 && g.di != 64) return false;
+  if (g.Hi < 1 || g.Hi > 32 || (32 % g.Hi) != 0) return false;
+  DecParams p = {};
+  if (!fused_layout(g, n_q, cap, nsplit, &p)) return false;
+  const void* kern = fp8 ? fused_kernel<true>(g.di) : fused_kernel<false>(g.di);
+  const int smem = decode_smem(g, n_q, cap);
+  if (set_max_dynamic_smem(kern, smem) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return cluster_fits(kern, nsplit, smem);
+}
+
+cudaError_t launch_decode_fused(const Geom& g, int batch, int n_q, int cap, int nsplit,
+                                int per_split, const int* kv_len, const void* q, const void* kc,
+                                const void* vc, const void* gate, const DecodeSelIn& si,
+                                void* out, float* lse, int* err, cudaStream_t st, Pages pg,
+                                Fp8Kv f8) {
+  if (batch == 0) return cudaSuccess;
+  CUtensorMap mk, mv;
+  if (!make_maps(g, batch, cap, kc, vc, pg, f8.on, &mk, &mv)) return cudaErrorInvalidValue;
+  DecParams p = base_params(g, n_q, cap, nsplit, per_split, kv_len, q, gate, out, lse, err, pg, f8);
+  if (!fused_layout(g, n_q, cap, nsplit, &p)) return cudaErrorInvalidValue;
+  p.cluster = 1;
+  p.iq = static_cast<const __nv_bfloat16*>(si.iq);
+  p.ik_cache = static_cast<const __nv_bfloat16*>(si.ik_cache);
+  p.iw = si.iw;
+  p.pooled = si.pooled;
+  p.sel_w = si.sel;
+  p.nsel_w = si.nsel;
+  const int smem = decode_smem(g, n_q, cap);
+  const void* kern = f8.on ? fused_kernel<true>(g.di) : fused_kernel<false>(g.di);
+  const cudaError_t e = set_max_dynamic_smem(kern, smem);
+  if (e != cudaSuccess) return e;
+  return launch_decode_kernel(kern, dim3(nsplit, batch, g.Hkv), smem, nsplit, st, mk, mv, p);
 }
 
 }  // namespace qsa

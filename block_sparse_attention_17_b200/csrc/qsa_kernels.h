@@ -112,6 +112,27 @@ cudaError_t launch_attn_decode_mma(const Geom& g, int batch, int n_q, int cap, i
                                    cudaStream_t st, Pages pg = Pages(), const int* ready = nullptr,
                                    Fp8Kv f8 = Fp8Kv());
 bool attn_decode_fp8_supported(const Geom& g, int n_q);
+
+// The selection of a decode step done inside the decode attention kernel (one
+// launch per step): the indexer inputs, the pooled-key cache the kernel updates
+// and reads, and the selection lists it writes ([batch, n_q, k + 1], [batch, n_q]).
+struct DecodeSelIn {
+  const void* iq = nullptr;
+  const void* ik_cache = nullptr;
+  const float* iw = nullptr;
+  float* pooled = nullptr;
+  int* sel = nullptr;
+  int* nsel = nullptr;
+};
+// Whether launch_decode_fused can run this geometry (bf16, the tensor-map
+// decode path, indexer dim 32 or 64, the selection's shared memory within the
+// ring, a resident cluster of nsplit CTAs).
+bool decode_fused_supported(const Geom& g, int n_q, int cap, int nsplit, bool fp8);
+cudaError_t launch_decode_fused(const Geom& g, int batch, int n_q, int cap, int nsplit,
+                                int per_split, const int* kv_len, const void* q, const void* kc,
+                                const void* vc, const void* gate, const DecodeSelIn& si,
+                                void* out, float* lse, int* err, cudaStream_t st,
+                                Pages pg = Pages(), Fp8Kv f8 = Fp8Kv());
 bool attn_prefill_tc_supported(const Geom& g);
 cudaError_t launch_attn_prefill_tc(const Geom& g, const int* cu, int batch, int total_tokens,
                                    int max_seqlen, int words, const uint32_t* bitmask,

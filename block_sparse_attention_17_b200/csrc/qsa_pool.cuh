@@ -1,0 +1,65 @@
+// Mean pooling of one B-row block of indexer keys (instagit MTPLX page, "Qwen
+// Sparse Attention (QSA)": each block is represented by the mean of its keys).
+// Every kernel that pools calls pool_block(), so the prefill pooling, the
+// incremental decode finalisation and the cache rebuild write identical bits.
+#pragma once
+
+#include "qsa_common.cuh"
+
+namespace qsa {
+
+template <typename T>
+__device__ __forceinline__ float2 load_pair(const T* p);
+template <>
+__device__ __forceinline__ float2 load_pair<float>(const float* p) {
+  return *reinterpret_cast<const float2*>(p);
+}
+template <>
+__device__ __forceinline__ float2 load_pair<__nv_bfloat16>(const __nv_bfloat16* p) {
+  const uint32_t u = *reinterpret_cast<const uint32_t*>(p);
+  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+
+// Pools rows[0 .. B) (di <= 64 dims each) into dst[0 .. di) with the whole CTA
+// (nwarps warps, all threads call it). The order of the sums is fixed whatever
+// nwarps is: eight partial sums, partial v over rows v, v + 8, v + 16, ... in
+// ascending order (lane l owns dims 2l and 2l + 1), combined in the tree
+// ((p0 + p1) + (p2 + p3)) + ((p4 + p5) + (p6 + p7)) and scaled by 1/B (B is a
+// power of two). part: 8 x 32 float2 of shared memory.
+template <typename T>
+__device__ __forceinline__ void pool_block(const T* __restrict__ rows, int B, int di,
+                                           float* dst, float2 (*part)[32], int nwarps) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool active = 2 * lane < di;
+  for (int v = warp; v < 8; v += nwarps) {
+    float2 acc = make_float2(0.f, 0.f);
+    if (active) {
+      for (int i0 = v; i0 < B; i0 += 64) {   // eight rows' loads in flight, then their sums in order
+        float2 x[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          x[u] = i0 + 8 * u < B ? load_pair<T>(rows + (size_t)(i0 + 8 * u) * di + 2 * lane)
+                                : make_float2(0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (i0 + 8 * u < B) {
+            acc.x += x[u].x;
+            acc.y += x[u].y;
+          }
+      }
+    }
+    part[v][lane] = acc;
+  }
+  __syncthreads();
+  if (warp == 0 && active) {
+    float2 q[8];
+#pragma unroll
+    for (int w = 0; w < 8; ++w) q[w] = part[w][lane];
+    const float inv = 1.0f / (float)B;
+    const float sx = ((q[0].x + q[1].x) + (q[2].x + q[3].x)) + ((q[4].x + q[5].x) + (q[6].x + q[7].x));
+    const float sy = ((q[0].y + q[1].y) + (q[2].y + q[3].y)) + ((q[4].y + q[5].y) + (q[6].y + q[7].y));
+    *reinterpret_cast<float2*>(dst + 2 * lane) = make_float2(sx * inv, sy * inv);
+  }
+}
+
+}  // namespace qsa

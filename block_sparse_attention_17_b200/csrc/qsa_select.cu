@@ -15,56 +15,20 @@
 
 #include "qsa_common.cuh"
 #include "qsa_kernels.h"
+#include "qsa_pool.cuh"
 
 namespace qsa {
 
 // ----------------------------------------------------------------- pooling
-// One CTA of 256 threads pools one block: warp w sums rows w, w + 8, ... of
-// the block (coalesced rows; lane l owns dims 2l and 2l + 1) in ascending
-// order, then the 8 partial sums are combined in a fixed tree
-// ((p0 + p1) + (p2 + p3)) + ((p4 + p5) + (p6 + p7)) and scaled by 1/B (B is a
-// power of two). The prefill pooling, the incremental decode finalisation and
-// the cache rebuild all call this one function, so they write identical bits.
+// One CTA of 256 threads pools one block (pool_block: warp w sums rows w, w + 8,
+// ... of the block in ascending order, then a fixed tree and the 1/B scale).
 constexpr int kPoolThreads = 256;
-
-template <typename T>
-__device__ __forceinline__ float2 load_pair(const T* p);
-template <>
-__device__ __forceinline__ float2 load_pair<float>(const float* p) {
-  return *reinterpret_cast<const float2*>(p);
-}
-template <>
-__device__ __forceinline__ float2 load_pair<__nv_bfloat16>(const __nv_bfloat16* p) {
-  const uint32_t u = *reinterpret_cast<const uint32_t*>(p);
-  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
-}
 
 template <typename T>
 __device__ __forceinline__ void pool_block_cta(const T* __restrict__ rows, int B, int di,
                                                float* __restrict__ dst) {
   __shared__ float2 part[8][32];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool active = 2 * lane < di;
-  float2 acc = make_float2(0.f, 0.f);
-  if (active) {
-#pragma unroll 4
-    for (int i = warp; i < B; i += 8) {
-      const float2 x = load_pair<T>(rows + (size_t)i * di + 2 * lane);
-      acc.x += x.x;
-      acc.y += x.y;
-    }
-  }
-  part[warp][lane] = acc;
-  __syncthreads();
-  if (warp == 0 && active) {
-    float2 q[8];
-#pragma unroll
-    for (int w = 0; w < 8; ++w) q[w] = part[w][lane];
-    const float inv = 1.0f / (float)B;
-    const float sx = ((q[0].x + q[1].x) + (q[2].x + q[3].x)) + ((q[4].x + q[5].x) + (q[6].x + q[7].x));
-    const float sy = ((q[0].y + q[1].y) + (q[2].y + q[3].y)) + ((q[4].y + q[5].y) + (q[6].y + q[7].y));
-    *reinterpret_cast<float2*>(dst + 2 * lane) = make_float2(sx * inv, sy * inv);
-  }
+  pool_block<T>(rows, B, di, dst, part, kPoolThreads / 32);
 }
 
 // Grid (blocks of the longest sequence, batch).
