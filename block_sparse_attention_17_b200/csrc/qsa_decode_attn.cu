@@ -45,7 +45,7 @@ constexpr int kThreads = 32 * (kConsumers + 1);
 constexpr int kQStride = kD * 2 + 16;           // padded bf16 row of Q in shared memory
 constexpr int kMaxUnion = 4 * (kMaxTopK + 1);
 constexpr int kMaxClusterSplits = 16;           // CTAs of one cluster-merged (sequence, KV head)
-constexpr int kSelRows = 128;                   // in-kernel selection: blocks per scoring pass
+constexpr int kSelRows = 160;                   // in-kernel selection: blocks per scoring pass
 
 // fp8 caches: a stage holds the K and V rows as e4m3 bytes (one 128-byte box
 // each) and the 64 rows' scales for every KV head (K, then V); each consumer
@@ -188,17 +188,18 @@ __device__ __forceinline__ uint32_t tile_off(int row, int dim) {
 // ------------------------------------------------- selection in the cluster
 // The k largest of keys[0 .. n) (shared memory), a lower position winning a
 // tie, written as a bitmap: bits[w] for w < ceil(n / 32), bit j % 32 of word
-// j / 32 set for a chosen position j. Radix select over the 32-bit keys: the
-// bits above the highest bit where the largest and smallest key differ are
-// common to all keys; below them, 8-bit digits, most significant first. Each
+// j / 32 set for a chosen position j; hi and lo are the largest and smallest
+// key. Radix select over the 32-bit keys: the bits above the highest bit where
+// hi and lo differ are common to all keys; below them, 8-bit digits, most
+// significant first. Each
 // pass histograms the digit of the keys that still match the chosen prefix
 // (shared-memory atomics), warp 0 finds the digit value holding the k-th
 // largest key by a suffix scan, and the passes stop as soon as every key with
 // that digit value is taken. Otherwise the last pass ends on the k-th largest
 // key itself, and of the keys equal to it the lowest positions are taken.
-// hist: 256 ints, ctl: 16 ints of shared memory. All threads call it.
-__device__ __forceinline__ void cta_topk_radix(const uint32_t* keys, int n, int k, uint32_t* bits, int* hist,
-                               int* ctl) {
+// hist: 256 ints, ctl: 4 ints of shared memory. All threads call it.
+__device__ __forceinline__ void cta_topk_radix(const uint32_t* keys, int n, int k, uint32_t* bits,
+                                               int* hist, int* ctl, uint32_t hi, uint32_t lo) {
   const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31, warp = tid >> 5;
   const int nwarps = nthr >> 5;
   const int nwords = (n + 31) >> 5;
@@ -208,24 +209,8 @@ __device__ __forceinline__ void cta_topk_radix(const uint32_t* keys, int n, int 
     __syncthreads();
     return;
   }
-  uint32_t hi = 0u, lo = 0xffffffffu;
-  for (int j = tid; j < n; j += nthr) {
-    const uint32_t key = keys[j];
-    hi = max(hi, key);
-    lo = min(lo, key);
-  }
-  hi = __reduce_max_sync(kFull, hi);
-  lo = __reduce_min_sync(kFull, lo);
-  if (lane == 0) {
-    ctl[4 + warp] = (int)hi;
-    ctl[10 + warp] = (int)lo;
-  }
   for (int e = tid; e < 256; e += nthr) hist[e] = 0;
   __syncthreads();
-  for (int w = 0; w < nwarps; ++w) {
-    hi = max(hi, (uint32_t)ctl[4 + w]);
-    lo = min(lo, (uint32_t)ctl[10 + w]);
-  }
   const int top = hi == lo ? -1 : 31 - __clz(hi ^ lo);   // highest differing bit
   uint32_t pmask = top < 0 ? 0xffffffffu : top == 31 ? 0u : ~((2u << top) - 1u);   // common bits
   uint32_t prefix = hi & pmask;
@@ -382,14 +367,16 @@ __device__ __forceinline__ void select_in_cluster(const DecParams& P, uint8_t* s
   const int per = select_range(nc_last, P.nsplit);
   const int j0 = split * per, j1 = min(nc_last, j0 + per);
   uint8_t* ring = smem + kOffStages;
-  uint32_t* keys_mine = reinterpret_cast<uint32_t*>(ring);                  // [n_q][per]
+  uint32_t* mm_mine = reinterpret_cast<uint32_t*>(ring);                    // [4][2] largest, smallest key
+  uint32_t* keys_mine = reinterpret_cast<uint32_t*>(ring + 32);             // [n_q][per]
   uint32_t* keys_all = reinterpret_cast<uint32_t*>(ring + P.fo_keys);       // [nblk_cap]
   float* kbar_s = reinterpret_cast<float*>(ring + P.fo_kbar);               // [kRows][kStride]
   float* iq_s = reinterpret_cast<float*>(ring + P.fo_iq);                   // [n_q][Hi][kDI]
   float* iw_s = reinterpret_cast<float*>(ring + P.fo_iw);                   // [n_q][Hi]
   float* new_s = reinterpret_cast<float*>(ring + P.fo_new);                 // [2][kDI]
   int* hist = reinterpret_cast<int*>(ring + P.fo_hist);                     // [256] + ctl [16]
-  float2(*part)[32] = reinterpret_cast<float2(*)[32]>(hist + 272);           // [8][32]
+  uint32_t* gmm = reinterpret_cast<uint32_t*>(hist + 272);                   // [4][2]
+  float2(*part)[32] = reinterpret_cast<float2(*)[32]>(hist + 280);           // [8][32]
 
   // paged caches: every page the step may gather must be in the pool
   if (P.table && hk == 0) {
@@ -398,6 +385,10 @@ __device__ __forceinline__ void select_in_cluster(const DecParams& P, uint8_t* s
       const int page = P.table[(size_t)b * nblk_cap + j];
       if ((page < 0 || page >= P.num_pages) && P.err) atomicExch(P.err, 3);
     }
+  }
+  if (tid < 4) {
+    mm_mine[2 * tid] = 0u;
+    mm_mine[2 * tid + 1] = 0xffffffffu;
   }
   __syncthreads();   // the caller staged iq_s and iw_s
   // blocks completed by this step's tokens (at most two: n_q <= 4 < B)
@@ -412,7 +403,7 @@ __device__ __forceinline__ void select_in_cluster(const DecParams& P, uint8_t* s
     }
     float* dst = new_s + (j - jn_lo) * kDI;
     if (ok) {   // uniform across the CTA
-      pool_block<__nv_bfloat16>(P.ik_cache + (ok ? r0 : 0) * kDI, g.B, kDI, dst, part, nthr >> 5);
+      pool_block_halves<__nv_bfloat16, kDI>(P.ik_cache + (ok ? r0 : 0) * kDI, g.B, dst, part);
     } else {    // a page outside the pool (reported): the cached row stands
       for (int d = tid; d < kDI; d += nthr) dst[d] = P.pooled[((size_t)b * nblk_cap + j) * kDI + d];
     }
@@ -420,7 +411,9 @@ __device__ __forceinline__ void select_in_cluster(const DecParams& P, uint8_t* s
     if (hk == 0 && ok)
       for (int d = tid; d < kDI; d += nthr) P.pooled[((size_t)b * nblk_cap + j) * kDI + d] = dst[d];
   }
-  // score the range, kRows blocks at a time
+  // score the range, kRows blocks at a time (with each query's largest and
+  // smallest key)
+  uint32_t qhi[4] = {0u, 0u, 0u, 0u}, qlo[4] = {~0u, ~0u, ~0u, ~0u};
   for (int r0 = j0; r0 < j1; r0 += kRows) {
     const int rows = min(kRows, j1 - r0);
     {   // every load of the pass is issued before the first store
@@ -444,57 +437,91 @@ __device__ __forceinline__ void select_in_cluster(const DecParams& P, uint8_t* s
       }
     }
     __syncthreads();
-    // Thread t takes head t % Hi of the (query, block) slots t / Hi + m * hpr
-    // (hpr = nthr / Hi; nthr is a multiple of Hi, so a slot's heads are adjacent
-    // lanes of one warp), two slots per pass. Each dot product is one fma chain
-    // over the dims in ascending order, as in the selection kernel; the heads'
-    // terms are summed by shuffles. iq rows are padded to kQStride floats so
-    // that the heads of a warp read distinct banks.
+    // For each query, thread t takes head t % Hi of blocks r = t / Hi + m * hpr,
+    // m < 4 (hpr = nthr / Hi; nthr is a multiple of Hi, so a block's heads are
+    // adjacent lanes of one warp): four blocks share each q load. Each dot
+    // product is one fma chain over the dims in ascending order, as in the
+    // selection kernel; the heads' terms are summed by shuffles. iq rows are
+    // padded to kQStrideI floats so that the heads of a warp read distinct banks.
     const int hpr = nthr / Hi, h = tid % Hi, slot = tid / Hi;
-    for (int base = 0; base < n_q * kRows; base += 2 * hpr) {
-      int ii[2], rr[2];
-      bool live[2];
+    for (int i = 0; i < n_q; ++i) {
+      const int lim = kv - n_q + 1 + i;   // block j is complete for query i iff (j + 1) B <= lim
+      const float4* qv = reinterpret_cast<const float4*>(iq_s + (i * Hi + h) * kQStrideI);
+      const float wq = iw_s[i * Hi + h];
+      for (int rb = 0; rb < rows; rb += 4 * hpr) {   // uniform
+        int rr[4];
+        bool live[4];
+        const float4* kr[4];
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const int sl = base + slot + t * hpr;
-        ii[t] = sl / kRows;
-        rr[t] = sl % kRows;
-        // block r0 + rr is complete for query ii: (r0 + rr + 1) B <= kv - n_q + 1 + ii
-        live[t] = ii[t] < n_q && rr[t] < rows && (r0 + rr[t] + 1) * g.B <= kv - n_q + 1 + ii[t];
-      }
-      const float4* kr0 = reinterpret_cast<const float4*>(kbar_s + (live[0] ? rr[0] : 0) * kStride);
-      const float4* kr1 = reinterpret_cast<const float4*>(kbar_s + (live[1] ? rr[1] : 0) * kStride);
-      const float4* q0 = reinterpret_cast<const float4*>(iq_s + ((live[0] ? ii[0] : 0) * Hi + h) * kQStrideI);
-      const float4* q1 = reinterpret_cast<const float4*>(iq_s + ((live[1] ? ii[1] : 0) * Hi + h) * kQStrideI);
-      float d0 = 0.f, d1 = 0.f;
+        for (int m = 0; m < 4; ++m) {
+          rr[m] = rb + slot + m * hpr;
+          live[m] = rr[m] < rows && (r0 + rr[m] + 1) * g.B <= lim;
+          kr[m] = reinterpret_cast<const float4*>(kbar_s + (live[m] ? rr[m] : 0) * kStride);
+        }
+        float dt[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int d4 = 0; d4 < kDI / 4; ++d4) {
-        const float4 ka = kr0[d4], qa = q0[d4], kb = kr1[d4], qb = q1[d4];
-        d0 = fmaf(qa.x, ka.x, d0);
-        d1 = fmaf(qb.x, kb.x, d1);
-        d0 = fmaf(qa.y, ka.y, d0);
-        d1 = fmaf(qb.y, kb.y, d1);
-        d0 = fmaf(qa.z, ka.z, d0);
-        d1 = fmaf(qb.z, kb.z, d1);
-        d0 = fmaf(qa.w, ka.w, d0);
-        d1 = fmaf(qb.w, kb.w, d1);
-      }
-      float t0 = live[0] ? iw_s[ii[0] * Hi + h] * fmaxf(d0, 0.f) : 0.f;
-      float t1 = live[1] ? iw_s[ii[1] * Hi + h] * fmaxf(d1, 0.f) : 0.f;
-      for (int o = 1; o < Hi; o <<= 1) {
-        t0 += __shfl_xor_sync(kFull, t0, o);
-        t1 += __shfl_xor_sync(kFull, t1, o);
-      }
-      if (h == 0) {
-        if (live[0]) keys_mine[ii[0] * per + (r0 + rr[0] - j0)] = score_key(t0 * g.idx_scale);
-        if (live[1]) keys_mine[ii[1] * per + (r0 + rr[1] - j0)] = score_key(t1 * g.idx_scale);
+        for (int d4 = 0; d4 < kDI / 4; ++d4) {
+          const float4 qa = qv[d4];
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const float4 ka = kr[m][d4];
+            dt[m] = fmaf(qa.x, ka.x, dt[m]);
+            dt[m] = fmaf(qa.y, ka.y, dt[m]);
+            dt[m] = fmaf(qa.z, ka.z, dt[m]);
+            dt[m] = fmaf(qa.w, ka.w, dt[m]);
+          }
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          float t = live[m] ? wq * fmaxf(dt[m], 0.f) : 0.f;
+          for (int o = 1; o < Hi; o <<= 1) t += __shfl_xor_sync(kFull, t, o);
+          if (h == 0 && live[m]) {
+            const uint32_t y = score_key(t * g.idx_scale);
+            keys_mine[i * per + (r0 + rr[m] - j0)] = y;
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              if (q == i) {
+                qhi[q] = max(qhi[q], y);
+                qlo[q] = min(qlo[q], y);
+              }
+          }
+        }
       }
     }
     __syncthreads();
   }
-  cluster_sync_all();   // every CTA's keys are in place
-  const uint32_t mine_s = smem_u32(keys_mine);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    if (q < n_q) {
+      const uint32_t hw = __reduce_max_sync(kFull, qhi[q]), lw = __reduce_min_sync(kFull, qlo[q]);
+      if (lane == 0 && hw >= lw) {
+        atomicMax(&mm_mine[2 * q], hw);
+        atomicMin(&mm_mine[2 * q + 1], lw);
+      }
+    }
+  }
+  cluster_sync_all();   // every CTA's keys (and their extremes) are in place
+  const uint32_t mine_s = smem_u32(keys_mine), mm_s = smem_u32(mm_mine);
+  // With several queries, CTA s selects queries s, s + nsplit, ... and the
+  // others read the bitmaps afterwards; one query is selected by every CTA.
+  const bool spread = n_q > 1;
+  if (warp == 0) {   // the queries' largest and smallest keys over the cluster
+    for (int i = 0; i < n_q; ++i) {
+      uint2 m = make_uint2(0u, 0xffffffffu);
+      if (lane < P.nsplit) {
+        const uint32_t a = cluster_map(mm_s + 8u * i, lane);
+        m.x = (uint32_t)__float_as_uint(ld_cluster_f32(a));
+        m.y = (uint32_t)__float_as_uint(ld_cluster_f32(a + 4));
+      }
+      const uint32_t hw = __reduce_max_sync(kFull, m.x), lw = __reduce_min_sync(kFull, m.y);
+      if (lane == 0) {
+        gmm[2 * i] = hw;
+        gmm[2 * i + 1] = lw;
+      }
+    }
+  }
   for (int i = 0; i < n_q; ++i) {
+    if (spread && i % P.nsplit != split) continue;   // uniform across the CTA
     const int n = kv - n_q + 1 + i;
     const int nc_i = n / g.B;
     // gather: 16-byte groups of four positions, each owned by one CTA; four
@@ -517,11 +544,11 @@ __device__ __forceinline__ void select_in_cluster(const DecParams& P, uint8_t* s
     }
     __syncthreads();
     uint32_t* qb = qbits + i * words;
-    cta_topk_radix(keys_all, nc_i, k, qb, hist, hist + 256);
+    cta_topk_radix(keys_all, nc_i, k, qb, hist, hist + 256, gmm[2 * i], gmm[2 * i + 1]);
     const int tail = n - nc_i * g.B;
     if (tid == 0 && tail > 0) qb[nc_i >> 5] |= 1u << (nc_i & 31);
     __syncthreads();
-    if (split == 0 && hk == 0 && warp == 0) {   // the selection list: ascending, tail last
+    if ((spread || split == 0) && hk == 0 && warp == 0) {   // the selection list: ascending, tail last
       int* srow = P.sel_w + ((size_t)b * n_q + i) * kp1;
       const int nw = min(words, (nc_i + 1 + 31) >> 5);
       int base = 0;
@@ -547,6 +574,16 @@ __device__ __forceinline__ void select_in_cluster(const DecParams& P, uint8_t* s
       for (int e = base + lane; e < kp1; e += 32) srow[e] = -1;
       if (lane == 0) P.nsel_w[(size_t)b * n_q + i] = min(base, kp1);
     }
+  }
+  if (spread) {   // the other queries' bitmaps, from the CTAs that selected them
+    cluster_sync_all();
+    const uint32_t qbits_s = smem_u32(qbits);
+    for (int e = tid; e < n_q * words; e += nthr) {
+      const int i = e / words;
+      if (i % P.nsplit != split)
+        qbits[e] = (uint32_t)__float_as_uint(ld_cluster_f32(cluster_map(qbits_s + 4u * e, i % P.nsplit)));
+    }
+    __syncthreads();
   }
   cluster_arrive_all();   // this CTA has read the other CTAs' keys
 }
@@ -1381,7 +1418,7 @@ bool fused_layout(const Geom& g, int n_q, int cap, int nsplit, DecParams* p) {
   auto a16 = [](long long x) { return (x + 15) & ~15LL; };
   const int nblk_cap = cap / g.B;
   const long long per = select_range(nblk_cap, nsplit);
-  long long off = a16(4LL * n_q * per);
+  long long off = a16(32 + 4LL * n_q * per);   // extremes, then this CTA's keys
   p->fo_keys = (int)off;
   off += a16(4LL * (nblk_cap + 4));
   p->fo_kbar = (int)off;
@@ -1393,7 +1430,7 @@ bool fused_layout(const Geom& g, int n_q, int cap, int nsplit, DecParams* p) {
   p->fo_new = (int)off;
   off += a16(4LL * 2 * g.di);
   p->fo_hist = (int)off;
-  off += 4LL * 272 + 8LL * 8 * 32;
+  off += 4LL * 280 + 8LL * 8 * 32;
   return off <= (long long)kStages * kStageBytes;
 }
 

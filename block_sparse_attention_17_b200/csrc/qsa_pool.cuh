@@ -63,3 +63,55 @@ __device__ __forceinline__ void pool_block(const T* __restrict__ rows, int B, in
 }
 
 }  // namespace qsa
+
+namespace qsa {
+
+// pool_block for a CTA of at least four warps and kDI = 32 or 64, in one round:
+// half-warp v of warps 0-3 sums partial v (lane l' of it owns dims
+// [kDI/16 * l', kDI/16 * (l' + 1))), with the same rows, order and final tree
+// as pool_block, so both write identical bits.
+template <typename T, int kDI>
+__device__ __forceinline__ void pool_block_halves(const T* __restrict__ rows, int B, float* dst,
+                                                  float2 (*part)[32]) {
+  static_assert(kDI == 32 || kDI == 64, "indexer dim");
+  constexpr int kPer = kDI / 16;                  // dims per lane: 2 or 4
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp < 4) {
+    const int v = 2 * warp + (lane >> 4), l = lane & 15;
+    float acc[kPer];
+#pragma unroll
+    for (int d = 0; d < kPer; ++d) acc[d] = 0.f;
+    for (int i0 = v; i0 < B; i0 += 64) {   // eight rows in flight, then their sums in order
+      float x[8][kPer];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int r = i0 + 8 * u;
+#pragma unroll
+        for (int d = 0; d < kPer; d += 2) {
+          const float2 p = r < B ? load_pair<T>(rows + (size_t)r * kDI + kPer * l + d) : make_float2(0.f, 0.f);
+          x[u][d] = p.x;
+          x[u][d + 1] = p.y;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (i0 + 8 * u < B)
+#pragma unroll
+          for (int d = 0; d < kPer; ++d) acc[d] += x[u][d];
+    }
+#pragma unroll
+    for (int d = 0; d < kPer; d += 2) part[v][(kPer * l + d) / 2] = make_float2(acc[d], acc[d + 1]);
+  }
+  __syncthreads();
+  if (warp == 0 && 2 * lane < kDI) {
+    float2 q[8];
+#pragma unroll
+    for (int w = 0; w < 8; ++w) q[w] = part[w][lane];
+    const float inv = 1.0f / (float)B;
+    const float sx = ((q[0].x + q[1].x) + (q[2].x + q[3].x)) + ((q[4].x + q[5].x) + (q[6].x + q[7].x));
+    const float sy = ((q[0].y + q[1].y) + (q[2].y + q[3].y)) + ((q[4].y + q[5].y) + (q[6].y + q[7].y));
+    *reinterpret_cast<float2*>(dst + 2 * lane) = make_float2(sx * inv, sy * inv);
+  }
+}
+
+}  // namespace qsa
