@@ -334,6 +334,7 @@ def run_ours(args, w, rank, world, dist):
         esz = 2 if w.dtype == "bf16" else 4
         io = w.batch * w.n_q * (2 * w.num_q_heads * w.head_dim * esz)   # q + out
         io += w.batch * w.n_q * w.num_q_heads * w.head_dim * esz         # gate
+        io += decode_selection_bytes(w, inp["kv_len"])
         alg = {"bound": "hbm", "work": kv_bytes + io, "peak_key": "hbm_gbs", "unit": "GB/s"}
         in_names = ["q", "iq", "iw", "gate", "kv_len"]   # one decode step's new inputs
 
@@ -357,7 +358,9 @@ def run_ours(args, w, rank, world, dist):
             ends[i].record(stream)
             torch.cuda.synchronize()       # read this step's stage events before reuse
             if stages:
-                attn.append(ev_stage[1].elapsed_time(ev_stage[2]))
+                # prefill: the attention kernel; decode: the whole step (the
+                # selection runs inside the decode kernel)
+                attn.append(ev_stage[0 if w.kind == "decode" else 1].elapsed_time(ev_stage[2]))
         return [starts[i].elapsed_time(ends[i]) for i in range(args.steps)], attn
 
     # one step captured as a CUDA graph (the library makes no host sync, reads
@@ -420,7 +423,8 @@ def run_ours(args, w, rank, world, dist):
     roof = {"bound": alg["bound"], "achieved": round(achieved, 3), "peak": peak,
             "unit": alg["unit"], "frac": round(achieved / peak, 5),
             "traffic": recorded_traffic(kfile, w.name),
-            "kernel": "qsa attention" + (" + combine" if w.kind == "decode" else ""),
+            "kernel": ("qsa decode step (selection + attention + merge, one kernel)"
+                       if w.kind == "decode" else "qsa attention"),
             "kernel_ms": round(attn_ms, 5), "peak_source": f"{peak_kind} ({alg['peak_key']})",
             "algorithmic_per_launch": alg["work"]}
 
@@ -485,6 +489,22 @@ def ctypes_voidp_array(ptrs):
     import ctypes
     arr = (ctypes.c_void_p * len(ptrs))(*[ctypes.c_void_p(p) for p in ptrs])
     return ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
+
+
+def decode_selection_bytes(w, kv_len):
+    """Bytes the selection of one decode step must move: the pooled keys of every
+    complete block (fp32, read once), the indexer rows of the blocks the step
+    completes (read) and their pooled rows (written), the queries' indexer q and
+    weights, and the selection lists written."""
+    esz = 2 if w.dtype == "bf16" else 4
+    total = 0
+    for kv in np.asarray(kv_len).tolist():
+        total += (kv // w.block_size) * w.idx_dim * 4
+        new_blocks = kv // w.block_size - (kv - w.n_q) // w.block_size
+        total += new_blocks * w.block_size * w.idx_dim * esz + new_blocks * w.idx_dim * 4
+    total += w.batch * w.n_q * w.idx_heads * (w.idx_dim * esz + 4)
+    total += w.batch * w.n_q * (w.topk + 2) * 4
+    return total
 
 
 def decode_selected_kv_bytes(w, sel, nsel, kv_len, kv_format="bf16"):
