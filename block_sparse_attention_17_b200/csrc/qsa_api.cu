@@ -251,6 +251,9 @@ qsa_status check_decode_dims(const qsa_config* cfg, int batch, int n_q, int cap)
   if (n_q > kMaxDecodeQ) return fail(QSA_ERR_UNSUPPORTED, "n_q > %d", kMaxDecodeQ);
   if (n_q * (cfg->num_q_heads / cfg->num_kv_heads) > kMaxDecodeRows)
     return fail(QSA_ERR_UNSUPPORTED, "n_q * group size > %d", kMaxDecodeRows);
+  // the decode selection sums a block's indexer heads over adjacent lanes of a warp
+  if (cfg->idx_heads & (cfg->idx_heads - 1))
+    return fail(QSA_ERR_UNSUPPORTED, "decode: idx_heads must be a power of two");
   return QSA_OK;
 }
 

@@ -121,6 +121,7 @@ def test_decode_rejects_bad_geometry():
     g16 = cfg(num_kv_heads=1)                                          # group size 16
     assert call(n_q=3, c=g16) == _lib.QSA_ERR_UNSUPPORTED              # 3 * 16 rows > 32
     assert call(ws_bytes=ws - 256) == _lib.QSA_ERR_WORKSPACE
+    assert call(c=cfg(idx_heads=6)) == _lib.QSA_ERR_UNSUPPORTED        # heads summed by lane groups
 
 
 def test_workspace_sizes_grow_with_the_problem():

@@ -160,8 +160,8 @@ def run_decode(w, inp, d=None):
     return r
 
 
-def decode_parity(w, inp, pairs=None):
-    gpu = run_decode(w, inp)
+def decode_parity(w, inp, pairs=None, d=None):
+    gpu = run_decode(w, inp, d)
     assert gpu["err"] == 0
     orc = O.qsa_decode(w, inp, pairs=pairs)
     rep = TL.check_queries(orc["queries"], gpu, lambda bi: bi, w)

@@ -1,14 +1,17 @@
 """Parity of the kernel variants the workloads above do not reach: the fp32
 decode path (CUDA-core attention + split combine), bf16 decode with more than
-16 query rows per KV head (the same CUDA-core path), head-wise gates on the
-tensor-core prefill and the tensor-map decode, and bf16 prefill with
-head_dim 64 (CUDA-core prefill). Every query is compared with the fp64 oracle.
+16 query rows per KV head (the same CUDA-core path), bf16 decode with more
+indexer heads than the one-launch decode takes (the selection kernel, then the
+tensor-map attention kernel), head-wise gates on the tensor-core prefill and the
+tensor-map decode, and bf16 prefill with head_dim 64 (CUDA-core prefill). Every
+query is compared with the fp64 oracle.
 """
 import numpy as np
 import pytest
 import torch
 
 import block_sparse_attention_17_b200 as qsa
+from block_sparse_attention_17_b200 import _lib
 from block_sparse_attention_17_b200.workloads import (WORKLOADS, make_decode_inputs,
                                                       make_prefill_inputs)
 from oracle import qsa_oracle as O
@@ -64,3 +67,44 @@ def test_prefill_bf16_head_dim_64_cuda_core_path():
     w, inp = _prefill("prefill_bf16_t8192", seqlens=(1200,), head_dim=64)
     rep = prefill_parity(w, inp, None)
     assert len(rep["excused_near_ties"]) <= 2, rep
+
+
+def _decode_launches(w, d):
+    """Kernel launches of one qsa.decode call on the uploaded inputs d (after a
+    warm-up call)."""
+    cfg = qsa.QSAConfig.from_workload(w)
+    kv = d["kv_len"]
+    pooled = qsa.pool_build(cfg, d["ik_cache"], (kv - w.n_q).to(torch.int32))
+
+    def call():
+        qsa.decode(cfg, d["q"], d["k_cache"], d["v_cache"], d["iq"], d["ik_cache"], d["iw"],
+                   d["gate"], pooled, kv)
+    call()
+    torch.cuda.synchronize()
+    lib = _lib.lib()
+    n0 = lib.qsa_kernel_launch_count()
+    call()
+    torch.cuda.synchronize()
+    return lib.qsa_kernel_launch_count() - n0
+
+
+@pytest.mark.parametrize("name,kv_lens,cap", [
+    ("decode_bf16_b32_kv32768", (4100, 2048, 70), 4160),
+    ("mtp_verify_bf16_b4_kv262144", (9000, 129, 2), 9088),
+])
+def test_decode_one_launch_and_two_launch_paths(name, kv_lens, cap):
+    # A cache of a few thousand blocks: one launch (selection inside the decode
+    # kernel's clusters). The same rows at the start of a 12800-block cache: the
+    # selection's keys no longer fit the kernel's shared memory, so the selection
+    # kernel and then the attention kernel run. Both match the oracle.
+    w, inp = _decode(name, batch=len(kv_lens), cap=cap, kv_lens=kv_lens)
+    d = TL.upload(inp, w)
+    assert _decode_launches(w, d) == 1
+    big = 12800 * w.block_size
+    for key in ("k_cache", "v_cache", "ik_cache"):
+        t = torch.zeros((t0 := d[key]).shape[0], big, *t0.shape[2:], dtype=t0.dtype, device="cuda")
+        t[:, :cap] = t0
+        d[key] = t
+    assert _decode_launches(w, d) == 2
+    rep = decode_parity(w, inp, d=d)
+    assert len(rep["excused_near_ties"]) <= 1, rep
