@@ -139,6 +139,13 @@ __device__ __forceinline__ uint32_t pack2h(float a, float b) {
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
   return r;
 }
+// two e4m3 codes (low byte first) -> fp16x2
+__device__ __forceinline__ uint32_t e4m3x2(uint32_t two_bytes) {
+  uint32_t h;
+  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}"
+      : "=r"(h) : "r"(two_bytes));
+  return h;
+}
 // two e4m3 codes (low byte first) -> fp16x2 times an fp16x2 scale
 __device__ __forceinline__ uint32_t e4m3x2_scaled(uint32_t two_bytes, uint32_t scale2) {
   uint32_t h, r;
@@ -712,11 +719,16 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
     }
     __syncthreads();
     if (P.rotated) fwht128_rows(qf, 16, (int)threadIdx.x, (int)blockDim.x, [] { __syncthreads(); });
+    // Within each 16-dim block the MMA's k order is permuted (the same on the K
+    // side, so the dot products are unchanged): fragment positions 2t, 2t + 1,
+    // 2t + 8, 2t + 9 hold dims 4t .. 4t + 3, so that a thread's K fragment is
+    // one 32-bit word of four e4m3 codes. Logical 8-group c8 holds dims
+    // (c8 % 2) * 2 + 4m + {0, 1}, m < 4, of its block.
     for (int e = threadIdx.x; e < 16 * (kD / 8); e += blockDim.x) {
       const int r = e / (kD / 8), c8 = e % (kD / 8);
-      const float* src = qf + r * kD + c8 * 8;
-      const uint4 v = make_uint4(pack2h(src[0], src[1]), pack2h(src[2], src[3]),
-                                 pack2h(src[4], src[5]), pack2h(src[6], src[7]));
+      const float* src = qf + r * kD + (c8 >> 1) * 16 + (c8 & 1) * 2;
+      const uint4 v = make_uint4(pack2h(src[0], src[1]), pack2h(src[4], src[5]),
+                                 pack2h(src[8], src[9]), pack2h(src[12], src[13]));
       *reinterpret_cast<uint4*>(smem + kOffQ + r * kQStride + c8 * 16) = v;
     }
   }
@@ -936,41 +948,39 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
       int lim_all = 0;
       for (int i = 0; i < n_q; ++i)
         if ((qm >> i) & 1) lim_all = max(lim_all, min(kChunk, max(0, kv - n_q + i + 1 - key0)));
-      uint32_t kt, vt;   // this warp's K and V tiles (64-key bf16 tiles, or 16-key fp16 tiles)
+      uint32_t kt = 0, vt;   // K and V tiles (64-key bf16 tiles; fp8: this warp's 16-key fp16 V tile)
+      const uint32_t st8 = kOffStages + s * kF8StageBytes;   // fp8 stage: K codes, V codes, scales
       if constexpr (!kFp8) {
         kt = sbase + kOffStages + s * kStageBytes;
         vt = kt + kTileBytes;
       } else {
-        // widen this warp's 16 keys (rows 16w .. 16w + 15 of the chunk) from
-        // e4m3 times the row scale into fp16, then release the stage
-        const uint32_t st8 = kOffStages + s * kF8StageBytes;
-        const float* ks = reinterpret_cast<const float*>(smem + st8 + 2 * kF8BoxBytes);
-        const float* vs = reinterpret_cast<const float*>(smem + st8 + 2 * kF8BoxBytes + kF8ScaleBytes);
+        // widen this warp's 16 V rows (rows 16w .. 16w + 15 of the chunk) from
+        // e4m3 times the row scale to fp16; rows no query may see are zero. K is
+        // read as e4m3 straight into the MMA fragments below (its row scales
+        // multiply the scores).
         const uint32_t tiles = kOffStages + kStages * kF8StageBytes + warp * 2 * kWarpTileBytes;
-        kt = sbase + tiles;
-        vt = kt + kWarpTileBytes;
+        vt = sbase + tiles + kWarpTileBytes;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 4; ++i) {
           const int u = lane + 32 * i;
-          const int which = u >> 7, rr = (u >> 3) & 15, ch = u & 7;   // K/V, row, 16-dim chunk
-          const int row = warp * 16 + rr;                               // row in the chunk
+          const int rr = u >> 3, ch = u & 7;   // row of the warp's 16, 16-dim chunk
+          const int row = warp * 16 + rr;      // row in the chunk
           uint4 out0 = make_uint4(0, 0, 0, 0), out1 = make_uint4(0, 0, 0, 0);
-          if (!(which == 1 && row >= lim_all)) {
+          if (row < lim_all) {
             const uint4 in = *reinterpret_cast<const uint4*>(
-                smem + st8 + which * kF8BoxBytes + row * 128 + ((ch ^ (row & 7)) << 4));
-            const float scl = (which ? vs : ks)[row * g.Hkv + hk];
+                smem + st8 + kF8BoxBytes + row * 128 + ((ch ^ (row & 7)) << 4));
+            const float scl = reinterpret_cast<const float*>(
+                smem + st8 + 2 * kF8BoxBytes + kF8ScaleBytes)[row * g.Hkv + hk];
             const uint32_t s2 = pack2h(scl, scl);
             out0 = make_uint4(e4m3x2_scaled(in.x & 0xffffu, s2), e4m3x2_scaled(in.x >> 16, s2),
                               e4m3x2_scaled(in.y & 0xffffu, s2), e4m3x2_scaled(in.y >> 16, s2));
             out1 = make_uint4(e4m3x2_scaled(in.z & 0xffffu, s2), e4m3x2_scaled(in.z >> 16, s2),
                               e4m3x2_scaled(in.w & 0xffffu, s2), e4m3x2_scaled(in.w >> 16, s2));
           }
-          uint8_t* dst = smem + tiles + which * kWarpTileBytes;
+          uint8_t* dst = smem + tiles + kWarpTileBytes;
           *reinterpret_cast<uint4*>(dst + tile16_off(rr, 16 * ch)) = out0;
           *reinterpret_cast<uint4*>(dst + tile16_off(rr, 16 * ch + 8)) = out1;
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
       }
       // visible keys of this chunk per held row: keys key0 + j with j < lim
       int lim[2];
@@ -990,13 +1000,34 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
           mma_bf16(sfr[0], qa[kk], b0, b1);
           mma_bf16(sfr[1], qa[kk], b2, b3);
         } else {
-          const int key = (mi >> 1) * 8 + ri;
-          ldsm_x4(kt + tile16_off(key, kk * 16 + (mi & 1) * 8), b0, b1, b2, b3);
-          mma_f16(sfr[0], qa[kk], b0, b1);
-          mma_f16(sfr[1], qa[kk], b2, b3);
+          // B fragment of key row 16w + 8 nt + gq: the four e4m3 codes of dims
+          // kk * 16 + 4 tq .. + 3 of the 128-byte-swizzled row (the permuted k
+          // order of the Q staging), widened to two fp16x2
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            const int row = warp * 16 + nt * 8 + gq;
+            const uint32_t w4 = *reinterpret_cast<const uint32_t*>(
+                smem + st8 + row * 128 + ((kk ^ (row & 7)) << 4) + 4 * tq);
+            b0 = e4m3x2(w4 & 0xffffu);
+            b1 = e4m3x2(w4 >> 16);
+            mma_f16(sfr[nt], qa[kk], b0, b1);
+          }
+          (void)b2;
+          (void)b3;
         }
       }
-      // mask, scale, online softmax (per row across the quad's 4 threads)
+      // mask, scale, online softmax (per row across the quad's 4 threads); fp8:
+      // the K row scales multiply the scores
+      float ksc[2][2] = {{1.f, 1.f}, {1.f, 1.f}};
+      if constexpr (kFp8) {
+        const float* ks = reinterpret_cast<const float*>(smem + st8 + 2 * kF8BoxBytes);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int c = 0; c < 2; ++c) ksc[nt][c] = ks[(warp * 16 + nt * 8 + 2 * tq + c) * g.Hkv + hk];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);   // K and its scales are read, V is widened
+      }
       float x[2][4];
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
@@ -1004,7 +1035,7 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
         for (int e = 0; e < 4; ++e) {
           const int h2 = e >> 1;
           const int j = warp * 16 + nt * 8 + 2 * tq + (e & 1);
-          x[nt][e] = j < lim[h2] ? sfr[nt][e] * sc : -INFINITY;
+          x[nt][e] = j < lim[h2] ? sfr[nt][e] * (kFp8 ? sc * ksc[nt][e & 1] : sc) : -INFINITY;
         }
       float alpha[2];
 #pragma unroll
