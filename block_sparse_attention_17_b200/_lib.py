@@ -27,7 +27,7 @@ EXPORTED = [
     "qsa_prefill_workspace_size", "qsa_prefill", "qsa_select",
     "qsa_decode_workspace_size", "qsa_decode", "qsa_select_decode",
     "qsa_pool_build", "qsa_decode_noalloc", "qsa_decode_paged", "qsa_pool_build_paged",
-    "qsa_decode_fp8",
+    "qsa_decode_fp8", "qsa_decode_attend",
 ]
 
 
@@ -84,6 +84,7 @@ def _declare(lib):
         # cfg, batch, n_q, cap, kv_len, q, k, k_scale, v, v_scale, rotated, iq, ik, iw, gate,
         # pooled, out, lse, sel, nsel, dev_err, ws, ws_bytes, stream
         "qsa_decode_fp8": (I, [CFG, I, I, I, P, P, P, P, P, P, I] + [P] * 11 + [SZ, P]),
+        "qsa_decode_attend": (I, [CFG, I, I, I] + [P] * 11 + [SZ, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

@@ -253,6 +253,37 @@ def decode_noalloc(cfg: QSAConfig, q, k_cache, v_cache, iq, ik_cache, iw, gate, 
     return {"out": out, "lse": lse, "sel": sel, "nsel": nsel}
 
 
+def decode_attend(cfg: QSAConfig, q, k_cache, v_cache, gate, kv_len, sel, nsel, *, out=None,
+                  lse=None, want_lse=False, dev_err=None, workspace=None, stream=None) -> dict:
+    """Decode attention over caller-given selections (qsa_decode_attend):
+    sel [batch, n_q, k + 1] int32 block ids (ascending, nsel[b, i] used),
+    nsel [batch, n_q] int32; returns {"out", "lse"}."""
+    dt = cfg.dtype
+    batch, n_q = q.shape[0], q.shape[1]
+    cap = k_cache.shape[1]
+    _need(q, "q", dt, (batch, n_q, cfg.num_q_heads, cfg.head_dim))
+    _need(k_cache, "k_cache", dt, (batch, cap, cfg.num_kv_heads, cfg.head_dim))
+    _need(v_cache, "v_cache", dt, (batch, cap, cfg.num_kv_heads, cfg.head_dim))
+    gshape = ((batch, n_q, cfg.num_q_heads) if cfg.gate_headwise
+              else (batch, n_q, cfg.num_q_heads, cfg.head_dim))
+    _need(gate, "gate", dt, gshape)
+    _need(kv_len, "kv_len", torch.int32, (batch,))
+    _need(sel, "sel", torch.int32, (batch, n_q, cfg.topk + 1))
+    _need(nsel, "nsel", torch.int32, (batch, n_q))
+    dev = q.device
+    out = out if out is not None else torch.empty_like(q)
+    if want_lse and lse is None:
+        lse = torch.empty(batch, n_q, cfg.num_q_heads, dtype=torch.float32, device=dev)
+    ws = _workspace(decode_workspace_size(cfg, batch, n_q, cap), dev, workspace)
+    c = cfg.c()
+    st = _lib.lib().qsa_decode_attend(ctypes.byref(c), batch, n_q, cap, _ptr(kv_len), _ptr(q),
+                                      _ptr(k_cache), _ptr(v_cache), _ptr(gate), _ptr(sel),
+                                      _ptr(nsel), _ptr(out), _ptr(lse), _ptr(dev_err), _ptr(ws),
+                                      ws.numel(), _stream(stream))
+    _lib.check(st, "qsa_decode_attend")
+    return {"out": out, "lse": lse}
+
+
 def select_decode(cfg: QSAConfig, iq, ik_cache, iw, pooled_cache, kv_len, *, want_scores=False,
                   dev_err=None, workspace=None, stream=None) -> dict:
     """Decode selection only (qsa_select_decode); also finalises the pooled

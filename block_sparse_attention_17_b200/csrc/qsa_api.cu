@@ -515,6 +515,45 @@ qsa_status qsa_decode_fp8(const qsa_config* cfg, int batch, int n_q, int cap,
                      stream, Pages(), f8);
 }
 
+qsa_status qsa_decode_attend(const qsa_config* cfg, int batch, int n_q, int cap,
+                             const int32_t* kv_len, const void* q, const void* k_cache,
+                             const void* v_cache, const void* gate, const int32_t* sel,
+                             const int32_t* nsel, void* out, float* lse, int32_t* dev_err,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+  g_err[0] = 0;
+  qsa_status s = check_decode_dims(cfg, batch, n_q, cap);
+  if (s != QSA_OK) return s;
+  if (batch == 0) return QSA_OK;
+  QSA_REQUIRE(kv_len, "kv_len");
+  QSA_REQUIRE(q, "q"); QSA_REQUIRE(k_cache, "k_cache"); QSA_REQUIRE(v_cache, "v_cache");
+  QSA_REQUIRE(gate, "gate"); QSA_REQUIRE(sel, "sel"); QSA_REQUIRE(nsel, "nsel");
+  QSA_REQUIRE(out, "out");
+  if (lse) QSA_REQUIRE(lse, "lse");
+  const Geom g = make_geom(cfg);
+  const DecodeWs need = carve_decode(cfg, g, nullptr, batch, n_q, cap);
+  if (!workspace || workspace_bytes < need.bytes || ((uintptr_t)workspace & 255u))
+    return fail(QSA_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned", need.bytes);
+  const DecodeWs w = carve_decode(cfg, g, workspace, batch, n_q, cap);
+  cudaStream_t st = (cudaStream_t)stream;
+  QSA_CUDA(cudaMemsetAsync(w.counters, 0, sizeof(int) * (size_t)batch * (2 + g.Hkv), st),
+           "clear counters");
+  stage_mark(0, st);
+  stage_mark(1, st);
+  if (decode_uses_mma(cfg, g, n_q)) {
+    QSA_CUDA(launch_attn_decode_mma(g, batch, n_q, cap, w.nsplit, w.per_split, kv_len, q,
+                                    k_cache, v_cache, gate, sel, nsel, w.part_ml, w.part_o,
+                                    w.counters + batch, out, lse, dev_err ? dev_err : w.err, st),
+             "decode attention");
+  } else {
+    QSA_CUDA(launch_attn_decode_simt(cfg->dtype, g, batch, n_q, cap, w.nsplit, w.per_split,
+                                     kv_len, q, k_cache, v_cache, gate, sel, nsel, w.part_ml,
+                                     w.part_o, out, lse, st),
+             "decode attention");
+  }
+  stage_mark(2, st);
+  return QSA_OK;
+}
+
 static qsa_status check_pages(const qsa_config* cfg, int max_blocks, const int32_t* block_table,
                               int num_pages) {
   if (max_blocks <= 0 || num_pages <= 0)

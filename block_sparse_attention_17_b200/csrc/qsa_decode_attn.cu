@@ -652,13 +652,13 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
   const int kv = P.kv_len[b];
   const size_t row0 = (((size_t)b * g.Hkv + hk) * P.nsplit + split) * R;
   if (kv < n_q || kv > P.cap) {   // reported by the selection; outputs are zero
-    if constexpr (kSelDI > 0) {
-      if (split == 0 && hk == 0) {
+    if (split == 0 && hk == 0) {
+      if constexpr (kSelDI > 0) {
         const int kp1 = g.k + 1;
         for (int e = threadIdx.x; e < n_q * kp1; e += blockDim.x) P.sel_w[(size_t)b * n_q * kp1 + e] = -1;
         for (int e = threadIdx.x; e < n_q; e += blockDim.x) P.nsel_w[(size_t)b * n_q + e] = 0;
-        if (P.err && threadIdx.x == 0) atomicExch(P.err, 1);
       }
+      if (P.err && threadIdx.x == 0) atomicExch(P.err, 1);
     }
     if (split == 0)
       for (int e = threadIdx.x; e < R * kD; e += blockDim.x) {

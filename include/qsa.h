@@ -175,6 +175,24 @@ qsa_status qsa_decode(const qsa_config* cfg, int batch, int n_q, int cap,
                       float* lse, int32_t* sel, int32_t* nsel, int32_t* dev_err,
                       void* workspace, size_t workspace_bytes, void* stream);
 
+/* Decode attention over selections the caller provides: qsa_decode without
+ * its selection step (no pooling, no scoring). Used by a context-parallel
+ * decode, where each process attends its share of a global selection over its
+ * shard of the cache.
+ *   sel   [batch, n_q, k + 1] int32 (device): block ids of the caches for each
+ *         new query, ascending; the first nsel[b, i] entries are used. Ids
+ *         outside [0, cap / B) are ignored. A listed block is attended over the
+ *         positions the query can see (keys below kv_len - n_q + 1 + i); the
+ *         caller lists the query's incomplete block if it is to be attended.
+ *   nsel  [batch, n_q] int32 (device).
+ * Other arguments, the outputs and the workspace as qsa_decode; a query with
+ * no listed block gets out = 0 and lse = -inf. */
+qsa_status qsa_decode_attend(const qsa_config* cfg, int batch, int n_q, int cap,
+                             const int32_t* kv_len, const void* q, const void* k_cache,
+                             const void* v_cache, const void* gate, const int32_t* sel,
+                             const int32_t* nsel, void* out, float* lse, int32_t* dev_err,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
 /* Selection only, for decode geometry (same arguments as qsa_decode; it also
  * finalises the pooled rows completed by this step). scores: optional
  * [batch, n_q, cap/B] fp32, -inf past a query's candidates. */
