@@ -437,9 +437,9 @@ static qsa_status decode_impl(const qsa_config* cfg, int batch, int n_q, int cap
   int* sel_p = sel ? sel : w.sel;
   int* nsel_p = nsel ? nsel : w.nsel;
   stage_mark(0, st);
-  const bool vec_ok = (((uintptr_t)iq | (uintptr_t)ik_cache | (uintptr_t)pooled_cache) & 15u) == 0;
-  if (decode_uses_mma(cfg, g, n_q) && vec_ok &&
-      decode_fused_supported(g, n_q, cap, w.nsplit, f8.on)) {
+  // (every pointer was checked for 16-byte alignment above, as the fused
+  // selection's vector loads need)
+  if (decode_uses_mma(cfg, g, n_q) && decode_fused_supported(g, n_q, cap, w.nsplit, f8.on)) {
     // one launch: each (sequence, KV head) cluster pools, scores and selects,
     // then gathers K/V and merges its partials
     stage_mark(1, st);

@@ -161,11 +161,12 @@ qsa_status qsa_select(const qsa_config* cfg, int batch, int total_tokens, int ma
  *   dev_err       optional int32 (device): set to a non-zero code when a
  *                 kv_len entry is out of range; those sequences are skipped.
  * cap must be a multiple of B.
- * Execution: on bf16 geometries with indexer dim 32 or 64, at most 8 indexer
- * heads, n_q * G <= 16 and 16-byte aligned iq/ik_cache/pooled_cache, the step
- * is one kernel launch (each (sequence, KV head) thread-block cluster selects,
- * gathers and merges in on-chip memory); otherwise a selection kernel and an
- * attention kernel. Results are the same either way. */
+ * Execution: on bf16 geometries with head_dim 128, n_q * G <= 16 and a cache
+ * whose selection keys fit the kernel's shared memory (about 12000 blocks per
+ * sequence), the step is one kernel launch (each (sequence, KV head)
+ * thread-block cluster selects, gathers and merges in on-chip memory);
+ * otherwise a selection kernel and an attention kernel. Results are the same
+ * either way. */
 size_t qsa_decode_workspace_size(const qsa_config* cfg, int batch, int n_q, int cap);
 
 qsa_status qsa_decode(const qsa_config* cfg, int batch, int n_q, int cap,
