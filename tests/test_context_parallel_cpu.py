@@ -125,3 +125,42 @@ def test_global_topk_order_and_ties():
     cid = torch.tensor([[[9, 1]], [[3, 2 ** 62]]])
     ids, count = cp.global_topk(cs, cid, 2)
     assert ids.tolist() == [[1, 3]] and count.tolist() == [2]
+
+
+def test_shard_blocks_cover_the_cache_once():
+    for nblk in (1, 7, 64, 513):
+        for world in (1, 2, 3, 8):
+            ranges = [cp.shard_blocks(nblk, world, r) for r in range(world)]
+            covered = [j for b0, b1 in ranges for j in range(b0, b1)]
+            assert covered == list(range(nblk))
+
+
+def test_local_candidates_skip_the_tail_and_unused_slots():
+    # local selection: blocks 1, 5 (complete) and the tail block 7 (score -inf)
+    sel = torch.tensor([[[1, 5, 7, -1]]], dtype=torch.int32)
+    nsel = torch.tensor([[3]], dtype=torch.int32)
+    scores = torch.tensor([[[0.1, 2.0, 0.3, 0.4, 0.5, 1.5, 0.0, float("-inf")]]])
+    sc, gid = cp.local_candidates(sel, nsel, scores, 3, b0=100)
+    assert gid.tolist() == [[101, 105, 2 ** 62]]
+    assert sc[0, :2].tolist() == [2.0, 1.5] and sc[0, 2].item() == float("-inf")
+
+
+def test_local_share_adds_the_tail_on_the_last_rank_only():
+    gids = torch.tensor([[3, 10, 25, -1], [8, 9, -1, -1]])
+    kv = torch.tensor([16 * 16 + 5, 16 * 16], dtype=torch.int32)   # rows in the shard
+    sel, nsel = cp.local_share(gids, 8, 24, kv, 16, 4, is_last=True)
+    assert sel[0, 0].tolist() == [2, 16, -1, -1, -1] and nsel[0, 0].item() == 2   # tail block 16
+    assert sel[1, 0].tolist() == [0, 1, -1, -1, -1] and nsel[1, 0].item() == 2    # no tail
+    sel, nsel = cp.local_share(gids, 8, 24, kv, 16, 4, is_last=False)
+    assert sel[0, 0].tolist() == [2, -1, -1, -1, -1] and nsel[0, 0].item() == 1
+
+
+def test_merge_partials_weights_and_empty_ranks():
+    outs = torch.tensor([[[[1.0, 2.0]]], [[[3.0, 4.0]]], [[[9.0, 9.0]]]])     # [R, b, 1, 2]
+    lses = torch.tensor([[[0.0]], [[float(np.log(3.0))]], [[float("-inf")]]])  # [R, b, 1]
+    out, lse = cp.merge_partials(outs[..., None, :].squeeze(-2), lses)
+    # weights 1/4 and 3/4; the rank with nothing attended weighs nothing
+    assert torch.allclose(out, torch.tensor([[[2.5, 3.5]]]))
+    assert torch.allclose(lse, torch.tensor([[float(np.log(4.0))]]))
+    out, lse = cp.merge_partials(outs[:1] * 0, torch.full((1, 1, 1), float("-inf")))
+    assert torch.equal(out, torch.zeros(1, 1, 2)) and lse.item() == float("-inf")
