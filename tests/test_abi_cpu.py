@@ -156,3 +156,23 @@ def test_paged_decode_rejects_bad_arguments():
     st = lib.qsa_pool_build_paged(ctypes.byref(c), 32, max_blocks, None, 16, FAKE, FAKE, FAKE,
                                   None, None)
     assert st == _lib.QSA_ERR_INVALID_ARG
+
+
+def test_decode_attend_rejects_bad_arguments():
+    # attention over caller-given selections: every check happens before a launch
+    lib = _lib.lib()
+    c = cfg()
+    ws = lib.qsa_decode_workspace_size(ctypes.byref(c), 32, 1, 32768)
+
+    def call(n_q=1, cap=32768, sel=FAKE, nsel=FAKE, q=FAKE, ws_bytes=ws, c=c):
+        return lib.qsa_decode_attend(ctypes.byref(c), 32, n_q, cap, FAKE, q, FAKE, FAKE, FAKE,
+                                     sel, nsel, FAKE, None, None, ctypes.c_void_p(0x20000),
+                                     ws_bytes, None)
+    assert call(sel=None) == _lib.QSA_ERR_INVALID_ARG
+    assert call(nsel=None) == _lib.QSA_ERR_INVALID_ARG
+    assert call(q=MISALIGNED) == _lib.QSA_ERR_INVALID_ARG
+    assert call(cap=32768 + 1) == _lib.QSA_ERR_INVALID_ARG
+    assert call(n_q=5) == _lib.QSA_ERR_UNSUPPORTED
+    assert call(ws_bytes=ws - 256) == _lib.QSA_ERR_WORKSPACE
+    assert lib.qsa_decode_attend(ctypes.byref(c), 0, 1, 32768, *([None] * 11), 0,
+                                 None) == _lib.QSA_OK             # empty batch: nothing to do
