@@ -57,15 +57,25 @@ def workload_units(w):
     return sum(selected_tokens(n, w.block_size, w.topk) for n in ns), ns
 
 
+def code_sha(text: str) -> str:
+    """sha256 of C/CUDA source with its comments, trailing spaces and blank
+    lines removed: the code a counter capture describes (a comment edit does
+    not void it)."""
+    import hashlib
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = [re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines()]
+    return hashlib.sha256("\n".join(ln for ln in lines if ln).encode()).hexdigest()
+
+
 def recorded_traffic(kernel_file: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the kernel source as it is now (sha256 prefix match); else None."""
-    import hashlib
+    the kernel code as it is now (code_sha prefix match); else None."""
     src = os.path.join(ROOT, "block_sparse_attention_17_b200", "csrc", kernel_file)
     table = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not (os.path.exists(src) and os.path.exists(table)):
         return None
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    sha = code_sha(open(src).read())
     for line in open(table):
         parts = line.split()
         if len(parts) == 4 and not line.startswith("#") and parts[0] == kernel_file \

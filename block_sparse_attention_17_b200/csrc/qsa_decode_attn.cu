@@ -1,24 +1,30 @@
-// QSA decode attention, split-KV over the selected blocks (sm_100a).
+// QSA decode step (sm_100a): selection, gather and attention in one kernel.
 //
 // One decode step reads, per (sequence, KV head), only the K/V rows of the
 // union of the step's n_q queries' selections (selected complete blocks plus
 // tail blocks): the gather consumer of the selection, never a mask over the
 // whole cache (ramgpt "Porting Qwen4 to llama.cpp", section "CUDA Optimization
-// Should Follow State Correctness"). The step is bound by HBM bandwidth, so
-// the kernel is built around streaming: the union is cut into 64-key chunks,
-// each CTA takes a contiguous range of chunks of one (sequence, KV head), and
-// a producer warp streams each chunk's K and V tiles with TMA through a
-// 3-stage ring (two CTAs per SM keep about 190 KB in flight per SM).
-//
-// The arithmetic per chunk is tiny (at most 16 query rows = n_q x group
-// heads), so the four consumer warps use warp-level bf16 MMAs (m16n8k16,
-// fp32 accumulation): warp w takes keys [16w, 16w + 16) of each chunk and
-// keeps its own online-softmax state (log2 domain); the four states are
-// merged at the end into one (m, l, O) partial per row. The CTAs of one
-// (sequence, KV head) form a thread-block cluster and merge their partials by
-// log-sum-exp through distributed shared memory (each CTA takes some rows),
-// applying the sigmoid output gate; where such a cluster cannot be resident,
-// the partials go through global memory and the last CTA merges them.
+// Should Follow State Correctness"). The nsplit CTAs of one (sequence, KV head)
+// form a thread-block cluster:
+//  1. (kSelDI > 0) the cluster selects: each CTA pools the block this step
+//     completes if it owns it, scores its range of candidate blocks, and after
+//     a cluster barrier gathers a query's score keys from all CTAs through
+//     distributed shared memory and runs a radix top-k (select_in_cluster);
+//     with kSelDI == 0 the selections come from the selection kernel, which
+//     releases a per-sequence flag the CTAs wait on;
+//  2. the union is cut into 64-key chunks; each CTA takes a contiguous range,
+//     and a producer warp streams each chunk's K and V tiles with TMA through
+//     a 3-stage ring (two CTAs per SM keep about 190 KB in flight per SM);
+//  3. the per-chunk arithmetic is tiny (at most 16 query rows = n_q x group
+//     heads), so the four consumer warps use warp-level MMAs (m16n8k16, fp32
+//     accumulation): warp w takes keys [16w, 16w + 16) of each chunk with its
+//     own online-softmax state (log2 domain), merged at the end into one
+//     (m, l, O) partial per row;
+//  4. the cluster merges the partials by log-sum-exp through distributed
+//     shared memory (each CTA takes some rows) and applies the sigmoid output
+//     gate; where such a cluster cannot be resident (two-launch path only), the
+//     partials go through global memory and the last CTA merges them.
+// kFp8 reads e4m3 K/V codes with per-row scales instead of bf16 rows.
 #include <map>
 #include <mutex>
 #include <tuple>

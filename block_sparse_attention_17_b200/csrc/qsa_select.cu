@@ -520,7 +520,9 @@ __device__ int cta_topk_bits(const uint32_t* keys, int n, int k, int* out) {
   return k;
 }
 
-// ------------------------------------------------ decode: fused selection
+// ------------------------------------------------ decode: selection kernel
+// The decode step's selection as its own kernel: qsa_select_decode, and the
+// two-launch decode where the one-launch decode kernel does not apply.
 // Grid (ceil(cap/B / 64), batch); 256 threads (8 warps). CTA c owns candidate blocks
 // [64c, 64c + 64) of sequence b and
 //  1. pools the blocks of its range that this step's tokens complete (the
