@@ -76,8 +76,22 @@ def _need(t: torch.Tensor, name: str, dtype, shape=None):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
 
 
+def _one_device(dev, stream=None, **tensors):
+    """Every tensor argument must live on ``dev``, the GPU the call runs on (the
+    library launches on the current device and takes device pointers as they
+    are); a mismatch raises instead of launching."""
+    for name, t in tensors.items():
+        if t is not None and t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, expected {dev}: every tensor of one "
+                             "call must be on the same GPU")
+    if stream is not None and stream.device != dev:
+        raise ValueError(f"stream is on {stream.device}, expected {dev}")
+
+
 def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]):
     if workspace is not None:
+        if workspace.device != device:
+            raise ValueError(f"workspace is on {workspace.device}, expected {device}")
         if workspace.numel() * workspace.element_size() < nbytes:
             raise ValueError(f"workspace smaller than {nbytes} bytes")
         return workspace
@@ -137,12 +151,15 @@ def prefill(cfg: QSAConfig, q, k, v, iq, ik, iw, gate, cu_seqlens, max_seqlen: i
         pooled = torch.zeros(batch, nb, cfg.idx_dim, dtype=torch.float32, device=dev)
     ws_bytes = prefill_workspace_size(cfg, batch, T, max_seqlen)
     ws = _workspace(ws_bytes, dev, workspace)
+    _one_device(dev, stream, q=q, k=k, v=v, iq=iq, ik=ik, iw=iw, gate=gate, cu_seqlens=cu_seqlens,
+                out=out, lse=lse, sel=sel, nsel=nsel, pooled=pooled)
     c = cfg.c()
-    st = _lib.lib().qsa_prefill(ctypes.byref(c), batch, T, int(max_seqlen), _ptr(cu_seqlens),
-                                _ptr(q), _ptr(k), _ptr(v), _ptr(iq), _ptr(ik), _ptr(iw),
-                                _ptr(gate), _ptr(out), _ptr(lse), _ptr(sel), _ptr(nsel),
-                                _ptr(pooled), _ptr(ws), ws.numel(), _stream(stream))
-    _lib.check(st, "qsa_prefill")
+    with torch.cuda.device(dev):
+        st = _lib.lib().qsa_prefill(ctypes.byref(c), batch, T, int(max_seqlen), _ptr(cu_seqlens),
+                                    _ptr(q), _ptr(k), _ptr(v), _ptr(iq), _ptr(ik), _ptr(iw),
+                                    _ptr(gate), _ptr(out), _ptr(lse), _ptr(sel), _ptr(nsel),
+                                    _ptr(pooled), _ptr(ws), ws.numel(), _stream(stream))
+        _lib.check(st, "qsa_prefill")
     # int32 error word at the start of the workspace: non-zero once the call
     # has run if a kernel gave up on a bounded wait
     return {"out": out, "lse": lse, "sel": sel, "nsel": nsel, "pooled": pooled,
@@ -170,12 +187,14 @@ def select(cfg: QSAConfig, iq, ik, iw, cu_seqlens, max_seqlen: int, *, want_scor
         nb = -(-max_seqlen // cfg.block_size)
         pooled = torch.zeros(batch, nb, cfg.idx_dim, dtype=torch.float32, device=dev)
     ws = _workspace(prefill_workspace_size(cfg, batch, T, max_seqlen), dev, workspace)
+    _one_device(dev, stream, ik=ik, iw=iw, cu_seqlens=cu_seqlens)
     c = cfg.c()
-    st = _lib.lib().qsa_select(ctypes.byref(c), batch, T, int(max_seqlen), _ptr(cu_seqlens),
-                               _ptr(iq), _ptr(ik), _ptr(iw), _ptr(sel), _ptr(nsel),
-                               _ptr(scores), _ptr(pooled), _ptr(ws), ws.numel(),
-                               _stream(stream))
-    _lib.check(st, "qsa_select")
+    with torch.cuda.device(dev):
+        st = _lib.lib().qsa_select(ctypes.byref(c), batch, T, int(max_seqlen), _ptr(cu_seqlens),
+                                   _ptr(iq), _ptr(ik), _ptr(iw), _ptr(sel), _ptr(nsel),
+                                   _ptr(scores), _ptr(pooled), _ptr(ws), ws.numel(),
+                                   _stream(stream))
+        _lib.check(st, "qsa_select")
     return {"sel": sel, "nsel": nsel, "scores": scores, "pooled": pooled}
 
 
@@ -216,12 +235,16 @@ def decode(cfg: QSAConfig, q, k_cache, v_cache, iq, ik_cache, iw, gate, pooled_c
     if nsel is None and want_sel:
         nsel = torch.empty(batch, n_q, dtype=torch.int32, device=dev)
     ws = _workspace(decode_workspace_size(cfg, batch, n_q, cap), dev, workspace)
+    _one_device(dev, stream, k_cache=k_cache, v_cache=v_cache, iq=iq, ik_cache=ik_cache, iw=iw,
+                gate=gate, pooled_cache=pooled_cache, kv_len=kv_len, out=out, lse=lse, sel=sel,
+                nsel=nsel, dev_err=dev_err)
     c = cfg.c()
-    st = _lib.lib().qsa_decode(ctypes.byref(c), batch, n_q, cap, _ptr(kv_len), _ptr(q),
-                               _ptr(k_cache), _ptr(v_cache), _ptr(iq), _ptr(ik_cache), _ptr(iw),
-                               _ptr(gate), _ptr(pooled_cache), _ptr(out), _ptr(lse), _ptr(sel),
-                               _ptr(nsel), _ptr(dev_err), _ptr(ws), ws.numel(), _stream(stream))
-    _lib.check(st, "qsa_decode")
+    with torch.cuda.device(dev):
+        st = _lib.lib().qsa_decode(ctypes.byref(c), batch, n_q, cap, _ptr(kv_len), _ptr(q),
+                                   _ptr(k_cache), _ptr(v_cache), _ptr(iq), _ptr(ik_cache), _ptr(iw),
+                                   _ptr(gate), _ptr(pooled_cache), _ptr(out), _ptr(lse), _ptr(sel),
+                                   _ptr(nsel), _ptr(dev_err), _ptr(ws), ws.numel(), _stream(stream))
+        _lib.check(st, "qsa_decode")
     return {"out": out, "lse": lse, "sel": sel, "nsel": nsel}
 
 
@@ -243,13 +266,17 @@ def decode_noalloc(cfg: QSAConfig, q, k_cache, v_cache, iq, ik_cache, iw, gate, 
         sel = torch.empty(batch, n_q, cfg.topk + 1, dtype=torch.int32, device=dev)
     if nsel is None and want_sel:
         nsel = torch.empty(batch, n_q, dtype=torch.int32, device=dev)
+    _one_device(dev, stream, k_cache=k_cache, v_cache=v_cache, iq=iq, ik_cache=ik_cache, iw=iw,
+                gate=gate, pooled_cache=pooled_cache, kv_len=kv_len, out=out, lse=lse, sel=sel,
+                nsel=nsel, dev_err=dev_err)
     c = cfg.c()
-    st = _lib.lib().qsa_decode_noalloc(ctypes.byref(c), batch, n_q, cap, _ptr(kv_len), _ptr(q),
-                                       _ptr(k_cache), _ptr(v_cache), _ptr(iq), _ptr(ik_cache),
-                                       _ptr(iw), _ptr(gate), _ptr(pooled_cache), _ptr(out),
-                                       _ptr(lse), _ptr(sel), _ptr(nsel), _ptr(dev_err),
-                                       _stream(stream))
-    _lib.check(st, "qsa_decode_noalloc")
+    with torch.cuda.device(dev):
+        st = _lib.lib().qsa_decode_noalloc(ctypes.byref(c), batch, n_q, cap, _ptr(kv_len), _ptr(q),
+                                           _ptr(k_cache), _ptr(v_cache), _ptr(iq), _ptr(ik_cache),
+                                           _ptr(iw), _ptr(gate), _ptr(pooled_cache), _ptr(out),
+                                           _ptr(lse), _ptr(sel), _ptr(nsel), _ptr(dev_err),
+                                           _stream(stream))
+        _lib.check(st, "qsa_decode_noalloc")
     return {"out": out, "lse": lse, "sel": sel, "nsel": nsel}
 
 
@@ -275,12 +302,15 @@ def decode_attend(cfg: QSAConfig, q, k_cache, v_cache, gate, kv_len, sel, nsel, 
     if want_lse and lse is None:
         lse = torch.empty(batch, n_q, cfg.num_q_heads, dtype=torch.float32, device=dev)
     ws = _workspace(decode_workspace_size(cfg, batch, n_q, cap), dev, workspace)
+    _one_device(dev, stream, k_cache=k_cache, v_cache=v_cache, gate=gate, kv_len=kv_len, sel=sel,
+                nsel=nsel, out=out, lse=lse, dev_err=dev_err)
     c = cfg.c()
-    st = _lib.lib().qsa_decode_attend(ctypes.byref(c), batch, n_q, cap, _ptr(kv_len), _ptr(q),
-                                      _ptr(k_cache), _ptr(v_cache), _ptr(gate), _ptr(sel),
-                                      _ptr(nsel), _ptr(out), _ptr(lse), _ptr(dev_err), _ptr(ws),
-                                      ws.numel(), _stream(stream))
-    _lib.check(st, "qsa_decode_attend")
+    with torch.cuda.device(dev):
+        st = _lib.lib().qsa_decode_attend(ctypes.byref(c), batch, n_q, cap, _ptr(kv_len), _ptr(q),
+                                          _ptr(k_cache), _ptr(v_cache), _ptr(gate), _ptr(sel),
+                                          _ptr(nsel), _ptr(out), _ptr(lse), _ptr(dev_err), _ptr(ws),
+                                          ws.numel(), _stream(stream))
+        _lib.check(st, "qsa_decode_attend")
     return {"out": out, "lse": lse}
 
 
@@ -302,12 +332,15 @@ def select_decode(cfg: QSAConfig, iq, ik_cache, iw, pooled_cache, kv_len, *, wan
     scores = (torch.empty(batch, n_q, cap // cfg.block_size, dtype=torch.float32, device=dev)
               if want_scores else None)
     ws = _workspace(decode_workspace_size(cfg, batch, n_q, cap), dev, workspace)
+    _one_device(dev, stream, ik_cache=ik_cache, iw=iw, pooled_cache=pooled_cache, kv_len=kv_len,
+                dev_err=dev_err)
     c = cfg.c()
-    st = _lib.lib().qsa_select_decode(ctypes.byref(c), batch, n_q, cap, _ptr(kv_len), _ptr(iq),
-                                      _ptr(ik_cache), _ptr(iw), _ptr(pooled_cache), _ptr(sel),
-                                      _ptr(nsel), _ptr(scores), _ptr(dev_err), _ptr(ws),
-                                      ws.numel(), _stream(stream))
-    _lib.check(st, "qsa_select_decode")
+    with torch.cuda.device(dev):
+        st = _lib.lib().qsa_select_decode(ctypes.byref(c), batch, n_q, cap, _ptr(kv_len), _ptr(iq),
+                                          _ptr(ik_cache), _ptr(iw), _ptr(pooled_cache), _ptr(sel),
+                                          _ptr(nsel), _ptr(scores), _ptr(dev_err), _ptr(ws),
+                                          ws.numel(), _stream(stream))
+        _lib.check(st, "qsa_select_decode")
     return {"sel": sel, "nsel": nsel, "scores": scores}
 
 
@@ -320,10 +353,13 @@ def pool_build(cfg: QSAConfig, ik_cache, kv_len, pooled_cache=None, *, dev_err=N
     if pooled_cache is None:
         pooled_cache = torch.zeros(batch, cap // cfg.block_size, cfg.idx_dim,
                                    dtype=torch.float32, device=ik_cache.device)
+    dev = ik_cache.device
+    _one_device(dev, stream, kv_len=kv_len, pooled_cache=pooled_cache, dev_err=dev_err)
     c = cfg.c()
-    st = _lib.lib().qsa_pool_build(ctypes.byref(c), batch, cap, _ptr(kv_len), _ptr(ik_cache),
-                                   _ptr(pooled_cache), _ptr(dev_err), _stream(stream))
-    _lib.check(st, "qsa_pool_build")
+    with torch.cuda.device(dev):
+        st = _lib.lib().qsa_pool_build(ctypes.byref(c), batch, cap, _ptr(kv_len), _ptr(ik_cache),
+                                       _ptr(pooled_cache), _ptr(dev_err), _stream(stream))
+        _lib.check(st, "qsa_pool_build")
     return pooled_cache
 
 
@@ -359,14 +395,18 @@ def decode_paged(cfg: QSAConfig, q, k_pages, v_pages, iq, ik_pages, iw, gate, po
     if nsel is None and want_sel:
         nsel = torch.empty(batch, n_q, dtype=torch.int32, device=dev)
     ws = _workspace(decode_workspace_size(cfg, batch, n_q, max_blocks * B), dev, workspace)
+    _one_device(dev, stream, k_pages=k_pages, v_pages=v_pages, iq=iq, ik_pages=ik_pages, iw=iw,
+                gate=gate, pooled_cache=pooled_cache, kv_len=kv_len, block_table=block_table,
+                out=out, lse=lse, sel=sel, nsel=nsel, dev_err=dev_err)
     c = cfg.c()
-    st = _lib.lib().qsa_decode_paged(ctypes.byref(c), batch, n_q, max_blocks, _ptr(block_table),
-                                     num_pages, _ptr(kv_len), _ptr(q), _ptr(k_pages),
-                                     _ptr(v_pages), _ptr(iq), _ptr(ik_pages), _ptr(iw),
-                                     _ptr(gate), _ptr(pooled_cache), _ptr(out), _ptr(lse),
-                                     _ptr(sel), _ptr(nsel), _ptr(dev_err), _ptr(ws), ws.numel(),
-                                     _stream(stream))
-    _lib.check(st, "qsa_decode_paged")
+    with torch.cuda.device(dev):
+        st = _lib.lib().qsa_decode_paged(ctypes.byref(c), batch, n_q, max_blocks, _ptr(block_table),
+                                         num_pages, _ptr(kv_len), _ptr(q), _ptr(k_pages),
+                                         _ptr(v_pages), _ptr(iq), _ptr(ik_pages), _ptr(iw),
+                                         _ptr(gate), _ptr(pooled_cache), _ptr(out), _ptr(lse),
+                                         _ptr(sel), _ptr(nsel), _ptr(dev_err), _ptr(ws), ws.numel(),
+                                         _stream(stream))
+        _lib.check(st, "qsa_decode_paged")
     return {"out": out, "lse": lse, "sel": sel, "nsel": nsel}
 
 
@@ -381,11 +421,15 @@ def pool_build_paged(cfg: QSAConfig, ik_pages, kv_len, block_table, pooled_cache
     if pooled_cache is None:
         pooled_cache = torch.zeros(batch, max_blocks, cfg.idx_dim, dtype=torch.float32,
                                    device=ik_pages.device)
+    dev = ik_pages.device
+    _one_device(dev, stream, kv_len=kv_len, block_table=block_table, pooled_cache=pooled_cache,
+                dev_err=dev_err)
     c = cfg.c()
-    st = _lib.lib().qsa_pool_build_paged(ctypes.byref(c), batch, max_blocks, _ptr(block_table),
-                                         num_pages, _ptr(kv_len), _ptr(ik_pages),
-                                         _ptr(pooled_cache), _ptr(dev_err), _stream(stream))
-    _lib.check(st, "qsa_pool_build_paged")
+    with torch.cuda.device(dev):
+        st = _lib.lib().qsa_pool_build_paged(ctypes.byref(c), batch, max_blocks, _ptr(block_table),
+                                             num_pages, _ptr(kv_len), _ptr(ik_pages),
+                                             _ptr(pooled_cache), _ptr(dev_err), _stream(stream))
+        _lib.check(st, "qsa_pool_build_paged")
     return pooled_cache
 
 
@@ -424,12 +468,16 @@ def decode_fp8(cfg: QSAConfig, q, k_cache, k_scale, v_cache, v_scale, iq, ik_cac
     if nsel is None and want_sel:
         nsel = torch.empty(batch, n_q, dtype=torch.int32, device=dev)
     ws = _workspace(decode_workspace_size(cfg, batch, n_q, cap), dev, workspace)
+    _one_device(dev, stream, k_cache=k_cache, k_scale=k_scale, v_cache=v_cache, v_scale=v_scale,
+                iq=iq, ik_cache=ik_cache, iw=iw, gate=gate, pooled_cache=pooled_cache,
+                kv_len=kv_len, out=out, lse=lse, sel=sel, nsel=nsel, dev_err=dev_err)
     c = cfg.c()
-    st = _lib.lib().qsa_decode_fp8(ctypes.byref(c), batch, n_q, cap, _ptr(kv_len), _ptr(q),
-                                   _ptr(k_cache), _ptr(k_scale), _ptr(v_cache), _ptr(v_scale),
-                                   1 if rotated else 0, _ptr(iq), _ptr(ik_cache), _ptr(iw),
-                                   _ptr(gate), _ptr(pooled_cache), _ptr(out), _ptr(lse),
-                                   _ptr(sel), _ptr(nsel), _ptr(dev_err), _ptr(ws), ws.numel(),
-                                   _stream(stream))
-    _lib.check(st, "qsa_decode_fp8")
+    with torch.cuda.device(dev):
+        st = _lib.lib().qsa_decode_fp8(ctypes.byref(c), batch, n_q, cap, _ptr(kv_len), _ptr(q),
+                                       _ptr(k_cache), _ptr(k_scale), _ptr(v_cache), _ptr(v_scale),
+                                       1 if rotated else 0, _ptr(iq), _ptr(ik_cache), _ptr(iw),
+                                       _ptr(gate), _ptr(pooled_cache), _ptr(out), _ptr(lse),
+                                       _ptr(sel), _ptr(nsel), _ptr(dev_err), _ptr(ws), ws.numel(),
+                                       _stream(stream))
+        _lib.check(st, "qsa_decode_fp8")
     return {"out": out, "lse": lse, "sel": sel, "nsel": nsel}

@@ -51,11 +51,18 @@ extern "C" qsa_status qsa_decode_noalloc(const qsa_config* cfg, int batch, int n
   }
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+  if (e != cudaSuccess) {
     snprintf(msg, sizeof(msg), "qsa_decode_noalloc: no usable current device (%s)",
              cudaGetErrorString(e));
     qsa::set_last_error(msg);
     return QSA_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) {
+    snprintf(msg, sizeof(msg),
+             "qsa_decode_noalloc: device ordinal %d is beyond the %d devices it serves", dev,
+             kMaxDevices);
+    qsa::set_last_error(msg);
+    return QSA_ERR_UNSUPPORTED;
   }
   void* ptr = nullptr;
   {

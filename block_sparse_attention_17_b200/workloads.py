@@ -120,19 +120,33 @@ WORKLOAD_ORDER = [
 
 def round_to_bf16(x: np.ndarray) -> np.ndarray:
     """Round float32 values to the nearest bf16 value (ties to even), returned
-    as float32. Inputs are finite draws, so NaN handling is not needed."""
-    x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32)
-    lsb = (u >> np.uint32(16)) & np.uint32(1)
-    r = (u + np.uint32(0x7FFF) + lsb) & np.uint32(0xFFFF0000)
-    return r.view(np.float32)
+    as a new float32 array. Inputs are finite draws, so NaN handling is not
+    needed."""
+    return _round_bf16_inplace(np.array(x, dtype=np.float32, order="C"))
+
+
+def _round_bf16_inplace(x: np.ndarray) -> np.ndarray:
+    """round_to_bf16 on a C-contiguous float32 array that the caller owns,
+    in place, one slice at a time (no array-sized temporaries)."""
+    u = x.reshape(-1).view(np.uint32)
+    step = 1 << 20
+    buf = np.empty(min(step, u.size), dtype=np.uint32)
+    for s0 in range(0, u.size, step):
+        seg = u[s0:s0 + step]
+        lsb = buf[:seg.size]
+        np.right_shift(seg, np.uint32(16), out=lsb)
+        lsb &= np.uint32(1)
+        lsb += np.uint32(0x7FFF)
+        seg += lsb
+        seg &= np.uint32(0xFFFF0000)
+    return x
 
 
 def _normal(rng, shape, scale, dtype):
     x = rng.standard_normal(size=shape, dtype=np.float32)
     if scale != 1.0:
         x *= np.float32(scale)
-    return round_to_bf16(x) if dtype == "bf16" else x
+    return _round_bf16_inplace(x) if dtype == "bf16" else x
 
 
 def _uniform(rng, shape, dtype_unused=None):

@@ -214,7 +214,10 @@ qsa_status qsa_select_decode(const qsa_config* cfg, int batch, int n_q, int cap,
  *   QSA_ERR_WORKSPACE (qsa_last_error() says how much it needs).
  * - The first call on a device looks up the array's device address (once per
  *   device, with that device current), so make the first call on each device
- *   before any stream capture.
+ *   before any stream capture. The address is kept for the life of the
+ *   process: after cudaDeviceReset() on a device, this entry point must not be
+ *   called on that device again. Devices with ordinal 64 or more are refused
+ *   (QSA_ERR_UNSUPPORTED).
  * - All calls on a device share the one array, which keeps the last call's
  *   contents (no part of it needs to start at zero): calls that overlap on the
  *   GPU, on different streams or host threads, race and corrupt each other. */
