@@ -144,6 +144,23 @@ def config_of(w, world=1):
     return c
 
 
+def host_cores() -> int:
+    """CPU cores this process may use: its affinity mask, capped by a cgroup
+    CPU quota when one is set."""
+    try:
+        n = len(os.sched_getaffinity(0))
+    except Exception:
+        n = os.cpu_count() or 1
+    try:
+        with open("/sys/fs/cgroup/cpu.max") as f:
+            quota, period = f.read().split()[:2]
+        if quota != "max":
+            n = min(n, max(1, int(int(quota) // int(period))))
+    except Exception:
+        pass
+    return max(1, n)
+
+
 def make_inputs(w):
     return make_prefill_inputs(w) if w.kind == "prefill" else make_decode_inputs(w)
 
@@ -700,7 +717,7 @@ def run_ours(args, rank, world, dist):
         gen_s[w.name] = round(time.perf_counter() - t0, 2)
     cpu, oracle_sel = {}, {}
     do_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
-    cores = args.cpu_cores or (os.cpu_count() or 1)
+    cores = args.cpu_cores or host_cores()
     if do_cpu:
         for w in all_ws:
             cpu[w.name], oracle_sel[w.name], _ = cpu_leg(w, inputs[w.name], args.cpu_seconds,
@@ -775,7 +792,7 @@ def run_reference(args):
     random sample of the workload's queries, spread over all cores."""
     w = WORKLOADS[args.workload]
     inp = make_inputs(w)
-    cores = args.cpu_cores or (os.cpu_count() or 1)
+    cores = args.cpu_cores or host_cores()
     tot_tok, tot_s, tot_q = 0.0, 0.0, 0
     one = None
     for i in range(args.warmup + args.steps):

@@ -25,6 +25,7 @@
 //     gate; where such a cluster cannot be resident (two-launch path only), the
 //     partials go through global memory and the last CTA merges them.
 // kFp8 reads e4m3 K/V codes with per-row scales instead of bf16 rows.
+#include <cstdlib>
 #include <map>
 #include <mutex>
 #include <tuple>
@@ -106,6 +107,10 @@ struct DecParams {
   int* sel_w;                        // [batch, n_q, k + 1] selections out
   int* nsel_w;                       // [batch, n_q]
   int fo_keys, fo_kbar, fo_iq, fo_iw, fo_new, fo_hist;   // byte offsets in the ring's space
+  int spec_m;                        // blocks per query whose K/V each CTA prefetches into L2
+                                     // before the cluster's top-k (its best-scored ones)
+  int early;                         // the first scoring pass's pooled rows are copied into
+                                     // shared memory at kernel entry (stage_pooled_early)
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
@@ -235,9 +240,17 @@ __device__ __forceinline__ void cta_topk_radix(const uint32_t* keys, int n, int 
       for (int e = tid; e < 256; e += nthr) hist[e] = 0;
       __syncthreads();
     }
-    for (int j = tid; j < n; j += nthr) {
-      const uint32_t key = keys[j];
-      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+    // lanes with the same digit add their count with one atomic (the keys of a
+    // query crowd into few digit values, which would serialise plain atomics)
+    for (int j0 = warp * 32; j0 < n; j0 += nthr) {   // warp-uniform
+      const int j = j0 + lane;
+      int bin = -1;
+      if (j < n) {
+        const uint32_t key = keys[j];
+        if ((key & pmask) == prefix) bin = (int)((key >> shift) & 255u);
+      }
+      const unsigned peers = __match_any_sync(kFull, bin);
+      if (bin >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
     }
     __syncthreads();
     if (warp == 0) {
@@ -322,10 +335,33 @@ __device__ __forceinline__ uint4 ld_cluster_u32x4(uint32_t addr) {
 }
 
 // Chunk of candidate blocks one CTA of the cluster scores: a multiple of 4, so
-// that the gather below moves 16-byte groups owned by one CTA.
-__host__ __device__ __forceinline__ int select_range(int nc_last, int nsplit) {
-  const int per = ((nc_last > 1 ? nc_last : 1) + nsplit - 1) / nsplit;
+// that the gather below moves 16-byte groups owned by one CTA. The ranges split
+// the cache's blocks (cap / B, known before the sequence's length is read), so
+// that a CTA can start loading its pooled rows at once.
+__host__ __device__ __forceinline__ int select_range(int nblk_cap, int nsplit) {
+  const int per = ((nblk_cap > 1 ? nblk_cap : 1) + nsplit - 1) / nsplit;
   return (per + 3) & ~3;
+}
+
+// Starts the copies of the first scoring pass's pooled rows of this CTA's range
+// into shared memory (cp.async, padded rows), before the sequence's length is
+// known; rows past the sequence's complete blocks are never scored, and the row
+// of a block this step completes is replaced by its fresh pooling.
+template <int kDI>
+__device__ __forceinline__ void stage_pooled_early(const DecParams& P, uint8_t* smem, int split,
+                                                   int b) {
+  constexpr int kStride = kDI + 4;
+  const int nblk_cap = P.cap / P.g.B;
+  const int per = select_range(nblk_cap, P.nsplit);
+  const int j0 = split * per;
+  const int rows = min(min(kSelRows, per), nblk_cap - j0);
+  float* kbar_s = reinterpret_cast<float*>(smem + kOffStages + P.fo_kbar);
+  const float* src = P.pooled + ((size_t)b * nblk_cap + j0) * kDI;
+  for (int e = threadIdx.x; e < rows * (kDI / 4); e += blockDim.x) {
+    const int r = e / (kDI / 4), d4 = e - r * (kDI / 4);
+    cp_async16(smem_u32(kbar_s + r * kStride + 4 * d4), src + (size_t)r * kDI + 4 * d4);
+  }
+  cp_async_commit();
 }
 
 // The selection step of one decode step, done by the cluster of one (sequence,
@@ -348,7 +384,7 @@ template <int kDI>
 __device__ __forceinline__ void select_prefetch(const DecParams& P, int kv, int split, int b) {
   const Geom& g = P.g;
   const int nblk_cap = P.cap / g.B, nc_last = kv / g.B;
-  const int per = select_range(nc_last, P.nsplit);
+  const int per = select_range(nblk_cap, P.nsplit);
   const int j0 = split * per, j1 = min(nc_last, j0 + per);
   if (j1 > j0)
     bulk_prefetch_l2(P.pooled + ((size_t)b * nblk_cap + j0) * kDI, (uint32_t)(j1 - j0) * kDI * 4u);
@@ -366,9 +402,72 @@ __device__ __forceinline__ void select_prefetch(const DecParams& P, int kv, int 
     bulk_prefetch_l2(P.iq + (size_t)b * P.n_q * g.Hi * kDI, (uint32_t)(P.n_q * g.Hi * kDI * 2));
 }
 
+// Speculation while the cluster's top-k runs: the K and V rows (this CTA's KV
+// head) of the spec_m best-scored blocks of this CTA's own candidate range, per
+// query, are prefetched into L2. The blocks the top-k then selects in this range
+// are the range's best ones (a range holds about k / nsplit of them), so most of
+// the selected bytes are on their way from HBM before the selection is known;
+// a prefetched block that is not selected only costs its bandwidth. Warp 0;
+// keys_mine holds the range's keys per query (keys of complete blocks only).
+__device__ __forceinline__ void spec_prefetch(const DecParams& P, const CUtensorMap* tmK,
+                                              const CUtensorMap* tmV, const uint32_t* keys_mine,
+                                              int per, int j0, int j1, int kv, int b, int hk,
+                                              bool fp8) {
+  const Geom& g = P.g;
+  const int lane = threadIdx.x & 31;
+  const int nblk_cap = P.cap / g.B;
+  for (int i = 0; i < P.n_q; ++i) {
+    const int nc_i = (kv - P.n_q + 1 + i) / g.B;
+    const int cnt = min(min(j1, nc_i) - j0, 32 * 32);   // keys of query i in the range (scan cap)
+    uint32_t taken = 0u;                                 // bit t: key lane + 32 t already taken
+    for (int it = 0; it < P.spec_m && cnt > 0; ++it) {
+      uint32_t best = 0u;
+      int bestr = -1;
+      for (int r = lane, t = 0; r < cnt; r += 32, ++t) {
+        if ((taken >> t) & 1u) continue;
+        const uint32_t key = keys_mine[i * per + r];
+        if (bestr < 0 || key > best) {
+          best = key;
+          bestr = r;
+        }
+      }
+      const uint32_t wmax = __reduce_max_sync(kFull, bestr >= 0 ? best : 0u);
+      const uint32_t cand = __ballot_sync(kFull, bestr >= 0 && best == wmax);
+      if (!cand) break;
+      const int src = __ffs(cand) - 1;
+      const int rsel = __shfl_sync(kFull, bestr, src);
+      if (lane == src) taken |= 1u << (rsel >> 5);
+      if (lane == 0) {
+        const int j = j0 + rsel;
+        long long row = (long long)b * P.cap + (long long)j * g.B;
+        bool ok = true;
+        if (P.table) {
+          const int page = P.table[(size_t)b * nblk_cap + j];
+          ok = page >= 0 && page < P.num_pages;
+          row = (long long)page * g.B;
+        }
+        if (ok) {
+          for (int off = 0; off < g.B; off += kChunk) {
+            if (fp8) {
+              tma_prefetch_l2_3d(tmK, 0, hk, (int)(row + off));
+              tma_prefetch_l2_3d(tmV, 0, hk, (int)(row + off));
+            } else {
+              tma_prefetch_l2_3d(tmK, 0, hk, (int)(row + off));
+              tma_prefetch_l2_3d(tmK, 64, hk, (int)(row + off));
+              tma_prefetch_l2_3d(tmV, 0, hk, (int)(row + off));
+              tma_prefetch_l2_3d(tmV, 64, hk, (int)(row + off));
+            }
+          }
+        }
+      }
+    }
+  }
+}
+
 template <int kDI>
 __device__ __forceinline__ void select_in_cluster(const DecParams& P, uint8_t* smem, int kv, int split, int b,
-                                  int hk, uint32_t* qbits, int words) {
+                                  int hk, uint32_t* qbits, int words, const CUtensorMap* tmK,
+                                  const CUtensorMap* tmV, bool fp8) {
   constexpr int kStride = kDI + 4;                 // 16-byte rows; 8 rows of a warp hit distinct banks
   constexpr int kQStrideI = kDI + 4;
   constexpr int kRows = kSelRows;                 // candidate blocks per scoring pass
@@ -377,7 +476,7 @@ __device__ __forceinline__ void select_in_cluster(const DecParams& P, uint8_t* s
   const int tid = threadIdx.x, nthr = blockDim.x, warp = tid >> 5, lane = tid & 31;
   const int nblk_cap = P.cap / g.B;
   const int nc_last = kv / g.B;
-  const int per = select_range(nc_last, P.nsplit);
+  const int per = select_range(nblk_cap, P.nsplit);
   const int j0 = split * per, j1 = min(nc_last, j0 + per);
   uint8_t* ring = smem + kOffStages;
   uint32_t* mm_mine = reinterpret_cast<uint32_t*>(ring);                    // [4][2] largest, smallest key
@@ -429,7 +528,18 @@ __device__ __forceinline__ void select_in_cluster(const DecParams& P, uint8_t* s
   uint32_t qhi[4] = {0u, 0u, 0u, 0u}, qlo[4] = {~0u, ~0u, ~0u, ~0u};
   for (int r0 = j0; r0 < j1; r0 += kRows) {
     const int rows = min(kRows, j1 - r0);
-    {   // every load of the pass is issued before the first store
+    if (r0 == j0 && P.early) {
+      // the rows came by the copies started at kernel entry; the rows of the
+      // blocks this step completes are the fresh poolings
+      cp_async_wait_all();
+      __syncthreads();
+      for (int e = tid; e < (jn_hi - jn_lo) * (kDI / 4); e += nthr) {
+        const int r = e / (kDI / 4), d4 = e - r * (kDI / 4);
+        if (jn_lo + r - r0 < rows)
+          *reinterpret_cast<float4*>(kbar_s + (jn_lo + r - r0) * kStride + 4 * d4) =
+              *reinterpret_cast<const float4*>(new_s + r * kDI + 4 * d4);
+      }
+    } else {   // every load of the pass is issued before the first store
       constexpr int kLd = (kRows * (kDI / 4) + kThreads - 1) / kThreads;   // float4 per thread
       float4 v[kLd];
 #pragma unroll
@@ -513,6 +623,8 @@ __device__ __forceinline__ void select_in_cluster(const DecParams& P, uint8_t* s
       }
     }
   }
+  cp_async_wait_all();   // (a CTA with no candidates never waited on its early copies)
+  if (P.spec_m > 0 && warp == 0) spec_prefetch(P, tmK, tmV, keys_mine, per, j0, j1, kv, b, hk, fp8);
   cluster_sync_all();   // every CTA's keys (and their extremes) are in place
   const uint32_t mine_s = smem_u32(keys_mine), mm_s = smem_u32(mm_mine);
   // With several queries, CTA s selects queries s, s + nsplit, ... and the
@@ -613,7 +725,10 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
   const int split = blockIdx.x, b = blockIdx.y, hk = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = g.G, n_q = P.n_q, R = n_q * G;
-  if constexpr (kSelDI > 0) grid_dependency_wait();   // every input may come from the previous kernel
+  if constexpr (kSelDI > 0) {
+    grid_dependency_wait();   // every input may come from the previous kernel
+    if (P.early) stage_pooled_early<kSelDI>(P, smem, split, b);
+  }
   // Inputs that do not depend on the sequence's length are loaded together
   // with it, into registers: Q rows r = i * G + gi (query i, head hk * G + gi;
   // zero beyond R), the gate rows this CTA merges (cluster merge: rows split,
@@ -658,6 +773,7 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
   const int kv = P.kv_len[b];
   const size_t row0 = (((size_t)b * g.Hkv + hk) * P.nsplit + split) * R;
   if (kv < n_q || kv > P.cap) {   // reported by the selection; outputs are zero
+    if constexpr (kSelDI > 0) cp_async_wait_all();   // no copy may land after the CTA left
     if (split == 0 && hk == 0) {
       if constexpr (kSelDI > 0) {
         const int kp1 = g.k + 1;
@@ -789,7 +905,7 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
       float* iw_s = reinterpret_cast<float*>(smem + kOffStages + P.fo_iw);
       if (threadIdx.x < n_q * g.Hi) iw_s[threadIdx.x] = iwreg;
     }
-    select_in_cluster<kSelDI>(P, smem, kv, split, b, hk, qbits, words);
+    select_in_cluster<kSelDI>(P, smem, kv, split, b, hk, qbits, words, &tmK, &tmV, kFp8);
   } else {
     // the selections come from the selection kernel: wait for this sequence's
     // flag (bounded), or for the whole selection grid
@@ -1471,6 +1587,17 @@ bool fused_layout(const Geom& g, int n_q, int cap, int nsplit, DecParams* p) {
   return off <= (long long)kStages * kStageBytes;
 }
 
+// Blocks per query each CTA of a decode cluster prefetches into L2 ahead of the
+// cluster's top-k (QSA_SPEC_BLOCKS overrides the default, 0 turns it off).
+int spec_prefetch_blocks(const Geom& g, int nsplit) {
+  static const int env = [] {
+    const char* e = getenv("QSA_SPEC_BLOCKS");
+    return e ? atoi(e) : -1;
+  }();
+  if (env >= 0) return env;
+  return (g.k + nsplit - 1) / nsplit + 1;
+}
+
 template <bool kFp8>
 const void* fused_kernel(int di) {
   return di == 64 ? reinterpret_cast<const void*>(attn_decode_mma_kernel<kFp8, 64>)
@@ -1596,6 +1723,11 @@ cudaError_t launch_decode_fused(const Geom& g, int batch, int n_q, int cap, int 
   p.pooled = si.pooled;
   p.sel_w = si.sel;
   p.nsel_w = si.nsel;
+  // about k / nsplit of a range's blocks are selected; one more is prefetched
+  p.spec_m = spec_prefetch_blocks(g, nsplit);
+  // the fp8 kernel stages its query rows at the end of the fp8 ring, which the
+  // early pooled rows must not reach
+  p.early = !f8.on || p.fo_iq <= kStages * kF8StageBytes;
   const int smem = decode_smem(g, n_q, cap);
   const void* kern = f8.on ? fused_kernel<true>(g.di) : fused_kernel<false>(g.di);
   const cudaError_t e = set_max_dynamic_smem(kern, smem);

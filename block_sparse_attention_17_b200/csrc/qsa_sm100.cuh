@@ -145,6 +145,27 @@ __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes
                "r"(bytes)
                : "memory");
 }
+// 16-byte asynchronous copy global -> shared (both addresses 16-byte aligned),
+// tracked by the issuing thread's cp.async groups.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src))
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+// Prefetch of one tiled box of a tensor map into L2 (no shared memory, no
+// completion to wait for; a hint that the box will be loaded soon).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -298,10 +319,11 @@ __device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t addr) {
 // 2^x without the MUFU unit, for part of the softmax exponentials: range
 // reduction x = j + f with j = round(x), f in [-1/2, 1/2] (the rounding done by
 // adding 1.5 * 2^23), a cubic for 2^f, and 2^j added into the exponent bits.
-// The cubic's coefficients are a relative-error least-squares fit of 2^f on
-// [-1/2, 1/2] made for this library (max relative error 7.6e-5, far below the
-// 2^-9 rounding of the bf16 probabilities it feeds). Inputs below -126 give
-// about 2^-126 instead of 0.
+// The cubic's coefficients were fitted for this library to keep the largest
+// relative error of 2^f on [-1/2, 1/2] small; the error curve is close to
+// equi-ripple (minimax), with a maximum of 7.6e-5, far below the 2^-9 rounding
+// of the bf16 probabilities it feeds. Inputs below -126 give about 2^-126
+// instead of 0.
 __device__ __forceinline__ float exp2_poly(float x) {
   constexpr float kMagic = 12582912.0f;    // 1.5 * 2^23
   x = fmaxf(x, -126.0f);

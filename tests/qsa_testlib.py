@@ -5,6 +5,7 @@ from __future__ import annotations
 import numpy as np
 import torch
 
+from block_sparse_attention_17_b200.workloads import round_to_bf16
 from oracle import qsa_oracle as O
 
 # tolerances on outputs (max abs error), by input dtype
@@ -17,6 +18,12 @@ NEAR_TIE_REL = 1e-5
 
 def tdtype(w):
     return torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+
+def round_like(x: np.ndarray, w) -> np.ndarray:
+    """fp32 draws as the workload's dtype sees them (bf16 values for bf16
+    workloads), so that the oracle and the GPU get the same numbers."""
+    return round_to_bf16(x) if w.dtype == "bf16" else np.asarray(x, np.float32)
 
 
 def upload(inp: dict, w, device="cuda") -> dict:
