@@ -28,6 +28,7 @@ EXPORTED = [
     "qsa_decode_workspace_size", "qsa_decode", "qsa_select_decode",
     "qsa_pool_build", "qsa_decode_noalloc", "qsa_decode_paged", "qsa_pool_build_paged",
     "qsa_decode_fp8", "qsa_decode_attend",
+    "qsa_cp_select", "qsa_cp_global_topk", "qsa_cp_attend", "qsa_cp_merge",
 ]
 
 
@@ -85,6 +86,16 @@ def _declare(lib):
         # pooled, out, lse, sel, nsel, dev_err, ws, ws_bytes, stream
         "qsa_decode_fp8": (I, [CFG, I, I, I, P, P, P, P, P, P, I] + [P] * 11 + [SZ, P]),
         "qsa_decode_attend": (I, [CFG, I, I, I] + [P] * 11 + [SZ, P]),
+        # cfg, batch, n_q, cap, block_lo, kv_len, iq, ik, iw, pooled, cand_score, cand_id,
+        # dev_err, ws, ws_bytes, stream
+        "qsa_cp_select": (I, [CFG, I, I, I, I] + [P] * 9 + [SZ, P]),
+        # cfg, batch, n_q, world, kv_len, cand_score, cand_id, sel, nsel, stream
+        "qsa_cp_global_topk": (I, [CFG, I, I, I] + [P] * 6),
+        # cfg, batch, n_q, cap, block_lo, kv_len, q, k, v, gate, sel, nsel, part_out,
+        # part_lse, dev_err, ws, ws_bytes, stream
+        "qsa_cp_attend": (I, [CFG, I, I, I, I] + [P] * 11 + [SZ, P]),
+        # cfg, batch, n_q, world, part_out, part_lse, out, lse, stream
+        "qsa_cp_merge": (I, [CFG, I, I, I] + [P] * 5),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

@@ -481,3 +481,111 @@ def decode_fp8(cfg: QSAConfig, q, k_cache, k_scale, v_cache, v_scale, iq, ik_cac
                                        _stream(stream))
         _lib.check(st, "qsa_decode_fp8")
     return {"out": out, "lse": lse, "sel": sel, "nsel": nsel}
+
+
+# ------------------------------------------------- context-parallel decode
+def cp_select(cfg: QSAConfig, iq, ik_shard, iw, pooled_shard, kv_len, block_lo: int, *,
+              dev_err=None, workspace=None, stream=None) -> dict:
+    """Shard selection of a context-parallel decode step (qsa_cp_select):
+    this process holds blocks [block_lo, block_lo + cap / B) of every sequence
+    (ik_shard [batch, cap, di], pooled_shard [batch, cap / B, di]); kv_len are
+    the full lengths. Returns the shard's candidates {"score" [batch, n_q, k]
+    fp32, "id" [batch, n_q, k] int32 global block ids}."""
+    dt = cfg.dtype
+    batch, n_q = iq.shape[0], iq.shape[1]
+    cap = ik_shard.shape[1]
+    _need(iq, "iq", dt, (batch, n_q, cfg.idx_heads, cfg.idx_dim))
+    _need(ik_shard, "ik_shard", dt, (batch, cap, cfg.idx_dim))
+    _need(iw, "iw", torch.float32, (batch, n_q, cfg.idx_heads))
+    _need(pooled_shard, "pooled_shard", torch.float32, (batch, cap // cfg.block_size, cfg.idx_dim))
+    _need(kv_len, "kv_len", torch.int32, (batch,))
+    dev = iq.device
+    score = torch.empty(batch, n_q, cfg.topk, dtype=torch.float32, device=dev)
+    ids = torch.empty(batch, n_q, cfg.topk, dtype=torch.int32, device=dev)
+    ws = _workspace(decode_workspace_size(cfg, batch, n_q, cap), dev, workspace)
+    _one_device(dev, stream, ik_shard=ik_shard, iw=iw, pooled_shard=pooled_shard, kv_len=kv_len,
+                dev_err=dev_err)
+    c = cfg.c()
+    with torch.cuda.device(dev):
+        st = _lib.lib().qsa_cp_select(ctypes.byref(c), batch, n_q, cap, int(block_lo),
+                                      _ptr(kv_len), _ptr(iq), _ptr(ik_shard), _ptr(iw),
+                                      _ptr(pooled_shard), _ptr(score), _ptr(ids), _ptr(dev_err),
+                                      _ptr(ws), ws.numel(), _stream(stream))
+        _lib.check(st, "qsa_cp_select")
+    return {"score": score, "id": ids}
+
+
+def cp_global_topk(cfg: QSAConfig, cand_score, cand_id, kv_len, *, stream=None) -> dict:
+    """Global selection from every process's candidates (qsa_cp_global_topk):
+    cand_score / cand_id [world, batch, n_q, k]. Returns {"sel" [batch, n_q,
+    k + 1], "nsel" [batch, n_q]} as qsa_decode writes them (global ids)."""
+    world, batch, n_q, k = cand_score.shape
+    _need(cand_score, "cand_score", torch.float32, (world, batch, n_q, cfg.topk))
+    _need(cand_id, "cand_id", torch.int32, (world, batch, n_q, cfg.topk))
+    _need(kv_len, "kv_len", torch.int32, (batch,))
+    dev = cand_score.device
+    sel = torch.empty(batch, n_q, cfg.topk + 1, dtype=torch.int32, device=dev)
+    nsel = torch.empty(batch, n_q, dtype=torch.int32, device=dev)
+    _one_device(dev, stream, cand_id=cand_id, kv_len=kv_len)
+    c = cfg.c()
+    with torch.cuda.device(dev):
+        st = _lib.lib().qsa_cp_global_topk(ctypes.byref(c), batch, n_q, world, _ptr(kv_len),
+                                           _ptr(cand_score), _ptr(cand_id), _ptr(sel),
+                                           _ptr(nsel), _stream(stream))
+        _lib.check(st, "qsa_cp_global_topk")
+    return {"sel": sel, "nsel": nsel}
+
+
+def cp_attend(cfg: QSAConfig, q, k_shard, v_shard, gate, kv_len, sel, nsel, block_lo: int, *,
+              dev_err=None, workspace=None, stream=None) -> dict:
+    """Attention over the shard's share of the global selection
+    (qsa_cp_attend). Returns {"out" [batch, n_q, Hq, D] fp32 gated partials,
+    "lse" [batch, n_q, Hq]}."""
+    dt = cfg.dtype
+    batch, n_q = q.shape[0], q.shape[1]
+    cap = k_shard.shape[1]
+    _need(q, "q", dt, (batch, n_q, cfg.num_q_heads, cfg.head_dim))
+    _need(k_shard, "k_shard", dt, (batch, cap, cfg.num_kv_heads, cfg.head_dim))
+    _need(v_shard, "v_shard", dt, (batch, cap, cfg.num_kv_heads, cfg.head_dim))
+    gshape = ((batch, n_q, cfg.num_q_heads) if cfg.gate_headwise
+              else (batch, n_q, cfg.num_q_heads, cfg.head_dim))
+    _need(gate, "gate", dt, gshape)
+    _need(kv_len, "kv_len", torch.int32, (batch,))
+    _need(sel, "sel", torch.int32, (batch, n_q, cfg.topk + 1))
+    _need(nsel, "nsel", torch.int32, (batch, n_q))
+    dev = q.device
+    out = torch.empty(batch, n_q, cfg.num_q_heads, cfg.head_dim, dtype=torch.float32, device=dev)
+    lse = torch.empty(batch, n_q, cfg.num_q_heads, dtype=torch.float32, device=dev)
+    ws = _workspace(decode_workspace_size(cfg, batch, n_q, cap), dev, workspace)
+    _one_device(dev, stream, k_shard=k_shard, v_shard=v_shard, gate=gate, kv_len=kv_len, sel=sel,
+                nsel=nsel, dev_err=dev_err)
+    c = cfg.c()
+    with torch.cuda.device(dev):
+        st = _lib.lib().qsa_cp_attend(ctypes.byref(c), batch, n_q, cap, int(block_lo),
+                                      _ptr(kv_len), _ptr(q), _ptr(k_shard), _ptr(v_shard),
+                                      _ptr(gate), _ptr(sel), _ptr(nsel), _ptr(out), _ptr(lse),
+                                      _ptr(dev_err), _ptr(ws), ws.numel(), _stream(stream))
+        _lib.check(st, "qsa_cp_attend")
+    return {"out": out, "lse": lse}
+
+
+def cp_merge(cfg: QSAConfig, part_out, part_lse, *, out=None, stream=None) -> dict:
+    """Log-sum-exp merge of every process's gated partials (qsa_cp_merge):
+    part_out [world, batch, n_q, Hq, D] fp32, part_lse [world, batch, n_q, Hq].
+    Returns {"out" (cfg.dtype), "lse"}."""
+    world, batch, n_q = part_out.shape[0], part_out.shape[1], part_out.shape[2]
+    _need(part_out, "part_out", torch.float32,
+          (world, batch, n_q, cfg.num_q_heads, cfg.head_dim))
+    _need(part_lse, "part_lse", torch.float32, (world, batch, n_q, cfg.num_q_heads))
+    dev = part_out.device
+    if out is None:
+        out = torch.empty(batch, n_q, cfg.num_q_heads, cfg.head_dim, dtype=cfg.dtype, device=dev)
+    _need(out, "out", cfg.dtype, (batch, n_q, cfg.num_q_heads, cfg.head_dim))
+    lse = torch.empty(batch, n_q, cfg.num_q_heads, dtype=torch.float32, device=dev)
+    _one_device(dev, stream, part_lse=part_lse, out=out)
+    c = cfg.c()
+    with torch.cuda.device(dev):
+        st = _lib.lib().qsa_cp_merge(ctypes.byref(c), batch, n_q, world, _ptr(part_out),
+                                     _ptr(part_lse), _ptr(out), _ptr(lse), _stream(stream))
+        _lib.check(st, "qsa_cp_merge")
+    return {"out": out, "lse": lse}

@@ -554,6 +554,134 @@ qsa_status qsa_decode_attend(const qsa_config* cfg, int batch, int n_q, int cap,
   return QSA_OK;
 }
 
+// ------------------------------------------------------- context-parallel decode
+static qsa_status check_shard(const qsa_config* cfg, int batch, int n_q, int cap, int block_lo) {
+  qsa_status s = check_decode_dims(cfg, batch, n_q, cap);
+  if (s != QSA_OK) return s;
+  if (block_lo < 0) return fail(QSA_ERR_INVALID_ARG, "block_lo must be >= 0");
+  if ((long long)block_lo * cfg->block_size + cap > 2147483647LL)
+    return fail(QSA_ERR_UNSUPPORTED, "shard rows past 2^31");
+  return QSA_OK;
+}
+
+qsa_status qsa_cp_select(const qsa_config* cfg, int batch, int n_q, int cap, int block_lo,
+                         const int32_t* kv_len, const void* iq, const void* ik_shard,
+                         const float* iw, float* pooled_shard, float* cand_score,
+                         int32_t* cand_id, int32_t* dev_err, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  g_err[0] = 0;
+  qsa_status s = check_shard(cfg, batch, n_q, cap, block_lo);
+  if (s != QSA_OK) return s;
+  if (batch == 0) return QSA_OK;
+  QSA_REQUIRE(kv_len, "kv_len");
+  QSA_REQUIRE(iq, "iq"); QSA_REQUIRE(ik_shard, "ik_shard"); QSA_REQUIRE(iw, "iw");
+  QSA_REQUIRE(pooled_shard, "pooled_shard");
+  QSA_REQUIRE(cand_score, "cand_score"); QSA_REQUIRE(cand_id, "cand_id");
+  const Geom g = make_geom(cfg);
+  const DecodeWs need = carve_decode(cfg, g, nullptr, batch, n_q, cap);
+  if (!workspace || workspace_bytes < need.bytes || ((uintptr_t)workspace & 255u))
+    return fail(QSA_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned", need.bytes);
+  const DecodeWs w = carve_decode(cfg, g, workspace, batch, n_q, cap);
+  cudaStream_t st = (cudaStream_t)stream;
+  CpShard cp;
+  cp.on = true;
+  cp.row_off = block_lo * cfg->block_size;
+  cp.block_lo = block_lo;
+  cp.cand_score = cand_score;
+  cp.cand_id = cand_id;
+  QSA_CUDA(cudaMemsetAsync(w.counters, 0, sizeof(int) * (size_t)batch * (2 + g.Hkv), st),
+           "clear counters");
+  QSA_CUDA(launch_decode_select(cfg->dtype, g, batch, n_q, cap, kv_len, iq, ik_shard, iw,
+                                pooled_shard, nullptr, w.keys, w.counters, w.sel, w.nsel,
+                                dev_err ? dev_err : w.err, st, Pages(), nullptr, cp),
+           "shard select");
+  return QSA_OK;
+}
+
+qsa_status qsa_cp_global_topk(const qsa_config* cfg, int batch, int n_q, int world,
+                              const int32_t* kv_len, const float* cand_score,
+                              const int32_t* cand_id, int32_t* sel, int32_t* nsel,
+                              void* stream) {
+  g_err[0] = 0;
+  qsa_status s = check_cfg(cfg);
+  if (s != QSA_OK) return s;
+  if (batch < 0 || n_q <= 0 || world <= 0)
+    return fail(QSA_ERR_INVALID_ARG, "batch >= 0, n_q > 0 and world > 0 are required");
+  if (n_q > kMaxDecodeQ) return fail(QSA_ERR_UNSUPPORTED, "n_q > %d", kMaxDecodeQ);
+  if ((long long)world * (cfg->budget / cfg->block_size) > 4096)
+    return fail(QSA_ERR_UNSUPPORTED, "world * budget / block_size > 4096");
+  if (batch == 0) return QSA_OK;
+  QSA_REQUIRE(kv_len, "kv_len");
+  QSA_REQUIRE(cand_score, "cand_score"); QSA_REQUIRE(cand_id, "cand_id");
+  QSA_REQUIRE(sel, "sel"); QSA_REQUIRE(nsel, "nsel");
+  const Geom g = make_geom(cfg);
+  QSA_CUDA(launch_cp_global_topk(g, batch, n_q, world, kv_len, cand_score, cand_id, sel, nsel,
+                                 (cudaStream_t)stream),
+           "global top-k");
+  return QSA_OK;
+}
+
+qsa_status qsa_cp_attend(const qsa_config* cfg, int batch, int n_q, int cap, int block_lo,
+                         const int32_t* kv_len, const void* q, const void* k_shard,
+                         const void* v_shard, const void* gate, const int32_t* sel,
+                         const int32_t* nsel, float* part_out, float* part_lse,
+                         int32_t* dev_err, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  g_err[0] = 0;
+  qsa_status s = check_shard(cfg, batch, n_q, cap, block_lo);
+  if (s != QSA_OK) return s;
+  const Geom g = make_geom(cfg);
+  if (batch == 0) return QSA_OK;
+  QSA_REQUIRE(kv_len, "kv_len");
+  QSA_REQUIRE(q, "q"); QSA_REQUIRE(k_shard, "k_shard"); QSA_REQUIRE(v_shard, "v_shard");
+  QSA_REQUIRE(gate, "gate"); QSA_REQUIRE(sel, "sel"); QSA_REQUIRE(nsel, "nsel");
+  QSA_REQUIRE(part_out, "part_out"); QSA_REQUIRE(part_lse, "part_lse");
+  const DecodeWs need = carve_decode(cfg, g, nullptr, batch, n_q, cap);
+  if (!workspace || workspace_bytes < need.bytes || ((uintptr_t)workspace & 255u))
+    return fail(QSA_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned", need.bytes);
+  const DecodeWs w = carve_decode(cfg, g, workspace, batch, n_q, cap);
+  cudaStream_t st = (cudaStream_t)stream;
+  CpShard cp;
+  cp.on = true;
+  cp.row_off = block_lo * cfg->block_size;
+  cp.block_lo = block_lo;
+  cp.out_f32 = part_out;
+  QSA_CUDA(cudaMemsetAsync(w.counters, 0, sizeof(int) * (size_t)batch * (2 + g.Hkv), st),
+           "clear counters");
+  if (decode_uses_mma(cfg, g, n_q)) {
+    QSA_CUDA(launch_attn_decode_mma(g, batch, n_q, cap, w.nsplit, w.per_split, kv_len, q,
+                                    k_shard, v_shard, gate, sel, nsel, w.part_ml, w.part_o,
+                                    w.counters + batch, nullptr, part_lse,
+                                    dev_err ? dev_err : w.err, st, Pages(), nullptr, Fp8Kv(), cp),
+             "shard attention");
+  } else {
+    QSA_CUDA(launch_attn_decode_simt(cfg->dtype, g, batch, n_q, cap, w.nsplit, w.per_split,
+                                     kv_len, q, k_shard, v_shard, gate, sel, nsel, w.part_ml,
+                                     w.part_o, nullptr, part_lse, st, cp),
+             "shard attention");
+  }
+  return QSA_OK;
+}
+
+qsa_status qsa_cp_merge(const qsa_config* cfg, int batch, int n_q, int world,
+                        const float* part_out, const float* part_lse, void* out, float* lse,
+                        void* stream) {
+  g_err[0] = 0;
+  qsa_status s = check_cfg(cfg);
+  if (s != QSA_OK) return s;
+  if (batch < 0 || n_q <= 0 || world <= 0)
+    return fail(QSA_ERR_INVALID_ARG, "batch >= 0, n_q > 0 and world > 0 are required");
+  if (batch == 0) return QSA_OK;
+  QSA_REQUIRE(part_out, "part_out"); QSA_REQUIRE(part_lse, "part_lse"); QSA_REQUIRE(out, "out");
+  if (lse) QSA_REQUIRE(lse, "lse");
+  if ((long long)batch * n_q * cfg->num_q_heads > 2147483647LL)
+    return fail(QSA_ERR_UNSUPPORTED, "too many rows");
+  QSA_CUDA(launch_cp_merge(cfg->dtype, batch * n_q * cfg->num_q_heads, cfg->head_dim, world,
+                           part_out, part_lse, out, lse, (cudaStream_t)stream),
+           "merge");
+  return QSA_OK;
+}
+
 static qsa_status check_pages(const qsa_config* cfg, int max_blocks, const int32_t* block_table,
                               int num_pages) {
   if (max_blocks <= 0 || num_pages <= 0)

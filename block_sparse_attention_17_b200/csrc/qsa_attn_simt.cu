@@ -220,8 +220,10 @@ attn_prefill_simt_kernel(Geom g, const int* __restrict__ cu, const T* __restrict
 // ------------------------------------------------------------------- decode
 // Union of the n_q selection lists of one sequence, ascending, deduplicated.
 // Each entry also carries a bitmask of the queries that see it.
+// Block ids are taken relative to `lo` (a context-parallel shard's first
+// block; 0 otherwise) and those outside [0, nblk) are skipped.
 __device__ int build_union(const int* sel_b, const int* nsel_b, int n_q, int kp1, int* u_blk,
-                           int* u_qmask) {
+                           int* u_qmask, int lo, int nblk) {
   // serial merge by thread 0: at most n_q * (k + 1) entries
   int cnt = 0;
   int idx[4] = {0, 0, 0, 0};
@@ -233,9 +235,11 @@ __device__ int build_union(const int* sel_b, const int* nsel_b, int n_q, int kp1
     int qm = 0;
     for (int i = 0; i < n_q; ++i)
       if (idx[i] < nsel_b[i] && sel_b[i * kp1 + idx[i]] == best) { qm |= 1 << i; ++idx[i]; }
-    u_blk[cnt] = best;
-    u_qmask[cnt] = qm;
-    ++cnt;
+    if (best - lo >= 0 && best - lo < nblk) {
+      u_blk[cnt] = best - lo;
+      u_qmask[cnt] = qm;
+      ++cnt;
+    }
   }
   return cnt;
 }
@@ -246,7 +250,7 @@ attn_decode_simt_kernel(Geom g, int n_q, int cap, int nsplit, int per_split,
                         const int* __restrict__ kv_len, const T* __restrict__ q,
                         const T* __restrict__ kc, const T* __restrict__ vc,
                         const int* __restrict__ sel, const int* __restrict__ nsel,
-                        float* __restrict__ part_ml, float* __restrict__ part_o) {
+                        float* __restrict__ part_ml, float* __restrict__ part_o, CpShard cp) {
   constexpr int kMaxRows = 32;
   constexpr int kMaxOwn = kMaxRows * D / kChunkKeys;
   __shared__ __align__(16) float q_s[kMaxRows * D];
@@ -259,9 +263,9 @@ attn_decode_simt_kernel(Geom g, int n_q, int cap, int nsplit, int per_split,
   const int split = blockIdx.x, b = blockIdx.y, hk = blockIdx.z;
   const int tid = threadIdx.x;
   const int G = g.G, R = n_q * G;
-  const int kv = kv_len[b];
+  const int kv = kv_len[b] - cp.row_off;   // (a shard's rows: may be past either end)
   const size_t part_row0 = (((size_t)b * g.Hkv + hk) * nsplit + split) * R;
-  if (kv < n_q || kv > cap) {
+  if (!cp.on && (kv < n_q || kv > cap)) {
     for (int r = tid; r < R; r += blockDim.x) {
       part_ml[2 * (part_row0 + r)] = -INFINITY;
       part_ml[2 * (part_row0 + r) + 1] = 0.f;
@@ -276,7 +280,7 @@ attn_decode_simt_kernel(Geom g, int n_q, int cap, int nsplit, int per_split,
   }
   if (tid == 0)
     u_cnt = build_union(sel + (size_t)b * n_q * (g.k + 1), nsel + (size_t)b * n_q, n_q,
-                        g.k + 1, u_blk, u_qm);
+                        g.k + 1, u_blk, u_qm, cp.block_lo, cap / g.B);
   if (tid < R) { m_s[tid] = -INFINITY; l_s[tid] = 0.f; }
   __syncthreads();
 
@@ -322,7 +326,7 @@ __global__ void decode_combine_kernel(Geom g, int n_q, int cap, int nsplit,
                                       const float* __restrict__ part_ml,
                                       const float* __restrict__ part_o,
                                       const T* __restrict__ gate, T* __restrict__ out,
-                                      float* __restrict__ lse) {
+                                      float* __restrict__ lse, CpShard cp) {
   const int b = blockIdx.y;
   const int i = blockIdx.x / g.Hq, h = blockIdx.x - i * g.Hq;
   const int d = threadIdx.x;
@@ -330,7 +334,7 @@ __global__ void decode_combine_kernel(Geom g, int n_q, int cap, int nsplit,
   const int R = n_q * g.G, r = i * g.G + gi;
   const int kv = kv_len[b];
   const size_t orow = ((size_t)b * n_q + i) * g.Hq + h;
-  if (kv < n_q || kv > cap) {
+  if (!cp.on && (kv < n_q || kv > cap)) {
     out[orow * D + d] = from_f32<T>(0.f);
     if (lse && d == 0) lse[orow] = -INFINITY;
     return;
@@ -353,7 +357,10 @@ __global__ void decode_combine_kernel(Geom g, int n_q, int cap, int nsplit,
   }
   const float val = Lsum > 0.f ? o / Lsum : 0.f;
   const float gl = g.gate_headwise ? to_f32(gate[orow]) : to_f32(gate[orow * D + d]);
-  out[orow * D + d] = from_f32<T>(sigmoidf_(gl) * val);
+  if (cp.out_f32)
+    cp.out_f32[orow * D + d] = sigmoidf_(gl) * val;
+  else
+    out[orow * D + d] = from_f32<T>(sigmoidf_(gl) * val);
   if (lse && d == 0) lse[orow] = Lsum > 0.f ? (M + log2f(Lsum)) * kLn2 : -INFINITY;
 }
 
@@ -381,12 +388,12 @@ cudaError_t launch_attn_prefill_simt(qsa_dtype dt, const Geom& g, const int* cu,
 cudaError_t launch_decode_combine(qsa_dtype dt, const Geom& g, int batch, int n_q, int cap,
                                   int nsplit, const int* kv_len, const float* part_ml,
                                   const float* part_o, const void* gate, void* out, float* lse,
-                                  cudaStream_t st) {
+                                  cudaStream_t st, CpShard cp) {
   if (batch == 0) return cudaSuccess;
   dim3 cgrid(n_q * g.Hq, batch);
 #define QSA_CB(T, DD)                                                                     \
   decode_combine_kernel<T, DD><<<cgrid, DD, 0, st>>>(g, n_q, cap, nsplit, kv_len, part_ml,  \
-                                                     part_o, (const T*)gate, (T*)out, lse)
+                                                     part_o, (const T*)gate, (T*)out, lse, cp)
   if (dt == QSA_BF16) {
     if (g.D == 128) { QSA_CB(__nv_bfloat16, 128); } else { QSA_CB(__nv_bfloat16, 64); }
   } else {
@@ -401,7 +408,8 @@ cudaError_t launch_attn_decode_simt(qsa_dtype dt, const Geom& g, int batch, int 
                                     int nsplit, int per_split, const int* kv_len, const void* q,
                                     const void* kc, const void* vc, const void* gate,
                                     const int* sel, const int* nsel, float* part_ml,
-                                    float* part_o, void* out, float* lse, cudaStream_t st) {
+                                    float* part_o, void* out, float* lse, cudaStream_t st,
+                                    CpShard cp) {
   if (batch == 0) return cudaSuccess;
   dim3 grid(nsplit, batch, g.Hkv);
   dim3 cgrid(n_q * g.Hq, batch);
@@ -409,9 +417,9 @@ cudaError_t launch_attn_decode_simt(qsa_dtype dt, const Geom& g, int batch, int 
   attn_decode_simt_kernel<T, DD><<<grid, 128, 0, st>>>(g, n_q, cap, nsplit, per_split,      \
                                                        kv_len, (const T*)q, (const T*)kc,   \
                                                        (const T*)vc, sel, nsel, part_ml,    \
-                                                       part_o);                             \
+                                                       part_o, cp);                         \
   decode_combine_kernel<T, DD><<<cgrid, DD, 0, st>>>(g, n_q, cap, nsplit, kv_len, part_ml,  \
-                                                     part_o, (const T*)gate, (T*)out, lse)
+                                                     part_o, (const T*)gate, (T*)out, lse, cp)
   if (dt == QSA_BF16) {
     if (g.D == 128) { QSA_AD(__nv_bfloat16, 128); } else { QSA_AD(__nv_bfloat16, 64); }
   } else {

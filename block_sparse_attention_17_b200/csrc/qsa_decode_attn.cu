@@ -111,6 +111,11 @@ struct DecParams {
                                      // before the cluster's top-k (its best-scored ones)
   int early;                         // the first scoring pass's pooled rows are copied into
                                      // shared memory at kernel entry (stage_pooled_early)
+  // context-parallel shard (attention over given selections only): kv_len are
+  // full lengths, the caches hold rows [row_off, row_off + cap), sel holds
+  // global block ids; outputs are fp32 gated partials in out_f32
+  int cp, row_off, block_lo;
+  float* out_f32;
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
@@ -770,9 +775,9 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
       if (threadIdx.x + u * kThreads < nq8) iqreg[u] = iqb[threadIdx.x + u * kThreads];
     if (threadIdx.x < n_q * g.Hi) iwreg = P.iw[(size_t)b * n_q * g.Hi + threadIdx.x];
   }
-  const int kv = P.kv_len[b];
+  const int kv = P.kv_len[b] - P.row_off;   // (a shard's rows: may be past either end)
   const size_t row0 = (((size_t)b * g.Hkv + hk) * P.nsplit + split) * R;
-  if (kv < n_q || kv > P.cap) {   // reported by the selection; outputs are zero
+  if (!P.cp && (kv < n_q || kv > P.cap)) {   // reported by the selection; outputs are zero
     if constexpr (kSelDI > 0) cp_async_wait_all();   // no copy may land after the CTA left
     if (split == 0 && hk == 0) {
       if constexpr (kSelDI > 0) {
@@ -940,7 +945,7 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
       for (int e = threadIdx.x; e < n_q * kp1; e += blockDim.x) {
         const int i = e / kp1, j = e - i * kp1;
         if (j < P.nsel[(size_t)b * n_q + i]) {
-          const int blk = P.sel[((size_t)b * n_q + i) * kp1 + j];
+          const int blk = P.sel[((size_t)b * n_q + i) * kp1 + j] - P.block_lo;
           if (blk >= 0 && blk < nblk) atomicOr(&qbits[i * words + (blk >> 5)], 1u << (blk & 31));
         }
       }
@@ -1350,9 +1355,14 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
       }
       const int i = r / G, gi = r % G;
       const size_t orow = ((size_t)b * n_q + i) * g.Hq + hk * G + gi;
-      *reinterpret_cast<uint2*>(P.out + orow * kD + 4 * f) =
-          make_uint2(pack2(acc.x * inv * gs[0], acc.y * inv * gs[1]),
-                     pack2(acc.z * inv * gs[2], acc.w * inv * gs[3]));
+      if (P.out_f32)
+        *reinterpret_cast<float4*>(P.out_f32 + orow * kD + 4 * f) =
+            make_float4(acc.x * inv * gs[0], acc.y * inv * gs[1], acc.z * inv * gs[2],
+                        acc.w * inv * gs[3]);
+      else
+        *reinterpret_cast<uint2*>(P.out + orow * kD + 4 * f) =
+            make_uint2(pack2(acc.x * inv * gs[0], acc.y * inv * gs[1]),
+                       pack2(acc.z * inv * gs[2], acc.w * inv * gs[3]));
       if (P.lse && f == 0) P.lse[orow] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
     }
     cluster_sync_relaxed();   // no CTA leaves while another may still read its partial
@@ -1444,13 +1454,21 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
           gsig[2 * d + 1] = sigmoidf_(__uint_as_float(gw[d] & 0xffff0000u));
         }
       }
-      uint32_t packed[8];
+      if (P.out_f32) {
+        float4* dst = reinterpret_cast<float4*>(P.out_f32 + orow * kD + d0);
 #pragma unroll
-      for (int d = 0; d < 16; d += 2)
-        packed[d / 2] = pack2(acc[d] * inv * gsig[d], acc[d + 1] * inv * gsig[d + 1]);
-      uint4* dst = reinterpret_cast<uint4*>(P.out + orow * kD + d0);
-      dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-      dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+        for (int d = 0; d < 16; d += 4)
+          dst[d / 4] = make_float4(acc[d] * inv * gsig[d], acc[d + 1] * inv * gsig[d + 1],
+                                   acc[d + 2] * inv * gsig[d + 2], acc[d + 3] * inv * gsig[d + 3]);
+      } else {
+        uint32_t packed[8];
+#pragma unroll
+        for (int d = 0; d < 16; d += 2)
+          packed[d / 2] = pack2(acc[d] * inv * gsig[d], acc[d + 1] * inv * gsig[d + 1]);
+        uint4* dst = reinterpret_cast<uint4*>(P.out + orow * kD + d0);
+        dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+      }
       if (P.lse && d0 == 0) P.lse[orow] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
     }
     if (threadIdx.x == 0) P.counter[(size_t)b * g.Hkv + hk] = 0;
@@ -1670,11 +1688,16 @@ cudaError_t launch_attn_decode_mma(const Geom& g, int batch, int n_q, int cap, i
                                    const void* kc, const void* vc, const void* gate,
                                    const int* sel, const int* nsel, float* part_ml,
                                    float* part_o, int* counter, void* out, float* lse, int* err,
-                                   cudaStream_t st, Pages pg, const int* ready, Fp8Kv f8) {
+                                   cudaStream_t st, Pages pg, const int* ready, Fp8Kv f8,
+                                   CpShard cp) {
   if (batch == 0) return cudaSuccess;
   CUtensorMap mk, mv;
   if (!make_maps(g, batch, cap, kc, vc, pg, f8.on, &mk, &mv)) return cudaErrorInvalidValue;
   DecParams p = base_params(g, n_q, cap, nsplit, per_split, kv_len, q, gate, out, lse, err, pg, f8);
+  p.cp = cp.on ? 1 : 0;
+  p.row_off = cp.row_off;
+  p.block_lo = cp.block_lo;
+  p.out_f32 = cp.out_f32;
   p.sel = sel;
   p.nsel = nsel;
   p.part_ml = part_ml;

@@ -41,6 +41,22 @@ struct Fp8Kv {
   int rotated = 0;
 };
 
+// Context-parallel decode: this process holds the rows [row_off, row_off +
+// cap) of every sequence (blocks [block_lo, ...), row_off = block_lo * B);
+// kv_len stays the sequences' full lengths. The selection kernel then scores
+// the shard's complete visible blocks and writes each query's top-k of them
+// as candidates (cand_score: the scores, cand_id: global block ids; -inf / -1
+// padding); the attention kernel reads global block ids, attends those inside
+// the shard, and writes fp32 gated partials (out_f32) with their lse.
+struct CpShard {
+  bool on = false;
+  int row_off = 0;
+  int block_lo = 0;
+  float* cand_score = nullptr;
+  int* cand_id = nullptr;
+  float* out_f32 = nullptr;
+};
+
 // ready: [batch] flags the selection kernel sets (release) once a sequence's
 // selections are written, zero before the launch; the decode attention kernel
 // waits on its sequence's flag instead of on the whole selection grid.
@@ -87,7 +103,7 @@ cudaError_t launch_decode_select(qsa_dtype dt, const Geom& g, int batch, int n_q
                                  const float* iw, float* pooled, float* scores_out,
                                  uint32_t* keys_ws, int* counter, int* sel, int* nsel,
                                  int* dev_err, cudaStream_t st, Pages pg = Pages(),
-                                 int* ready = nullptr);
+                                 int* ready = nullptr, CpShard cp = CpShard());
 cudaError_t launch_attn_prefill_simt(qsa_dtype dt, const Geom& g, const int* cu, int batch,
                                      int max_seqlen, const void* q, const void* k, const void* v,
                                      const void* gate, const int* sel, const int* nsel,
@@ -96,12 +112,13 @@ cudaError_t launch_attn_decode_simt(qsa_dtype dt, const Geom& g, int batch, int 
                                     int nsplit, int per_split, const int* kv_len, const void* q,
                                     const void* kc, const void* vc, const void* gate,
                                     const int* sel, const int* nsel, float* part_ml,
-                                    float* part_o, void* out, float* lse, cudaStream_t st);
+                                    float* part_o, void* out, float* lse, cudaStream_t st,
+                                    CpShard cp = CpShard());
 
 cudaError_t launch_decode_combine(qsa_dtype dt, const Geom& g, int batch, int n_q, int cap,
                                   int nsplit, const int* kv_len, const float* part_ml,
                                   const float* part_o, const void* gate, void* out, float* lse,
-                                  cudaStream_t st);
+                                  cudaStream_t st, CpShard cp = CpShard());
 bool attn_decode_mma_supported(const Geom& g, int n_q);
 void decode_mma_split(const Geom& g, int batch, int n_q, int* nsplit, int* per_split);
 cudaError_t launch_attn_decode_mma(const Geom& g, int batch, int n_q, int cap, int nsplit,
@@ -110,7 +127,7 @@ cudaError_t launch_attn_decode_mma(const Geom& g, int batch, int n_q, int cap, i
                                    const int* sel, const int* nsel, float* part_ml,
                                    float* part_o, int* counter, void* out, float* lse, int* err,
                                    cudaStream_t st, Pages pg = Pages(), const int* ready = nullptr,
-                                   Fp8Kv f8 = Fp8Kv());
+                                   Fp8Kv f8 = Fp8Kv(), CpShard cp = CpShard());
 bool attn_decode_fp8_supported(const Geom& g, int n_q);
 
 // The selection of a decode step done inside the decode attention kernel (one
@@ -134,6 +151,15 @@ cudaError_t launch_decode_fused(const Geom& g, int batch, int n_q, int cap, int 
                                 void* out, float* lse, int* err, cudaStream_t st,
                                 Pages pg = Pages(), Fp8Kv f8 = Fp8Kv());
 bool attn_prefill_tc_supported(const Geom& g);
+// Context-parallel decode: the global top-k over every process's candidates
+// ([world, batch, n_q, k] scores and global ids) plus each query's tail block
+// (sel [batch, n_q, k + 1], nsel [batch, n_q], as qsa_decode writes them), and
+// the log-sum-exp merge of the processes' gated fp32 partials.
+cudaError_t launch_cp_global_topk(const Geom& g, int batch, int n_q, int world,
+                                  const int* kv_len, const float* cand_score,
+                                  const int* cand_id, int* sel, int* nsel, cudaStream_t st);
+cudaError_t launch_cp_merge(qsa_dtype dt, int rows, int D, int world, const float* part_out,
+                            const float* part_lse, void* out, float* lse, cudaStream_t st);
 cudaError_t launch_attn_prefill_tc(const Geom& g, const int* cu, int batch, int total_tokens,
                                    int max_seqlen, int words, const uint32_t* bitmask,
                                    const void* q, const void* k, const void* v, const void* gate,

@@ -543,7 +543,7 @@ decode_select_kernel(Geom g, int n_q, int cap, const int* __restrict__ kv_len,
                      const float* __restrict__ iw, float* __restrict__ pooled,
                      float* __restrict__ scores_out, uint32_t* __restrict__ keys_ws,
                      int* __restrict__ counter, int* __restrict__ sel, int* __restrict__ nsel,
-                     int* dev_err, Pages pg, int* ready) {
+                     int* dev_err, Pages pg, int* ready, CpShard cp) {
   grid_dependents_launch();   // the attention kernel may start its prologue
   extern __shared__ __align__(16) float smem[];
   constexpr int kStride = kDI + 1;
@@ -557,9 +557,11 @@ decode_select_kernel(Geom g, int n_q, int cap, const int* __restrict__ kv_len,
   __shared__ int last_s;
 
   const int c = blockIdx.x, b = blockIdx.y;
-  const int kv = kv_len[b];
+  // (context-parallel shard: lengths in the shard's rows; a query sees at most
+  // the shard's cap rows and possibly none)
+  const int kv = cp.on ? kv_len[b] - cp.row_off : kv_len[b];
   const int kp1 = k + 1;
-  if (kv < n_q || kv > cap) {
+  if (!cp.on && (kv < n_q || kv > cap)) {
     if (c == 0) {
       for (int e = threadIdx.x; e < n_q * kp1; e += blockDim.x) sel[(size_t)b * n_q * kp1 + e] = -1;
       for (int e = threadIdx.x; e < n_q; e += blockDim.x) nsel[(size_t)b * n_q + e] = 0;
@@ -567,7 +569,7 @@ decode_select_kernel(Geom g, int n_q, int cap, const int* __restrict__ kv_len,
     }
     return;
   }
-  const int nc_last = kv / g.B;                    // candidates of the last query
+  const int nc_last = min(max(kv, 0), cap) / g.B;   // candidates of the last query
   const int nparts = max(1, (nc_last + kPart - 1) / kPart);
   if (c >= nparts) return;
   const int j0 = c * kPart;
@@ -584,7 +586,8 @@ decode_select_kernel(Geom g, int n_q, int cap, const int* __restrict__ kv_len,
     }
   }
   // 1. blocks completed by this step's tokens (pool_block_cta needs the whole CTA)
-  const int jnew_lo = max((kv - n_q) / g.B, j0), jnew_hi = min(nc_last, j0 + kPart);
+  const int jnew_lo = max(min(max(kv - n_q, 0), cap) / g.B, j0),
+            jnew_hi = min(nc_last, j0 + kPart);
   for (int j = jnew_lo; j < jnew_hi; ++j) {
     size_t row0 = (size_t)b * cap + (size_t)j * g.B;
     if (pg.table) {
@@ -642,7 +645,7 @@ decode_select_kernel(Geom g, int n_q, int cap, const int* __restrict__ kv_len,
     const int r = rem / g.Hi, h = rem - r * g.Hi;
     float term = 0.f;
     const int j = j0 + r;
-    const int nc_i = i < n_q ? (kv - n_q + 1 + i) / g.B : 0;
+    const int nc_i = i < n_q ? min(max(kv - n_q + 1 + i, 0), cap) / g.B : 0;
     const bool live = i < n_q && j < nc_i;
     if (live) {
       const float* krow = kbar_s + r * kStride;
@@ -673,7 +676,7 @@ decode_select_kernel(Geom g, int n_q, int cap, const int* __restrict__ kv_len,
   if (!last_s) return;
   __threadfence();
   for (int i = 0; i < n_q; ++i) {
-    const int n = kv - n_q + 1 + i;
+    const int n = min(max(kv - n_q + 1 + i, 0), cap);
     const int nc_i = n / g.B;
     {   // eight loads in flight per thread before any store
       const uint32_t* kq = keys_ws + ((size_t)b * n_q + i) * nblk_cap;
@@ -702,6 +705,13 @@ decode_select_kernel(Geom g, int n_q, int cap, const int* __restrict__ kv_len,
       srow[e] = v;
     }
     if (threadIdx.x == 0) nsel[(size_t)b * n_q + i] = m + (tail > 0 ? 1 : 0);
+    if (cp.cand_score) {   // the shard's candidates: scores (keys decoded) and global ids
+      for (int e = threadIdx.x; e < k; e += blockDim.x) {
+        const size_t o = ((size_t)b * n_q + i) * k + e;
+        cp.cand_score[o] = e < m ? key_score(keys_s[pos_s[e]]) : -INFINITY;
+        cp.cand_id[o] = e < m ? pos_s[e] + cp.block_lo : -1;
+      }
+    }
     __syncthreads();
   }
   if (threadIdx.x == 0) counter[b] = 0;
@@ -816,14 +826,15 @@ static cudaError_t launch_decode_select_t(const Geom& g, int batch, int n_q, int
                                           const int* kv_len, const void* iq, const void* ik_cache,
                                           const float* iw, float* pooled, float* scores_out,
                                           uint32_t* keys_ws, int* counter, int* sel, int* nsel,
-                                          int* dev_err, cudaStream_t st, Pages pg, int* ready) {
+                                          int* dev_err, cudaStream_t st, Pages pg, int* ready,
+                                          CpShard cp) {
   const size_t smem = decode_select_smem(g, n_q, cap);
   auto kern = decode_select_kernel<T, kDI>;
   cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(kern), (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<dim3(decode_select_parts(g, cap), batch), kSelThreads, smem, st>>>(
       g, n_q, cap, kv_len, (const T*)iq, (const T*)ik_cache, iw, pooled, scores_out, keys_ws,
-      counter, sel, nsel, dev_err, pg, ready);
+      counter, sel, nsel, dev_err, pg, ready, cp);
   note_launch();
   return cudaGetLastError();
 }
@@ -832,12 +843,13 @@ cudaError_t launch_decode_select(qsa_dtype dt, const Geom& g, int batch, int n_q
                                  const int* kv_len, const void* iq, const void* ik_cache,
                                  const float* iw, float* pooled, float* scores_out,
                                  uint32_t* keys_ws, int* counter, int* sel, int* nsel,
-                                 int* dev_err, cudaStream_t st, Pages pg, int* ready) {
+                                 int* dev_err, cudaStream_t st, Pages pg, int* ready,
+                                 CpShard cp) {
   if (batch == 0) return cudaSuccess;
 #define QSA_DS(T, DI)                                                                       \
   return launch_decode_select_t<T, DI>(g, batch, n_q, cap, kv_len, iq, ik_cache, iw, pooled, \
                                        scores_out, keys_ws, counter, sel, nsel, dev_err, st, pg, \
-                                       ready)
+                                       ready, cp)
   if (dt == QSA_BF16) {
     if (g.di == 64) QSA_DS(__nv_bfloat16, 64);
     QSA_DS(__nv_bfloat16, 32);

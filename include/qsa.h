@@ -228,6 +228,76 @@ qsa_status qsa_decode_noalloc(const qsa_config* cfg, int batch, int n_q, int cap
                               void* out, float* lse, int32_t* sel, int32_t* nsel,
                               int32_t* dev_err, void* stream);
 
+/* ----------------------------------------------- context-parallel decode --
+ * A sequence whose KV cache does not fit one GPU is split by blocks over the
+ * processes of a group, one per GPU (the pages describe no multi-GPU QSA; the
+ * split follows the step's data dependencies). The process with shard
+ * [block_lo, block_lo + cap / B) holds cache rows [block_lo * B, block_lo * B
+ * + cap) of every sequence at local rows 0 .. cap - 1: k_shard, v_shard
+ * [batch, cap, Hkv, D], ik_shard [batch, cap, di], pooled_shard
+ * [batch, cap / B, di] (the shard's pooled keys, as qsa_pool_build writes them
+ * for the shard). kv_len [batch] are the sequences' FULL lengths after this
+ * step's n_q tokens were appended (to the shard that holds those rows); a
+ * shard may hold none, some or all of a sequence's visible rows. One step:
+ *   1. qsa_cp_select on every process: pools the shard's blocks completed by
+ *      this step, scores the shard's complete visible blocks, and writes each
+ *      query's top-k of them as candidates;
+ *   2. the caller all-gathers the candidates (cand_score, cand_id) of every
+ *      process into [world, batch, n_q, k] arrays, ordered by process;
+ *   3. qsa_cp_global_topk: the global selection, identical to qsa_decode's
+ *      (every globally selected block is in its own shard's top-k);
+ *   4. qsa_cp_attend on every process: gated attention over the selected
+ *      blocks inside the shard, as fp32 partials with their log-sum-exp;
+ *   5. the caller all-gathers the partials, and qsa_cp_merge merges them by
+ *      log-sum-exp (the sigmoid gate commutes with the weighted sum).
+ * The scores are computed by the same arithmetic as qsa_decode's, so the
+ * selection is bit-identical to the single-GPU one.
+ *
+ * qsa_cp_select: iq [batch, n_q, Hi, di], iw [batch, n_q, Hi] fp32 as for
+ *   qsa_decode; writes the pooled rows of the shard's blocks this step
+ *   completes, and cand_score [batch, n_q, k] fp32 / cand_id [batch, n_q, k]
+ *   int32 (global block ids; -inf / -1 in unused slots, k = budget / B). The
+ *   workspace is qsa_decode_workspace_size(cfg, batch, n_q, cap)'s.
+ *   dev_err (optional) is set if a kernel finds an inconsistent length. */
+qsa_status qsa_cp_select(const qsa_config* cfg, int batch, int n_q, int cap, int block_lo,
+                         const int32_t* kv_len, const void* iq, const void* ik_shard,
+                         const float* iw, float* pooled_shard, float* cand_score,
+                         int32_t* cand_id, int32_t* dev_err, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/* qsa_cp_global_topk: cand_score / cand_id [world, batch, n_q, k] gathered
+ * from every process; writes sel [batch, n_q, k + 1] (global ids of the
+ * selected complete blocks in ascending order, then the query's tail block
+ * floor(n / B) when n % B != 0, then -1) and nsel [batch, n_q], exactly as
+ * qsa_decode writes them. Supported: world * k <= 4096. */
+qsa_status qsa_cp_global_topk(const qsa_config* cfg, int batch, int n_q, int world,
+                              const int32_t* kv_len, const float* cand_score,
+                              const int32_t* cand_id, int32_t* sel, int32_t* nsel,
+                              void* stream);
+
+/* qsa_cp_attend: attention of q [batch, n_q, Hq, D] over the blocks of the
+ * global selection (sel / nsel from qsa_cp_global_topk) that lie in this
+ * shard, each over the positions the query sees; part_out [batch, n_q, Hq, D]
+ * fp32 receives the gated partial output and part_lse [batch, n_q, Hq] fp32
+ * its natural-log sum-exp (-inf and 0 where the shard holds none of the
+ * query's keys). Workspace as qsa_cp_select. Every geometry qsa_decode
+ * supports; bf16 with head_dim 128 and n_q * (Hq / Hkv) <= 16 runs on the
+ * tensor-map kernel, the rest on the CUDA-core kernels. */
+qsa_status qsa_cp_attend(const qsa_config* cfg, int batch, int n_q, int cap, int block_lo,
+                         const int32_t* kv_len, const void* q, const void* k_shard,
+                         const void* v_shard, const void* gate, const int32_t* sel,
+                         const int32_t* nsel, float* part_out, float* part_lse,
+                         int32_t* dev_err, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
+/* qsa_cp_merge: part_out [world, batch, n_q, Hq, D] fp32 and part_lse
+ * [world, batch, n_q, Hq] gathered from every process; writes out
+ * [batch, n_q, Hq, D] in the config's dtype and lse (optional) [batch, n_q,
+ * Hq]. */
+qsa_status qsa_cp_merge(const qsa_config* cfg, int batch, int n_q, int world,
+                        const float* part_out, const float* part_lse, void* out, float* lse,
+                        void* stream);
+
 /* --------------------------------------------------------- paged decode --
  * qsa_decode over a paged KV cache (a speed lever the llama.cpp PR #27739
  * page lists: "continuous batching and paged KV"; the QSA block is the page).

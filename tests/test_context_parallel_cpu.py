@@ -1,9 +1,13 @@
 """Context-parallel decode's host logic (block_sparse_attention_17_b200.
-context_parallel) on CPU: world_size-2 and -3 gloo ranks, each rank's compute
-steps (local pooling, scoring, top-k; attention over a given block list) done
-by the fp64 oracle, the candidate exchange and the partial merge by the module
-under test. The result must equal the oracle's single-process decode: the same
-selected blocks and the same gated outputs."""
+context_parallel) on CPU: world_size-2 and -3 gloo ranks. Each rank's four
+compute steps, which the library runs as kernels on a GPU (shard selection,
+global top-k, shard attention, log-sum-exp merge), are done here by fp64
+stand-ins written from the pages' definitions with the oracle's functions;
+the module under test drives them and moves the candidates and partials
+between the ranks with all-gathers. The result must equal the oracle's
+single-process decode: the same selected blocks and the same gated outputs,
+for one and two new tokens per sequence and for sequences that end inside an
+early shard."""
 import datetime
 import os
 import socket
@@ -22,68 +26,99 @@ from block_sparse_attention_17_b200.workloads import WORKLOADS, make_decode_inpu
 from oracle import qsa_oracle as O  # noqa: E402
 
 
-def _case():
-    # 3 sequences of a few hundred blocks, one new token each; B = 16 keeps it small
+def _case(n_q):
+    # 3 sequences of up to 60 blocks; B = 16 keeps it small; the third one
+    # ends in the first half of the cache (inside an early shard)
     w = WORKLOADS["decode_bf16_b32_kv32768"].with_(dtype="f32", batch=3, block_size=16,
-                                                   budget=16 * 8, cap=16 * 60, kv_len=16 * 60)
-    kv = np.array([16 * 60, 16 * 53 + 7, 16 * 45 + 1], np.int32)
+                                                   budget=16 * 8, cap=16 * 60, kv_len=16 * 60,
+                                                   n_q=n_q)
+    kv = np.array([16 * 60, 16 * 53 + 7, 16 * 21 + 1], np.int32)
     return w, make_decode_inputs(w, kv_lens=kv)
 
 
 def _oracle_fns(w, inp, b0, b1):
-    """This rank's compute steps on its shard, by the oracle (fp64)."""
-    B, k = w.block_size, w.topk
+    """This rank's four steps on shard [b0, b1), in fp64 with the oracle's
+    functions (global block ids; the shard sees the full cache rows)."""
+    B, k, n_q = w.block_size, w.topk, w.n_q
     sm, isc = w.head_dim ** -0.5, w.idx_dim ** -0.5
-    nloc = b1 - b0
-    ik = inp["ik_cache"][:, b0 * B:b1 * B]
-    K, V = inp["k_cache"][:, b0 * B:b1 * B], inp["v_cache"][:, b0 * B:b1 * B]
 
-    def select_fn(kv_loc):
-        batch = kv_loc.shape[0]
-        sel = torch.full((batch, 1, k + 1), -1, dtype=torch.int32)
-        nsel = torch.zeros(batch, 1, dtype=torch.int32)
-        scores = torch.full((batch, 1, nloc), float("-inf"), dtype=torch.float64)
-        for b in range(batch):
-            n = int(kv_loc[b])
-            kbar = O.pool_blocks(ik[b, :n], B)
-            s = O.index_scores(inp["iq"][b, 0], inp["iw"][b, 0], kbar, isc)
-            chosen = list(O.select_topk(s, k)) + ([n // B] if n % B else [])
-            sel[b, 0, :len(chosen)] = torch.tensor(chosen, dtype=torch.int32)
-            nsel[b, 0] = len(chosen)
-            scores[b, 0, :len(s)] = torch.from_numpy(s)
-        return {"sel": sel, "nsel": nsel, "scores": scores}
+    def visible(kv, i):
+        return int(kv) - n_q + 1 + i
 
-    def attend_fn(kv_loc, sel, nsel):
-        batch = kv_loc.shape[0]
-        out = torch.zeros(batch, 1, w.num_q_heads, w.head_dim, dtype=torch.float64)
-        lse = torch.full((batch, 1, w.num_q_heads), float("-inf"), dtype=torch.float64)
+    def select(kv_len):
+        batch = kv_len.shape[0]
+        score = torch.full((batch, n_q, k), float("-inf"), dtype=torch.float64)
+        ids = torch.full((batch, n_q, k), -1, dtype=torch.int32)
         for b in range(batch):
-            n = int(kv_loc[b])
-            pos = [np.arange(j * B, min((j + 1) * B, n)) for j in sel[b, 0, :int(nsel[b, 0])].tolist()]
-            pos = np.concatenate(pos) if pos else np.zeros(0, np.int64)
-            o, l = O.gated_attention(inp["q"][b, 0], K[b], V[b], pos, inp["gate"][b, 0], sm)
-            out[b, 0], lse[b, 0] = torch.from_numpy(o), torch.from_numpy(l)
+            kbar = O.pool_blocks(inp["ik_cache"][b, :int(kv_len[b])], B)
+            for i in range(n_q):
+                nc = visible(kv_len[b], i) // B
+                mine = list(range(b0, min(b1, nc)))
+                if not mine:
+                    continue
+                s = O.index_scores(inp["iq"][b, i], inp["iw"][b, i], kbar[mine], isc)
+                top = O.select_topk(s, k)
+                score[b, i, :len(top)] = torch.from_numpy(s[top])
+                ids[b, i, :len(top)] = torch.tensor([mine[t] for t in top], dtype=torch.int32)
+        return {"score": score, "id": ids}
+
+    def global_topk(cs, cid, kv_len):
+        W, batch = cs.shape[0], cs.shape[1]
+        sel = torch.full((batch, n_q, k + 1), -1, dtype=torch.int32)
+        nsel = torch.zeros(batch, n_q, dtype=torch.int32)
+        for b in range(batch):
+            for i in range(n_q):
+                cands = [(float(cs[r, b, i, j]), int(cid[r, b, i, j]))
+                         for r in range(W) for j in range(k) if int(cid[r, b, i, j]) >= 0]
+                cands.sort(key=lambda c: (-c[0], c[1]))
+                chosen = sorted(c[1] for c in cands[:k])
+                n = visible(kv_len[b], i)
+                if n % B:
+                    chosen.append(n // B)
+                sel[b, i, :len(chosen)] = torch.tensor(chosen, dtype=torch.int32)
+                nsel[b, i] = len(chosen)
+        return {"sel": sel, "nsel": nsel}
+
+    def attend(kv_len, sel, nsel):
+        batch = kv_len.shape[0]
+        out = torch.zeros(batch, n_q, w.num_q_heads, w.head_dim, dtype=torch.float64)
+        lse = torch.full((batch, n_q, w.num_q_heads), float("-inf"), dtype=torch.float64)
+        for b in range(batch):
+            for i in range(n_q):
+                n = visible(kv_len[b], i)
+                blocks = [j for j in sel[b, i, :int(nsel[b, i])].tolist() if b0 <= j < b1]
+                pos = [np.arange(j * B, min((j + 1) * B, n)) for j in blocks]
+                pos = np.concatenate(pos) if pos else np.zeros(0, np.int64)
+                if len(pos) == 0:
+                    continue
+                o, l = O.gated_attention(inp["q"][b, i], inp["k_cache"][b], inp["v_cache"][b],
+                                         pos, inp["gate"][b, i], sm)
+                out[b, i], lse[b, i] = torch.from_numpy(o), torch.from_numpy(l)
         return {"out": out, "lse": lse}
-    return select_fn, attend_fn
+
+    def merge(po, pl):
+        lse = torch.logsumexp(pl, dim=0)
+        wgt = torch.nan_to_num(torch.exp(pl - lse[None]), nan=0.0)
+        return {"out": (wgt[..., None] * po).sum(dim=0), "lse": lse}
+
+    return cp.CpFns(select=select, global_topk=global_topk, attend=attend, merge=merge)
 
 
-def _rank_main(rank, world, port, results):
+def _rank_main(rank, world, n_q, port, results):
     import torch.distributed as dist
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world,
                             timeout=datetime.timedelta(seconds=60))
     try:
-        w, inp = _case()
+        w, inp = _case(n_q)
         nblk = w.cap // w.block_size
         b0, b1 = cp.shard_blocks(nblk, world, rank)
-        select_fn, attend_fn = _oracle_fns(w, inp, b0, b1)
         cfg = cp.qsa.QSAConfig.from_workload(w)
-        q = torch.from_numpy(inp["q"]).double()
-        r = cp.decode_step(cfg, q, None, None, None, None, None, None, None,
-                           torch.from_numpy(inp["kv_len"]), b0=b0, b1=b1,
-                           is_last=rank == world - 1, select_fn=select_fn, attend_fn=attend_fn)
-        results[rank] = (r["out"].numpy(), r["lse"].numpy(), r["sel"].numpy(), r["count"].numpy())
+        r = cp.decode_step(cfg, None, None, None, None, None, None, None, None,
+                           torch.from_numpy(inp["kv_len"]), b0=b0,
+                           fns=_oracle_fns(w, inp, b0, b1))
+        results[rank] = (r["out"].numpy(), r["lse"].numpy(), r["sel"].numpy(), r["nsel"].numpy())
     finally:
         dist.destroy_process_group()
 
@@ -94,37 +129,25 @@ def _free_port():
         return s.getsockname()[1]
 
 
-@pytest.mark.parametrize("world", [2, 3])
-def test_context_parallel_decode_gloo_matches_single_process(world):
+@pytest.mark.parametrize("world,n_q", [(2, 1), (3, 1), (3, 2)])
+def test_context_parallel_decode_gloo_matches_single_process(world, n_q):
     mgr = mp.get_context("spawn").Manager()
     results = mgr.dict()
-    mp.start_processes(_rank_main, args=(world, _free_port(), results), nprocs=world,
+    mp.start_processes(_rank_main, args=(world, n_q, _free_port(), results), nprocs=world,
                        join=True, start_method="spawn")
     assert sorted(results.keys()) == list(range(world))
-    w, inp = _case()
+    w, inp = _case(n_q)
     orc = O.qsa_decode(w, inp)["queries"]
     for rank in range(world):
-        out, lse, sel, count = results[rank]
+        out, lse, sel, nsel = results[rank]
         for b in range(w.batch):
-            ref = orc[(b, 0)]
-            got = [j for j in sel[b].tolist() if j >= 0]
-            assert got == list(ref.selected), (rank, b)
-            assert int(count[b]) == len(ref.selected)
-            np.testing.assert_allclose(out[b, 0], ref.out, rtol=1e-10, atol=1e-12)
-            np.testing.assert_allclose(lse[b, 0], ref.lse, rtol=1e-10, atol=1e-12)
+            for i in range(n_q):
+                ref = orc[(b, i)]
+                exp = list(ref.selected) + ([ref.nc] if ref.tail else [])
+                assert sel[b, i, :int(nsel[b, i])].tolist() == exp, (rank, b, i)
+                np.testing.assert_allclose(out[b, i], ref.out, rtol=1e-10, atol=1e-12)
+                np.testing.assert_allclose(lse[b, i], ref.lse, rtol=1e-10, atol=1e-12)
         np.testing.assert_array_equal(out, results[0][0])   # every rank holds the same result
-
-
-def test_global_topk_order_and_ties():
-    # scores tie across ranks: the lower block id wins; -0 ties +0
-    cs = torch.tensor([[[3.0, 1.0, -0.0]], [[1.0, 2.0, float("-inf")]]])
-    cid = torch.tensor([[[10, 4, 7]], [[2, 30, 2 ** 62]]])
-    ids, count = cp.global_topk(cs, cid, 3)
-    assert ids.tolist() == [[2, 10, 30]] and count.tolist() == [3]
-    cs = torch.tensor([[[0.0, 5.0]], [[-0.0, float("-inf")]]])
-    cid = torch.tensor([[[9, 1]], [[3, 2 ** 62]]])
-    ids, count = cp.global_topk(cs, cid, 2)
-    assert ids.tolist() == [[1, 3]] and count.tolist() == [2]
 
 
 def test_shard_blocks_cover_the_cache_once():
@@ -135,32 +158,29 @@ def test_shard_blocks_cover_the_cache_once():
             assert covered == list(range(nblk))
 
 
-def test_local_candidates_skip_the_tail_and_unused_slots():
-    # local selection: blocks 1, 5 (complete) and the tail block 7 (score -inf)
-    sel = torch.tensor([[[1, 5, 7, -1]]], dtype=torch.int32)
-    nsel = torch.tensor([[3]], dtype=torch.int32)
-    scores = torch.tensor([[[0.1, 2.0, 0.3, 0.4, 0.5, 1.5, 0.0, float("-inf")]]])
-    sc, gid = cp.local_candidates(sel, nsel, scores, 3, b0=100)
-    assert gid.tolist() == [[101, 105, 2 ** 62]]
-    assert sc[0, :2].tolist() == [2.0, 1.5] and sc[0, 2].item() == float("-inf")
+def test_decode_step_passes_each_rank_result_through_the_gather():
+    # a world of 2 emulated by a gather that stacks this rank's tensor with a
+    # second rank's (a fixed tensor): the global top-k and the merge must see
+    # [world, ...] arrays in rank order
+    seen = {}
 
+    def gather(t):
+        other = torch.full_like(t, 7)
+        return torch.stack([t, other])
 
-def test_local_share_adds_the_tail_on_the_last_rank_only():
-    gids = torch.tensor([[3, 10, 25, -1], [8, 9, -1, -1]])
-    kv = torch.tensor([16 * 16 + 5, 16 * 16], dtype=torch.int32)   # rows in the shard
-    sel, nsel = cp.local_share(gids, 8, 24, kv, 16, 4, is_last=True)
-    assert sel[0, 0].tolist() == [2, 16, -1, -1, -1] and nsel[0, 0].item() == 2   # tail block 16
-    assert sel[1, 0].tolist() == [0, 1, -1, -1, -1] and nsel[1, 0].item() == 2    # no tail
-    sel, nsel = cp.local_share(gids, 8, 24, kv, 16, 4, is_last=False)
-    assert sel[0, 0].tolist() == [2, -1, -1, -1, -1] and nsel[0, 0].item() == 1
-
-
-def test_merge_partials_weights_and_empty_ranks():
-    outs = torch.tensor([[[[1.0, 2.0]]], [[[3.0, 4.0]]], [[[9.0, 9.0]]]])     # [R, b, 1, 2]
-    lses = torch.tensor([[[0.0]], [[float(np.log(3.0))]], [[float("-inf")]]])  # [R, b, 1]
-    out, lse = cp.merge_partials(outs[..., None, :].squeeze(-2), lses)
-    # weights 1/4 and 3/4; the rank with nothing attended weighs nothing
-    assert torch.allclose(out, torch.tensor([[[2.5, 3.5]]]))
-    assert torch.allclose(lse, torch.tensor([[float(np.log(4.0))]]))
-    out, lse = cp.merge_partials(outs[:1] * 0, torch.full((1, 1, 1), float("-inf")))
-    assert torch.equal(out, torch.zeros(1, 1, 2)) and lse.item() == float("-inf")
+    fns = cp.CpFns(
+        select=lambda kv: {"score": torch.ones(1, 1, 2), "id": torch.tensor([[[1, 2]]])},
+        global_topk=lambda cs, cid, kv: seen.setdefault("g", (cs, cid)) and
+        {"sel": torch.tensor([[[1, 2, -1]]]), "nsel": torch.tensor([[2]])},
+        attend=lambda kv, sel, nsel: {"out": torch.zeros(1, 1, 1, 4), "lse": torch.zeros(1, 1, 1)},
+        merge=lambda po, pl: seen.setdefault("m", (po, pl)) and
+        {"out": po[0], "lse": pl[0]})
+    cfg = cp.qsa.QSAConfig(num_q_heads=1, num_kv_heads=1, head_dim=4, idx_heads=1, idx_dim=4,
+                           block_size=64, budget=128)
+    r = cp.decode_step(cfg, None, None, None, None, None, None, None, None,
+                       torch.tensor([300], dtype=torch.int32), b0=0, fns=fns, gather_fn=gather)
+    cs, cid = seen["g"]
+    assert cs.shape == (2, 1, 1, 2) and cid[0].tolist() == [[[1, 2]]] and cid[1].eq(7).all()
+    po, pl = seen["m"]
+    assert po.shape == (2, 1, 1, 1, 4) and pl.shape == (2, 1, 1, 1)
+    assert r["nsel"].tolist() == [[2]]
