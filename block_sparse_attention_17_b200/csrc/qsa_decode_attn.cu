@@ -25,7 +25,6 @@
 //     gate; where such a cluster cannot be resident (two-launch path only), the
 //     partials go through global memory and the last CTA merges them.
 // kFp8 reads e4m3 K/V codes with per-row scales instead of bf16 rows.
-#include <cstdlib>
 #include <map>
 #include <mutex>
 #include <tuple>
@@ -107,8 +106,6 @@ struct DecParams {
   int* sel_w;                        // [batch, n_q, k + 1] selections out
   int* nsel_w;                       // [batch, n_q]
   int fo_keys, fo_kbar, fo_iq, fo_iw, fo_new, fo_hist;   // byte offsets in the ring's space
-  int spec_m;                        // blocks per query whose K/V each CTA prefetches into L2
-                                     // before the cluster's top-k (its best-scored ones)
   int early;                         // the first scoring pass's pooled rows are copied into
                                      // shared memory at kernel entry (stage_pooled_early)
   // context-parallel shard (attention over given selections only): kv_len are
@@ -407,72 +404,9 @@ __device__ __forceinline__ void select_prefetch(const DecParams& P, int kv, int 
     bulk_prefetch_l2(P.iq + (size_t)b * P.n_q * g.Hi * kDI, (uint32_t)(P.n_q * g.Hi * kDI * 2));
 }
 
-// Speculation while the cluster's top-k runs: the K and V rows (this CTA's KV
-// head) of the spec_m best-scored blocks of this CTA's own candidate range, per
-// query, are prefetched into L2. The blocks the top-k then selects in this range
-// are the range's best ones (a range holds about k / nsplit of them), so most of
-// the selected bytes are on their way from HBM before the selection is known;
-// a prefetched block that is not selected only costs its bandwidth. Warp 0;
-// keys_mine holds the range's keys per query (keys of complete blocks only).
-__device__ __forceinline__ void spec_prefetch(const DecParams& P, const CUtensorMap* tmK,
-                                              const CUtensorMap* tmV, const uint32_t* keys_mine,
-                                              int per, int j0, int j1, int kv, int b, int hk,
-                                              bool fp8) {
-  const Geom& g = P.g;
-  const int lane = threadIdx.x & 31;
-  const int nblk_cap = P.cap / g.B;
-  for (int i = 0; i < P.n_q; ++i) {
-    const int nc_i = (kv - P.n_q + 1 + i) / g.B;
-    const int cnt = min(min(j1, nc_i) - j0, 32 * 32);   // keys of query i in the range (scan cap)
-    uint32_t taken = 0u;                                 // bit t: key lane + 32 t already taken
-    for (int it = 0; it < P.spec_m && cnt > 0; ++it) {
-      uint32_t best = 0u;
-      int bestr = -1;
-      for (int r = lane, t = 0; r < cnt; r += 32, ++t) {
-        if ((taken >> t) & 1u) continue;
-        const uint32_t key = keys_mine[i * per + r];
-        if (bestr < 0 || key > best) {
-          best = key;
-          bestr = r;
-        }
-      }
-      const uint32_t wmax = __reduce_max_sync(kFull, bestr >= 0 ? best : 0u);
-      const uint32_t cand = __ballot_sync(kFull, bestr >= 0 && best == wmax);
-      if (!cand) break;
-      const int src = __ffs(cand) - 1;
-      const int rsel = __shfl_sync(kFull, bestr, src);
-      if (lane == src) taken |= 1u << (rsel >> 5);
-      if (lane == 0) {
-        const int j = j0 + rsel;
-        long long row = (long long)b * P.cap + (long long)j * g.B;
-        bool ok = true;
-        if (P.table) {
-          const int page = P.table[(size_t)b * nblk_cap + j];
-          ok = page >= 0 && page < P.num_pages;
-          row = (long long)page * g.B;
-        }
-        if (ok) {
-          for (int off = 0; off < g.B; off += kChunk) {
-            if (fp8) {
-              tma_prefetch_l2_3d(tmK, 0, hk, (int)(row + off));
-              tma_prefetch_l2_3d(tmV, 0, hk, (int)(row + off));
-            } else {
-              tma_prefetch_l2_3d(tmK, 0, hk, (int)(row + off));
-              tma_prefetch_l2_3d(tmK, 64, hk, (int)(row + off));
-              tma_prefetch_l2_3d(tmV, 0, hk, (int)(row + off));
-              tma_prefetch_l2_3d(tmV, 64, hk, (int)(row + off));
-            }
-          }
-        }
-      }
-    }
-  }
-}
-
 template <int kDI>
 __device__ __forceinline__ void select_in_cluster(const DecParams& P, uint8_t* smem, int kv, int split, int b,
-                                  int hk, uint32_t* qbits, int words, const CUtensorMap* tmK,
-                                  const CUtensorMap* tmV, bool fp8) {
+                                  int hk, uint32_t* qbits, int words) {
   constexpr int kStride = kDI + 4;                 // 16-byte rows; 8 rows of a warp hit distinct banks
   constexpr int kQStrideI = kDI + 4;
   constexpr int kRows = kSelRows;                 // candidate blocks per scoring pass
@@ -629,7 +563,6 @@ __device__ __forceinline__ void select_in_cluster(const DecParams& P, uint8_t* s
     }
   }
   cp_async_wait_all();   // (a CTA with no candidates never waited on its early copies)
-  if (P.spec_m > 0 && warp == 0) spec_prefetch(P, tmK, tmV, keys_mine, per, j0, j1, kv, b, hk, fp8);
   cluster_sync_all();   // every CTA's keys (and their extremes) are in place
   const uint32_t mine_s = smem_u32(keys_mine), mm_s = smem_u32(mm_mine);
   // With several queries, CTA s selects queries s, s + nsplit, ... and the
@@ -910,7 +843,7 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
       float* iw_s = reinterpret_cast<float*>(smem + kOffStages + P.fo_iw);
       if (threadIdx.x < n_q * g.Hi) iw_s[threadIdx.x] = iwreg;
     }
-    select_in_cluster<kSelDI>(P, smem, kv, split, b, hk, qbits, words, &tmK, &tmV, kFp8);
+    select_in_cluster<kSelDI>(P, smem, kv, split, b, hk, qbits, words);
   } else {
     // the selections come from the selection kernel: wait for this sequence's
     // flag (bounded), or for the whole selection grid
@@ -1605,17 +1538,6 @@ bool fused_layout(const Geom& g, int n_q, int cap, int nsplit, DecParams* p) {
   return off <= (long long)kStages * kStageBytes;
 }
 
-// Blocks per query each CTA of a decode cluster prefetches into L2 ahead of the
-// cluster's top-k (QSA_SPEC_BLOCKS overrides the default, 0 turns it off).
-int spec_prefetch_blocks(const Geom& g, int nsplit) {
-  static const int env = [] {
-    const char* e = getenv("QSA_SPEC_BLOCKS");
-    return e ? atoi(e) : -1;
-  }();
-  if (env >= 0) return env;
-  return (g.k + nsplit - 1) / nsplit + 1;
-}
-
 template <bool kFp8>
 const void* fused_kernel(int di) {
   return di == 64 ? reinterpret_cast<const void*>(attn_decode_mma_kernel<kFp8, 64>)
@@ -1746,8 +1668,6 @@ cudaError_t launch_decode_fused(const Geom& g, int batch, int n_q, int cap, int 
   p.pooled = si.pooled;
   p.sel_w = si.sel;
   p.nsel_w = si.nsel;
-  // about k / nsplit of a range's blocks are selected; one more is prefetched
-  p.spec_m = spec_prefetch_blocks(g, nsplit);
   // the fp8 kernel stages its query rows at the end of the fp8 ring, which the
   // early pooled rows must not reach
   p.early = !f8.on || p.fo_iq <= kStages * kF8StageBytes;

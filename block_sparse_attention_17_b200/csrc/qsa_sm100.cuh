@@ -158,14 +158,6 @@ __device__ __forceinline__ void cp_async_commit() {
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_all;" ::: "memory");
 }
-// Prefetch of one tiled box of a tensor map into L2 (no shared memory, no
-// completion to wait for; a hint that the box will be loaded soon).
-__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int c0, int c1, int c2) {
-  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(c0), "r"(c1), "r"(c2)
-               : "memory");
-}
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -322,7 +314,9 @@ __device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t addr) {
 // The cubic's coefficients were fitted for this library to keep the largest
 // relative error of 2^f on [-1/2, 1/2] small; the error curve is close to
 // equi-ripple (minimax), with a maximum of 7.6e-5, far below the 2^-9 rounding
-// of the bf16 probabilities it feeds. Inputs below -126 give about 2^-126
+// of the bf16 probabilities it feeds. A result under 2^-126 (x within 1e-3 of
+// -126) comes out of the exponent addition as a subnormal without its implicit
+// bit, accurate to 1.5e-4 relative; inputs below -126 give about 2^-126
 // instead of 0.
 __device__ __forceinline__ float exp2_poly(float x) {
   constexpr float kMagic = 12582912.0f;    // 1.5 * 2^23
