@@ -706,7 +706,8 @@ qsa_status qsa_decode_paged(const qsa_config* cfg, int batch, int n_q, int max_b
   if ((s = check_pages(cfg, max_blocks, block_table, num_pages)) != QSA_OK) return s;
   const Geom g = make_geom(cfg);
   if (!decode_uses_mma(cfg, g, n_q))
-    return fail(QSA_ERR_UNSUPPORTED, "paged decode needs bf16 and n_q * group size <= 16");
+    return fail(QSA_ERR_UNSUPPORTED,
+                "paged decode needs bf16, head_dim 128 and n_q * group size <= 32");
   return decode_impl(cfg, batch, n_q, max_blocks * cfg->block_size, kv_len, q, k_pages, v_pages,
                      iq, ik_pages, iw, gate, pooled_cache, out, lse, sel, nsel, dev_err,
                      workspace, workspace_bytes, stream, Pages{block_table, num_pages});

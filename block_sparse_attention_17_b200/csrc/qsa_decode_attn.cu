@@ -68,13 +68,19 @@ static_assert(kStages * kF8StageBytes + kF8ConvBytes <= kStages * kStageBytes,
               "the fp8 layout fits in the bf16 ring's space");
 
 constexpr int kOffStages = 0;
-constexpr int kOffQ = kOffStages + kStages * kStageBytes;
-constexpr int kOffBar = kOffQ + 16 * kQStride;
-constexpr int kOffMisc = kOffBar + 8 * 2 * kStages;
-constexpr int kOffUnion = kOffMisc + 64;
-constexpr int kOffGate = kOffUnion + 8 * kMaxUnion;   // cluster merge: [16 rows][128] gate bf16
-constexpr int kOffBits = kOffGate + 16 * kD * 2;      // [n_q][cap / B / 32] words
-// dynamic shared memory: kOffBits + 4 * n_q * words + 1024 (alignment slack)
+// Shared memory of a kernel that holds kRT tiles of 16 query rows (rows
+// r = i * G + gi: new query i, head gi of the KV head). Dynamic shared memory:
+// kOffBits + 4 * n_q * words + 1024 (alignment slack).
+template <int kRT>
+struct DecLayout {
+  static constexpr int kRows = 16 * kRT;
+  static constexpr int kOffQ = kOffStages + kStages * kStageBytes;
+  static constexpr int kOffBar = kOffQ + kRows * kQStride;
+  static constexpr int kOffMisc = kOffBar + 8 * 2 * kStages;
+  static constexpr int kOffUnion = kOffMisc + 64;
+  static constexpr int kOffGate = kOffUnion + 8 * kMaxUnion;   // cluster merge: [rows][128] gate
+  static constexpr int kOffBits = kOffGate + kRows * kD * 2;   // [n_q][cap / B / 32] words
+};
 
 struct DecParams {
   Geom g;
@@ -106,8 +112,6 @@ struct DecParams {
   int* sel_w;                        // [batch, n_q, k + 1] selections out
   int* nsel_w;                       // [batch, n_q]
   int fo_keys, fo_kbar, fo_iq, fo_iw, fo_new, fo_hist;   // byte offsets in the ring's space
-  int early;                         // the first scoring pass's pooled rows are copied into
-                                     // shared memory at kernel entry (stage_pooled_early)
   // context-parallel shard (attention over given selections only): kv_len are
   // full lengths, the caches hold rows [row_off, row_off + cap), sel holds
   // global block ids; outputs are fp32 gated partials in out_f32
@@ -242,17 +246,9 @@ __device__ __forceinline__ void cta_topk_radix(const uint32_t* keys, int n, int 
       for (int e = tid; e < 256; e += nthr) hist[e] = 0;
       __syncthreads();
     }
-    // lanes with the same digit add their count with one atomic (the keys of a
-    // query crowd into few digit values, which would serialise plain atomics)
-    for (int j0 = warp * 32; j0 < n; j0 += nthr) {   // warp-uniform
-      const int j = j0 + lane;
-      int bin = -1;
-      if (j < n) {
-        const uint32_t key = keys[j];
-        if ((key & pmask) == prefix) bin = (int)((key >> shift) & 255u);
-      }
-      const unsigned peers = __match_any_sync(kFull, bin);
-      if (bin >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+    for (int j = tid; j < n; j += nthr) {
+      const uint32_t key = keys[j];
+      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
     }
     __syncthreads();
     if (warp == 0) {
@@ -337,33 +333,10 @@ __device__ __forceinline__ uint4 ld_cluster_u32x4(uint32_t addr) {
 }
 
 // Chunk of candidate blocks one CTA of the cluster scores: a multiple of 4, so
-// that the gather below moves 16-byte groups owned by one CTA. The ranges split
-// the cache's blocks (cap / B, known before the sequence's length is read), so
-// that a CTA can start loading its pooled rows at once.
-__host__ __device__ __forceinline__ int select_range(int nblk_cap, int nsplit) {
-  const int per = ((nblk_cap > 1 ? nblk_cap : 1) + nsplit - 1) / nsplit;
+// that the gather below moves 16-byte groups owned by one CTA.
+__host__ __device__ __forceinline__ int select_range(int nc_last, int nsplit) {
+  const int per = ((nc_last > 1 ? nc_last : 1) + nsplit - 1) / nsplit;
   return (per + 3) & ~3;
-}
-
-// Starts the copies of the first scoring pass's pooled rows of this CTA's range
-// into shared memory (cp.async, padded rows), before the sequence's length is
-// known; rows past the sequence's complete blocks are never scored, and the row
-// of a block this step completes is replaced by its fresh pooling.
-template <int kDI>
-__device__ __forceinline__ void stage_pooled_early(const DecParams& P, uint8_t* smem, int split,
-                                                   int b) {
-  constexpr int kStride = kDI + 4;
-  const int nblk_cap = P.cap / P.g.B;
-  const int per = select_range(nblk_cap, P.nsplit);
-  const int j0 = split * per;
-  const int rows = min(min(kSelRows, per), nblk_cap - j0);
-  float* kbar_s = reinterpret_cast<float*>(smem + kOffStages + P.fo_kbar);
-  const float* src = P.pooled + ((size_t)b * nblk_cap + j0) * kDI;
-  for (int e = threadIdx.x; e < rows * (kDI / 4); e += blockDim.x) {
-    const int r = e / (kDI / 4), d4 = e - r * (kDI / 4);
-    cp_async16(smem_u32(kbar_s + r * kStride + 4 * d4), src + (size_t)r * kDI + 4 * d4);
-  }
-  cp_async_commit();
 }
 
 // The selection step of one decode step, done by the cluster of one (sequence,
@@ -386,7 +359,7 @@ template <int kDI>
 __device__ __forceinline__ void select_prefetch(const DecParams& P, int kv, int split, int b) {
   const Geom& g = P.g;
   const int nblk_cap = P.cap / g.B, nc_last = kv / g.B;
-  const int per = select_range(nblk_cap, P.nsplit);
+  const int per = select_range(nc_last, P.nsplit);
   const int j0 = split * per, j1 = min(nc_last, j0 + per);
   if (j1 > j0)
     bulk_prefetch_l2(P.pooled + ((size_t)b * nblk_cap + j0) * kDI, (uint32_t)(j1 - j0) * kDI * 4u);
@@ -415,7 +388,7 @@ __device__ __forceinline__ void select_in_cluster(const DecParams& P, uint8_t* s
   const int tid = threadIdx.x, nthr = blockDim.x, warp = tid >> 5, lane = tid & 31;
   const int nblk_cap = P.cap / g.B;
   const int nc_last = kv / g.B;
-  const int per = select_range(nblk_cap, P.nsplit);
+  const int per = select_range(nc_last, P.nsplit);
   const int j0 = split * per, j1 = min(nc_last, j0 + per);
   uint8_t* ring = smem + kOffStages;
   uint32_t* mm_mine = reinterpret_cast<uint32_t*>(ring);                    // [4][2] largest, smallest key
@@ -467,18 +440,7 @@ __device__ __forceinline__ void select_in_cluster(const DecParams& P, uint8_t* s
   uint32_t qhi[4] = {0u, 0u, 0u, 0u}, qlo[4] = {~0u, ~0u, ~0u, ~0u};
   for (int r0 = j0; r0 < j1; r0 += kRows) {
     const int rows = min(kRows, j1 - r0);
-    if (r0 == j0 && P.early) {
-      // the rows came by the copies started at kernel entry; the rows of the
-      // blocks this step completes are the fresh poolings
-      cp_async_wait_all();
-      __syncthreads();
-      for (int e = tid; e < (jn_hi - jn_lo) * (kDI / 4); e += nthr) {
-        const int r = e / (kDI / 4), d4 = e - r * (kDI / 4);
-        if (jn_lo + r - r0 < rows)
-          *reinterpret_cast<float4*>(kbar_s + (jn_lo + r - r0) * kStride + 4 * d4) =
-              *reinterpret_cast<const float4*>(new_s + r * kDI + 4 * d4);
-      }
-    } else {   // every load of the pass is issued before the first store
+    {   // every load of the pass is issued before the first store
       constexpr int kLd = (kRows * (kDI / 4) + kThreads - 1) / kThreads;   // float4 per thread
       float4 v[kLd];
 #pragma unroll
@@ -562,7 +524,6 @@ __device__ __forceinline__ void select_in_cluster(const DecParams& P, uint8_t* s
       }
     }
   }
-  cp_async_wait_all();   // (a CTA with no candidates never waited on its early copies)
   cluster_sync_all();   // every CTA's keys (and their extremes) are in place
   const uint32_t mine_s = smem_u32(keys_mine), mm_s = smem_u32(mm_mine);
   // With several queries, CTA s selects queries s, s + nsplit, ... and the
@@ -651,10 +612,18 @@ __device__ __forceinline__ void select_in_cluster(const DecParams& P, uint8_t* s
   cluster_arrive_all();   // this CTA has read the other CTAs' keys
 }
 
-template <bool kFp8, int kSelDI>
-__global__ void __launch_bounds__(kThreads, 2)
+template <bool kFp8, int kSelDI, int kRT>
+__global__ void __launch_bounds__(kThreads, kRT == 1 ? 2 : 1)
 attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const DecParams P) {
+  static_assert(kRT == 1 || (kRT == 2 && !kFp8), "fp8 caches: one 16-row tile");
+  using L = DecLayout<kRT>;
+  // Consumer warp w works on row tile w / kWPT and keys [kKW (w % kWPT), + kKW)
+  // of every chunk: 16 keys with one row tile, 32 keys with two.
+  constexpr int kWPT = kConsumers / kRT;   // consumer warps per row tile
+  constexpr int kKW = kChunk / kWPT;       // keys per warp and chunk
+  constexpr int kNT = kKW / 8;             // n-tiles of 8 keys (QK^T)
+  constexpr int kKS = kKW / 16;            // k-steps of 16 keys (PV)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -663,30 +632,28 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
   const int split = blockIdx.x, b = blockIdx.y, hk = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = g.G, n_q = P.n_q, R = n_q * G;
-  if constexpr (kSelDI > 0) {
-    grid_dependency_wait();   // every input may come from the previous kernel
-    if (P.early) stage_pooled_early<kSelDI>(P, smem, split, b);
-  }
+  if constexpr (kSelDI > 0) grid_dependency_wait();   // every input may come from the previous kernel
   // Inputs that do not depend on the sequence's length are loaded together
   // with it, into registers: Q rows r = i * G + gi (query i, head hk * G + gi;
   // zero beyond R), the gate rows this CTA merges (cluster merge: rows split,
   // split + nsplit, ...), and for the in-kernel selection the queries' indexer
   // q and weights.
-  constexpr int kQLd = (16 * (kD / 8) + kThreads - 1) / kThreads;
+  constexpr int kQLd = (L::kRows * (kD / 8) + kThreads - 1) / kThreads;
   uint4 qreg[kQLd];
 #pragma unroll
   for (int u = 0; u < kQLd; ++u) {
     const int e = threadIdx.x + u * kThreads, r = e / (kD / 8), c8 = e % (kD / 8);
     qreg[u] = make_uint4(0, 0, 0, 0);
-    if (e < 16 * (kD / 8) && r < R)
+    if (e < L::kRows * (kD / 8) && r < R)
       qreg[u] = *reinterpret_cast<const uint4*>(
           P.q + (((size_t)b * n_q + r / G) * g.Hq + hk * G + r % G) * kD + c8 * 8);
   }
   const int g_per_row = g.gate_headwise ? 1 : kD / 8;   // uint4 per gate row (or one value)
   const int g_rows = P.cluster && split < R ? (R - split + P.nsplit - 1) / P.nsplit : 0;
-  uint4 greg[2];   // g_rows * g_per_row <= 16 * 16 <= 2 * kThreads
+  constexpr int kGLd = (L::kRows * (kD / 8) + kThreads - 1) / kThreads;
+  uint4 greg[kGLd];   // g_rows * g_per_row <= rows * 16
 #pragma unroll
-  for (int u = 0; u < 2; ++u) {
+  for (int u = 0; u < kGLd; ++u) {
     const int e = threadIdx.x + u * kThreads;
     greg[u] = make_uint4(0, 0, 0, 0);
     if (e < g_rows * g_per_row) {
@@ -711,7 +678,6 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
   const int kv = P.kv_len[b] - P.row_off;   // (a shard's rows: may be past either end)
   const size_t row0 = (((size_t)b * g.Hkv + hk) * P.nsplit + split) * R;
   if (!P.cp && (kv < n_q || kv > P.cap)) {   // reported by the selection; outputs are zero
-    if constexpr (kSelDI > 0) cp_async_wait_all();   // no copy may land after the CTA left
     if (split == 0 && hk == 0) {
       if constexpr (kSelDI > 0) {
         const int kp1 = g.k + 1;
@@ -731,11 +697,11 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
   }
   if constexpr (kSelDI > 0)
     if (threadIdx.x == 0) select_prefetch<kSelDI>(P, kv, split, b);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
   uint64_t* empty = full + kStages;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc);
-  int* n_chunks_s = reinterpret_cast<int*>(smem + kOffMisc + 4);
-  int* u_blk = reinterpret_cast<int*>(smem + kOffUnion);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc);
+  int* n_chunks_s = reinterpret_cast<int*>(smem + L::kOffMisc + 4);
+  int* u_blk = reinterpret_cast<int*>(smem + L::kOffUnion);
   int* u_qm = u_blk + kMaxUnion;
   const int cpb = g.B / kChunk;   // chunks per block
 
@@ -743,7 +709,7 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
   // with a mask of the queries that selected each block: per-query bitmaps in
   // shared memory, then one ordered scan by warp 0
   const int words = (P.cap / g.B + 31) / 32;
-  uint32_t* qbits = reinterpret_cast<uint32_t*>(smem + kOffBits);   // [n_q][words]
+  uint32_t* qbits = reinterpret_cast<uint32_t*>(smem + L::kOffBits);   // [n_q][words]
   for (int e = threadIdx.x; e < n_q * words; e += blockDim.x) qbits[e] = 0u;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -759,7 +725,8 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
 #pragma unroll
     for (int u = 0; u < kQLd; ++u) {
       const int e = threadIdx.x + u * kThreads, r = e / (kD / 8), c8 = e % (kD / 8);
-      if (e < 16 * (kD / 8)) *reinterpret_cast<uint4*>(smem + kOffQ + r * kQStride + c8 * 16) = qreg[u];
+      if (e < L::kRows * (kD / 8))
+        *reinterpret_cast<uint4*>(smem + L::kOffQ + r * kQStride + c8 * 16) = qreg[u];
     }
   } else {
     // fp32 rows in the (still unused) fp16 tile area, rotated into the cache's
@@ -789,15 +756,15 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
       const float* src = qf + r * kD + (c8 >> 1) * 16 + (c8 & 1) * 2;
       const uint4 v = make_uint4(pack2h(src[0], src[1]), pack2h(src[4], src[5]),
                                  pack2h(src[8], src[9]), pack2h(src[12], src[13]));
-      *reinterpret_cast<uint4*>(smem + kOffQ + r * kQStride + c8 * 16) = v;
+      *reinterpret_cast<uint4*>(smem + L::kOffQ + r * kQStride + c8 * 16) = v;
     }
   }
   // the gate rows this CTA merges (cluster merge), or the merging CTA's rows
   // into L2
-  __nv_bfloat16* gate_s = reinterpret_cast<__nv_bfloat16*>(smem + kOffGate);
+  __nv_bfloat16* gate_s = reinterpret_cast<__nv_bfloat16*>(smem + L::kOffGate);
   if (P.cluster) {
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < kGLd; ++u) {
       const int e = threadIdx.x + u * kThreads;
       if (e < g_rows * g_per_row) {
         const int lr = e / g_per_row, c8 = e - lr * g_per_row;
@@ -969,23 +936,25 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
   } else {
     // ------------------------------------------------------------ consumers
     const int gq = lane >> 2, tq = lane & 3;   // mma fragment row group / column pair
+    const int tile = warp / kWPT;                // this warp's 16 query rows
+    const int kw0 = (warp % kWPT) * kKW;         // and its keys of each chunk
     // Q as A fragments, all 8 k-slices of 16 dims
     uint32_t qa[8][4];
     {
       const int mi = lane >> 3, ri = lane & 7;
-      const int row = (mi & 1) * 8 + ri;
+      const int row = tile * 16 + (mi & 1) * 8 + ri;
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const int col = kk * 16 + (mi >> 1) * 8;
-        ldsm_x4(sbase + kOffQ + row * kQStride + col * 2, qa[kk][0], qa[kk][1], qa[kk][2],
+        ldsm_x4(sbase + L::kOffQ + row * kQStride + col * 2, qa[kk][0], qa[kk][1], qa[kk][2],
                 qa[kk][3]);
       }
     }
-    // the two rows this thread holds: gq and gq + 8
+    // the two rows this thread holds: gq and gq + 8 of the tile
     int qrow[2], qpos[2];
 #pragma unroll
     for (int h2 = 0; h2 < 2; ++h2) {
-      const int r = gq + 8 * h2;
+      const int r = tile * 16 + gq + 8 * h2;
       qrow[h2] = r < R ? r / G : -1;                    // query index, -1 for padding
       qpos[h2] = r < R ? kv - n_q + qrow[h2] : -1;      // last visible position
     }
@@ -1049,16 +1018,21 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
         lim[h2] = (qrow[h2] >= 0 && ((qm >> qrow[h2]) & 1))
                       ? max(0, min(kChunk, qpos[h2] + 1 - key0))
                       : 0;
-      // S = Q K^T for keys [16w, 16w + 16): two n-tiles of 8 keys
-      float sfr[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      // S = Q K^T for the warp's keys [kw0, kw0 + kKW): kNT n-tiles of 8 keys
+      float sfr[kNT][4];
+#pragma unroll
+      for (int nt = 0; nt < kNT; ++nt) sfr[nt][0] = sfr[nt][1] = sfr[nt][2] = sfr[nt][3] = 0.f;
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         uint32_t b0, b1, b2, b3;
         if constexpr (!kFp8) {
-          const int key = warp * 16 + (mi >> 1) * 8 + ri;
-          ldsm_x4(kt + tile_off(key, kk * 16 + (mi & 1) * 8), b0, b1, b2, b3);
-          mma_bf16(sfr[0], qa[kk], b0, b1);
-          mma_bf16(sfr[1], qa[kk], b2, b3);
+#pragma unroll
+          for (int n2 = 0; n2 < kNT / 2; ++n2) {
+            const int key = kw0 + n2 * 16 + (mi >> 1) * 8 + ri;
+            ldsm_x4(kt + tile_off(key, kk * 16 + (mi & 1) * 8), b0, b1, b2, b3);
+            mma_bf16(sfr[2 * n2], qa[kk], b0, b1);
+            mma_bf16(sfr[2 * n2 + 1], qa[kk], b2, b3);
+          }
         } else {
           // B fragment of key row 16w + 8 nt + gq: the four e4m3 codes of dims
           // kk * 16 + 4 tq .. + 3 of the 128-byte-swizzled row (the permuted k
@@ -1088,19 +1062,21 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);   // K and its scales are read, V is widened
       }
-      float x[2][4];
+      float x[kNT][4];
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+      for (int nt = 0; nt < kNT; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int h2 = e >> 1;
-          const int j = warp * 16 + nt * 8 + 2 * tq + (e & 1);
-          x[nt][e] = j < lim[h2] ? sfr[nt][e] * (kFp8 ? sc * ksc[nt][e & 1] : sc) : -INFINITY;
+          const int j = kw0 + nt * 8 + 2 * tq + (e & 1);
+          x[nt][e] = j < lim[h2] ? sfr[nt][e] * (kFp8 ? sc * ksc[nt & 1][e & 1] : sc) : -INFINITY;
         }
       float alpha[2];
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2) {
         float mx = fmaxf(fmaxf(x[0][2 * h2], x[0][2 * h2 + 1]), fmaxf(x[1][2 * h2], x[1][2 * h2 + 1]));
+#pragma unroll
+        for (int nt = 2; nt < kNT; ++nt) mx = fmax3(mx, x[nt][2 * h2], x[nt][2 * h2 + 1]);
         mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
         mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
         const float m_new = fmaxf(m[h2], mx);
@@ -1109,7 +1085,7 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
         m[h2] = m_new;
         float rs = 0.f;
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
+        for (int nt = 0; nt < kNT; ++nt)
 #pragma unroll
           for (int e = 2 * h2; e < 2 * h2 + 2; ++e) {
             x[nt][e] = ex2_approx(x[nt][e] - ref);
@@ -1124,9 +1100,9 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
         o[i][2] *= alpha[1];
         o[i][3] *= alpha[1];
       }
-      if (!kFp8 && lim_all < warp * 16 + 16) {
-        for (int e = lane; e < 16 * 16; e += 32) {   // 16 rows x 2 boxes x 8 chunks of 16 B
-          const int row = warp * 16 + (e >> 4);
+      if (!kFp8 && lim_all < kw0 + kKW) {
+        for (int e = lane; e < kKW * 16; e += 32) {   // kKW rows x 2 boxes x 8 chunks of 16 B
+          const int row = kw0 + (e >> 4);
           const int box = (e >> 3) & 1, ch = e & 7;
           if (row >= lim_all)
             *reinterpret_cast<uint4*>(smem + (vt - sbase) + box * kBoxBytes + row * 128 + ch * 16) =
@@ -1134,39 +1110,45 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
         }
         __syncwarp();
       }
-      // P as the A fragment of a 16x16 (rows x keys) tile
-      uint32_t pa[4];
-      if constexpr (!kFp8) {
-        pa[0] = pack2(x[0][0], x[0][1]);
-        pa[1] = pack2(x[0][2], x[0][3]);
-        pa[2] = pack2(x[1][0], x[1][1]);
-        pa[3] = pack2(x[1][2], x[1][3]);
-      } else {
-        pa[0] = pack2h(x[0][0], x[0][1]);
-        pa[1] = pack2h(x[0][2], x[0][3]);
-        pa[2] = pack2h(x[1][0], x[1][1]);
-        pa[3] = pack2h(x[1][2], x[1][3]);
+      // P as A fragments of 16x16 (rows x keys) tiles, one per 16 keys
+      uint32_t pa[kKS][4];
+#pragma unroll
+      for (int ks = 0; ks < kKS; ++ks) {
+        if constexpr (!kFp8) {
+          pa[ks][0] = pack2(x[2 * ks][0], x[2 * ks][1]);
+          pa[ks][1] = pack2(x[2 * ks][2], x[2 * ks][3]);
+          pa[ks][2] = pack2(x[2 * ks + 1][0], x[2 * ks + 1][1]);
+          pa[ks][3] = pack2(x[2 * ks + 1][2], x[2 * ks + 1][3]);
+        } else {
+          pa[ks][0] = pack2h(x[2 * ks][0], x[2 * ks][1]);
+          pa[ks][1] = pack2h(x[2 * ks][2], x[2 * ks][3]);
+          pa[ks][2] = pack2h(x[2 * ks + 1][0], x[2 * ks + 1][1]);
+          pa[ks][3] = pack2h(x[2 * ks + 1][2], x[2 * ks + 1][3]);
+        }
       }
-      // O += P V over the warp's 16 keys, 16 n-tiles of 8 dims
+      // O += P V over the warp's keys, 16 n-tiles of 8 dims
+#pragma unroll
+      for (int ks = 0; ks < kKS; ++ks)
 #pragma unroll
       for (int dn = 0; dn < 16; dn += 2) {
         uint32_t b0, b1, b2, b3;
         if constexpr (!kFp8) {
-          const int key = warp * 16 + (mi & 1) * 8 + ri;
+          const int key = kw0 + ks * 16 + (mi & 1) * 8 + ri;
           ldsm_x4_t(vt + tile_off(key, dn * 8 + (mi >> 1) * 8), b0, b1, b2, b3);
-          mma_bf16(o[dn], pa, b0, b1);
-          mma_bf16(o[dn + 1], pa, b2, b3);
+          mma_bf16(o[dn], pa[ks], b0, b1);
+          mma_bf16(o[dn + 1], pa[ks], b2, b3);
         } else {
           const int key = (mi & 1) * 8 + ri;
           ldsm_x4_t(vt + tile16_off(key, dn * 8 + (mi >> 1) * 8), b0, b1, b2, b3);
-          mma_f16(o[dn], pa, b0, b1);
-          mma_f16(o[dn + 1], pa, b2, b3);
+          mma_f16(o[dn], pa[ks], b0, b1);
+          mma_f16(o[dn + 1], pa[ks], b2, b3);
         }
       }
       __syncwarp();
       if (!kFp8 && lane == 0) mbar_arrive(&empty[s]);
     }
-    // merge the four warps' states through shared memory (the ring is free)
+    // merge the states of the warps of each row tile through shared memory
+    // (the ring is free): warp w's 16 rows are rows 16 (w / kWPT) + 0 .. 15
 #pragma unroll
     for (int h2 = 0; h2 < 2; ++h2) {
       l[h2] += __shfl_xor_sync(kFull, l[h2], 1);
@@ -1189,48 +1171,54 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
       sm[(warp * 16 + gq + 8) * 2 + 1] = l[1];
     }
     named_bar_sync(1, 32 * kConsumers);
-    // thread t of the 128 consumers: row t / 8, dims [16 (t % 8), + 16)
+    // thread t of the 128 consumers: rows t / 8 + 16 u (u < kRT), dims [16 (t % 8), + 16)
     const int t = threadIdx.x;
-    const int r = t >> 3, d0 = (t & 7) * 16;
+    const int d0 = (t & 7) * 16;
     // a rotated fp8 cache gives O' = H O: the merged rows are rotated back
     // (H is symmetric and orthonormal) before they leave as the partial
     // (cluster merge: every CTA's partial stays in its own shared memory, O in
     // urow and (m, l) in pml, for the cluster's CTAs to read)
-    float* urow = sm + kConsumers * 16 * 2;                    // [16 rows][128]
-    float* pml = urow + 16 * kD;                               // [16 rows][2]
+    float* urow = sm + kConsumers * 16 * 2;                    // [rows][128]
+    float* pml = urow + L::kRows * kD;                         // [rows][2]
     const bool unrotate = kFp8 && P.rotated;
     const bool local = unrotate || P.cluster;
-    if (r < R) {
-      float M = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < kConsumers; ++w) M = fmaxf(M, sm[(w * 16 + r) * 2]);
-      float wsc[kConsumers], L = 0.f;
+    for (int u = 0; u < kRT; ++u) {
+      const int rt = t >> 3, r = rt + 16 * u;   // row of tile u
+      if (r < R) {
+        float M = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < kConsumers; ++w) {
-        const float mw = sm[(w * 16 + r) * 2];
-        wsc[w] = mw == -INFINITY ? 0.f : ex2_approx(mw - M);
-        L += sm[(w * 16 + r) * 2 + 1] * wsc[w];
-      }
-      float* dst = local ? urow + r * kD + d0 : P.part_o + (row0 + r) * kD + d0;
+        for (int ww = 0; ww < kWPT; ++ww) M = fmaxf(M, sm[((u * kWPT + ww) * 16 + rt) * 2]);
+        float wsc[kWPT], Ls = 0.f;
 #pragma unroll
-      for (int d = 0; d < 16; d += 4) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int w = 0; w < kConsumers; ++w) {
-          const float4 v = *reinterpret_cast<const float4*>(so + (w * 16 + r) * kD + d0 + d);
-          acc.x += v.x * wsc[w];
-          acc.y += v.y * wsc[w];
-          acc.z += v.z * wsc[w];
-          acc.w += v.w * wsc[w];
+        for (int ww = 0; ww < kWPT; ++ww) {
+          const float mw = sm[((u * kWPT + ww) * 16 + rt) * 2];
+          wsc[ww] = mw == -INFINITY ? 0.f : ex2_approx(mw - M);
+          Ls += sm[((u * kWPT + ww) * 16 + rt) * 2 + 1] * wsc[ww];
         }
-        *reinterpret_cast<float4*>(dst + d) = acc;
-      }
-      if ((t & 7) == 0) {
-        float* ml = P.cluster ? pml + 2 * r : P.part_ml + 2 * (row0 + r);
-        ml[0] = M;
-        ml[1] = L;
+        float* dst = local ? urow + r * kD + d0 : P.part_o + (row0 + r) * kD + d0;
+#pragma unroll
+        for (int d = 0; d < 16; d += 4) {
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int ww = 0; ww < kWPT; ++ww) {
+            const float4 v =
+                *reinterpret_cast<const float4*>(so + ((u * kWPT + ww) * 16 + rt) * kD + d0 + d);
+            acc.x += v.x * wsc[ww];
+            acc.y += v.y * wsc[ww];
+            acc.z += v.z * wsc[ww];
+            acc.w += v.w * wsc[ww];
+          }
+          *reinterpret_cast<float4*>(dst + d) = acc;
+        }
+        if ((t & 7) == 0) {
+          float* ml = P.cluster ? pml + 2 * r : P.part_ml + 2 * (row0 + r);
+          ml[0] = M;
+          ml[1] = Ls;
+        }
       }
     }
+    const int r = t >> 3;   // (fp8 caches: one row tile)
     if (unrotate) {
       named_bar_sync(1, 32 * kConsumers);
       fwht128_rows(urow, R, t, 32 * kConsumers, [] { named_bar_sync(1, 32 * kConsumers); });
@@ -1249,7 +1237,7 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
     // flight at once), then applies the sigmoid output gate staged at the start.
     cluster_sync_all();
     const int ns = P.nsplit;
-    const uint32_t pml_s = sbase + kOffStages + (uint32_t)(kConsumers * 16 * kD + kConsumers * 16 * 2 + 16 * kD) * 4u;
+    const uint32_t pml_s = sbase + kOffStages + (uint32_t)(kConsumers * 16 * kD + kConsumers * 16 * 2 + L::kRows * kD) * 4u;
     const uint32_t po_s = sbase + kOffStages + (uint32_t)(kConsumers * 16 * kD + kConsumers * 16 * 2) * 4u;
     const int mr = split < R ? (R - split + ns - 1) / ns : 0;
     for (int e = threadIdx.x; e < mr * (kD / 4); e += blockDim.x) {
@@ -1315,7 +1303,7 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
     // per-row max over the splits, then each split's weight, in parallel
     float* wgt = reinterpret_cast<float*>(smem + kOffStages);   // [nsplit][R] (ring is free)
     float* rowM = wgt + P.nsplit * R;                            // [R]
-    float* rowL = rowM + 16;                                     // [R]
+    float* rowL = rowM + L::kRows;                               // [R]
     for (int e = threadIdx.x; e < P.nsplit * R; e += blockDim.x)
       wgt[e] = __ldcg(P.part_ml + 2 * (rowb + e));
     __syncthreads();
@@ -1330,7 +1318,7 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
       wgt[e] = (ms == -INFINITY) ? 0.f : ex2_approx(ms - M);
     }
     __syncthreads();
-    float* lw = rowL + 16;                                        // [nsplit][R]
+    float* lw = rowL + L::kRows;                                  // [nsplit][R]
     for (int e = threadIdx.x; e < P.nsplit * R; e += blockDim.x)
       lw[e] = __ldcg(P.part_ml + 2 * (rowb + e) + 1) * wgt[e];
     __syncthreads();
@@ -1493,11 +1481,16 @@ bool cluster_fits(const void* kern, int size, int smem) {
 }  // namespace
 
 bool attn_decode_fp8_supported(const Geom& g, int n_q) {
-  return attn_decode_mma_supported(g, n_q) && g.Hkv <= kMaxHkvFp8;
+  return attn_decode_mma_supported(g, n_q) && g.Hkv <= kMaxHkvFp8 && n_q * g.G <= 16;
 }
 
+namespace {
+// Row tiles of 16 (query, head) rows the decode kernel holds: n_q * G rows.
+int row_tiles(const Geom& g, int n_q) { return n_q * g.G > 16 ? 2 : 1; }
+}  // namespace
+
 bool attn_decode_mma_supported(const Geom& g, int n_q) {
-  return g.D == kD && g.B % kChunk == 0 && n_q * g.G <= 16 && n_q <= 4;
+  return g.D == kD && g.B % kChunk == 0 && n_q * g.G <= 32 && n_q <= 4;
 }
 
 // Chunks per CTA for the split-KV grid: about two CTAs per SM in one wave, and
@@ -1506,7 +1499,8 @@ bool attn_decode_mma_supported(const Geom& g, int n_q) {
 void decode_mma_split(const Geom& g, int batch, int n_q, int* nsplit, int* per_split) {
   const int max_chunks = n_q * (g.k + 1) * (g.B / kChunk);
   const int pairs = batch * g.Hkv > 0 ? batch * g.Hkv : 1;
-  int ns = (2 * 148) / pairs;
+  // two CTAs per SM with one row tile, one with two (larger shared memory)
+  int ns = ((row_tiles(g, n_q) == 1 ? 2 : 1) * 148) / pairs;
   if (ns < 1) ns = 1;
   if (ns > kMaxClusterSplits) ns = kMaxClusterSplits;
   if (ns > (max_chunks + 7) / 8) ns = (max_chunks + 7) / 8;   // at least 8 chunks per CTA
@@ -1539,14 +1533,23 @@ bool fused_layout(const Geom& g, int n_q, int cap, int nsplit, DecParams* p) {
 }
 
 template <bool kFp8>
-const void* fused_kernel(int di) {
-  return di == 64 ? reinterpret_cast<const void*>(attn_decode_mma_kernel<kFp8, 64>)
-                  : reinterpret_cast<const void*>(attn_decode_mma_kernel<kFp8, 32>);
+const void* fused_kernel(int di, int rt) {
+  if constexpr (kFp8) {
+    return di == 64 ? reinterpret_cast<const void*>(attn_decode_mma_kernel<true, 64, 1>)
+                    : reinterpret_cast<const void*>(attn_decode_mma_kernel<true, 32, 1>);
+  } else {
+    if (rt == 2)
+      return di == 64 ? reinterpret_cast<const void*>(attn_decode_mma_kernel<false, 64, 2>)
+                      : reinterpret_cast<const void*>(attn_decode_mma_kernel<false, 32, 2>);
+    return di == 64 ? reinterpret_cast<const void*>(attn_decode_mma_kernel<false, 64, 1>)
+                    : reinterpret_cast<const void*>(attn_decode_mma_kernel<false, 32, 1>);
+  }
 }
 
 int decode_smem(const Geom& g, int n_q, int cap) {
   const int words = (cap / g.B + 31) / 32;
-  return kOffBits + 4 * n_q * words + 1024;
+  const int bits = row_tiles(g, n_q) == 1 ? DecLayout<1>::kOffBits : DecLayout<2>::kOffBits;
+  return bits + 4 * n_q * words + 1024;
 }
 
 DecParams base_params(const Geom& g, int n_q, int cap, int nsplit, int per_split,
@@ -1627,8 +1630,10 @@ cudaError_t launch_attn_decode_mma(const Geom& g, int batch, int n_q, int cap, i
   p.counter = counter;
   p.ready = ready;
   const int smem = decode_smem(g, n_q, cap);
-  const void* kern = f8.on ? reinterpret_cast<const void*>(attn_decode_mma_kernel<true, 0>)
-                           : reinterpret_cast<const void*>(attn_decode_mma_kernel<false, 0>);
+  const void* kern =
+      f8.on ? reinterpret_cast<const void*>(attn_decode_mma_kernel<true, 0, 1>)
+      : row_tiles(g, n_q) == 2 ? reinterpret_cast<const void*>(attn_decode_mma_kernel<false, 0, 2>)
+                               : reinterpret_cast<const void*>(attn_decode_mma_kernel<false, 0, 1>);
   cudaError_t e = set_max_dynamic_smem(kern, smem);
   if (e != cudaSuccess) return e;
   p.cluster = nsplit > 1 && cluster_fits(kern, nsplit, smem) ? 1 : 0;
@@ -1642,7 +1647,7 @@ bool decode_fused_supported(const Geom& g, int n_q, int cap, int nsplit, bool fp
   if (g.Hi < 1 || g.Hi > 32 || (32 % g.Hi) != 0) return false;
   DecParams p = {};
   if (!fused_layout(g, n_q, cap, nsplit, &p)) return false;
-  const void* kern = fp8 ? fused_kernel<true>(g.di) : fused_kernel<false>(g.di);
+  const void* kern = fp8 ? fused_kernel<true>(g.di, 1) : fused_kernel<false>(g.di, row_tiles(g, n_q));
   const int smem = decode_smem(g, n_q, cap);
   if (set_max_dynamic_smem(kern, smem) != cudaSuccess) {
     cudaGetLastError();
@@ -1668,11 +1673,9 @@ cudaError_t launch_decode_fused(const Geom& g, int batch, int n_q, int cap, int 
   p.pooled = si.pooled;
   p.sel_w = si.sel;
   p.nsel_w = si.nsel;
-  // the fp8 kernel stages its query rows at the end of the fp8 ring, which the
-  // early pooled rows must not reach
-  p.early = !f8.on || p.fo_iq <= kStages * kF8StageBytes;
   const int smem = decode_smem(g, n_q, cap);
-  const void* kern = f8.on ? fused_kernel<true>(g.di) : fused_kernel<false>(g.di);
+  const void* kern =
+      f8.on ? fused_kernel<true>(g.di, 1) : fused_kernel<false>(g.di, row_tiles(g, n_q));
   const cudaError_t e = set_max_dynamic_smem(kern, smem);
   if (e != cudaSuccess) return e;
   return launch_decode_kernel(kern, dim3(nsplit, batch, g.Hkv), smem, nsplit, st, mk, mv, p);

@@ -145,19 +145,6 @@ __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes
                "r"(bytes)
                : "memory");
 }
-// 16-byte asynchronous copy global -> shared (both addresses 16-byte aligned),
-// tracked by the issuing thread's cp.async groups.
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst),
-               "l"(reinterpret_cast<uint64_t>(src))
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.wait_all;" ::: "memory");
-}
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

@@ -161,7 +161,7 @@ qsa_status qsa_select(const qsa_config* cfg, int batch, int total_tokens, int ma
  *   dev_err       optional int32 (device): set to a non-zero code when a
  *                 kv_len entry is out of range; those sequences are skipped.
  * cap must be a multiple of B.
- * Execution: on bf16 geometries with head_dim 128, n_q * G <= 16 and a cache
+ * Execution: on bf16 geometries with head_dim 128, n_q * G <= 32 and a cache
  * whose selection keys fit the kernel's shared memory (about 12000 blocks per
  * sequence), the step is one kernel launch (each (sequence, KV head)
  * thread-block cluster selects, gathers and merges in on-chip memory);
@@ -312,8 +312,8 @@ qsa_status qsa_cp_merge(const qsa_config* cfg, int batch, int n_q, int world,
  * are bit-identical to qsa_decode on the same rows laid out contiguously.
  * A page id outside [0, num_pages) among a sequence's blocks sets *dev_err
  * to 3 (that sequence's outputs are then unspecified, and nothing outside the
- * pools is read). Supported: bf16 with n_q * (Hq / Hkv) <= 16; otherwise
- * QSA_ERR_UNSUPPORTED. */
+ * pools is read). Supported: bf16, head_dim 128, n_q * (Hq / Hkv) <= 32;
+ * otherwise QSA_ERR_UNSUPPORTED. */
 qsa_status qsa_decode_paged(const qsa_config* cfg, int batch, int n_q, int max_blocks,
                             const int32_t* block_table, int num_pages, const int32_t* kv_len,
                             const void* q, const void* k_pages, const void* v_pages,

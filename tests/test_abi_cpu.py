@@ -171,7 +171,8 @@ def test_paged_decode_rejects_bad_arguments():
     assert call(max_blocks=0) == _lib.QSA_ERR_INVALID_ARG
     assert call(num_pages=0) == _lib.QSA_ERR_INVALID_ARG
     assert call(n_q=0) == _lib.QSA_ERR_INVALID_ARG
-    assert call(n_q=3) == _lib.QSA_ERR_UNSUPPORTED                    # 3 * 8 rows > 16
+    assert call(n_q=5) == _lib.QSA_ERR_UNSUPPORTED                    # n_q > 4
+    assert call(n_q=3, c=cfg(num_kv_heads=1)) == _lib.QSA_ERR_UNSUPPORTED   # 3 * 16 rows > 32
     assert call(c=cfg(dtype=_lib.QSA_F32)) == _lib.QSA_ERR_UNSUPPORTED  # tensor-map gather: bf16
     assert call(ws_bytes=ws - 256) == _lib.QSA_ERR_WORKSPACE
     st = lib.qsa_pool_build_paged(ctypes.byref(c), 32, max_blocks, None, 16, FAKE, FAKE, FAKE,

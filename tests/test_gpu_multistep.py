@@ -51,10 +51,11 @@ def _prefill_pooled(cfg, w, d, b_lens, rng):
 
 
 @pytest.mark.parametrize("name,L,steps", [
-    # n_q = 1, B = 64: from 1277 tokens, steps 3 and 67 complete blocks 19 and 20
+    # n_q = 1, B = 64: from 1277 and 700 tokens: blocks 19 and 20, blocks 10 and 11
     ("decode_bf16_b32_kv32768", (1277, 700), 70),
-    # n_q = 2, B = 128: from 2301 tokens, 2 tokens a step, blocks 17, 18 and 19
-    ("mtp_verify_bf16_b4_kv262144", (2301, 1000), 70),
+    # n_q = 2, B = 128: from 2301 and 1020 tokens, 2 tokens a step: blocks 17
+    # and 18, blocks 7 and 8
+    ("mtp_verify_bf16_b4_kv262144", (2301, 1020), 70),
 ])
 def test_prefill_then_decode_steps_keep_the_side_cache(name, L, steps):
     w0 = WORKLOADS[name]

@@ -1,10 +1,11 @@
 """Parity of the kernel variants the workloads above do not reach: the fp32
-decode path (CUDA-core attention + split combine), bf16 decode with more than
-16 query rows per KV head (the same CUDA-core path), bf16 decode with more
-indexer heads than the one-launch decode takes (the selection kernel, then the
-tensor-map attention kernel), head-wise gates on the tensor-core prefill and the
-tensor-map decode, and bf16 prefill with head_dim 64 (CUDA-core prefill). Every
-query is compared with the fp64 oracle.
+decode path (CUDA-core attention + split combine), bf16 decode with 24 and 32
+query rows per KV head (the tensor-map decode with two 16-row tiles, in one
+launch and after the selection kernel; MTP verification of 2 and 3 draft
+tokens at full cache size), the selection kernel followed by the tensor-map
+attention kernel, head-wise gates on the tensor-core prefill and the
+tensor-map decode, and bf16 prefill with head_dim 64 (CUDA-core prefill).
+Every query is compared with the fp64 oracle.
 """
 import numpy as np
 import pytest
@@ -39,12 +40,35 @@ def test_decode_fp32_cuda_core_path():
     assert len(rep["excused_near_ties"]) <= 1, rep
 
 
-def test_decode_bf16_24_rows_per_kv_head():
-    # n_q = 3 new tokens x 8 query heads per KV head = 24 rows: past the
-    # 16-row tensor-map path, served by the CUDA-core decode
-    w, inp = _decode("decode_bf16_b32_kv32768", n_q=3, batch=3, cap=3008,
-                     kv_lens=(3000, 500, 3))
+@pytest.mark.parametrize("n_q", [3, 4])
+def test_decode_bf16_two_row_tiles(n_q):
+    # n_q new tokens x 8 query heads per KV head = 24 or 32 rows: the tensor-map
+    # decode holds two tiles of 16 rows; one launch with the selection inside
+    # the clusters, two when the cache is too large for that
+    w, inp = _decode("decode_bf16_b32_kv32768", n_q=n_q, batch=3, cap=3008,
+                     kv_lens=(3000, 500, n_q))
+    d = TL.upload(inp, w)
+    assert _decode_launches(w, d) == 1
+    rep = decode_parity(w, inp, d=d)
+    assert len(rep["excused_near_ties"]) <= 1, rep
+    big = 12800 * w.block_size
+    for key in ("k_cache", "v_cache", "ik_cache"):
+        t = torch.zeros((t0 := d[key]).shape[0], big, *t0.shape[2:], dtype=t0.dtype, device="cuda")
+        t[:, :3008] = t0
+        d[key] = t
+    assert _decode_launches(w, d) == 2
+    rep = decode_parity(w, inp, d=d)
+    assert len(rep["excused_near_ties"]) <= 1, rep
+
+
+@pytest.mark.parametrize("n_q", [3, 4])
+def test_mtp_verify_more_drafts_full_size(n_q):
+    # MTP verification of n_q - 1 draft tokens on the 4 x 262144-token caches
+    # (the pages measure n = 2 drafts; 24 and 32 rows per KV head)
+    w = WORKLOADS["mtp_verify_bf16_b4_kv262144"].with_(n_q=n_q)
+    inp = make_decode_inputs(w)
     rep = decode_parity(w, inp)
+    print(f"n_q {n_q}: excused near-ties {rep['excused_near_ties']}")
     assert len(rep["excused_near_ties"]) <= 1, rep
 
 
