@@ -7,17 +7,20 @@
 // Should Follow State Correctness"). The nsplit CTAs of one (sequence, KV head)
 // form a thread-block cluster:
 //  1. (kSelDI > 0) the cluster selects: each CTA pools the block this step
-//     completes if it owns it, scores its range of candidate blocks, and after
-//     a cluster barrier gathers a query's score keys from all CTAs through
-//     distributed shared memory and runs a radix top-k (select_in_cluster);
-//     with kSelDI == 0 the selections come from the selection kernel, which
-//     releases a per-sequence flag the CTAs wait on;
+//     completes if it owns it, scores its range of candidate blocks and keeps
+//     each query's top k of the range; after a cluster barrier every CTA
+//     gathers these candidates from all CTAs through distributed shared memory
+//     and takes the top k of them (select_in_cluster); with kSelDI == 0 the
+//     selections come from the selection kernel, which releases a per-sequence
+//     flag the CTAs wait on;
 //  2. the union is cut into 64-key chunks; each CTA takes a contiguous range,
 //     and a producer warp streams each chunk's K and V tiles with TMA through
 //     a 3-stage ring (two CTAs per SM keep about 190 KB in flight per SM);
-//  3. the per-chunk arithmetic is tiny (at most 16 query rows = n_q x group
-//     heads), so the four consumer warps use warp-level MMAs (m16n8k16, fp32
-//     accumulation): warp w takes keys [16w, 16w + 16) of each chunk with its
+//  3. the per-chunk arithmetic is tiny (at most 32 query rows = n_q x group
+//     heads, in one or two tiles of 16), so the four consumer warps use
+//     warp-level MMAs (m16n8k16, fp32 accumulation): with one tile warp w
+//     takes keys [16w, 16w + 16) of each chunk, with two tiles warps 2t, 2t + 1
+//     take tile t's rows over keys [0, 32) and [32, 64); each warp keeps its
 //     own online-softmax state (log2 domain), merged at the end into one
 //     (m, l, O) partial per row;
 //  4. the cluster merges the partials by log-sum-exp through distributed
@@ -111,7 +114,7 @@ struct DecParams {
   int num_pages;                     // paged caches: pages in the pool
   int* sel_w;                        // [batch, n_q, k + 1] selections out
   int* nsel_w;                       // [batch, n_q]
-  int fo_keys, fo_kbar, fo_iq, fo_iw, fo_new, fo_hist;   // byte offsets in the ring's space
+  int fo_cand, fo_gath, fo_kbar, fo_iq, fo_iw, fo_new, fo_hist;   // byte offsets in the ring's space
   // context-parallel shard (attention over given selections only): kv_len are
   // full lengths, the caches hold rows [row_off, row_off + cap), sel holds
   // global block ids; outputs are fp32 gated partials in out_f32
@@ -210,115 +213,6 @@ __device__ __forceinline__ uint32_t tile_off(int row, int dim) {
 }
 
 // ------------------------------------------------- selection in the cluster
-// The k largest of keys[0 .. n) (shared memory), a lower position winning a
-// tie, written as a bitmap: bits[w] for w < ceil(n / 32), bit j % 32 of word
-// j / 32 set for a chosen position j; hi and lo are the largest and smallest
-// key. Radix select over the 32-bit keys: the bits above the highest bit where
-// hi and lo differ are common to all keys; below them, 8-bit digits, most
-// significant first. Each
-// pass histograms the digit of the keys that still match the chosen prefix
-// (shared-memory atomics), warp 0 finds the digit value holding the k-th
-// largest key by a suffix scan, and the passes stop as soon as every key with
-// that digit value is taken. Otherwise the last pass ends on the k-th largest
-// key itself, and of the keys equal to it the lowest positions are taken.
-// hist: 256 ints, ctl: 4 ints of shared memory. All threads call it.
-__device__ __forceinline__ void cta_topk_radix(const uint32_t* keys, int n, int k, uint32_t* bits,
-                                               int* hist, int* ctl, uint32_t hi, uint32_t lo) {
-  const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31, warp = tid >> 5;
-  const int nwarps = nthr >> 5;
-  const int nwords = (n + 31) >> 5;
-  if (n <= k) {
-    for (int w = tid; w < nwords; w += nthr)
-      bits[w] = (w == nwords - 1 && (n & 31)) ? ((1u << (n & 31)) - 1u) : 0xffffffffu;
-    __syncthreads();
-    return;
-  }
-  for (int e = tid; e < 256; e += nthr) hist[e] = 0;
-  __syncthreads();
-  const int top = hi == lo ? -1 : 31 - __clz(hi ^ lo);   // highest differing bit
-  uint32_t pmask = top < 0 ? 0xffffffffu : top == 31 ? 0u : ~((2u << top) - 1u);   // common bits
-  uint32_t prefix = hi & pmask;
-  int krem = k;
-  bool exact = false;
-  for (int shift = top - 7 > 0 ? top - 7 : 0; top >= 0; shift = shift - 8 > 0 ? shift - 8 : 0) {
-    const bool last = shift == 0;
-    if (shift != (top - 7 > 0 ? top - 7 : 0)) {
-      for (int e = tid; e < 256; e += nthr) hist[e] = 0;
-      __syncthreads();
-    }
-    for (int j = tid; j < n; j += nthr) {
-      const uint32_t key = keys[j];
-      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
-    }
-    __syncthreads();
-    if (warp == 0) {
-      // lane l holds byte values 255 - 8l down to 248 - 8l
-      int c[8], sum = 0;
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        c[t] = hist[255 - 8 * lane - t];
-        sum += c[t];
-      }
-      int incl = sum;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(kFull, incl, o);
-        if (lane >= o) incl += v;
-      }
-      const int excl = incl - sum;
-      if (excl < krem && krem <= incl) {
-        int run = excl;
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          if (run + c[t] >= krem) {
-            ctl[0] = 255 - 8 * lane - t;   // the byte value
-            ctl[1] = run;                  // keys above it
-            ctl[2] = c[t];                 // keys with it
-            break;
-          }
-          run += c[t];
-        }
-      }
-    }
-    __syncthreads();
-    const int dv = ctl[0], above = ctl[1], with = ctl[2];
-    krem -= above;
-    prefix |= (uint32_t)dv << shift;
-    pmask |= 0xffu << shift;
-    if (with == krem) {
-      exact = true;
-      break;
-    }
-    if (last) break;
-  }
-  // exact: the keys whose prefix bits are >= prefix (k of them); else the keys
-  // above the k-th largest, then its ties below
-  for (int w = warp; w < nwords; w += nwarps) {
-    const int j = w * 32 + lane;
-    bool take = false;
-    if (j < n) {
-      const uint32_t key = keys[j];
-      take = exact ? (key & pmask) >= prefix : key > prefix;
-    }
-    const uint32_t m = __ballot_sync(kFull, take);
-    if (lane == 0) bits[w] = m;
-  }
-  if (!exact) {
-    __syncthreads();
-    if (warp == 0) {
-      int left = krem;
-      for (int w = 0; w < nwords && left > 0; ++w) {
-        const int j = w * 32 + lane;
-        uint32_t m = __ballot_sync(kFull, j < n && keys[j] == prefix);
-        while (__popc(m) > left) m &= ~(1u << (31 - __clz(m)));   // keep the lowest `left`
-        if (lane == 0) bits[w] |= m;
-        left -= __popc(m);
-      }
-    }
-  }
-  __syncthreads();
-}
-
 __device__ __forceinline__ void cluster_arrive_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
 }
@@ -332,8 +226,108 @@ __device__ __forceinline__ uint4 ld_cluster_u32x4(uint32_t addr) {
   return v;
 }
 
-// Chunk of candidate blocks one CTA of the cluster scores: a multiple of 4, so
-// that the gather below moves 16-byte groups owned by one CTA.
+__device__ __forceinline__ unsigned lane_mask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// One warp, keys[0 .. n) in shared memory: the threshold of the kk largest
+// keys, a lower index winning among equal keys. Afterwards the chosen keys are
+// those > tau plus the first `need` keys == tau in index order. tau is found
+// by deciding its bits from the highest bit where the largest and the
+// smallest key differ, each step counting the keys at or above the candidate
+// over the warp; it stops early once exactly kk keys are at or above it.
+__device__ __forceinline__ void warp_threshold(const uint32_t* keys, int n, int kk, uint32_t& tau,
+                                               int& need) {
+  const int lane = threadIdx.x & 31;
+  if (kk <= 0) {
+    tau = 0xffffffffu;   // above every score key: nothing is taken
+    need = 0;
+    return;
+  }
+  if (n <= kk) {
+    tau = 0u;            // score keys are never 0: every key is taken
+    need = 0;
+    return;
+  }
+  uint32_t hi = 0u, lo = 0xffffffffu;
+  for (int j = lane; j < n; j += 32) {
+    const uint32_t x = keys[j];
+    hi = max(hi, x);
+    lo = min(lo, x);
+  }
+  hi = __reduce_max_sync(kFull, hi);
+  lo = __reduce_min_sync(kFull, lo);
+  tau = hi;
+  if (hi != lo) {
+    const int top = 31 - __clz(hi ^ lo);
+    tau = top == 31 ? 0u : (hi & ~((2u << top) - 1u));
+    for (int bit = top; bit >= 0; --bit) {
+      const uint32_t cand = tau | (1u << bit);
+      int c = 0;
+      for (int j = lane; j < n; j += 32) c += keys[j] >= cand ? 1 : 0;
+      c = __reduce_add_sync(kFull, c);
+      if (c >= kk) tau = cand;
+      if (c == kk) break;
+    }
+  }
+  int gt = 0;
+  for (int j = lane; j < n; j += 32) gt += keys[j] > tau ? 1 : 0;
+  need = kk - __reduce_add_sync(kFull, gt);
+}
+
+// One warp: the kk largest of keys[0 .. n) (warp_threshold's rule), written in
+// index order to out_key / out_pos (pos0 + index); slots kk .. kpad - 1 get a
+// sentinel (key 0, below every score key).
+__device__ __forceinline__ void warp_topk_compact(const uint32_t* keys, int n, int kk, int pos0,
+                                                  uint32_t* out_key, int* out_pos, int kpad) {
+  const int lane = threadIdx.x & 31;
+  uint32_t tau;
+  int need;
+  warp_threshold(keys, n, kk, tau, need);
+  int base = 0;
+  for (int j0 = 0; j0 < n && base < kk; j0 += 32) {   // uniform
+    const int j = j0 + lane;
+    const uint32_t x = j < n ? keys[j] : 0u;
+    const bool eq = j < n && x == tau;
+    const unsigned eb = __ballot_sync(kFull, eq);
+    const bool t = (j < n && x > tau) || (eq && __popc(eb & lane_mask_lt()) < need);
+    need -= __popc(eb);
+    const unsigned tb = __ballot_sync(kFull, t);
+    if (t) {
+      const int sl = base + __popc(tb & lane_mask_lt());
+      out_key[sl] = x;
+      out_pos[sl] = pos0 + j;
+    }
+    base += __popc(tb);
+  }
+  for (int sl = kk + lane; sl < kpad; sl += 32) {
+    out_key[sl] = 0u;
+    out_pos[sl] = 0x7fffffff;
+  }
+}
+
+// One warp: the kk largest of keys[0 .. n) (warp_threshold's rule); sets bit
+// pos[j] % 32 of word pos[j] / 32 of bits for every chosen j.
+__device__ __forceinline__ void warp_topk_bits(const uint32_t* keys, const int* pos, int n, int kk,
+                                               uint32_t* bits) {
+  const int lane = threadIdx.x & 31;
+  uint32_t tau;
+  int need;
+  warp_threshold(keys, n, kk, tau, need);
+  for (int j0 = 0; j0 < n; j0 += 32) {
+    const int j = j0 + lane;
+    const uint32_t x = j < n ? keys[j] : 0u;
+    const bool eq = j < n && x == tau;
+    const unsigned eb = __ballot_sync(kFull, eq);
+    const bool t = (j < n && x > tau) || (eq && __popc(eb & lane_mask_lt()) < need);
+    need -= __popc(eb);
+    if (t) atomicOr(&bits[pos[j] >> 5], 1u << (pos[j] & 31));
+  }
+}
+
+// Chunk of candidate blocks one CTA of the cluster scores: a multiple of 4.
 __host__ __device__ __forceinline__ int select_range(int nc_last, int nsplit) {
   const int per = ((nc_last > 1 ? nc_last : 1) + nsplit - 1) / nsplit;
   return (per + 3) & ~3;
@@ -347,14 +341,16 @@ __host__ __device__ __forceinline__ int select_range(int nc_last, int nsplit) {
 // pooled-key cache once, from the KV head 0 cluster), scores its blocks for
 // every query, s = c * sum_h w_h relu(q_h . kbar) (one thread per (query,
 // block, head), the heads summed by shuffles; the same arithmetic as the
-// selection kernel), and keeps the score keys in its shared memory. After a
-// cluster barrier every CTA gathers each query's keys from all CTAs, selects
-// the top k (cta_topk_radix) into the query's bitmap and adds the tail block;
-// CTA (0, b, 0) also writes the selection lists. Ends with this CTA's arrival
-// on the cluster barrier that the caller waits on before reusing the space.
-// Starts moving what select_in_cluster reads into L2 (bulk prefetches by one
-// thread): the CTA's range of pooled rows, the indexer rows of the blocks this
-// step completes, and the queries' indexer q.
+// selection kernel), and keeps the score keys in its shared memory; warp i
+// takes query i's top k of the range as candidates. After a cluster barrier
+// every CTA gathers all CTAs' candidates, selects each query's top k of them
+// into the query's bitmap (warp_topk_bits) and adds the tail block; CTA
+// (0, b, 0) also writes the selection lists. Ends with this CTA's arrival on
+// the cluster barrier that the caller waits on before reusing the space.
+//
+// select_prefetch starts moving what select_in_cluster reads into L2 (bulk
+// prefetches by one thread): the CTA's range of pooled rows, the indexer rows
+// of the blocks this step completes, and the queries' indexer q.
 template <int kDI>
 __device__ __forceinline__ void select_prefetch(const DecParams& P, int kv, int split, int b) {
   const Geom& g = P.g;
@@ -391,15 +387,18 @@ __device__ __forceinline__ void select_in_cluster(const DecParams& P, uint8_t* s
   const int per = select_range(nc_last, P.nsplit);
   const int j0 = split * per, j1 = min(nc_last, j0 + per);
   uint8_t* ring = smem + kOffStages;
-  uint32_t* mm_mine = reinterpret_cast<uint32_t*>(ring);                    // [4][2] largest, smallest key
   uint32_t* keys_mine = reinterpret_cast<uint32_t*>(ring + 32);             // [n_q][per]
-  uint32_t* keys_all = reinterpret_cast<uint32_t*>(ring + P.fo_keys);       // [nblk_cap]
+  const int kpad = (k + 3) & ~3;                                            // candidate slots per query
+  uint32_t* cand_key = reinterpret_cast<uint32_t*>(ring + P.fo_cand);       // [n_q][kpad]
+  int* cand_pos = reinterpret_cast<int*>(cand_key + n_q * kpad);            // [n_q][kpad]
+  const int ng = P.nsplit * kpad;                                           // gathered per query
+  uint32_t* gkey = reinterpret_cast<uint32_t*>(ring + P.fo_gath);           // [n_q][ng]
+  int* gpos = reinterpret_cast<int*>(gkey + n_q * ng);                      // [n_q][ng]
   float* kbar_s = reinterpret_cast<float*>(ring + P.fo_kbar);               // [kRows][kStride]
   float* iq_s = reinterpret_cast<float*>(ring + P.fo_iq);                   // [n_q][Hi][kDI]
   float* iw_s = reinterpret_cast<float*>(ring + P.fo_iw);                   // [n_q][Hi]
   float* new_s = reinterpret_cast<float*>(ring + P.fo_new);                 // [2][kDI]
-  int* hist = reinterpret_cast<int*>(ring + P.fo_hist);                     // [256] + ctl [16]
-  uint32_t* gmm = reinterpret_cast<uint32_t*>(hist + 272);                   // [4][2]
+  int* hist = reinterpret_cast<int*>(ring + P.fo_hist);
   float2(*part)[32] = reinterpret_cast<float2(*)[32]>(hist + 280);           // [8][32]
 
   // paged caches: every page the step may gather must be in the pool
@@ -409,10 +408,6 @@ __device__ __forceinline__ void select_in_cluster(const DecParams& P, uint8_t* s
       const int page = P.table[(size_t)b * nblk_cap + j];
       if ((page < 0 || page >= P.num_pages) && P.err) atomicExch(P.err, 3);
     }
-  }
-  if (tid < 4) {
-    mm_mine[2 * tid] = 0u;
-    mm_mine[2 * tid + 1] = 0xffffffffu;
   }
   __syncthreads();   // the caller staged iq_s and iw_s
   // blocks completed by this step's tokens (at most two: n_q <= 4 < B)
@@ -435,9 +430,7 @@ __device__ __forceinline__ void select_in_cluster(const DecParams& P, uint8_t* s
     if (hk == 0 && ok)
       for (int d = tid; d < kDI; d += nthr) P.pooled[((size_t)b * nblk_cap + j) * kDI + d] = dst[d];
   }
-  // score the range, kRows blocks at a time (with each query's largest and
-  // smallest key)
-  uint32_t qhi[4] = {0u, 0u, 0u, 0u}, qlo[4] = {~0u, ~0u, ~0u, ~0u};
+  // score the range, kRows blocks at a time
   for (int r0 = j0; r0 < j1; r0 += kRows) {
     const int rows = min(kRows, j1 - r0);
     {   // every load of the pass is issued before the first store
@@ -499,117 +492,80 @@ __device__ __forceinline__ void select_in_cluster(const DecParams& P, uint8_t* s
         for (int m = 0; m < 4; ++m) {
           float t = live[m] ? wq * fmaxf(dt[m], 0.f) : 0.f;
           for (int o = 1; o < Hi; o <<= 1) t += __shfl_xor_sync(kFull, t, o);
-          if (h == 0 && live[m]) {
-            const uint32_t y = score_key(t * g.idx_scale);
-            keys_mine[i * per + (r0 + rr[m] - j0)] = y;
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              if (q == i) {
-                qhi[q] = max(qhi[q], y);
-                qlo[q] = min(qlo[q], y);
-              }
-          }
+          if (h == 0 && live[m]) keys_mine[i * per + (r0 + rr[m] - j0)] = score_key(t * g.idx_scale);
         }
       }
     }
     __syncthreads();
   }
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    if (q < n_q) {
-      const uint32_t hw = __reduce_max_sync(kFull, qhi[q]), lw = __reduce_min_sync(kFull, qlo[q]);
-      if (lane == 0 && hw >= lw) {
-        atomicMax(&mm_mine[2 * q], hw);
-        atomicMin(&mm_mine[2 * q + 1], lw);
-      }
+  // Top-k in two steps. Each CTA first takes the top k of its own range for
+  // every query (warp i, query i): every block of the cluster's top k is among
+  // them, since fewer than k blocks of the whole cache beat it, so fewer than k
+  // of its range. After a cluster barrier each CTA gathers all CTAs'
+  // candidates (CTA order is ascending block order, so a lower position still
+  // wins a tie) and takes the top k of those for every query itself: no bitmap
+  // has to cross the cluster afterwards.
+  if (warp < n_q) {
+    const int i = warp;
+    const int cnt = max(0, min(j1, (kv - n_q + 1 + i) / g.B) - j0);   // query i's blocks here
+    warp_topk_compact(keys_mine + i * per, cnt, min(k, cnt), j0, cand_key + i * kpad,
+                      cand_pos + i * kpad, kpad);
+  }
+  cluster_sync_all();   // every CTA's candidates are in place
+  {   // 16-byte groups of four candidates (keys, then positions) from every CTA
+    const int groups = n_q * P.nsplit * (kpad / 4);
+    const uint32_t ck_s = smem_u32(cand_key), cp_s = smem_u32(cand_pos);
+    for (int e = tid; e < groups; e += nthr) {
+      const int i = e / (P.nsplit * (kpad / 4)), rem = e - i * (P.nsplit * (kpad / 4));
+      const int c = rem / (kpad / 4), q4 = rem - c * (kpad / 4);
+      const uint32_t off = 4u * (uint32_t)(i * kpad + 4 * q4);
+      const uint4 kv4 = ld_cluster_u32x4(cluster_map(ck_s + off, c));
+      const uint4 pv4 = ld_cluster_u32x4(cluster_map(cp_s + off, c));
+      *reinterpret_cast<uint4*>(gkey + i * ng + c * kpad + 4 * q4) = kv4;
+      *reinterpret_cast<uint4*>(gpos + i * ng + c * kpad + 4 * q4) = pv4;
     }
   }
-  cluster_sync_all();   // every CTA's keys (and their extremes) are in place
-  const uint32_t mine_s = smem_u32(keys_mine), mm_s = smem_u32(mm_mine);
-  // With several queries, CTA s selects queries s, s + nsplit, ... and the
-  // others read the bitmaps afterwards; one query is selected by every CTA.
-  const bool spread = n_q > 1;
-  if (warp == 0) {   // the queries' largest and smallest keys over the cluster
-    for (int i = 0; i < n_q; ++i) {
-      uint2 m = make_uint2(0u, 0xffffffffu);
-      if (lane < P.nsplit) {
-        const uint32_t a = cluster_map(mm_s + 8u * i, lane);
-        m.x = (uint32_t)__float_as_uint(ld_cluster_f32(a));
-        m.y = (uint32_t)__float_as_uint(ld_cluster_f32(a + 4));
-      }
-      const uint32_t hw = __reduce_max_sync(kFull, m.x), lw = __reduce_min_sync(kFull, m.y);
-      if (lane == 0) {
-        gmm[2 * i] = hw;
-        gmm[2 * i + 1] = lw;
-      }
-    }
-  }
-  for (int i = 0; i < n_q; ++i) {
-    if (spread && i % P.nsplit != split) continue;   // uniform across the CTA
+  __syncthreads();
+  if (warp < n_q) {
+    const int i = warp;
     const int n = kv - n_q + 1 + i;
     const int nc_i = n / g.B;
-    // gather: 16-byte groups of four positions, each owned by one CTA; four
-    // groups per thread in flight
-    for (int jb = 4 * tid; jb < nc_i; jb += 16 * nthr) {
-      uint4 v[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int j = jb + 4 * u * nthr;
-        if (j < nc_i) {
-          const int c = j / per;
-          v[u] = ld_cluster_u32x4(cluster_map(mine_s + 4u * (uint32_t)(i * per + j - c * per), c));
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int j = jb + 4 * u * nthr;
-        if (j < nc_i) *reinterpret_cast<uint4*>(keys_all + j) = v[u];
-      }
-    }
-    __syncthreads();
     uint32_t* qb = qbits + i * words;
-    cta_topk_radix(keys_all, nc_i, k, qb, hist, hist + 256, gmm[2 * i], gmm[2 * i + 1]);
-    const int tail = n - nc_i * g.B;
-    if (tid == 0 && tail > 0) qb[nc_i >> 5] |= 1u << (nc_i & 31);
-    __syncthreads();
-    if ((spread || split == 0) && hk == 0 && warp == 0) {   // the selection list: ascending, tail last
-      int* srow = P.sel_w + ((size_t)b * n_q + i) * kp1;
-      const int nw = min(words, (nc_i + 1 + 31) >> 5);
-      int base = 0;
-      for (int w0 = 0; w0 < nw; w0 += 32) {
-        const int w = w0 + lane;
-        uint32_t m = w < nw ? qb[w] : 0u;
-        const int c = __popc(m);
-        int incl = c;
+    warp_topk_bits(gkey + i * ng, gpos + i * ng, ng, min(k, nc_i), qb);
+    __syncwarp();
+    if (lane == 0 && n - nc_i * g.B > 0) atomicOr(&qb[nc_i >> 5], 1u << (nc_i & 31));   // tail
+  }
+  __syncthreads();
+  if (split == 0 && hk == 0 && warp < n_q) {   // the selection lists: ascending, tail last
+    const int i = warp;
+    const int nc_i = (kv - n_q + 1 + i) / g.B;
+    const uint32_t* qb = qbits + i * words;
+    int* srow = P.sel_w + ((size_t)b * n_q + i) * kp1;
+    const int nw = min(words, (nc_i + 1 + 31) >> 5);
+    int base = 0;
+    for (int w0 = 0; w0 < nw; w0 += 32) {
+      const int w = w0 + lane;
+      uint32_t m = w < nw ? qb[w] : 0u;
+      const int c = __popc(m);
+      int incl = c;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int v = __shfl_up_sync(kFull, incl, o);
-          if (lane >= o) incl += v;
-        }
-        int off = base + incl - c;
-        while (m) {
-          const int bp = __ffs(m) - 1;
-          m &= m - 1;
-          if (off < kp1) srow[off] = w * 32 + bp;
-          ++off;
-        }
-        base += __shfl_sync(kFull, incl, 31);
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += v;
       }
-      for (int e = base + lane; e < kp1; e += 32) srow[e] = -1;
-      if (lane == 0) P.nsel_w[(size_t)b * n_q + i] = min(base, kp1);
+      int off = base + incl - c;
+      while (m) {
+        const int bp = __ffs(m) - 1;
+        m &= m - 1;
+        if (off < kp1) srow[off] = w * 32 + bp;
+        ++off;
+      }
+      base += __shfl_sync(kFull, incl, 31);
     }
+    for (int e = base + lane; e < kp1; e += 32) srow[e] = -1;
+    if (lane == 0) P.nsel_w[(size_t)b * n_q + i] = min(base, kp1);
   }
-  if (spread) {   // the other queries' bitmaps, from the CTAs that selected them
-    cluster_sync_all();
-    const uint32_t qbits_s = smem_u32(qbits);
-    for (int e = tid; e < n_q * words; e += nthr) {
-      const int i = e / words;
-      if (i % P.nsplit != split)
-        qbits[e] = (uint32_t)__float_as_uint(ld_cluster_f32(cluster_map(qbits_s + 4u * e, i % P.nsplit)));
-    }
-    __syncthreads();
-  }
-  cluster_arrive_all();   // this CTA has read the other CTAs' keys
+  cluster_arrive_all();   // this CTA has read the other CTAs' candidates
 }
 
 template <bool kFp8, int kSelDI, int kRT>
@@ -1516,9 +1472,12 @@ bool fused_layout(const Geom& g, int n_q, int cap, int nsplit, DecParams* p) {
   auto a16 = [](long long x) { return (x + 15) & ~15LL; };
   const int nblk_cap = cap / g.B;
   const long long per = select_range(nblk_cap, nsplit);
-  long long off = a16(32 + 4LL * n_q * per);   // extremes, then this CTA's keys
-  p->fo_keys = (int)off;
-  off += a16(4LL * (nblk_cap + 4));
+  const long long kpad = (g.k + 3) & ~3;
+  long long off = a16(32 + 4LL * n_q * per);   // this CTA's keys
+  p->fo_cand = (int)off;
+  off += a16(8LL * n_q * kpad);                 // its candidates
+  p->fo_gath = (int)off;
+  off += a16(8LL * n_q * nsplit * kpad);        // every CTA's candidates
   p->fo_kbar = (int)off;
   off += a16(4LL * kSelRows * (g.di + 4));
   p->fo_iq = (int)off;

@@ -299,8 +299,9 @@ qsa_status qsa_cp_merge(const qsa_config* cfg, int batch, int n_q, int world,
                         void* stream);
 
 /* --------------------------------------------------------- paged decode --
- * qsa_decode over a paged KV cache (a speed lever the llama.cpp PR #27739
- * page lists: "continuous batching and paged KV"; the QSA block is the page).
+ * qsa_decode over a paged KV cache (the llama.cpp PR #27739 page names paged
+ * KV storage, next to continuous batching, among its speed levers; the QSA
+ * block is the page).
  * A page holds the B consecutive rows of one block of one sequence:
  *   k_pages/v_pages [num_pages, B, Hkv, D]   ik_pages [num_pages, B, di]
  *   block_table     [batch, max_blocks] int32 (device): block j of sequence b
