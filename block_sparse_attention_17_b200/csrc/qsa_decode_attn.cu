@@ -237,7 +237,10 @@ __device__ __forceinline__ unsigned lane_mask_lt() {
 // those > tau plus the first `need` keys == tau in index order. tau is found
 // by deciding its bits from the highest bit where the largest and the
 // smallest key differ, each step counting the keys at or above the candidate
-// over the warp; it stops early once exactly kk keys are at or above it.
+// over the warp; it stops early once exactly kk keys are at or above it. Up to
+// 32 * kR keys are held in registers for the search (longer lists are re-read
+// from shared memory at every step).
+template <int kR>
 __device__ __forceinline__ void warp_threshold(const uint32_t* keys, int n, int kk, uint32_t& tau,
                                                int& need) {
   const int lane = threadIdx.x & 31;
@@ -251,12 +254,24 @@ __device__ __forceinline__ void warp_threshold(const uint32_t* keys, int n, int 
     need = 0;
     return;
   }
+  const bool regs = n <= 32 * kR;   // uniform
+  uint32_t kr[kR];
   uint32_t hi = 0u, lo = 0xffffffffu;
-  for (int j = lane; j < n; j += 32) {
-    const uint32_t x = keys[j];
-    hi = max(hi, x);
-    lo = min(lo, x);
+#pragma unroll
+  for (int u = 0; u < kR; ++u) {
+    const int j = lane + 32 * u;
+    kr[u] = (regs && j < n) ? keys[j] : 0u;
+    if (regs && j < n) {
+      hi = max(hi, kr[u]);
+      lo = min(lo, kr[u]);
+    }
   }
+  if (!regs)
+    for (int j = lane; j < n; j += 32) {
+      const uint32_t x = keys[j];
+      hi = max(hi, x);
+      lo = min(lo, x);
+    }
   hi = __reduce_max_sync(kFull, hi);
   lo = __reduce_min_sync(kFull, lo);
   tau = hi;
@@ -266,14 +281,24 @@ __device__ __forceinline__ void warp_threshold(const uint32_t* keys, int n, int 
     for (int bit = top; bit >= 0; --bit) {
       const uint32_t cand = tau | (1u << bit);
       int c = 0;
-      for (int j = lane; j < n; j += 32) c += keys[j] >= cand ? 1 : 0;
+      if (regs) {
+#pragma unroll
+        for (int u = 0; u < kR; ++u) c += kr[u] >= cand ? 1 : 0;   // padding keys are 0
+      } else {
+        for (int j = lane; j < n; j += 32) c += keys[j] >= cand ? 1 : 0;
+      }
       c = __reduce_add_sync(kFull, c);
       if (c >= kk) tau = cand;
       if (c == kk) break;
     }
   }
   int gt = 0;
-  for (int j = lane; j < n; j += 32) gt += keys[j] > tau ? 1 : 0;
+  if (regs) {
+#pragma unroll
+    for (int u = 0; u < kR; ++u) gt += kr[u] > tau ? 1 : 0;
+  } else {
+    for (int j = lane; j < n; j += 32) gt += keys[j] > tau ? 1 : 0;
+  }
   need = kk - __reduce_add_sync(kFull, gt);
 }
 
@@ -285,7 +310,7 @@ __device__ __forceinline__ void warp_topk_compact(const uint32_t* keys, int n, i
   const int lane = threadIdx.x & 31;
   uint32_t tau;
   int need;
-  warp_threshold(keys, n, kk, tau, need);
+  warp_threshold<8>(keys, n, kk, tau, need);
   int base = 0;
   for (int j0 = 0; j0 < n && base < kk; j0 += 32) {   // uniform
     const int j = j0 + lane;
@@ -315,7 +340,7 @@ __device__ __forceinline__ void warp_topk_bits(const uint32_t* keys, const int* 
   const int lane = threadIdx.x & 31;
   uint32_t tau;
   int need;
-  warp_threshold(keys, n, kk, tau, need);
+  warp_threshold<16>(keys, n, kk, tau, need);
   for (int j0 = 0; j0 < n; j0 += 32) {
     const int j = j0 + lane;
     const uint32_t x = j < n ? keys[j] : 0u;

@@ -40,24 +40,33 @@ def test_decode_fp32_cuda_core_path():
     assert len(rep["excused_near_ties"]) <= 1, rep
 
 
+def _two_kernel_parity(w, inp, d):
+    """The selection kernel (qsa_select_decode) followed by the attention
+    kernel over its lists (qsa_decode_attend): the kernels qsa_decode runs
+    when the in-cluster selection does not apply. Compared with the oracle."""
+    cfg = qsa.QSAConfig.from_workload(w)
+    kv = d["kv_len"]
+    pooled = qsa.pool_build(cfg, d["ik_cache"], (kv - w.n_q).to(torch.int32))
+    s = qsa.select_decode(cfg, d["iq"], d["ik_cache"], d["iw"], pooled, kv)
+    a = qsa.decode_attend(cfg, d["q"], d["k_cache"], d["v_cache"], d["gate"], kv, s["sel"],
+                          s["nsel"], want_lse=True)
+    torch.cuda.synchronize()
+    gpu = {"out": a["out"], "lse": a["lse"], "sel": s["sel"], "nsel": s["nsel"]}
+    return TL.check_queries(O.qsa_decode(w, inp)["queries"], gpu, lambda bi: bi, w)
+
+
 @pytest.mark.parametrize("n_q", [3, 4])
 def test_decode_bf16_two_row_tiles(n_q):
     # n_q new tokens x 8 query heads per KV head = 24 or 32 rows: the tensor-map
-    # decode holds two tiles of 16 rows; one launch with the selection inside
-    # the clusters, two when the cache is too large for that
+    # decode holds two tiles of 16 rows, in one launch (selection inside the
+    # clusters) and as the attention kernel after the selection kernel
     w, inp = _decode("decode_bf16_b32_kv32768", n_q=n_q, batch=3, cap=3008,
                      kv_lens=(3000, 500, n_q))
     d = TL.upload(inp, w)
     assert _decode_launches(w, d) == 1
     rep = decode_parity(w, inp, d=d)
     assert len(rep["excused_near_ties"]) <= 1, rep
-    big = 12800 * w.block_size
-    for key in ("k_cache", "v_cache", "ik_cache"):
-        t = torch.zeros((t0 := d[key]).shape[0], big, *t0.shape[2:], dtype=t0.dtype, device="cuda")
-        t[:, :3008] = t0
-        d[key] = t
-    assert _decode_launches(w, d) == 2
-    rep = decode_parity(w, inp, d=d)
+    rep = _two_kernel_parity(w, inp, d)
     assert len(rep["excused_near_ties"]) <= 1, rep
 
 
@@ -116,11 +125,11 @@ def _decode_launches(w, d):
     ("decode_bf16_b32_kv32768", (4100, 2048, 70), 4160),
     ("mtp_verify_bf16_b4_kv262144", (9000, 129, 2), 9088),
 ])
-def test_decode_one_launch_and_two_launch_paths(name, kv_lens, cap):
-    # A cache of a few thousand blocks: one launch (selection inside the decode
-    # kernel's clusters). The same rows at the start of a 12800-block cache: the
-    # selection's keys no longer fit the kernel's shared memory, so the selection
-    # kernel and then the attention kernel run. Both match the oracle.
+def test_decode_one_launch_and_two_kernel_paths(name, kv_lens, cap):
+    # A cache of a few thousand blocks, and the same rows at the start of a
+    # 12800-block cache: one launch each (the selection inside the decode
+    # kernel's clusters keeps only candidates, so it fits either cache). The
+    # selection kernel + attention kernel pair matches the oracle as well.
     w, inp = _decode(name, batch=len(kv_lens), cap=cap, kv_lens=kv_lens)
     d = TL.upload(inp, w)
     assert _decode_launches(w, d) == 1
@@ -129,6 +138,8 @@ def test_decode_one_launch_and_two_launch_paths(name, kv_lens, cap):
         t = torch.zeros((t0 := d[key]).shape[0], big, *t0.shape[2:], dtype=t0.dtype, device="cuda")
         t[:, :cap] = t0
         d[key] = t
-    assert _decode_launches(w, d) == 2
+    assert _decode_launches(w, d) == 1
     rep = decode_parity(w, inp, d=d)
+    assert len(rep["excused_near_ties"]) <= 1, rep
+    rep = _two_kernel_parity(w, inp, d)
     assert len(rep["excused_near_ties"]) <= 1, rep
