@@ -17,7 +17,7 @@ from block_sparse_attention_17_b200.workloads import (WORKLOADS, make_decode_inp
                                                       make_prefill_inputs)
 from oracle import qsa_oracle as O
 from tests import qsa_testlib as TL
-from tests.test_gpu_parity import decode_parity, prefill_parity
+from tests.test_gpu_parity import decode_parity, prefill_parity, run_decode
 
 pytestmark = pytest.mark.gpu
 
@@ -143,3 +143,29 @@ def test_decode_one_launch_and_two_kernel_paths(name, kv_lens, cap):
     assert len(rep["excused_near_ties"]) <= 1, rep
     rep = _two_kernel_parity(w, inp, d)
     assert len(rep["excused_near_ties"]) <= 1, rep
+
+
+@pytest.mark.parametrize("name", ["decode_bf16_b32_kv32768", "mtp_verify_bf16_b4_kv262144"])
+def test_decode_topk_concentrated_in_one_range(name):
+    # The one-launch decode's clusters first compare only the leading candidates
+    # of each CTA's range of blocks (about twice a range's share of the top k);
+    # when one range holds more of the top k than that, the query is selected
+    # again over every candidate. The indexer keys of the first 48 blocks are
+    # scaled by 8 (exact in bf16), so most of the top k lies in the first range.
+    B = WORKLOADS[name].block_size
+    kv = 800 * B + 3
+    w, inp = _decode(name, batch=2, cap=801 * B, kv_lens=(kv, kv - 70))
+    ik = inp["ik_cache"].copy()
+    ik[:, :48 * B] *= 8.0
+    inp["ik_cache"] = ik
+    d = TL.upload(inp, w)
+    assert _decode_launches(w, d) == 1
+    gpu = run_decode(w, inp, d)
+    assert gpu["err"] == 0
+    rep = TL.check_queries(O.qsa_decode(w, inp)["queries"], gpu, lambda bi: bi, w)
+    assert len(rep["excused_near_ties"]) <= 1, rep
+    sel = gpu["sel"].cpu().numpy()
+    k = w.topk
+    for b in range(w.batch):
+        for i in range(w.n_q):
+            assert (sel[b, i, :k] < 48).sum() >= 24, sel[b, i]
