@@ -28,7 +28,6 @@
 //     gate; where such a cluster cannot be resident (two-launch path only), the
 //     partials go through global memory and the last CTA merges them.
 // kFp8 reads e4m3 K/V codes with per-row scales instead of bf16 rows.
-#include <algorithm>
 #include <map>
 #include <mutex>
 #include <tuple>
@@ -116,7 +115,6 @@ struct DecParams {
   int* sel_w;                        // [batch, n_q, k + 1] selections out
   int* nsel_w;                       // [batch, n_q]
   int fo_cand, fo_gath, fo_kbar, fo_iq, fo_iw, fo_new, fo_hist;   // byte offsets in the ring's space
-  int cand_m;                        // candidates per CTA and query the top-k first looks at
   // context-parallel shard (attention over given selections only): kv_len are
   // full lengths, the caches hold rows [row_off, row_off + cap), sel holds
   // global block ids; outputs are fp32 gated partials in out_f32
@@ -234,35 +232,124 @@ __device__ __forceinline__ unsigned lane_mask_lt() {
   return m;
 }
 
-// How many of the keys[0 .. n4) (shared memory, n4 a multiple of 4; block
-// positions pos0 + index) come before (key, pos) in the selection's total
-// order: a larger score key, or the same key at a lower block position.
-__device__ __forceinline__ int rank_in_range(const uint32_t* keys, int n4, int pos0, uint32_t key,
-                                             int pos) {
-  int rank = 0;
-  for (int r = 0; r < n4; r += 4) {
-    const uint4 v = *reinterpret_cast<const uint4*>(keys + r);
-    const int p = pos0 + r - pos;   // < 0: the entry lies before (key, pos)
-    rank += (v.x > key) | ((v.x == key) & (p < 0));
-    rank += (v.y > key) | ((v.y == key) & (p + 1 < 0));
-    rank += (v.z > key) | ((v.z == key) & (p + 2 < 0));
-    rank += (v.w > key) | ((v.w == key) & (p + 3 < 0));
+// One warp, keys[0 .. n) in shared memory: the threshold of the kk largest
+// keys, a lower index winning among equal keys. Afterwards the chosen keys are
+// those > tau plus the first `need` keys == tau in index order. tau is found
+// by deciding its bits from the highest bit where the largest and the
+// smallest key differ, each step counting the keys at or above the candidate
+// over the warp; it stops early once exactly kk keys are at or above it. Up to
+// 32 * kR keys are held in registers for the search (longer lists are re-read
+// from shared memory at every step).
+template <int kR>
+__device__ __forceinline__ void warp_threshold(const uint32_t* keys, int n, int kk, uint32_t& tau,
+                                               int& need) {
+  const int lane = threadIdx.x & 31;
+  if (kk <= 0) {
+    tau = 0xffffffffu;   // above every score key: nothing is taken
+    need = 0;
+    return;
   }
-  return rank;
+  if (n <= kk) {
+    tau = 0u;            // score keys are never 0: every key is taken
+    need = 0;
+    return;
+  }
+  const bool regs = n <= 32 * kR;   // uniform
+  uint32_t kr[kR];
+  uint32_t hi = 0u, lo = 0xffffffffu;
+#pragma unroll
+  for (int u = 0; u < kR; ++u) {
+    const int j = lane + 32 * u;
+    kr[u] = (regs && j < n) ? keys[j] : 0u;
+    if (regs && j < n) {
+      hi = max(hi, kr[u]);
+      lo = min(lo, kr[u]);
+    }
+  }
+  if (!regs)
+    for (int j = lane; j < n; j += 32) {
+      const uint32_t x = keys[j];
+      hi = max(hi, x);
+      lo = min(lo, x);
+    }
+  hi = __reduce_max_sync(kFull, hi);
+  lo = __reduce_min_sync(kFull, lo);
+  tau = hi;
+  if (hi != lo) {
+    const int top = 31 - __clz(hi ^ lo);
+    tau = top == 31 ? 0u : (hi & ~((2u << top) - 1u));
+    for (int bit = top; bit >= 0; --bit) {
+      const uint32_t cand = tau | (1u << bit);
+      int c = 0;
+      if (regs) {
+#pragma unroll
+        for (int u = 0; u < kR; ++u) c += kr[u] >= cand ? 1 : 0;   // padding keys are 0
+      } else {
+        for (int j = lane; j < n; j += 32) c += keys[j] >= cand ? 1 : 0;
+      }
+      c = __reduce_add_sync(kFull, c);
+      if (c >= kk) tau = cand;
+      if (c == kk) break;
+    }
+  }
+  int gt = 0;
+  if (regs) {
+#pragma unroll
+    for (int u = 0; u < kR; ++u) gt += kr[u] > tau ? 1 : 0;
+  } else {
+    for (int j = lane; j < n; j += 32) gt += keys[j] > tau ? 1 : 0;
+  }
+  need = kk - __reduce_add_sync(kFull, gt);
 }
-// The same with explicit positions (poss[0 .. n4), also 16-byte aligned).
-__device__ __forceinline__ int rank_in_list(const uint32_t* keys, const int* poss, int n4,
-                                            uint32_t key, int pos) {
-  int rank = 0;
-  for (int r = 0; r < n4; r += 4) {
-    const uint4 v = *reinterpret_cast<const uint4*>(keys + r);
-    const int4 q = *reinterpret_cast<const int4*>(poss + r);
-    rank += (v.x > key) | ((v.x == key) & (q.x < pos));
-    rank += (v.y > key) | ((v.y == key) & (q.y < pos));
-    rank += (v.z > key) | ((v.z == key) & (q.z < pos));
-    rank += (v.w > key) | ((v.w == key) & (q.w < pos));
+
+// One warp: the kk largest of keys[0 .. n) (warp_threshold's rule), written in
+// index order to out_key / out_pos (pos0 + index); slots kk .. kpad - 1 get a
+// sentinel (key 0, below every score key).
+__device__ __forceinline__ void warp_topk_compact(const uint32_t* keys, int n, int kk, int pos0,
+                                                  uint32_t* out_key, int* out_pos, int kpad) {
+  const int lane = threadIdx.x & 31;
+  uint32_t tau;
+  int need;
+  warp_threshold<8>(keys, n, kk, tau, need);
+  int base = 0;
+  for (int j0 = 0; j0 < n && base < kk; j0 += 32) {   // uniform
+    const int j = j0 + lane;
+    const uint32_t x = j < n ? keys[j] : 0u;
+    const bool eq = j < n && x == tau;
+    const unsigned eb = __ballot_sync(kFull, eq);
+    const bool t = (j < n && x > tau) || (eq && __popc(eb & lane_mask_lt()) < need);
+    need -= __popc(eb);
+    const unsigned tb = __ballot_sync(kFull, t);
+    if (t) {
+      const int sl = base + __popc(tb & lane_mask_lt());
+      out_key[sl] = x;
+      out_pos[sl] = pos0 + j;
+    }
+    base += __popc(tb);
   }
-  return rank;
+  for (int sl = kk + lane; sl < kpad; sl += 32) {
+    out_key[sl] = 0u;
+    out_pos[sl] = 0x7fffffff;
+  }
+}
+
+// One warp: the kk largest of keys[0 .. n) (warp_threshold's rule); sets bit
+// pos[j] % 32 of word pos[j] / 32 of bits for every chosen j.
+__device__ __forceinline__ void warp_topk_bits(const uint32_t* keys, const int* pos, int n, int kk,
+                                               uint32_t* bits) {
+  const int lane = threadIdx.x & 31;
+  uint32_t tau;
+  int need;
+  warp_threshold<16>(keys, n, kk, tau, need);
+  for (int j0 = 0; j0 < n; j0 += 32) {
+    const int j = j0 + lane;
+    const uint32_t x = j < n ? keys[j] : 0u;
+    const bool eq = j < n && x == tau;
+    const unsigned eb = __ballot_sync(kFull, eq);
+    const bool t = (j < n && x > tau) || (eq && __popc(eb & lane_mask_lt()) < need);
+    need -= __popc(eb);
+    if (t) atomicOr(&bits[pos[j] >> 5], 1u << (pos[j] & 31));
+  }
 }
 
 // Chunk of candidate blocks one CTA of the cluster scores: a multiple of 4.
@@ -436,103 +523,42 @@ __device__ __forceinline__ void select_in_cluster(const DecParams& P, uint8_t* s
     }
     __syncthreads();
   }
-  // Top-k in two steps, under the selection's total order (score key
-  // descending, block position ascending), with ranks counted by every thread:
-  // 1. every key of this CTA's range is ranked among its query's keys of the
-  //    range; the first k in rank order are the CTA's candidates (every block
-  //    of the cluster's top k is among them: fewer than k blocks of the whole
-  //    cache come before it, so fewer than k of its range);
-  // 2. after a cluster barrier each CTA gathers the first cand_m candidates of
-  //    every CTA (about twice the k / nsplit blocks a range holds on average),
-  //    ranks them the same way and takes the top k for every query itself, so
-  //    no bitmap has to cross the cluster. A CTA whose cand_m gathered
-  //    candidates were all taken while its list goes on may hold more of the
-  //    top k: that query is then redone over the full lists.
-  int* redo = hist;   // [n_q] (the scratch of the pooling above is free again)
-  {
-    for (int i = 0; i < n_q; ++i) {   // keys padded to a multiple of 4 (0: below every score key)
-      const int cnt = max(0, min(j1, (kv - n_q + 1 + i) / g.B) - j0);
-      for (int r = cnt + tid; r < ((cnt + 3) & ~3); r += nthr) keys_mine[i * per + r] = 0u;
-    }
-    for (int e = tid; e < n_q * kpad; e += nthr) {
-      cand_key[e] = 0u;
-      cand_pos[e] = 0x7fffffff;
-    }
-    if (tid < n_q) redo[tid] = 0;
-    __syncthreads();
-    for (int e = tid; e < n_q * per; e += nthr) {
-      const int i = e / per, r = e - i * per;
-      const int cnt = max(0, min(j1, (kv - n_q + 1 + i) / g.B) - j0);
-      if (r >= cnt) continue;
-      const uint32_t* kq = keys_mine + i * per;
-      const uint32_t key = kq[r];
-      const int rank = rank_in_range(kq, (cnt + 3) & ~3, j0, key, j0 + r);
-      if (rank < k) {
-        cand_key[i * kpad + rank] = key;
-        cand_pos[i * kpad + rank] = j0 + r;
-      }
-    }
+  // Top-k in two steps. Each CTA first takes the top k of its own range for
+  // every query (warp i, query i): every block of the cluster's top k is among
+  // them, since fewer than k blocks of the whole cache beat it, so fewer than k
+  // of its range. After a cluster barrier each CTA gathers all CTAs'
+  // candidates (CTA order is ascending block order, so a lower position still
+  // wins a tie) and takes the top k of those for every query itself: no bitmap
+  // has to cross the cluster afterwards.
+  if (warp < n_q) {
+    const int i = warp;
+    const int cnt = max(0, min(j1, (kv - n_q + 1 + i) / g.B) - j0);   // query i's blocks here
+    warp_topk_compact(keys_mine + i * per, cnt, min(k, cnt), j0, cand_key + i * kpad,
+                      cand_pos + i * kpad, kpad);
   }
   cluster_sync_all();   // every CTA's candidates are in place
-  const uint32_t ck_s = smem_u32(cand_key), cp_s = smem_u32(cand_pos);
-  // 16-byte groups of four candidates (keys, then positions), slots [0, mg) of
-  // every CTA's list of query i, or of every query with i < 0
-  auto gather = [&](int i_only, int mg) {
-    const int nq = i_only < 0 ? n_q : 1;
-    const int groups = nq * P.nsplit * (mg / 4);
+  {   // 16-byte groups of four candidates (keys, then positions) from every CTA
+    const int groups = n_q * P.nsplit * (kpad / 4);
+    const uint32_t ck_s = smem_u32(cand_key), cp_s = smem_u32(cand_pos);
     for (int e = tid; e < groups; e += nthr) {
-      const int ii = e / (P.nsplit * (mg / 4)), rem = e - ii * (P.nsplit * (mg / 4));
-      const int i = i_only < 0 ? ii : i_only;
-      const int c = rem / (mg / 4), q4 = rem - c * (mg / 4);
+      const int i = e / (P.nsplit * (kpad / 4)), rem = e - i * (P.nsplit * (kpad / 4));
+      const int c = rem / (kpad / 4), q4 = rem - c * (kpad / 4);
       const uint32_t off = 4u * (uint32_t)(i * kpad + 4 * q4);
       const uint4 kv4 = ld_cluster_u32x4(cluster_map(ck_s + off, c));
       const uint4 pv4 = ld_cluster_u32x4(cluster_map(cp_s + off, c));
       *reinterpret_cast<uint4*>(gkey + i * ng + c * kpad + 4 * q4) = kv4;
       *reinterpret_cast<uint4*>(gpos + i * ng + c * kpad + 4 * q4) = pv4;
     }
-  };
-  // the top k of slots [0, m) of every gathered list of query i (or of every
-  // query with i < 0) into the query bitmaps; with check, flags a list whose
-  // slot m - 1 is taken while its slot m holds a candidate
-  auto select = [&](int i_only, int m, bool check) {
-    const int nq = i_only < 0 ? n_q : 1;
-    for (int e = tid; e < nq * P.nsplit * m; e += nthr) {
-      const int ii = e / (P.nsplit * m), rem = e - ii * (P.nsplit * m);
-      const int i = i_only < 0 ? ii : i_only;
-      const int c = rem / m, sl = rem - c * m;
-      const uint32_t key = gkey[i * ng + c * kpad + sl];
-      if (key == 0u) continue;   // padding
-      const int pos = gpos[i * ng + c * kpad + sl];
-      int rank = 0;
-      for (int c2 = 0; c2 < P.nsplit; ++c2)
-        rank += rank_in_list(gkey + i * ng + c2 * kpad, gpos + i * ng + c2 * kpad, m, key, pos);
-      const int nc_i = (kv - n_q + 1 + i) / g.B;
-      if (rank < min(k, nc_i)) {
-        atomicOr(&qbits[i * words + (pos >> 5)], 1u << (pos & 31));
-        if (check && sl == m - 1 && gkey[i * ng + c * kpad + m] != 0u) redo[i] = 1;
-      }
-    }
-  };
-  const int m = P.cand_m;                  // a multiple of 4, at most kpad
-  const bool cut = m < k;                  // lists longer than m exist
-  gather(-1, cut ? min(kpad, m + 4) : kpad);
-  __syncthreads();
-  select(-1, cut ? m : kpad, cut);
-  __syncthreads();
-  if (cut) {
-    for (int i = 0; i < n_q; ++i) {
-      if (!redo[i]) continue;   // uniform
-      for (int w = tid; w < words; w += nthr) qbits[i * words + w] = 0u;
-      gather(i, kpad);
-      __syncthreads();
-      select(i, kpad, false);
-      __syncthreads();
-    }
   }
-  if (warp < n_q && lane == 0) {   // the tail block
-    const int n = kv - n_q + 1 + warp;
+  __syncthreads();
+  if (warp < n_q) {
+    const int i = warp;
+    const int n = kv - n_q + 1 + i;
     const int nc_i = n / g.B;
-    if (n - nc_i * g.B > 0) atomicOr(&qbits[warp * words + (nc_i >> 5)], 1u << (nc_i & 31));
+    uint32_t* qb = qbits + i * words;
+    warp_topk_bits(gkey + i * ng, gpos + i * ng, ng, min(k, nc_i), qb);
+    __syncwarp();
+    if (lane == 0 && n - nc_i * g.B > 0) atomicOr(&qb[nc_i >> 5], 1u << (nc_i & 31));   // tail
   }
   __syncthreads();
   if (split == 0 && hk == 0 && warp < n_q) {   // the selection lists: ascending, tail last
@@ -1631,11 +1657,6 @@ cudaError_t launch_decode_fused(const Geom& g, int batch, int n_q, int cap, int 
   p.pooled = si.pooled;
   p.sel_w = si.sel;
   p.nsel_w = si.nsel;
-  {   // candidates per CTA the top-k first looks at: about twice a range's share, + 4
-    const int kpad = (g.k + 3) & ~3;
-    const int m = 2 * ((g.k + nsplit - 1) / nsplit) + 4;
-    p.cand_m = std::min(kpad, (m + 3) & ~3);
-  }
   const int smem = decode_smem(g, n_q, cap);
   const void* kern =
       f8.on ? fused_kernel<true>(g.di, 1) : fused_kernel<false>(g.di, row_tiles(g, n_q));

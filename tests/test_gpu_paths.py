@@ -147,11 +147,9 @@ def test_decode_one_launch_and_two_kernel_paths(name, kv_lens, cap):
 
 @pytest.mark.parametrize("name", ["decode_bf16_b32_kv32768", "mtp_verify_bf16_b4_kv262144"])
 def test_decode_topk_concentrated_in_one_range(name):
-    # The one-launch decode's clusters first compare only the leading candidates
-    # of each CTA's range of blocks (about twice a range's share of the top k);
-    # when one range holds more of the top k than that, the query is selected
-    # again over every candidate. The indexer keys of the first 48 blocks are
-    # scaled by 8 (exact in bf16), so most of the top k lies in the first range.
+    # The one-launch decode's clusters take each CTA's top k of its own range
+    # of blocks as candidates; here one range holds most of the top k. The
+    # indexer keys of the first 48 blocks are scaled by 8 (exact in bf16).
     B = WORKLOADS[name].block_size
     kv = 800 * B + 3
     w, inp = _decode(name, batch=2, cap=801 * B, kv_lens=(kv, kv - 70))
