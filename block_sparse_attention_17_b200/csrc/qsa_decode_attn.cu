@@ -352,6 +352,44 @@ __device__ __forceinline__ void warp_topk_bits(const uint32_t* keys, const int* 
   }
 }
 
+// Sorted top-32 lists held one value per lane. A value packs a score key and
+// a block position as (key << 32) | (0xffffffff - position): a larger value
+// comes first in the selection's order (a larger key, or the same key at a
+// lower position); 0 is padding, below every real value.
+__device__ __forceinline__ unsigned long long cand_value(uint32_t key, int pos) {
+  return ((unsigned long long)key << 32) | (0xffffffffu - (uint32_t)pos);
+}
+__device__ __forceinline__ unsigned long long shfl_xor_u64(unsigned long long v, int m) {
+  return __shfl_xor_sync(kFull, v, m);
+}
+// One warp: the 32 values (one per lane) sorted in descending order, lane =
+// rank (a bitonic sorting network over the lanes).
+__device__ __forceinline__ unsigned long long warp_sort32_desc(unsigned long long v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int sz = 2; sz <= 32; sz <<= 1)
+#pragma unroll
+    for (int j = sz >> 1; j > 0; j >>= 1) {
+      const unsigned long long o = shfl_xor_u64(v, j);
+      v = (((lane & j) == 0) == ((lane & sz) == 0 || sz == 32)) ? (v > o ? v : o) : (v < o ? v : o);
+    }
+  return v;
+}
+// One warp: the largest 32 of two descending lists (lane = rank), descending:
+// max(a[i], b[31 - i]) is bitonic and holds them; one bitonic merge sorts it.
+__device__ __forceinline__ unsigned long long warp_merge32_desc(unsigned long long a,
+                                                                unsigned long long b) {
+  const int lane = threadIdx.x & 31;
+  const unsigned long long br = __shfl_sync(kFull, b, 31 - lane);
+  unsigned long long v = a > br ? a : br;
+#pragma unroll
+  for (int j = 16; j > 0; j >>= 1) {
+    const unsigned long long o = shfl_xor_u64(v, j);
+    v = ((lane & j) == 0) ? (v > o ? v : o) : (v < o ? v : o);
+  }
+  return v;
+}
+
 // Chunk of candidate blocks one CTA of the cluster scores: a multiple of 4.
 __host__ __device__ __forceinline__ int select_range(int nc_last, int nsplit) {
   const int per = ((nc_last > 1 ? nc_last : 1) + nsplit - 1) / nsplit;
@@ -530,11 +568,30 @@ __device__ __forceinline__ void select_in_cluster(const DecParams& P, uint8_t* s
   // candidates (CTA order is ascending block order, so a lower position still
   // wins a tie) and takes the top k of those for every query itself: no bitmap
   // has to cross the cluster afterwards.
+  // With k <= 32 every list is a sorted top-32 held one value per lane: the
+  // range's keys are sorted 32 at a time and merged into the running top 32,
+  // and the candidate list is written in rank order.
   if (warp < n_q) {
     const int i = warp;
     const int cnt = max(0, min(j1, (kv - n_q + 1 + i) / g.B) - j0);   // query i's blocks here
-    warp_topk_compact(keys_mine + i * per, cnt, min(k, cnt), j0, cand_key + i * kpad,
-                      cand_pos + i * kpad, kpad);
+    if (k <= 32) {
+      const uint32_t* kq = keys_mine + i * per;
+      unsigned long long top = 0ull;
+      for (int r0 = 0; r0 < cnt; r0 += 32) {   // uniform
+        const int r = r0 + lane;
+        const unsigned long long v =
+            warp_sort32_desc(r < cnt ? cand_value(kq[r], j0 + r) : 0ull);
+        top = r0 == 0 ? v : warp_merge32_desc(top, v);
+      }
+      if (lane < kpad) {
+        const bool real = lane < k && top != 0ull;
+        cand_key[i * kpad + lane] = real ? (uint32_t)(top >> 32) : 0u;
+        cand_pos[i * kpad + lane] = real ? (int)(0xffffffffu - (uint32_t)top) : 0x7fffffff;
+      }
+    } else {
+      warp_topk_compact(keys_mine + i * per, cnt, min(k, cnt), j0, cand_key + i * kpad,
+                        cand_pos + i * kpad, kpad);
+    }
   }
   cluster_sync_all();   // every CTA's candidates are in place
   {   // 16-byte groups of four candidates (keys, then positions) from every CTA
@@ -556,7 +613,25 @@ __device__ __forceinline__ void select_in_cluster(const DecParams& P, uint8_t* s
     const int n = kv - n_q + 1 + i;
     const int nc_i = n / g.B;
     uint32_t* qb = qbits + i * words;
-    warp_topk_bits(gkey + i * ng, gpos + i * ng, ng, min(k, nc_i), qb);
+    if (k <= 32) {
+      // every CTA's list is sorted: merge them pairwise into the top 32
+      unsigned long long top = 0ull;
+      for (int c = 0; c < P.nsplit; c += 2) {   // uniform
+        const int a = i * ng + c * kpad + lane, bb = a + kpad;
+        unsigned long long v = lane < kpad ? cand_value(gkey[a], gpos[a]) : 0ull;
+        if (lane < kpad && gkey[a] == 0u) v = 0ull;
+        if (c + 1 < P.nsplit) {
+          unsigned long long w = lane < kpad ? cand_value(gkey[bb], gpos[bb]) : 0ull;
+          if (lane < kpad && gkey[bb] == 0u) w = 0ull;
+          v = warp_merge32_desc(v, w);
+        }
+        top = c == 0 ? v : warp_merge32_desc(top, v);
+      }
+      const int pos = (int)(0xffffffffu - (uint32_t)top);
+      if (lane < min(k, nc_i) && top != 0ull) atomicOr(&qb[pos >> 5], 1u << (pos & 31));
+    } else {
+      warp_topk_bits(gkey + i * ng, gpos + i * ng, ng, min(k, nc_i), qb);
+    }
     __syncwarp();
     if (lane == 0 && n - nc_i * g.B > 0) atomicOr(&qb[nc_i >> 5], 1u << (nc_i & 31));   // tail
   }
