@@ -44,7 +44,15 @@ design notes of the repository):
 * R10 attention scale: softmax_scale (default head_dim ** -0.5).
 * R11 decode: kv_len counts tokens after this step's n_q tokens were appended;
   new query i sees n = kv_len - n_q + 1 + i tokens.
-* R12 no rotary embedding is applied to indexer queries or pooled keys.
+* R12 indexer rotary embedding, optional (rope_dim = 0 turns it off and is the
+  default): the query of the indexer is rotated at its own position (the token
+  index within the sequence, n - 1 for a query that sees n tokens); the pooled
+  key of block j is the mean of the block's raw indexer keys rotated at the
+  block's first position j * B; both with one angle table. The rotation is the
+  ordinary partial rotary embedding: pairs (f, f + rope_dim / 2) of the first
+  rope_dim dims, frequency f has inverse wavelength theta ** (-2 f / rope_dim)
+  rounded to fp32, and the angle is the fp32 product of the position and that
+  value (cos and sin of the fp32 angle are then taken in fp64).
 
 Every pin of these functions lives in tests/test_oracle_pins.py.
 """
@@ -74,6 +82,61 @@ def pool_blocks(ik_rows: np.ndarray, block_size: int) -> np.ndarray:
     for j in range(nblk):
         out[j] = ik_rows[j * block_size:(j + 1) * block_size].sum(axis=0) / block_size
     return out
+
+
+# --------------------------------------------------------------------------
+# optional: rotary embedding of the indexer (R12)
+# (llama.cpp PR #27739 page, QSA block-composition commit text: the indexer is
+#  fed the roped query and the raw keys, and the pooled indexer keys take the
+#  same rope angles as the query; instagit MTPLX page, "Multidimensional Rotary
+#  Embeddings (M-RoPE)": for text the rotary embedding is the ordinary partial
+#  rotary embedding)
+# --------------------------------------------------------------------------
+def rope_params(cfg) -> tuple:
+    """(rope_dim, theta as an fp32 value) of a config; rope_dim 0 = no rotation."""
+    r = int(getattr(cfg, "rope_dim", 0) or 0)
+    theta = float(np.float32(getattr(cfg, "rope_theta", 10000.0) or 10000.0))
+    return r, theta
+
+
+def rope_inv_freq(rope_dim: int, theta: float) -> np.ndarray:
+    """theta ** (-2 f / rope_dim) for f < rope_dim / 2, each rounded to fp32."""
+    th = float(np.float32(theta))
+    return np.array([np.float32(th ** (-2.0 * f / rope_dim)) for f in range(rope_dim // 2)],
+                    dtype=np.float32)
+
+
+def rope_angles(pos: int, rope_dim: int, theta: float) -> np.ndarray:
+    """The fp32 products pos * inv_freq[f] (round to nearest even), as fp64."""
+    return (np.float32(pos) * rope_inv_freq(rope_dim, theta)).astype(np.float64)
+
+
+def rope_rotate(x, pos: int, rope_dim: int, theta: float) -> np.ndarray:
+    """Rotates the pairs (x[f], x[f + h]), h = rope_dim / 2, of the last axis
+    by angle[f] (counter-clockwise: (1, 0) goes to (cos, sin)); the dims from
+    rope_dim on are unchanged."""
+    x = np.array(x, dtype=np.float64)
+    if rope_dim == 0:
+        return x
+    h = rope_dim // 2
+    a = rope_angles(pos, rope_dim, theta)
+    c, s = np.cos(a), np.sin(a)
+    x1 = x[..., :h].copy()
+    x2 = x[..., h:rope_dim].copy()
+    x[..., :h] = x1 * c - x2 * s
+    x[..., h:rope_dim] = x2 * c + x1 * s
+    return x
+
+
+def pooled_keys(cfg, ik_rows) -> np.ndarray:
+    """Step 1 with R12: block means, row j rotated at position j * B."""
+    B = cfg.block_size
+    kbar = pool_blocks(ik_rows, B)
+    r, theta = rope_params(cfg)
+    if r:
+        for j in range(kbar.shape[0]):
+            kbar[j] = rope_rotate(kbar[j], j * B, r, theta)
+    return kbar
 
 
 # --------------------------------------------------------------------------
@@ -200,12 +263,16 @@ def qsa_query(cfg, n: int, kbar: np.ndarray, iq_t, iw_t, q_t=None, K=None, V=Non
               gate_t=None, attend: bool = True) -> QueryResult:
     """QSA for one query that sees n tokens of its sequence.
 
-    kbar: pooled keys of the sequence (at least floor(n/B) rows).
+    kbar: pooled keys of the sequence (at least floor(n/B) rows; rotated by
+    pooled_keys when the config has a rotary embedding).
     """
     B = cfg.block_size
     k = cfg.budget // B
     sm_scale, idx_scale = _scales(cfg)
     nc = n // B
+    r, theta = rope_params(cfg)
+    if r and nc > 0:
+        iq_t = rope_rotate(iq_t, n - 1, r, theta)     # R12: the query's own position
     s = index_scores(iq_t, iw_t, kbar[:nc], idx_scale) if nc > 0 else np.zeros(0)
     sel = select_topk(s, k)
     tail = n - nc * B
@@ -223,7 +290,7 @@ def qsa_prefill(cfg, inp: dict, queries: Optional[Iterable[int]] = None,
     of every sequence under key "pooled" (list of [floor(L/B), di])."""
     cu = np.asarray(inp["cu_seqlens"], dtype=np.int64)
     nseq = len(cu) - 1
-    pooled = [pool_blocks(inp["ik"][cu[b]:cu[b + 1]], cfg.block_size) for b in range(nseq)]
+    pooled = [pooled_keys(cfg, inp["ik"][cu[b]:cu[b + 1]]) for b in range(nseq)]
     T = int(cu[-1])
     qs = range(T) if queries is None else queries
     res = {}
@@ -259,7 +326,7 @@ def qsa_decode(cfg, inp: dict, pairs: Optional[Iterable[tuple]] = None,
     for b, i in pairs:
         L = int(kv[b])
         if b not in pooled_cache:
-            pooled_cache[b] = pool_blocks(inp["ik_cache"][b, :L], cfg.block_size)
+            pooled_cache[b] = pooled_keys(cfg, inp["ik_cache"][b, :L])
         n = decode_visible(L, n_q, i)
         r = qsa_query(cfg, n, pooled_cache[b], inp["iq"][b, i], inp["iw"][b, i],
                       q_t=inp["q"][b, i] if attend else None,

@@ -347,6 +347,104 @@ def test_workload_recipe_shapes():
     assert inp["q"].shape == (137, 4, 64) and inp["cu_seqlens"].tolist() == [0, 100, 100, 137]
 
 
+# ---------------------------------------------------------------- indexer rotary embedding (R12)
+COS1, SIN1 = 0.5403023058681398, 0.8414709848078965     # cos(1), sin(1)
+
+
+def pin_rope_closed_form(rotate=None, inv_freq=None):
+    rotate = rotate or O.rope_rotate
+    inv_freq = inv_freq or O.rope_inv_freq
+    # frequencies: theta ** (-2 f / r); 10000 ** (-1/2) = 0.01, 10000 ** 0 = 1
+    np.testing.assert_array_equal(inv_freq(4, 10000.0), np.float32([1.0, 0.01]))
+    np.testing.assert_array_equal(inv_freq(8, 256.0), np.float32([1.0, 0.25, 0.0625, 0.015625]))
+    # rope_dim 2: one pair rotated by pos radians; (1, 0) goes to (cos, sin)
+    np.testing.assert_allclose(rotate([1.0, 0.0], 1, 2, 10000.0), [COS1, SIN1], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(rotate([0.0, 1.0], 1, 2, 10000.0), [-SIN1, COS1], rtol=0, atol=1e-15)
+    # position 0 is the identity
+    x = np.array([0.3, -1.25, 2.0, 0.5, 7.0, -3.0])
+    np.testing.assert_array_equal(rotate(x, 0, 4, 10000.0), x)
+    # rope_dim 4 of 6 dims at position 100: frequency 1 turns by fp32(100 * fp32(0.01)) = 1 rad;
+    # the pair of dim 1 is dim 3 (half split), and dims 4, 5 are untouched
+    e1 = np.array([0.0, 1.0, 0.0, 0.0, 7.0, -3.0])
+    np.testing.assert_allclose(rotate(e1, 100, 4, 10000.0), [0.0, COS1, 0.0, SIN1, 7.0, -3.0],
+                               rtol=0, atol=1e-15)
+    # frequency 0 turns by 100 rad: e0 -> (cos 100, 0, sin 100, 0)
+    e0 = np.array([1.0, 0.0, 0.0, 0.0])
+    np.testing.assert_allclose(rotate(e0, 100, 4, 10000.0),
+                               [0.8623188722876839, 0.0, -0.5063656411097588, 0.0], rtol=0, atol=1e-15)
+
+
+def test_rope_closed_form():
+    pin_rope_closed_form()
+
+
+def pin_rope_complex_and_norm(rotate=None):
+    """Against complex multiplication z_f * exp(i a_f) with z_f = x_f + i x_{f+h},
+    and the norm of every pair is kept."""
+    rotate = rotate or O.rope_rotate
+    rng = np.random.default_rng(12)
+    for r, di, pos, theta in [(8, 8, 37, 10000.0), (16, 32, 1000, 500000.0), (4, 8, 262143, 10000.0)]:
+        x = rng.standard_normal(di)
+        y = rotate(x, pos, r, theta)
+        h = r // 2
+        a = O.rope_angles(pos, r, theta)
+        z = (x[:h] + 1j * x[h:r]) * np.exp(1j * a)
+        np.testing.assert_allclose(y[:h], z.real, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(y[h:r], z.imag, rtol=0, atol=1e-13)
+        np.testing.assert_array_equal(y[r:], x[r:])
+        np.testing.assert_allclose(y[:h] ** 2 + y[h:r] ** 2, x[:h] ** 2 + x[h:r] ** 2, rtol=1e-13)
+
+
+def test_rope_complex_and_norm():
+    pin_rope_complex_and_norm()
+
+
+def pin_rope_relative(rotate=None):
+    """rot(q, m) . rot(k, n) depends on m - n only (same frequencies and turning
+    direction on both sides); fp32 angles keep it to rounding at small positions."""
+    rotate = rotate or O.rope_rotate
+    rng = np.random.default_rng(13)
+    q, k = rng.standard_normal(16), rng.standard_normal(16)
+    for m, n, d in [(9, 3, 5), (40, 40, 17), (3, 30, 64)]:
+        a = rotate(q, m, 16, 10000.0) @ rotate(k, n, 16, 10000.0)
+        b = rotate(q, m + d, 16, 10000.0) @ rotate(k, n + d, 16, 10000.0)
+        c = rotate(q, m - n, 16, 10000.0) @ k if m >= n else q @ rotate(k, n - m, 16, 10000.0)
+        assert abs(a - b) < 2e-5 * (np.abs(q) @ np.abs(k)), (m, n, d)
+        assert abs(a - c) < 2e-5 * (np.abs(q) @ np.abs(k)), (m, n)
+
+
+def test_rope_relative_position():
+    pin_rope_relative()
+
+
+def pin_rope_positions_in_scores(query=None):
+    """With R12 the score of block j is the unrotated score of the query turned by
+    its offset (n - 1) - j * B from the block's first token: the query sits at
+    its own position and every pooled key at its block's first position."""
+    query = query or O.qsa_query
+    rng = np.random.default_rng(14)
+    B, di, Hi, r = 8, 16, 3, 12
+    cfg = Cfg(block_size=B, budget=4 * B, idx_dim=di, idx_heads=Hi, rope_dim=r, rope_theta=10000.0)
+    plain = Cfg(block_size=B, budget=4 * B, idx_dim=di, idx_heads=Hi)
+    n = 83
+    ik = rng.standard_normal((n, di))
+    iq, iw = rng.standard_normal((Hi, di)), rng.random(Hi)
+    res = query(cfg, n, O.pooled_keys(cfg, ik), iq, iw, attend=False)
+    raw = O.pool_blocks(ik, B)
+    c = di ** -0.5
+    for j in range(n // B):
+        qj = np.stack([O.rope_rotate(iq[h], (n - 1) - j * B, r, 10000.0) for h in range(Hi)])
+        expect = c * (np.maximum(qj @ raw[j], 0.0) @ iw)
+        assert abs(res.scores[j] - expect) <= 1e-5 * (1.0 + abs(expect)), j
+    # rope_dim 0 is the plain score
+    res0 = query(plain, n, O.pooled_keys(plain, ik), iq, iw, attend=False)
+    np.testing.assert_allclose(res0.scores, c * (np.maximum(raw[:n // B] @ iq.T, 0.0) @ iw), rtol=1e-14)
+
+
+def test_rope_positions_in_scores():
+    pin_rope_positions_in_scores()
+
+
 # ---------------------------------------------------------------- mutation battery
 def _mut_pool_divide_by_n(ik_rows, B):
     ik_rows = np.asarray(ik_rows, np.float64)
@@ -386,6 +484,32 @@ def _mut_topk_unstable_negzero(scores, k):
     return np.array(sorted(keyed[:min(k, nc)]), dtype=np.int64)
 
 
+def _mut_rope_clockwise(x, pos, r, theta):
+    return O.rope_rotate(x, -pos, r, theta)
+
+
+def _mut_rope_interleaved(x, pos, r, theta):
+    x = np.array(x, dtype=np.float64)
+    a = O.rope_angles(pos, r, theta)
+    c, s = np.cos(a), np.sin(a)
+    x1, x2 = x[0:r:2].copy(), x[1:r:2].copy()
+    x[0:r:2], x[1:r:2] = x1 * c - x2 * s, x2 * c + x1 * s
+    return x
+
+
+def _mut_rope_freq(r, theta):
+    return np.array([np.float32(float(theta) ** (-1.0 * f / r)) for f in range(r // 2)], np.float32)
+
+
+_rope_calls = [0]
+
+
+def _mut_rope_sign_by_parity(x, pos, r, theta):
+    # the second operand of every dot turned the other way
+    _rope_calls[0] += 1
+    return O.rope_rotate(x, pos if _rope_calls[0] % 2 else -pos, r, theta)
+
+
 @pytest.mark.parametrize("name,target,mut,pin", [
     ("pool/B+1", "pool_blocks", _mut_pool_divide_by_n, pin_pool_closed_form),
     ("pool/partial", "pool_blocks", _mut_pool_includes_partial, pin_pool_closed_form),
@@ -394,6 +518,12 @@ def _mut_topk_unstable_negzero(scores, k):
     ("score/weights-reversed", "index_scores", _mut_score_transposed, pin_scores_hand_example),
     ("topk/tie-high", "select_topk", _mut_topk_high_index_wins, pin_topk_brute_force),
     ("topk/negzero", "select_topk", _mut_topk_unstable_negzero, pin_topk_brute_force),
+    ("rope/clockwise", "rope_rotate", _mut_rope_clockwise, pin_rope_closed_form),
+    ("rope/interleaved", "rope_rotate", _mut_rope_interleaved, pin_rope_closed_form),
+    ("rope/interleaved-c", "rope_rotate", _mut_rope_interleaved, pin_rope_complex_and_norm),
+    ("rope/freq-f-over-r", "rope_inv_freq", _mut_rope_freq,
+     lambda m: pin_rope_closed_form(inv_freq=m)),
+    ("rope/k-other-way", "rope_rotate", _mut_rope_sign_by_parity, pin_rope_relative),
 ])
 def test_mutation_turns_a_pin_red(name, target, mut, pin):
     with pytest.raises(AssertionError):
@@ -420,3 +550,26 @@ def test_mutations_of_attention_turn_dense_pin_red(monkeypatch):
                         lambda n, B, sel: orig_vis((n // B) * B, B, sel))
     with pytest.raises(AssertionError):
         test_single_block_closed_form()
+
+
+def test_mutations_of_rope_positions_turn_score_pin_red(monkeypatch):
+    # the query rotated at n (the count) instead of its position n - 1
+    def query_at_n(cfg, n, kbar, iq_t, iw_t, **kw):
+        r, th = O.rope_params(cfg)
+        return O.qsa_query(cfg, n, kbar, O.rope_rotate(iq_t, 1, r, th), iw_t, **kw)
+    with pytest.raises(AssertionError):
+        pin_rope_positions_in_scores(query_at_n)
+
+    # pooled keys rotated at the block's last token instead of its first
+    orig_rot = O.rope_rotate
+
+    def pooled_at_last(cfg, ik_rows):
+        B = cfg.block_size
+        kbar = O.pool_blocks(ik_rows, B)
+        r, th = O.rope_params(cfg)
+        for j in range(kbar.shape[0]):
+            kbar[j] = orig_rot(kbar[j], j * B + B - 1, r, th) if r else kbar[j]
+        return kbar
+    monkeypatch.setattr(O, "pooled_keys", pooled_at_last)
+    with pytest.raises(AssertionError):
+        pin_rope_positions_in_scores()
