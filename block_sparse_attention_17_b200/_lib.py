@@ -29,6 +29,7 @@ EXPORTED = [
     "qsa_pool_build", "qsa_decode_noalloc", "qsa_decode_paged", "qsa_pool_build_paged",
     "qsa_decode_fp8", "qsa_decode_attend",
     "qsa_cp_select", "qsa_cp_global_topk", "qsa_cp_attend", "qsa_cp_merge",
+    "qsa_cp_pool_build",
 ]
 
 
@@ -45,6 +46,8 @@ class QsaConfigC(ctypes.Structure):
         ("index_scale", ctypes.c_float),
         ("gate_headwise", ctypes.c_int),
         ("dtype", ctypes.c_int),
+        ("rope_dim", ctypes.c_int),
+        ("rope_theta", ctypes.c_float),
     ]
 
 
@@ -89,6 +92,8 @@ def _declare(lib):
         # cfg, batch, n_q, cap, block_lo, kv_len, iq, ik, iw, pooled, cand_score, cand_id,
         # dev_err, ws, ws_bytes, stream
         "qsa_cp_select": (I, [CFG, I, I, I, I] + [P] * 9 + [SZ, P]),
+        # cfg, batch, cap, block_lo, kv_len, ik_shard, pooled_shard, dev_err, stream
+        "qsa_cp_pool_build": (I, [CFG, I, I, I, P, P, P, P, P]),
         # cfg, batch, n_q, world, kv_len, cand_score, cand_id, sel, nsel, stream
         "qsa_cp_global_topk": (I, [CFG, I, I, I] + [P] * 6),
         # cfg, batch, n_q, cap, block_lo, kv_len, q, k, v, gate, sel, nsel, part_out,

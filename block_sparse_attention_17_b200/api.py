@@ -32,6 +32,8 @@ class QSAConfig:
     index_scale: float = 0.0       # 0 => idx_dim ** -0.5
     gate_headwise: bool = False
     dtype: torch.dtype = torch.bfloat16
+    rope_dim: int = 0              # indexer rotary embedding (0 = off)
+    rope_theta: float = 10000.0
 
     @property
     def topk(self) -> int:
@@ -43,7 +45,8 @@ class QSAConfig:
                    head_dim=w.head_dim, idx_heads=w.idx_heads, idx_dim=w.idx_dim,
                    block_size=w.block_size, budget=w.budget,
                    gate_headwise=bool(w.gate_headwise),
-                   dtype=torch.bfloat16 if w.dtype == "bf16" else torch.float32)
+                   dtype=torch.bfloat16 if w.dtype == "bf16" else torch.float32,
+                   rope_dim=int(w.rope_dim), rope_theta=float(w.rope_theta))
 
     def c(self) -> _lib.QsaConfigC:
         if self.dtype not in _DT:
@@ -51,7 +54,8 @@ class QSAConfig:
         return _lib.QsaConfigC(self.num_q_heads, self.num_kv_heads, self.head_dim,
                                self.idx_heads, self.idx_dim, self.block_size, self.budget,
                                float(self.softmax_scale), float(self.index_scale),
-                               int(bool(self.gate_headwise)), _DT[self.dtype])
+                               int(bool(self.gate_headwise)), _DT[self.dtype],
+                               int(self.rope_dim), float(self.rope_theta))
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -484,6 +488,29 @@ def decode_fp8(cfg: QSAConfig, q, k_cache, k_scale, v_cache, v_scale, iq, ik_cac
 
 
 # ------------------------------------------------- context-parallel decode
+def cp_pool_build(cfg: QSAConfig, ik_shard, kv_len, block_lo: int, *, dev_err=None,
+                  stream=None) -> torch.Tensor:
+    """Pooled rows of a context-parallel shard (qsa_cp_pool_build): ik_shard
+    [batch, cap, di] holds blocks [block_lo, block_lo + cap / B); kv_len are the
+    full lengths. Returns pooled_shard [batch, cap / B, di] fp32 (rows of
+    incomplete blocks are zero)."""
+    dt = cfg.dtype
+    batch, cap = ik_shard.shape[0], ik_shard.shape[1]
+    _need(ik_shard, "ik_shard", dt, (batch, cap, cfg.idx_dim))
+    _need(kv_len, "kv_len", torch.int32, (batch,))
+    dev = ik_shard.device
+    pooled = torch.zeros(batch, cap // cfg.block_size, cfg.idx_dim, dtype=torch.float32,
+                         device=dev)
+    _one_device(dev, stream, kv_len=kv_len, dev_err=dev_err)
+    c = cfg.c()
+    with torch.cuda.device(dev):
+        st = _lib.lib().qsa_cp_pool_build(ctypes.byref(c), batch, cap, int(block_lo),
+                                          _ptr(kv_len), _ptr(ik_shard), _ptr(pooled),
+                                          _ptr(dev_err), _stream(stream))
+        _lib.check(st, "qsa_cp_pool_build")
+    return pooled
+
+
 def cp_select(cfg: QSAConfig, iq, ik_shard, iw, pooled_shard, kv_len, block_lo: int, *,
               dev_err=None, workspace=None, stream=None) -> dict:
     """Shard selection of a context-parallel decode step (qsa_cp_select):

@@ -124,6 +124,10 @@ qsa_status check_cfg(const qsa_config* c) {
   if (c->idx_dim != 32 && c->idx_dim != 64)
     return fail(QSA_ERR_UNSUPPORTED, "idx_dim %d (supported: 32, 64)", c->idx_dim);
   if (c->idx_heads > 16) return fail(QSA_ERR_UNSUPPORTED, "idx_heads > 16");
+  if (c->rope_dim < 0 || c->rope_dim > c->idx_dim || (c->rope_dim & 3))
+    return fail(QSA_ERR_INVALID_ARG, "rope_dim %d (a multiple of 4 in [0, idx_dim])", c->rope_dim);
+  if (c->rope_dim > 0 && !(c->rope_theta > 0.f && isfinite(c->rope_theta)))
+    return fail(QSA_ERR_INVALID_ARG, "rope_theta must be finite and > 0 when rope_dim > 0");
   return QSA_OK;
 }
 
@@ -141,6 +145,8 @@ Geom make_geom(const qsa_config* c) {
   g.sm_scale_log2 = sm * kLog2e;
   g.idx_scale = c->index_scale > 0.f ? c->index_scale : 1.0f / sqrtf((float)g.di);
   g.gate_headwise = c->gate_headwise ? 1 : 0;
+  g.rope_dim = c->rope_dim;
+  g.rope_theta = c->rope_dim > 0 ? c->rope_theta : 0.f;
   return g;
 }
 
@@ -286,7 +292,7 @@ const char* qsa_status_string(qsa_status s) {
 
 const char* qsa_last_error(void) { return g_err; }
 
-int qsa_version(void) { return 100; }
+int qsa_version(void) { return 101; }
 
 unsigned long long qsa_kernel_launch_count(void) { return g_launches.load(); }
 
@@ -313,8 +319,7 @@ static qsa_status prefill_select_common(const qsa_config* cfg, const Geom& g, in
   const int words = (max_nblk + 31) / 32;
   // the error word and the selection's work counter start at zero
   QSA_CUDA(cudaMemsetAsync(w.err, 0, 2 * sizeof(int), st), "clear error word");
-  QSA_CUDA(launch_pool_prefill(cfg->dtype, ik, cu, batch, max_seqlen, g.B, g.di, pooled,
-                               max_nblk, st),
+  QSA_CUDA(launch_pool_prefill(cfg->dtype, ik, cu, batch, max_seqlen, g, pooled, max_nblk, st),
            "pool");
   QSA_CUDA(launch_select_prefill(cfg->dtype, g, cu, batch, max_seqlen, max_nblk, words, iq, iw,
                                  pooled, w.sched, sel, nsel, w.bitmask, scores,
@@ -564,6 +569,22 @@ static qsa_status check_shard(const qsa_config* cfg, int batch, int n_q, int cap
   return QSA_OK;
 }
 
+qsa_status qsa_cp_pool_build(const qsa_config* cfg, int batch, int cap, int block_lo,
+                             const int32_t* kv_len, const void* ik_shard, float* pooled_shard,
+                             int32_t* dev_err, void* stream) {
+  g_err[0] = 0;
+  qsa_status s = check_shard(cfg, batch, 1, cap, block_lo);
+  if (s != QSA_OK) return s;
+  if (batch == 0) return QSA_OK;
+  QSA_REQUIRE(kv_len, "kv_len");
+  QSA_REQUIRE(ik_shard, "ik_shard");
+  QSA_REQUIRE(pooled_shard, "pooled_shard");
+  QSA_CUDA(launch_pool_cache(cfg->dtype, ik_shard, kv_len, batch, cap, 0, 0, make_geom(cfg),
+                             pooled_shard, dev_err, (cudaStream_t)stream, Pages(), block_lo),
+           "shard pool build");
+  return QSA_OK;
+}
+
 qsa_status qsa_cp_select(const qsa_config* cfg, int batch, int n_q, int cap, int block_lo,
                          const int32_t* kv_len, const void* iq, const void* ik_shard,
                          const float* iw, float* pooled_shard, float* cand_score,
@@ -746,8 +767,8 @@ qsa_status qsa_pool_build(const qsa_config* cfg, int batch, int cap, const int32
   QSA_REQUIRE(kv_len, "kv_len");
   QSA_REQUIRE(ik_cache, "ik_cache");
   QSA_REQUIRE(pooled_cache, "pooled_cache");
-  QSA_CUDA(launch_pool_cache(cfg->dtype, ik_cache, kv_len, batch, cap, 0, 0, cfg->block_size,
-                             cfg->idx_dim, pooled_cache, dev_err, (cudaStream_t)stream),
+  QSA_CUDA(launch_pool_cache(cfg->dtype, ik_cache, kv_len, batch, cap, 0, 0, make_geom(cfg),
+                             pooled_cache, dev_err, (cudaStream_t)stream),
            "pool build");
   return QSA_OK;
 }
@@ -766,8 +787,8 @@ qsa_status qsa_pool_build_paged(const qsa_config* cfg, int batch, int max_blocks
   QSA_REQUIRE(kv_len, "kv_len");
   QSA_REQUIRE(ik_pages, "ik_pages");
   QSA_REQUIRE(pooled_cache, "pooled_cache");
-  QSA_CUDA(launch_pool_cache(cfg->dtype, ik_pages, kv_len, batch, cap, 0, 0, cfg->block_size,
-                             cfg->idx_dim, pooled_cache, dev_err, (cudaStream_t)stream,
+  QSA_CUDA(launch_pool_cache(cfg->dtype, ik_pages, kv_len, batch, cap, 0, 0, make_geom(cfg),
+                             pooled_cache, dev_err, (cudaStream_t)stream,
                              Pages{block_table, num_pages}),
            "pool build");
   return QSA_OK;

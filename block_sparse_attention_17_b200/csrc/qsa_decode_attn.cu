@@ -473,6 +473,8 @@ __device__ __forceinline__ void select_in_cluster(const DecParams& P, uint8_t* s
     }
   }
   __syncthreads();   // the caller staged iq_s and iw_s
+  if (g.rope_dim)     // query i turned at its position kv - n_q + i (read after the next barrier)
+    rope_rows(iq_s, n_q * Hi, Hi, kQStrideI, kv - n_q, g.rope_dim, g.rope_theta, tid, nthr);
   // blocks completed by this step's tokens (at most two: n_q <= 4 < B)
   const int jn_lo = max((kv - n_q) / g.B, j0), jn_hi = min(nc_last, j1);
   for (int j = jn_lo; j < jn_hi; ++j) {
@@ -485,7 +487,8 @@ __device__ __forceinline__ void select_in_cluster(const DecParams& P, uint8_t* s
     }
     float* dst = new_s + (j - jn_lo) * kDI;
     if (ok) {   // uniform across the CTA
-      pool_block_halves<__nv_bfloat16, kDI>(P.ik_cache + (ok ? r0 : 0) * kDI, g.B, dst, part);
+      pool_block_halves<__nv_bfloat16, kDI>(P.ik_cache + (ok ? r0 : 0) * kDI, g.B, dst, part,
+                                            g.rope_dim, g.rope_theta, j * g.B);
     } else {    // a page outside the pool (reported): the cached row stands
       for (int d = tid; d < kDI; d += nthr) dst[d] = P.pooled[((size_t)b * nblk_cap + j) * kDI + d];
     }

@@ -84,11 +84,12 @@ cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, si
 void set_last_error(const char* msg);
 
 cudaError_t launch_pool_prefill(qsa_dtype dt, const void* ik, const int* cu, int batch,
-                                int max_seqlen, int B, int di, float* pooled, int max_nblk,
+                                int max_seqlen, const Geom& g, float* pooled, int max_nblk,
                                 cudaStream_t st);
 cudaError_t launch_pool_cache(qsa_dtype dt, const void* ik_cache, const int* kv_len, int batch,
-                              int cap, int n_q, int mode, int B, int di, float* pooled,
-                              int* dev_err, cudaStream_t st, Pages pg = Pages());
+                              int cap, int n_q, int mode, const Geom& g, float* pooled,
+                              int* dev_err, cudaStream_t st, Pages pg = Pages(),
+                              int block_lo = -1);
 size_t select_prefill_smem(const Geom& g, int nc_cap);
 // sched: one int the caller zeroed on the stream before the launch (the
 // kernel's work counter).

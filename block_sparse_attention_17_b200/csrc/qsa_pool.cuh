@@ -8,6 +8,24 @@
 
 namespace qsa {
 
+// Warp 0's last step of a pooling: the eight partial sums of lane l's dims
+// (2l, 2l + 1) combined in a fixed tree, scaled by 1/B, turned by the indexer
+// rotary embedding when rope_dim > 0, and stored (lanes with active set).
+__device__ __forceinline__ void pool_finish(float2 (*part)[32], int lane, bool active, int B,
+                                            float* dst, int rope_dim, float rope_theta, int pos) {
+  float sx = 0.f, sy = 0.f;
+  if (active) {
+    float2 q[8];
+#pragma unroll
+    for (int w = 0; w < 8; ++w) q[w] = part[w][lane];
+    const float inv = 1.0f / (float)B;
+    sx = (((q[0].x + q[1].x) + (q[2].x + q[3].x)) + ((q[4].x + q[5].x) + (q[6].x + q[7].x))) * inv;
+    sy = (((q[0].y + q[1].y) + (q[2].y + q[3].y)) + ((q[4].y + q[5].y) + (q[6].y + q[7].y))) * inv;
+  }
+  if (rope_dim > 0) rope_lane_pair(sx, sy, lane, pos, rope_dim, rope_theta);
+  if (active) *reinterpret_cast<float2*>(dst + 2 * lane) = make_float2(sx, sy);
+}
+
 template <typename T>
 __device__ __forceinline__ float2 load_pair(const T* p);
 template <>
@@ -25,10 +43,13 @@ __device__ __forceinline__ float2 load_pair<__nv_bfloat16>(const __nv_bfloat16* 
 // nwarps is: eight partial sums, partial v over rows v, v + 8, v + 16, ... in
 // ascending order (lane l owns dims 2l and 2l + 1), combined in the tree
 // ((p0 + p1) + (p2 + p3)) + ((p4 + p5) + (p6 + p7)) and scaled by 1/B (B is a
-// power of two). part: 8 x 32 float2 of shared memory.
+// power of two). With rope_dim > 0 the mean is then turned at position `pos`
+// (the block's first token) by rope_lane_pair. part: 8 x 32 float2 of shared
+// memory.
 template <typename T>
 __device__ __forceinline__ void pool_block(const T* __restrict__ rows, int B, int di,
-                                           float* dst, float2 (*part)[32], int nwarps) {
+                                           float* dst, float2 (*part)[32], int nwarps,
+                                           int rope_dim = 0, float rope_theta = 0.f, int pos = 0) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool active = 2 * lane < di;
   for (int v = warp; v < 8; v += nwarps) {
@@ -51,15 +72,7 @@ __device__ __forceinline__ void pool_block(const T* __restrict__ rows, int B, in
     part[v][lane] = acc;
   }
   __syncthreads();
-  if (warp == 0 && active) {
-    float2 q[8];
-#pragma unroll
-    for (int w = 0; w < 8; ++w) q[w] = part[w][lane];
-    const float inv = 1.0f / (float)B;
-    const float sx = ((q[0].x + q[1].x) + (q[2].x + q[3].x)) + ((q[4].x + q[5].x) + (q[6].x + q[7].x));
-    const float sy = ((q[0].y + q[1].y) + (q[2].y + q[3].y)) + ((q[4].y + q[5].y) + (q[6].y + q[7].y));
-    *reinterpret_cast<float2*>(dst + 2 * lane) = make_float2(sx * inv, sy * inv);
-  }
+  if (warp == 0) pool_finish(part, lane, active, B, dst, rope_dim, rope_theta, pos);
 }
 
 }  // namespace qsa
@@ -72,7 +85,8 @@ namespace qsa {
 // as pool_block, so both write identical bits.
 template <typename T, int kDI>
 __device__ __forceinline__ void pool_block_halves(const T* __restrict__ rows, int B, float* dst,
-                                                  float2 (*part)[32]) {
+                                                  float2 (*part)[32], int rope_dim = 0,
+                                                  float rope_theta = 0.f, int pos = 0) {
   static_assert(kDI == 32 || kDI == 64, "indexer dim");
   constexpr int kPer = kDI / 16;                  // dims per lane: 2 or 4
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -103,15 +117,7 @@ __device__ __forceinline__ void pool_block_halves(const T* __restrict__ rows, in
     for (int d = 0; d < kPer; d += 2) part[v][(kPer * l + d) / 2] = make_float2(acc[d], acc[d + 1]);
   }
   __syncthreads();
-  if (warp == 0 && 2 * lane < kDI) {
-    float2 q[8];
-#pragma unroll
-    for (int w = 0; w < 8; ++w) q[w] = part[w][lane];
-    const float inv = 1.0f / (float)B;
-    const float sx = ((q[0].x + q[1].x) + (q[2].x + q[3].x)) + ((q[4].x + q[5].x) + (q[6].x + q[7].x));
-    const float sy = ((q[0].y + q[1].y) + (q[2].y + q[3].y)) + ((q[4].y + q[5].y) + (q[6].y + q[7].y));
-    *reinterpret_cast<float2*>(dst + 2 * lane) = make_float2(sx * inv, sy * inv);
-  }
+  if (warp == 0) pool_finish(part, lane, 2 * lane < kDI, B, dst, rope_dim, rope_theta, pos);
 }
 
 }  // namespace qsa

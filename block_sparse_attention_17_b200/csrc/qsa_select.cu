@@ -26,22 +26,23 @@ constexpr int kPoolThreads = 256;
 
 template <typename T>
 __device__ __forceinline__ void pool_block_cta(const T* __restrict__ rows, int B, int di,
-                                               float* __restrict__ dst) {
+                                               float* __restrict__ dst, int rope_dim,
+                                               float rope_theta, int pos) {
   __shared__ float2 part[8][32];
-  pool_block<T>(rows, B, di, dst, part, kPoolThreads / 32);
+  pool_block<T>(rows, B, di, dst, part, kPoolThreads / 32, rope_dim, rope_theta, pos);
 }
 
 // Grid (blocks of the longest sequence, batch).
 template <typename T>
 __global__ void __launch_bounds__(kPoolThreads)
 pool_prefill_kernel(const T* __restrict__ ik, const int* __restrict__ cu, int B, int di,
-                    float* __restrict__ pooled, int max_nblk) {
+                    float* __restrict__ pooled, int max_nblk, int rope_dim, float rope_theta) {
   grid_dependents_launch();   // the selection kernel may start its prologue
   const int b = blockIdx.y, j = blockIdx.x;
   const int s0 = cu[b], L = cu[b + 1] - s0;
   if (j >= L / B) return;
   pool_block_cta(ik + ((size_t)s0 + (size_t)j * B) * di, B, di,
-                 pooled + ((size_t)b * max_nblk + j) * di);
+                 pooled + ((size_t)b * max_nblk + j) * di, rope_dim, rope_theta, j * B);
 }
 
 // mode 0: rebuild every complete block; mode 1: only the blocks completed by
@@ -50,9 +51,11 @@ template <typename T>
 __global__ void __launch_bounds__(kPoolThreads)
 pool_cache_kernel(const T* __restrict__ ik_cache, const int* __restrict__ kv_len, int cap,
                   int n_q, int mode, int B, int di, float* __restrict__ pooled, int* dev_err,
-                  Pages pg) {
+                  Pages pg, int rope_dim, float rope_theta, int block_lo) {
   const int b = blockIdx.y;
-  const int kv = kv_len[b];
+  // block_lo >= 0: a context-parallel shard starting at that block, kv_len
+  // the full lengths (the shard holds the clamped remainder)
+  const int kv = block_lo >= 0 ? min(max(kv_len[b] - block_lo * B, 0), cap) : kv_len[b];
   if (kv < (mode ? n_q : 0) || kv > cap) {
     if (dev_err && threadIdx.x == 0 && blockIdx.x == 0) atomicExch(dev_err, 1);
     return;
@@ -69,7 +72,8 @@ pool_cache_kernel(const T* __restrict__ ik_cache, const int* __restrict__ kv_len
     }
     row0 = (size_t)page * B;
   }
-  pool_block_cta(ik_cache + row0 * di, B, di, pooled + ((size_t)b * (cap / B) + j) * di);
+  pool_block_cta(ik_cache + row0 * di, B, di, pooled + ((size_t)b * (cap / B) + j) * di, rope_dim,
+                 rope_theta, (j + max(block_lo, 0)) * B);
 }
 
 // ----------------------------------------------------------------- top-k
@@ -283,6 +287,10 @@ select_prefill_kernel(Geom g, const int* __restrict__ cu, int batch, int n_group
         }
         for (int e = tid; e < kQc * Hi; e += kSelThreadsPrefill)
           iw_s[e] = e < nq * Hi ? iw[((size_t)s0 + p0) * Hi + e] : 0.f;
+      }
+      if (g.rope_dim) {   // query p0 + q turned at its position (read after the chunk barrier)
+        __syncthreads();
+        rope_rows(iq_s, nq * Hi, Hi, kDI, p0, g.rope_dim, g.rope_theta, tid, kSelThreadsPrefill);
       }
 
       grid_dependency_wait();   // pooled rows come from the pooling kernel
@@ -595,7 +603,8 @@ decode_select_kernel(Geom g, int n_q, int cap, const int* __restrict__ kv_len,
       row0 = (page >= 0 && page < pg.num_pages) ? (size_t)page * g.B : SIZE_MAX;
     }
     if (row0 != SIZE_MAX)   // uniform across the CTA
-      pool_block_cta(ik_cache + row0 * kDI, g.B, kDI, pooled + ((size_t)b * nblk_cap + j) * kDI);
+      pool_block_cta(ik_cache + row0 * kDI, g.B, kDI, pooled + ((size_t)b * nblk_cap + j) * kDI,
+                     g.rope_dim, g.rope_theta, (j + (cp.on ? cp.block_lo : 0)) * g.B);
     __syncthreads();
   }
   // 2. stage the range's pooled rows and the queries' indexer q / weights
@@ -636,6 +645,11 @@ decode_select_kernel(Geom g, int n_q, int cap, const int* __restrict__ kv_len,
     }
   }
   __syncthreads();
+  if (g.rope_dim) {   // query i turned at its position kv_len - n_q + i
+    rope_rows(iq_s, n_q * g.Hi, g.Hi, kDI, kv_len[b] - n_q, g.rope_dim, g.rope_theta, threadIdx.x,
+              blockDim.x);
+    __syncthreads();
+  }
   // scores: one (query, block, head) triple per thread; heads are adjacent
   // lanes (Hi divides 32), so the weighted relu terms are summed by shuffles
   const int per_q = kPart * g.Hi;
@@ -726,37 +740,40 @@ decode_select_kernel(Geom g, int n_q, int cap, const int* __restrict__ kv_len,
 // ------------------------------------------------------------ launchers
 template <typename T>
 static cudaError_t launch_pool_prefill_t(const void* ik, const int* cu, int batch, int max_seqlen,
-                                         int B, int di, float* pooled, int max_nblk,
+                                         const Geom& g, float* pooled, int max_nblk,
                                          cudaStream_t st) {
-  const int nblk = max_seqlen / B;
+  const int nblk = max_seqlen / g.B;
   if (nblk == 0 || batch == 0) return cudaSuccess;
-  pool_prefill_kernel<T><<<dim3(nblk, batch), kPoolThreads, 0, st>>>((const T*)ik, cu, B, di,
-                                                                     pooled, max_nblk);
+  pool_prefill_kernel<T><<<dim3(nblk, batch), kPoolThreads, 0, st>>>(
+      (const T*)ik, cu, g.B, g.di, pooled, max_nblk, g.rope_dim, g.rope_theta);
   note_launch();
   return cudaGetLastError();
 }
 
 cudaError_t launch_pool_prefill(qsa_dtype dt, const void* ik, const int* cu, int batch,
-                                int max_seqlen, int B, int di, float* pooled, int max_nblk,
+                                int max_seqlen, const Geom& g, float* pooled, int max_nblk,
                                 cudaStream_t st) {
   return dt == QSA_BF16
-             ? launch_pool_prefill_t<__nv_bfloat16>(ik, cu, batch, max_seqlen, B, di, pooled,
+             ? launch_pool_prefill_t<__nv_bfloat16>(ik, cu, batch, max_seqlen, g, pooled,
                                                     max_nblk, st)
-             : launch_pool_prefill_t<float>(ik, cu, batch, max_seqlen, B, di, pooled, max_nblk, st);
+             : launch_pool_prefill_t<float>(ik, cu, batch, max_seqlen, g, pooled, max_nblk, st);
 }
 
 cudaError_t launch_pool_cache(qsa_dtype dt, const void* ik_cache, const int* kv_len, int batch,
-                              int cap, int n_q, int mode, int B, int di, float* pooled,
-                              int* dev_err, cudaStream_t st, Pages pg) {
+                              int cap, int n_q, int mode, const Geom& g, float* pooled,
+                              int* dev_err, cudaStream_t st, Pages pg, int block_lo) {
+  const int B = g.B, di = g.di;
   const int span = mode ? (n_q + B - 1) / B + 1 : cap / B;
   if (batch == 0 || span == 0) return cudaSuccess;
   dim3 grid(span, batch);
   if (dt == QSA_BF16)
     pool_cache_kernel<__nv_bfloat16><<<grid, kPoolThreads, 0, st>>>(
-        (const __nv_bfloat16*)ik_cache, kv_len, cap, n_q, mode, B, di, pooled, dev_err, pg);
+        (const __nv_bfloat16*)ik_cache, kv_len, cap, n_q, mode, B, di, pooled, dev_err, pg,
+        g.rope_dim, g.rope_theta, block_lo);
   else
     pool_cache_kernel<float><<<grid, kPoolThreads, 0, st>>>((const float*)ik_cache, kv_len, cap,
-                                                            n_q, mode, B, di, pooled, dev_err, pg);
+                                                            n_q, mode, B, di, pooled, dev_err, pg,
+                                                            g.rope_dim, g.rope_theta, block_lo);
   note_launch();
   return cudaGetLastError();
 }

@@ -59,6 +59,8 @@ class Workload:
     n_q: int = 0
     cap: int = 0                 # cache rows per sequence (0 => kv_len rounded up to B)
     gate_headwise: bool = False
+    rope_dim: int = 0            # indexer rotary embedding (0 = off)
+    rope_theta: float = 10000.0
     description: str = ""
 
     @property

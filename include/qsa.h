@@ -74,6 +74,20 @@ typedef struct {
   float index_scale;   /* indexer score scale c; 0 => idx_dim^-0.5 */
   int gate_headwise;   /* 0: gate [.., Hq, D] elementwise; 1: gate [.., Hq] */
   qsa_dtype dtype;     /* dtype of q, k, v, iq, ik, gate, out */
+  /* Indexer rotary embedding (llama.cpp PR #27739 page, QSA block-composition
+   * commit text: the indexer scores the roped query against pooled keys that
+   * take the same rope angles; instagit MTPLX page, "Multidimensional Rotary
+   * Embeddings (M-RoPE)": for text it is the ordinary partial rotary
+   * embedding). rope_dim = 0 turns it off. Otherwise the first rope_dim dims
+   * (a multiple of 4, <= idx_dim) of every indexer query and pooled key are
+   * turned in pairs (f, f + rope_dim/2) by the fp32 angle pos * fp32(rope_theta
+   * ^ (-2f / rope_dim)): an indexer query at its own position (its token index
+   * in the sequence), the pooled key of block j at position j * B. The caches
+   * hold the raw indexer keys; the pooled-key cache and pooled_out hold the
+   * turned means. Every call that pools or scores must be given the same two
+   * values. */
+  int rope_dim;
+  float rope_theta;    /* > 0 when rope_dim > 0 */
 } qsa_config;
 
 /* Human-readable name of a status code (static storage). */
@@ -235,8 +249,8 @@ qsa_status qsa_decode_noalloc(const qsa_config* cfg, int batch, int n_q, int cap
  * [block_lo, block_lo + cap / B) holds cache rows [block_lo * B, block_lo * B
  * + cap) of every sequence at local rows 0 .. cap - 1: k_shard, v_shard
  * [batch, cap, Hkv, D], ik_shard [batch, cap, di], pooled_shard
- * [batch, cap / B, di] (the shard's pooled keys, as qsa_pool_build writes them
- * for the shard). kv_len [batch] are the sequences' FULL lengths after this
+ * [batch, cap / B, di] (the shard's pooled keys, as qsa_cp_pool_build writes
+ * them). kv_len [batch] are the sequences' FULL lengths after this
  * step's n_q tokens were appended (to the shard that holds those rows); a
  * shard may hold none, some or all of a sequence's visible rows. One step:
  *   1. qsa_cp_select on every process: pools the shard's blocks completed by
@@ -265,6 +279,17 @@ qsa_status qsa_cp_select(const qsa_config* cfg, int batch, int n_q, int cap, int
                          int32_t* cand_id, int32_t* dev_err, void* workspace,
                          size_t workspace_bytes, void* stream);
 
+/* qsa_cp_pool_build: (re)builds pooled_shard [batch, cap / B, di] from
+ * ik_shard for every block of the shard that is complete under kv_len [batch]
+ * (FULL lengths, as for qsa_cp_select: the shard holds min(max(kv_len -
+ * block_lo * B, 0), cap) of a sequence's rows). The same bits as qsa_pool_build
+ * of the whole cache, rows [block_lo, block_lo + cap / B); with the indexer
+ * rotary embedding, block j of the shard turns at its global position
+ * (block_lo + j) * B. Rows of blocks that are not complete are not written. */
+qsa_status qsa_cp_pool_build(const qsa_config* cfg, int batch, int cap, int block_lo,
+                             const int32_t* kv_len, const void* ik_shard, float* pooled_shard,
+                             int32_t* dev_err, void* stream);
+
 /* qsa_cp_global_topk: cand_score / cand_id [world, batch, n_q, k] gathered
  * from every process; writes sel [batch, n_q, k + 1] (global ids of the
  * selected complete blocks in ascending order, then the query's tail block
@@ -281,7 +306,7 @@ qsa_status qsa_cp_global_topk(const qsa_config* cfg, int batch, int n_q, int wor
  * fp32 receives the gated partial output and part_lse [batch, n_q, Hq] fp32
  * its natural-log sum-exp (-inf and 0 where the shard holds none of the
  * query's keys). Workspace as qsa_cp_select. Every geometry qsa_decode
- * supports; bf16 with head_dim 128 and n_q * (Hq / Hkv) <= 16 runs on the
+ * supports; bf16 with head_dim 128 and n_q * (Hq / Hkv) <= 32 runs on the
  * tensor-map kernel, the rest on the CUDA-core kernels. */
 qsa_status qsa_cp_attend(const qsa_config* cfg, int batch, int n_q, int cap, int block_lo,
                          const int32_t* kv_len, const void* q, const void* k_shard,

@@ -40,7 +40,7 @@ def test_library_exports_every_declared_symbol():
     for s in syms:
         assert hasattr(lib, s), s
     assert set(syms) == set(_lib.EXPORTED)
-    assert lib.qsa_version() == 100
+    assert lib.qsa_version() == 101
 
 
 def test_status_strings():
@@ -85,6 +85,11 @@ def call_prefill(c, T=8192, ws_bytes=None, ptrs=None, batch=1, max_seqlen=8192):
     (dict(idx_dim=48), _lib.QSA_ERR_UNSUPPORTED),
     (dict(budget=64 * 65), _lib.QSA_ERR_UNSUPPORTED),         # k > 64
     (dict(num_q_heads=34, num_kv_heads=2), _lib.QSA_ERR_UNSUPPORTED),   # G > 16
+    (dict(rope_dim=6, rope_theta=1e4), _lib.QSA_ERR_INVALID_ARG),         # not a multiple of 4
+    (dict(rope_dim=128, rope_theta=1e4), _lib.QSA_ERR_INVALID_ARG),       # > idx_dim
+    (dict(rope_dim=-4, rope_theta=1e4), _lib.QSA_ERR_INVALID_ARG),
+    (dict(rope_dim=32, rope_theta=0.0), _lib.QSA_ERR_INVALID_ARG),
+    (dict(rope_dim=32, rope_theta=float("nan")), _lib.QSA_ERR_INVALID_ARG),
 ])
 def test_prefill_rejects_bad_config(kw, code):
     assert call_prefill(cfg(**kw)) == code

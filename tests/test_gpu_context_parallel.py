@@ -30,8 +30,7 @@ def _emulated_cp(cfg, w, d, world):
     for b0, b1 in shards:
         # the shard's pooled rows hold the blocks completed before this step
         ik = rows(d["ik_cache"], b0, b1)
-        kv_prev = torch.clamp(kv - w.n_q - b0 * B, 0, (b1 - b0) * B).to(torch.int32)
-        pooled = qsa.pool_build(cfg, ik, kv_prev)
+        pooled = qsa.cp_pool_build(cfg, ik, (kv - w.n_q).to(torch.int32), b0)
         f = cp.library_fns(cfg, d["q"], rows(d["k_cache"], b0, b1), rows(d["v_cache"], b0, b1),
                            d["iq"], ik, d["iw"], d["gate"], pooled, b0)
         fns.append(f)
@@ -44,17 +43,28 @@ def _emulated_cp(cfg, w, d, world):
     return merged, glob
 
 
-@pytest.mark.parametrize("world,n_q,dtype", [(2, 1, "bf16"), (3, 1, "bf16"), (4, 2, "bf16"),
-                                             (3, 1, "f32"), (2, 3, "bf16")])
-def test_context_parallel_decode_emulated_ranks(world, n_q, dtype):
+@pytest.mark.parametrize("world,n_q,dtype,rope_dim", [
+    (2, 1, "bf16", 0), (3, 1, "bf16", 0), (4, 2, "bf16", 0), (3, 1, "f32", 0), (2, 3, "bf16", 0),
+    (3, 1, "bf16", 64), (2, 2, "f32", 32)])
+def test_context_parallel_decode_emulated_ranks(world, n_q, dtype, rope_dim):
+    # rope_dim > 0: the indexer rotary embedding, where every shard must turn its
+    # pooled rows at their global block positions
     w = WORKLOADS["decode_bf16_b32_kv32768"].with_(batch=4, cap=64 * 120, kv_len=64 * 120,
-                                                   n_q=n_q, dtype=dtype)
+                                                   n_q=n_q, dtype=dtype, rope_dim=rope_dim,
+                                                   rope_theta=10000.0)
     # full, ragged, ending inside an early shard, and a short one
     kv = np.array([64 * 120, 64 * 117 + 5, 64 * 37 + 63, 200], np.int32)
     inp = make_decode_inputs(w, kv_lens=kv)
     cfg = qsa.QSAConfig.from_workload(w)
     d = TL.upload(inp, w)
     pooled = qsa.pool_build(cfg, d["ik_cache"], (d["kv_len"] - n_q).to(torch.int32))
+    # each shard's pool build gives the whole cache's rows, bit for bit
+    B, nblk = w.block_size, w.cap // w.block_size
+    for r in range(world):
+        b0, b1 = cp.shard_blocks(nblk, world, r)
+        ps = qsa.cp_pool_build(cfg, d["ik_cache"][:, b0 * B:b1 * B].contiguous(),
+                               (d["kv_len"] - n_q).to(torch.int32), b0)
+        assert torch.equal(ps, pooled[:, b0:b1]), r
     ref = qsa.decode(cfg, d["q"], d["k_cache"], d["v_cache"], d["iq"], d["ik_cache"], d["iw"],
                      d["gate"], pooled, d["kv_len"], want_lse=True, want_sel=True)
     merged, glob = _emulated_cp(cfg, w, d, world)

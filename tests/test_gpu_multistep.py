@@ -50,15 +50,18 @@ def _prefill_pooled(cfg, w, d, b_lens, rng):
     return r["pooled"]
 
 
-@pytest.mark.parametrize("name,L,steps", [
+@pytest.mark.parametrize("name,L,steps,rope_dim", [
     # n_q = 1, B = 64: from 1277 and 700 tokens: blocks 19 and 20, blocks 10 and 11
-    ("decode_bf16_b32_kv32768", (1277, 700), 70),
+    ("decode_bf16_b32_kv32768", (1277, 700), 70, 0),
     # n_q = 2, B = 128: from 2301 and 1020 tokens, 2 tokens a step: blocks 17
     # and 18, blocks 7 and 8
-    ("mtp_verify_bf16_b4_kv262144", (2301, 1020), 70),
+    ("mtp_verify_bf16_b4_kv262144", (2301, 1020), 70, 0),
+    # with the indexer rotary embedding (pooled rows turned at their blocks'
+    # positions by the prefill, the steps and the rebuild alike)
+    ("decode_bf16_b32_kv32768", (1277, 700), 70, 64),
 ])
-def test_prefill_then_decode_steps_keep_the_side_cache(name, L, steps):
-    w0 = WORKLOADS[name]
+def test_prefill_then_decode_steps_keep_the_side_cache(name, L, steps, rope_dim):
+    w0 = WORKLOADS[name].with_(rope_dim=rope_dim, rope_theta=1e4)
     n_q = w0.n_q
     cap = ((max(L) + steps * n_q) // w0.block_size + 1) * w0.block_size
     w = w0.with_(batch=len(L), kv_len=cap, cap=cap)
