@@ -29,7 +29,7 @@ EXPORTED = [
     "qsa_pool_build", "qsa_decode_noalloc", "qsa_decode_paged", "qsa_pool_build_paged",
     "qsa_decode_fp8", "qsa_decode_attend",
     "qsa_cp_select", "qsa_cp_global_topk", "qsa_cp_attend", "qsa_cp_merge",
-    "qsa_cp_pool_build",
+    "qsa_cp_pool_build", "qsa_append",
 ]
 
 
@@ -94,6 +94,9 @@ def _declare(lib):
         "qsa_cp_select": (I, [CFG, I, I, I, I] + [P] * 9 + [SZ, P]),
         # cfg, batch, cap, block_lo, kv_len, ik_shard, pooled_shard, dev_err, stream
         "qsa_cp_pool_build": (I, [CFG, I, I, I, P, P, P, P, P]),
+        # cfg, batch, n_q, cap, kv_len, k_new, v_new, ik_new, k_cache, v_cache, ik_cache,
+        # pooled_cache, block_table, num_pages, dev_err, stream
+        "qsa_append": (I, [CFG, I, I, I] + [P] * 9 + [I, P, P]),
         # cfg, batch, n_q, world, kv_len, cand_score, cand_id, sel, nsel, stream
         "qsa_cp_global_topk": (I, [CFG, I, I, I] + [P] * 6),
         # cfg, batch, n_q, cap, block_lo, kv_len, q, k, v, gate, sel, nsel, part_out,

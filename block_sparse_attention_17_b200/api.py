@@ -367,6 +367,46 @@ def pool_build(cfg: QSAConfig, ik_cache, kv_len, pooled_cache=None, *, dev_err=N
     return pooled_cache
 
 
+def append(cfg: QSAConfig, ik_new, ik_cache, pooled_cache, kv_len, *, k_new=None, v_new=None,
+           k_cache=None, v_cache=None, block_table=None, dev_err=None, stream=None) -> None:
+    """Indexer front end of a decode step (qsa_append): writes the step's new
+    rows (ik_new [batch, n_q, di]; k_new / v_new [batch, n_q, Hkv, D], optional)
+    at positions kv_len - n_q .. kv_len - 1 of the caches and pools the blocks
+    they complete into pooled_cache, in one launch. block_table [batch,
+    max_blocks] int32 selects paged caches ([num_pages, B, ...])."""
+    dt = cfg.dtype
+    batch, n_q = ik_new.shape[0], ik_new.shape[1]
+    _need(ik_new, "ik_new", dt, (batch, n_q, cfg.idx_dim))
+    _need(kv_len, "kv_len", torch.int32, (batch,))
+    B = cfg.block_size
+    if block_table is not None:
+        _need(block_table, "block_table", torch.int32, (batch, block_table.shape[1]))
+        cap, num_pages = block_table.shape[1] * B, ik_cache.shape[0]
+        _need(ik_cache, "ik_cache", dt, (num_pages, B, cfg.idx_dim))
+        kv_shape = (num_pages, B, cfg.num_kv_heads, cfg.head_dim)
+    else:
+        cap, num_pages = ik_cache.shape[1], 0
+        _need(ik_cache, "ik_cache", dt, (batch, cap, cfg.idx_dim))
+        kv_shape = (batch, cap, cfg.num_kv_heads, cfg.head_dim)
+    _need(pooled_cache, "pooled_cache", torch.float32, (batch, cap // B, cfg.idx_dim))
+    if k_new is not None:
+        _need(k_new, "k_new", dt, (batch, n_q, cfg.num_kv_heads, cfg.head_dim))
+        _need(v_new, "v_new", dt, (batch, n_q, cfg.num_kv_heads, cfg.head_dim))
+        _need(k_cache, "k_cache", dt, kv_shape)
+        _need(v_cache, "v_cache", dt, kv_shape)
+    dev = ik_new.device
+    _one_device(dev, stream, ik_cache=ik_cache, pooled_cache=pooled_cache, kv_len=kv_len,
+                k_new=k_new, v_new=v_new, k_cache=k_cache, v_cache=v_cache,
+                block_table=block_table, dev_err=dev_err)
+    c = cfg.c()
+    with torch.cuda.device(dev):
+        st = _lib.lib().qsa_append(ctypes.byref(c), batch, n_q, cap, _ptr(kv_len), _ptr(k_new),
+                                   _ptr(v_new), _ptr(ik_new), _ptr(k_cache), _ptr(v_cache),
+                                   _ptr(ik_cache), _ptr(pooled_cache), _ptr(block_table),
+                                   num_pages, _ptr(dev_err), _stream(stream))
+        _lib.check(st, "qsa_append")
+
+
 def decode_paged(cfg: QSAConfig, q, k_pages, v_pages, iq, ik_pages, iw, gate, pooled_cache,
                  kv_len, block_table, *, out=None, lse=None, sel=None, nsel=None, dev_err=None,
                  workspace=None, want_lse=False, want_sel=False, stream=None) -> dict:

@@ -714,6 +714,34 @@ static qsa_status check_pages(const qsa_config* cfg, int max_blocks, const int32
   return QSA_OK;
 }
 
+qsa_status qsa_append(const qsa_config* cfg, int batch, int n_q, int cap, const int32_t* kv_len,
+                      const void* k_new, const void* v_new, const void* ik_new, void* k_cache,
+                      void* v_cache, void* ik_cache, float* pooled_cache,
+                      const int32_t* block_table, int num_pages, int32_t* dev_err, void* stream) {
+  g_err[0] = 0;
+  qsa_status s = check_decode_dims(cfg, batch, n_q, cap);
+  if (s != QSA_OK) return s;
+  if (block_table && (s = check_pages(cfg, cap / cfg->block_size, block_table, num_pages)) != QSA_OK)
+    return s;
+  if (batch == 0) return QSA_OK;
+  QSA_REQUIRE(kv_len, "kv_len");
+  QSA_REQUIRE(ik_new, "ik_new"); QSA_REQUIRE(ik_cache, "ik_cache");
+  QSA_REQUIRE(pooled_cache, "pooled_cache");
+  if ((k_new == nullptr) != (v_new == nullptr) || (k_new == nullptr) != (k_cache == nullptr) ||
+      (k_new == nullptr) != (v_cache == nullptr))
+    return fail(QSA_ERR_INVALID_ARG, "k_new, v_new, k_cache and v_cache are given together or not at all");
+  if (k_new) {
+    QSA_REQUIRE(k_new, "k_new"); QSA_REQUIRE(v_new, "v_new");
+    QSA_REQUIRE(k_cache, "k_cache"); QSA_REQUIRE(v_cache, "v_cache");
+  }
+  QSA_CUDA(launch_append(cfg->dtype, make_geom(cfg), batch, n_q, cap, kv_len, k_new, v_new, ik_new,
+                         k_cache, v_cache, ik_cache, pooled_cache, dev_err,
+                         block_table ? Pages{block_table, num_pages} : Pages(),
+                         (cudaStream_t)stream),
+           "append");
+  return QSA_OK;
+}
+
 qsa_status qsa_decode_paged(const qsa_config* cfg, int batch, int n_q, int max_blocks,
                             const int32_t* block_table, int num_pages, const int32_t* kv_len,
                             const void* q, const void* k_pages, const void* v_pages,

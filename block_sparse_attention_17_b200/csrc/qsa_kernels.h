@@ -90,6 +90,12 @@ cudaError_t launch_pool_cache(qsa_dtype dt, const void* ik_cache, const int* kv_
                               int cap, int n_q, int mode, const Geom& g, float* pooled,
                               int* dev_err, cudaStream_t st, Pages pg = Pages(),
                               int block_lo = -1);
+// Appends the step's new K / V (optional: k_new == nullptr) and indexer-key
+// rows and pools the blocks they complete (one launch).
+cudaError_t launch_append(qsa_dtype dt, const Geom& g, int batch, int n_q, int cap,
+                          const int* kv_len, const void* k_new, const void* v_new,
+                          const void* ik_new, void* k_cache, void* v_cache, void* ik_cache,
+                          float* pooled, int* dev_err, Pages pg, cudaStream_t st);
 size_t select_prefill_smem(const Geom& g, int nc_cap);
 // sched: one int the caller zeroed on the stream before the launch (the
 // kernel's work counter).

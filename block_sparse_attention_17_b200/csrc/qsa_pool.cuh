@@ -44,12 +44,16 @@ __device__ __forceinline__ float2 load_pair<__nv_bfloat16>(const __nv_bfloat16* 
 // ascending order (lane l owns dims 2l and 2l + 1), combined in the tree
 // ((p0 + p1) + (p2 + p3)) + ((p4 + p5) + (p6 + p7)) and scaled by 1/B (B is a
 // power of two). With rope_dim > 0 the mean is then turned at position `pos`
-// (the block's first token) by rope_lane_pair. part: 8 x 32 float2 of shared
+// (the block's first token) by rope_lane_pair. Rows r >= split come from
+// new_rows[r - split] instead of rows[r] (a block completed by rows that are
+// not in the cache yet); the sums are the same. part: 8 x 32 float2 of shared
 // memory.
 template <typename T>
 __device__ __forceinline__ void pool_block(const T* __restrict__ rows, int B, int di,
                                            float* dst, float2 (*part)[32], int nwarps,
-                                           int rope_dim = 0, float rope_theta = 0.f, int pos = 0) {
+                                           int rope_dim = 0, float rope_theta = 0.f, int pos = 0,
+                                           const T* __restrict__ new_rows = nullptr,
+                                           int split = 1 << 30) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool active = 2 * lane < di;
   for (int v = warp; v < 8; v += nwarps) {
@@ -59,8 +63,11 @@ __device__ __forceinline__ void pool_block(const T* __restrict__ rows, int B, in
         float2 x[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u)
-          x[u] = i0 + 8 * u < B ? load_pair<T>(rows + (size_t)(i0 + 8 * u) * di + 2 * lane)
-                                : make_float2(0.f, 0.f);
+          x[u] = i0 + 8 * u < B
+                     ? load_pair<T>((i0 + 8 * u < split ? rows + (size_t)(i0 + 8 * u) * di
+                                                        : new_rows + (size_t)(i0 + 8 * u - split) * di) +
+                                    2 * lane)
+                     : make_float2(0.f, 0.f);
 #pragma unroll
         for (int u = 0; u < 8; ++u)
           if (i0 + 8 * u < B) {

@@ -76,6 +76,70 @@ pool_cache_kernel(const T* __restrict__ ik_cache, const int* __restrict__ kv_len
                  rope_theta, (j + max(block_lo, 0)) * B);
 }
 
+// --------------------------------------------- append (indexer front end)
+// One CTA per sequence: writes the step's n_q new rows of K and V (optional)
+// and of the indexer keys into the caches at rows kv - n_q .. kv - 1 (kv the
+// post-append length), and in the same pass pools the blocks those rows
+// complete (with the indexer rotary embedding), reading the block's earlier
+// rows from the cache and its new rows from the inputs, in pool_block's order:
+// the same bits as the cache rebuild. Paged caches (pg.table): token p of
+// sequence b is row p % B of page table[b * (cap / B) + p / B].
+template <typename T>
+__global__ void __launch_bounds__(kPoolThreads)
+append_kernel(Geom g, int n_q, int cap, const int* __restrict__ kv_len, const T* __restrict__ k_new,
+              const T* __restrict__ v_new, const T* __restrict__ ik_new, T* __restrict__ k_cache,
+              T* __restrict__ v_cache, T* __restrict__ ik_cache, float* __restrict__ pooled,
+              int* dev_err, Pages pg) {
+  constexpr int kVec = 16 / sizeof(T);
+  const int b = blockIdx.x, tid = threadIdx.x;
+  const int kv = kv_len[b];
+  const int nblk_cap = cap / g.B;
+  if (kv < n_q || kv > cap) {
+    if (dev_err && tid == 0) atomicExch(dev_err, 1);
+    return;
+  }
+  const int p0 = kv - n_q;
+  // cache row of token p (-1: a page outside the pool, reported)
+  auto row_of = [&](int p) -> long long {
+    if (!pg.table) return (long long)b * cap + p;
+    const int page = pg.table[(size_t)b * nblk_cap + p / g.B];
+    if (page < 0 || page >= pg.num_pages) return -1;
+    return (long long)page * g.B + p % g.B;
+  };
+  const int kvr = g.Hkv * g.D / kVec, ikr = g.di / kVec;   // 16-byte vectors per token row
+  for (int e = tid; e < n_q * (ikr + (k_new ? 2 * kvr : 0)); e += blockDim.x) {
+    const int per = ikr + (k_new ? 2 * kvr : 0);
+    const int i = e / per, c = e - i * per;
+    const long long r = row_of(p0 + i);
+    if (r < 0) {
+      if (dev_err) atomicExch(dev_err, 3);
+      continue;
+    }
+    if (c < ikr) {
+      reinterpret_cast<uint4*>(ik_cache + r * g.di)[c] =
+          reinterpret_cast<const uint4*>(ik_new + ((size_t)b * n_q + i) * g.di)[c];
+    } else if (c < ikr + kvr) {
+      reinterpret_cast<uint4*>(k_cache + r * g.Hkv * g.D)[c - ikr] =
+          reinterpret_cast<const uint4*>(k_new + ((size_t)b * n_q + i) * g.Hkv * g.D)[c - ikr];
+    } else {
+      reinterpret_cast<uint4*>(v_cache + r * g.Hkv * g.D)[c - ikr - kvr] =
+          reinterpret_cast<const uint4*>(v_new + ((size_t)b * n_q + i) * g.Hkv * g.D)[c - ikr - kvr];
+    }
+  }
+  // blocks completed by the new rows (n_q < B: the new rows of block j start
+  // at split = p0 - j * B > 0)
+  for (int j = p0 / g.B; j < kv / g.B; ++j) {
+    const long long r0 = row_of(j * g.B);
+    if (r0 < 0) continue;   // uniform across the CTA; reported above or by the decode step
+    __shared__ float2 part[8][32];
+    const int split = p0 - j * g.B;
+    pool_block<T>(ik_cache + r0 * g.di, g.B, g.di, pooled + ((size_t)b * nblk_cap + j) * g.di, part,
+                  kPoolThreads / 32, g.rope_dim, g.rope_theta, j * g.B,
+                  ik_new + (size_t)b * n_q * g.di, split);
+    __syncthreads();
+  }
+}
+
 // ----------------------------------------------------------------- top-k
 __device__ __forceinline__ unsigned lanemask_lt() {
   unsigned m;
@@ -774,6 +838,24 @@ cudaError_t launch_pool_cache(qsa_dtype dt, const void* ik_cache, const int* kv_
     pool_cache_kernel<float><<<grid, kPoolThreads, 0, st>>>((const float*)ik_cache, kv_len, cap,
                                                             n_q, mode, B, di, pooled, dev_err, pg,
                                                             g.rope_dim, g.rope_theta, block_lo);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append(qsa_dtype dt, const Geom& g, int batch, int n_q, int cap,
+                          const int* kv_len, const void* k_new, const void* v_new,
+                          const void* ik_new, void* k_cache, void* v_cache, void* ik_cache,
+                          float* pooled, int* dev_err, Pages pg, cudaStream_t st) {
+  if (batch == 0) return cudaSuccess;
+  if (dt == QSA_BF16)
+    append_kernel<__nv_bfloat16><<<batch, kPoolThreads, 0, st>>>(
+        g, n_q, cap, kv_len, (const __nv_bfloat16*)k_new, (const __nv_bfloat16*)v_new,
+        (const __nv_bfloat16*)ik_new, (__nv_bfloat16*)k_cache, (__nv_bfloat16*)v_cache,
+        (__nv_bfloat16*)ik_cache, pooled, dev_err, pg);
+  else
+    append_kernel<float><<<batch, kPoolThreads, 0, st>>>(
+        g, n_q, cap, kv_len, (const float*)k_new, (const float*)v_new, (const float*)ik_new,
+        (float*)k_cache, (float*)v_cache, (float*)ik_cache, pooled, dev_err, pg);
   note_launch();
   return cudaGetLastError();
 }

@@ -384,6 +384,26 @@ qsa_status qsa_pool_build_paged(const qsa_config* cfg, int batch, int max_blocks
                                 const int32_t* kv_len, const void* ik_pages,
                                 float* pooled_cache, int32_t* dev_err, void* stream);
 
+/* Indexer front end of a decode step (one launch): writes the step's n_q new
+ * rows into the caches and, in the same pass, pools (and, with the indexer
+ * rotary embedding, turns) every block those rows complete, the bits of
+ * qsa_pool_build. Rows go to cache positions kv_len[b] - n_q + i (kv_len the
+ * post-append lengths, device [batch]); the block's earlier rows are read from
+ * the cache, its new rows from the inputs. Inputs: ik_new [batch, n_q, di];
+ * k_new, v_new [batch, n_q, Hkv, D] (both NULL: only the indexer keys are
+ * appended), all in cfg->dtype. Caches: block_table NULL: ik_cache
+ * [batch, cap, di], k_cache / v_cache [batch, cap, Hkv, D], pooled_cache
+ * [batch, cap / B, di] fp32; block_table [batch, cap / B] int32: paged caches
+ * of num_pages pages of B rows ([num_pages, B, di], [num_pages, B, Hkv, D]).
+ * A following qsa_decode (or its paged form) on the same lengths pools the same
+ * blocks again to the same bits (the write-back is idempotent). Errors: a
+ * length outside [n_q, cap] sets *dev_err to 1 and writes nothing for that
+ * sequence; a bad page id sets it to 3 and skips that row or block. */
+qsa_status qsa_append(const qsa_config* cfg, int batch, int n_q, int cap, const int32_t* kv_len,
+                      const void* k_new, const void* v_new, const void* ik_new, void* k_cache,
+                      void* v_cache, void* ik_cache, float* pooled_cache,
+                      const int32_t* block_table, int num_pages, int32_t* dev_err, void* stream);
+
 /* Rebuild the pooled-key cache of every complete block j < kv_len[b]/B from
  * the indexer-key cache (restore after a state reload). The rows it writes are
  * bit-identical to the ones the incremental decode path writes. */

@@ -215,3 +215,29 @@ def test_binding_refuses_tensors_on_another_device():
     with pytest.raises(ValueError, match="same GPU"):
         api._one_device(cuda0, None, q=torch.zeros(1))
     api._one_device(torch.device("cpu"), None, q=torch.zeros(1), k=None)
+
+
+@fake_pointers
+def test_append_rejects_bad_arguments():
+    lib = _lib.lib()
+    c = cfg()
+    P = FAKE
+    # K / V given without their caches
+    assert lib.qsa_append(ctypes.byref(c), 2, 1, 4096, P, P, P, P, None, None, P, P, None, 0,
+                          None, None) == _lib.QSA_ERR_INVALID_ARG
+    # no indexer rows
+    assert lib.qsa_append(ctypes.byref(c), 2, 1, 4096, P, None, None, None, None, None, P, P, None,
+                          0, None, None) == _lib.QSA_ERR_INVALID_ARG
+    # misaligned pooled cache, cap not a multiple of B, n_q past the limit
+    assert lib.qsa_append(ctypes.byref(c), 2, 1, 4096, P, None, None, P, None, None, P, MISALIGNED,
+                          None, 0, None, None) == _lib.QSA_ERR_INVALID_ARG
+    assert lib.qsa_append(ctypes.byref(c), 2, 1, 4000, P, None, None, P, None, None, P, P, None, 0,
+                          None, None) == _lib.QSA_ERR_INVALID_ARG
+    assert lib.qsa_append(ctypes.byref(c), 2, 5, 4096, P, None, None, P, None, None, P, P, None, 0,
+                          None, None) == _lib.QSA_ERR_UNSUPPORTED
+    # a block table with no pages
+    assert lib.qsa_append(ctypes.byref(c), 2, 1, 4096, P, None, None, P, None, None, P, P, P, 0,
+                          None, None) == _lib.QSA_ERR_INVALID_ARG
+    # an empty batch launches nothing
+    assert lib.qsa_append(ctypes.byref(c), 0, 1, 4096, None, None, None, None, None, None, None,
+                          None, None, 0, None, None) == _lib.QSA_OK
