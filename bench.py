@@ -703,7 +703,11 @@ def run_ours(args, rank, world, dist):
     import torch
     local = int(os.environ.get("LOCAL_RANK", "0"))
     peaks, peak_kind = load_peaks()
-    head_w = rank_workload(WORKLOADS[args.workload], rank)
+    head_w = WORKLOADS[args.workload]
+    if args.seqlens:   # a smaller case of the prefill workload (profiling captures)
+        head_w = head_w.with_(seqlens=tuple(int(x) for x in args.seqlens.split(",")),
+                              ragged_range=None)
+    head_w = rank_workload(head_w, rank)
     dec_names = [] if args.decode in ("", "none") else [x for x in args.decode.split(",") if x]
     dec_ws = [rank_workload(WORKLOADS[n], rank) for n in dec_names]
     all_ws = [head_w] + dec_ws
@@ -840,6 +844,9 @@ def main():
                     help="seconds of the one-thread oracle sample per workload")
     ap.add_argument("--cpu-cores", type=int, default=0, help="0: every host core")
     ap.add_argument("--ref-step-seconds", type=float, default=2.0)
+    ap.add_argument("--seqlens", default="",
+                    help="prefill workload: comma-separated sequence lengths replacing the "
+                         "workload's (a smaller case for profiling captures)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

@@ -81,8 +81,10 @@ __device__ __forceinline__ void grid_dependents_launch() {
 // Embeddings (M-RoPE)": for text, the ordinary partial rotary embedding).
 // Frequency f < rope_dim / 2 turns the pair (x[f], x[f + rope_dim / 2]) by the
 // fp32 product of the position and fp32(theta^(-2f / rope_dim)); the power is
-// taken in double precision so that its fp32 rounding is the correct one.
-__device__ __forceinline__ float2 rope_cos_sin(int f, int pos, int rope_dim, float theta) {
+// taken in double precision so that its fp32 rounding is the correct one. The
+// rotary helpers are kept out of line: the kernels that carry them run them
+// only when rope_dim > 0, and their code stays out of the hot paths' fetch.
+static __device__ __noinline__ float2 rope_cos_sin(int f, int pos, int rope_dim, float theta) {
   const float inv = (float)pow((double)theta, -2.0 * f / rope_dim);
   const float a = __fmul_rn((float)pos, inv);
   float s, c;
@@ -101,7 +103,7 @@ __device__ __forceinline__ void rope_turn(float& lo, float& hi, float2 cs) {
 // Rotates nrows rows of shared memory in place: row r starts at base + r *
 // stride and belongs to query r / per_q, whose position is pos0 + r / per_q.
 // All threads of the CTA call it (tid, nthr); the caller synchronises around it.
-__device__ __forceinline__ void rope_rows(float* base, int nrows, int per_q, int stride, int pos0,
+static __device__ __noinline__ void rope_rows(float* base, int nrows, int per_q, int stride, int pos0,
                                           int rope_dim, float theta, int tid, int nthr) {
   const int hp = rope_dim >> 1;
   for (int e = tid; e < nrows * hp; e += nthr) {
@@ -114,7 +116,7 @@ __device__ __forceinline__ void rope_rows(float* base, int nrows, int per_q, int
 // One warp holds a row two dims per lane (lane l: dims 2l and 2l + 1, as x and
 // y); turns its first rope_dim dims (rope_dim a multiple of 4) at `pos` with
 // rope_turn's roundings. Every lane of the warp calls it.
-__device__ __forceinline__ void rope_lane_pair(float& x, float& y, int lane, int pos, int rope_dim,
+static __device__ __noinline__ void rope_lane_pair(float& x, float& y, int lane, int pos, int rope_dim,
                                                float theta) {
   const int qo = rope_dim >> 2;                 // lanes holding the first half
   const bool in = lane < 2 * qo;
