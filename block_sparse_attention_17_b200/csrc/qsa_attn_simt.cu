@@ -11,8 +11,8 @@
 // Decode: split-KV over the union of the n_q new queries' selected blocks.
 // One CTA per (sequence, KV head, split) writes partial (m, l, O) for every
 // query row of the group; qsa_combine merges the splits by log-sum-exp and
-// applies the sigmoid output gate (llama.cpp PR #27739 page: sigmoid output
-// gate).
+// applies the sigmoid gate on the output (llama.cpp PR #27739 page, QSA
+// block-composition commit text).
 #include "qsa_common.cuh"
 #include "qsa_kernels.h"
 

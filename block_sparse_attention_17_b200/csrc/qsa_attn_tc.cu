@@ -25,7 +25,7 @@
 //               softmax in the log2 domain with lazy rescaling (O is rescaled
 //               only when the running max grows by more than 2^8), write P as
 //               bf16 over S, and in the epilogue apply 1/l and the sigmoid
-//               gate (llama.cpp PR #27739 page: sigmoid output gate).
+//               gate (llama.cpp PR #27739 page, QSA block-composition commit text).
 // Every wait is bounded; a timeout sets the workspace error word and the CTA
 // unwinds (drains its TMA loads and MMAs, frees TMEM).
 #include "qsa_common.cuh"

@@ -16,7 +16,7 @@
 //     partials with their log-sum-exp) and the partials are all-gathered,
 //     cp_merge_kernel merges them: with M = max_r lse_r and
 //     w_r = exp(lse_r - M) / sum_r exp(lse_r - M), out = sum_r w_r out_r and
-//     lse = M + log sum_r exp(lse_r - M). The sigmoid output gate is
+//     lse = M + log sum_r exp(lse_r - M). The sigmoid gate on the output is
 //     elementwise, so it commutes with this weighted sum.
 #include <math.h>
 

@@ -24,7 +24,7 @@
 //     own online-softmax state (log2 domain), merged at the end into one
 //     (m, l, O) partial per row;
 //  4. the cluster merges the partials by log-sum-exp through distributed
-//     shared memory (each CTA takes some rows) and applies the sigmoid output
+//     shared memory (each CTA takes some rows) and applies the output's sigmoid
 //     gate; where such a cluster cannot be resident (two-launch path only), the
 //     partials go through global memory and the last CTA merges them.
 // kFp8 reads e4m3 K/V codes with per-row scales instead of bf16 rows.
@@ -1293,7 +1293,7 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
     // The cluster's CTAs merge the partials by log-sum-exp straight from each
     // other's shared memory: CTA `split` takes rows split, split + nsplit, ...,
     // and each of its threads four dims of one row (all partials' loads in
-    // flight at once), then applies the sigmoid output gate staged at the start.
+    // flight at once), then applies the sigmoid gate on the output staged at the start.
     cluster_sync_all();
     const int ns = P.nsplit;
     const uint32_t pml_s = sbase + kOffStages + (uint32_t)(kConsumers * 16 * kD + kConsumers * 16 * 2 + L::kRows * kD) * 4u;
@@ -1350,7 +1350,7 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
     return;
   }
   // the last CTA of this (sequence, KV head) merges the splits' partials by
-  // log-sum-exp and applies the sigmoid output gate
+  // log-sum-exp and applies the sigmoid gate on the output
   __threadfence();
   __syncthreads();
   __shared__ int last_s;

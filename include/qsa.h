@@ -14,7 +14,7 @@
  *   out[h]   = sigmoid(gate[h]) * softmax_{s in S}(scale * q[h] . k[s, h/G]) v[s, h/G]
  *
  * The indexer settings (per-head weights, no n_head scale, c = idx_dim^-0.5,
- * candidates = complete visible blocks) and the sigmoid output gate follow the
+ * candidates = complete visible blocks) and the sigmoid gate on the output follow the
  * QSA block-composition commit text on the llama.cpp PR #27739 page.
  *
  * Conventions for every entry point

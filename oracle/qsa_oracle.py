@@ -20,7 +20,7 @@ What QSA computes, as the pages state it:
 * llama.cpp PR #27739 page, the QSA block-composition commit text ("The value
   gate ..."): the indexer settings -- weights per head, n_head_scale = 1,
   softmax_scale = index_head_dim ** -0.5, candidate window end = kv_len / ratio
-  (complete blocks only) -- and the sigmoid output gate; worked example at
+  (complete blocks only) -- and the sigmoid gate on the output; worked example at
   kv_len 3002, budget 2048, ratio 4.
 * ramgpt "Porting Qwen4 to llama.cpp", sections "QSA Should First Be
   Implemented as Selection Semantics" (visible width bound
@@ -188,7 +188,7 @@ def visible_positions(n: int, block_size: int, selected: Sequence[int]) -> np.nd
 
 # --------------------------------------------------------------------------
 # step 5: gated GQA attention over a token set
-# (instagit MTPLX page: standard gated GQA; PR #27739 page: the sigmoid output gate)
+# (instagit MTPLX page: standard gated GQA; PR #27739 page: the sigmoid gate on the output)
 # --------------------------------------------------------------------------
 def sigmoid(x):
     x = np.asarray(x, dtype=np.float64)
