@@ -23,7 +23,7 @@ QSA_BF16 = 1
 # every symbol include/qsa.h declares
 EXPORTED = [
     "qsa_status_string", "qsa_last_error", "qsa_version", "qsa_kernel_launch_count",
-    "qsa_set_stage_events",
+    "qsa_set_stage_events", "qsa_set_keys_visited",
     "qsa_prefill_workspace_size", "qsa_prefill", "qsa_select",
     "qsa_decode_workspace_size", "qsa_decode", "qsa_select_decode",
     "qsa_pool_build", "qsa_decode_noalloc", "qsa_decode_paged", "qsa_pool_build_paged",
@@ -72,6 +72,7 @@ def _declare(lib):
         "qsa_version": (I, []),
         "qsa_kernel_launch_count": (ctypes.c_ulonglong, []),
         "qsa_set_stage_events": (I, [ctypes.POINTER(ctypes.c_void_p), I]),
+        "qsa_set_keys_visited": (None, [P]),
         "qsa_prefill_workspace_size": (SZ, [CFG, I, I, I]),
         "qsa_prefill": (I, [CFG, I, I, I, P, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]),
         "qsa_select": (I, [CFG, I, I, I, P, P, P, P, P, P, P, P, P, SZ, P]),

@@ -58,6 +58,18 @@ class QSAConfig:
                                int(self.rope_dim), float(self.rope_theta))
 
 
+def set_keys_visited(counter: Optional[torch.Tensor]) -> None:
+    """Debug counter of visited keys for this host thread (qsa_set_keys_visited):
+    counter is a one-element int64 CUDA tensor the caller zeroes; the attention
+    kernels of later calls add the (query, head, key) triples they attend over.
+    None turns it off."""
+    if counter is not None:
+        if not (isinstance(counter, torch.Tensor) and counter.is_cuda and
+                counter.dtype == torch.int64 and counter.numel() == 1):
+            raise ValueError("counter must be a one-element int64 CUDA tensor")
+    _lib.lib().qsa_set_keys_visited(None if counter is None else ctypes.c_void_p(counter.data_ptr()))
+
+
 def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 

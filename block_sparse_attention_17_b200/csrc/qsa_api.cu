@@ -74,6 +74,7 @@ void stage_mark(int i, cudaStream_t st) {
 }
 
 thread_local char g_err[512] = "";
+thread_local unsigned long long* g_keys_visited = nullptr;   // see qsa_set_keys_visited()
 
 qsa_status fail(qsa_status s, const char* fmt, ...) {
   va_list ap;
@@ -147,6 +148,7 @@ Geom make_geom(const qsa_config* c) {
   g.gate_headwise = c->gate_headwise ? 1 : 0;
   g.rope_dim = c->rope_dim;
   g.rope_theta = c->rope_dim > 0 ? c->rope_theta : 0.f;
+  g.keys_visited = g_keys_visited;
   return g;
 }
 
@@ -295,6 +297,8 @@ const char* qsa_last_error(void) { return g_err; }
 int qsa_version(void) { return 101; }
 
 unsigned long long qsa_kernel_launch_count(void) { return g_launches.load(); }
+
+void qsa_set_keys_visited(unsigned long long* counter) { g_keys_visited = counter; }
 
 qsa_status qsa_set_stage_events(void* const* events, int count) {
   if (count < 0 || count > 4 || (count > 0 && !events))

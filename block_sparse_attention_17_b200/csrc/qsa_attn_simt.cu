@@ -45,10 +45,12 @@ template <> __device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bflo
 template <typename T, int D, int kMaxOwn>
 struct SimtAttn {
   float acc[kMaxOwn];
+  unsigned visited;   // debug count: (row, key) pairs this thread's key slots let through
 
   __device__ void init() {
 #pragma unroll
     for (int i = 0; i < kMaxOwn; ++i) acc[i] = 0.f;
+    visited = 0;
   }
 
   // rowmask_s[r]: bit e of the chunk-entry visibility is handled by the caller
@@ -62,7 +64,11 @@ struct SimtAttn {
     // -1), so unselected rows cannot leak into the result even through 0 * NaN.
     if (tid < cnt) {
       bool seen = false;
-      for (int r = 0; r < R; ++r) seen |= vis(r, tid);
+      for (int r = 0; r < R; ++r) {
+        const bool v = vis(r, tid);
+        seen |= v;
+        visited += v ? 1u : 0u;
+      }
       if (seen) {
         const T* krow = kbase + (size_t)pos_s[tid] * kv_row_stride;
         float dots[32];
@@ -198,6 +204,7 @@ attn_prefill_simt_kernel(Geom g, const int* __restrict__ cu, const T* __restrict
     core.chunk(G, q_s, lg_s, m_s, l_s, alpha_s, pos_s, cnt, kbase, vbase, kv_stride,
                [](int, int) { return true; });
   }
+  if (g.keys_visited) add_keys_visited(g.keys_visited, core.visited);
 
   constexpr int kRowsPerPass = kChunkKeys / D;
   const int d = tid % D, r0 = tid / D;
@@ -305,6 +312,7 @@ attn_decode_simt_kernel(Geom g, int n_q, int cap, int nsplit, int per_split,
                  });
     }
   }
+  if (g.keys_visited) add_keys_visited(g.keys_visited, core.visited);
   constexpr int kRowsPerPass = kChunkKeys / D;
   const int d = tid % D, r0 = tid / D;
 #pragma unroll

@@ -329,6 +329,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
     };
     uint32_t wn = 0u;
     int bn = -1;
+    unsigned visited = 0;   // debug count of the row's visible keys in these columns
     if (ok) fetch(0, wn, bn);
     for (int j = 0; ok && j < n_iter; ++j) {
       // visible keys among this thread's 64 columns: all of a selected
@@ -338,6 +339,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
         const int col0 = bn * kB + (kB == 128 ? 64 * hf : 0);   // position of column 0
         lim = max(0, min(64, pos + 1 - col0));
       }
+      visited += lim;
       if (j + 1 < n_iter) fetch(j + 1, wn, bn);
       const bool any_vis = __any_sync(kFull, lim > 0);
       const bool partial = __any_sync(kFull, lim > 0 && lim < 64);
@@ -430,6 +432,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
       mbar_arrive(&p_full[t]);
       m_used = m_tgt;
     }
+    if (g.keys_visited) add_keys_visited(g.keys_visited, visited);
     // ------------------------------------------------------------ epilogue
     // each thread writes its 64 output dims; l is the sum of both halves
     if (ok && n_iter > 0 &&

@@ -16,7 +16,7 @@ constexpr int kMaxTopK = 64;          // budget / block_size
 constexpr int kMaxBlocksPerSeq = 4096;        // prefill
 constexpr int kMaxDecodeBlocksPerSeq = 16384; // decode cache blocks (cap / B)
 
-// Geometry passed by value to every kernel.
+// Geometry (and the per-call debug counter) passed by value to every kernel.
 struct Geom {
   int Hq, Hkv, G, D;
   int Hi, di;
@@ -26,7 +26,15 @@ struct Geom {
   int gate_headwise;
   int rope_dim;         // indexer rotary embedding: dims rotated (0 = none)
   float rope_theta;
+  unsigned long long* keys_visited;   // debug: (query, head, key) triples attended, or null
 };
+
+// Adds a warp's per-lane counts to the visited-keys counter (every lane calls it).
+__device__ __forceinline__ void add_keys_visited(unsigned long long* ctr, unsigned v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if ((threadIdx.x & 31) == 0 && v) atomicAdd(ctr, (unsigned long long)v);
+}
 
 template <typename T> __device__ __forceinline__ float to_f32(T x);
 template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }

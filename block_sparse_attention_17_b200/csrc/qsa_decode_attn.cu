@@ -671,7 +671,7 @@ __device__ __forceinline__ void select_in_cluster(const DecParams& P, uint8_t* s
   cluster_arrive_all();   // this CTA has read the other CTAs' candidates
 }
 
-template <bool kFp8, int kSelDI, int kRT>
+template <bool kFp8, int kSelDI, int kRT, bool kCount>
 __global__ void __launch_bounds__(kThreads, kRT == 1 ? 2 : 1)
 attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const DecParams P) {
@@ -760,6 +760,7 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
   uint64_t* empty = full + kStages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc);
   int* n_chunks_s = reinterpret_cast<int*>(smem + L::kOffMisc + 4);
+  unsigned* visited_s = reinterpret_cast<unsigned*>(smem + L::kOffMisc + 8);   // debug, [kConsumers]
   int* u_blk = reinterpret_cast<int*>(smem + L::kOffUnion);
   int* u_qm = u_blk + kMaxUnion;
   const int cpb = g.B / kChunk;   // chunks per block
@@ -776,6 +777,8 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
       mbar_init(&empty[s], kConsumers);
     }
     *abort_flag = 0;
+    if constexpr (kCount)
+      for (int w = 0; w < kConsumers; ++w) visited_s[w] = 0u;
     fence_barrier_init();
     fence_proxy_async();
   }
@@ -1077,6 +1080,10 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
         lim[h2] = (qrow[h2] >= 0 && ((qm >> qrow[h2]) & 1))
                       ? max(0, min(kChunk, qpos[h2] + 1 - key0))
                       : 0;
+      if (kCount && tq == 0)   // debug count of the visible (row, key) pairs of this
+                               // warp's keys (a quad's threads share two rows)
+        atomicAdd(reinterpret_cast<unsigned*>(smem + L::kOffMisc + 8) + warp, (unsigned)(min(kKW, max(0, lim[0] - kw0)) +
+                                               min(kKW, max(0, lim[1] - kw0))));
       // S = Q K^T for the warp's keys [kw0, kw0 + kKW): kNT n-tiles of 8 keys
       float sfr[kNT][4];
 #pragma unroll
@@ -1230,6 +1237,9 @@ attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK,
       sm[(warp * 16 + gq + 8) * 2 + 1] = l[1];
     }
     named_bar_sync(1, 32 * kConsumers);
+    if (kCount && threadIdx.x == 0)   // (every consumer warp's count is complete)
+      atomicAdd(g.keys_visited, (unsigned long long)visited_s[0] + visited_s[1] + visited_s[2] +
+                                    visited_s[3]);
     // thread t of the 128 consumers: rows t / 8 + 16 u (u < kRT), dims [16 (t % 8), + 16)
     const int t = threadIdx.x;
     const int d0 = (t & 7) * 16;
@@ -1594,18 +1604,30 @@ bool fused_layout(const Geom& g, int n_q, int cap, int nsplit, DecParams* p) {
   return off <= (long long)kStages * kStageBytes;
 }
 
-template <bool kFp8>
-const void* fused_kernel(int di, int rt) {
+// The kernel for (fp8, indexer dim, row tiles); kCount: the instantiation that
+// adds to the visited-keys debug counter (the others carry no counting code).
+template <bool kFp8, bool kCount>
+const void* fused_kernel_c(int di, int rt) {
   if constexpr (kFp8) {
-    return di == 64 ? reinterpret_cast<const void*>(attn_decode_mma_kernel<true, 64, 1>)
-                    : reinterpret_cast<const void*>(attn_decode_mma_kernel<true, 32, 1>);
+    return di == 64 ? reinterpret_cast<const void*>(attn_decode_mma_kernel<true, 64, 1, kCount>)
+                    : reinterpret_cast<const void*>(attn_decode_mma_kernel<true, 32, 1, kCount>);
   } else {
     if (rt == 2)
-      return di == 64 ? reinterpret_cast<const void*>(attn_decode_mma_kernel<false, 64, 2>)
-                      : reinterpret_cast<const void*>(attn_decode_mma_kernel<false, 32, 2>);
-    return di == 64 ? reinterpret_cast<const void*>(attn_decode_mma_kernel<false, 64, 1>)
-                    : reinterpret_cast<const void*>(attn_decode_mma_kernel<false, 32, 1>);
+      return di == 64 ? reinterpret_cast<const void*>(attn_decode_mma_kernel<false, 64, 2, kCount>)
+                      : reinterpret_cast<const void*>(attn_decode_mma_kernel<false, 32, 2, kCount>);
+    return di == 64 ? reinterpret_cast<const void*>(attn_decode_mma_kernel<false, 64, 1, kCount>)
+                    : reinterpret_cast<const void*>(attn_decode_mma_kernel<false, 32, 1, kCount>);
   }
+}
+template <bool kFp8>
+const void* fused_kernel(const Geom& g, int rt) {
+  return g.keys_visited ? fused_kernel_c<kFp8, true>(g.di, rt) : fused_kernel_c<kFp8, false>(g.di, rt);
+}
+template <bool kCount>
+const void* attend_kernel(bool fp8, int rt) {
+  return fp8 ? reinterpret_cast<const void*>(attn_decode_mma_kernel<true, 0, 1, kCount>)
+         : rt == 2 ? reinterpret_cast<const void*>(attn_decode_mma_kernel<false, 0, 2, kCount>)
+                   : reinterpret_cast<const void*>(attn_decode_mma_kernel<false, 0, 1, kCount>);
 }
 
 int decode_smem(const Geom& g, int n_q, int cap) {
@@ -1692,10 +1714,8 @@ cudaError_t launch_attn_decode_mma(const Geom& g, int batch, int n_q, int cap, i
   p.counter = counter;
   p.ready = ready;
   const int smem = decode_smem(g, n_q, cap);
-  const void* kern =
-      f8.on ? reinterpret_cast<const void*>(attn_decode_mma_kernel<true, 0, 1>)
-      : row_tiles(g, n_q) == 2 ? reinterpret_cast<const void*>(attn_decode_mma_kernel<false, 0, 2>)
-                               : reinterpret_cast<const void*>(attn_decode_mma_kernel<false, 0, 1>);
+  const void* kern = g.keys_visited ? attend_kernel<true>(f8.on, row_tiles(g, n_q))
+                                    : attend_kernel<false>(f8.on, row_tiles(g, n_q));
   cudaError_t e = set_max_dynamic_smem(kern, smem);
   if (e != cudaSuccess) return e;
   p.cluster = nsplit > 1 && cluster_fits(kern, nsplit, smem) ? 1 : 0;
@@ -1709,7 +1729,7 @@ bool decode_fused_supported(const Geom& g, int n_q, int cap, int nsplit, bool fp
   if (g.Hi < 1 || g.Hi > 32 || (32 % g.Hi) != 0) return false;
   DecParams p = {};
   if (!fused_layout(g, n_q, cap, nsplit, &p)) return false;
-  const void* kern = fp8 ? fused_kernel<true>(g.di, 1) : fused_kernel<false>(g.di, row_tiles(g, n_q));
+  const void* kern = fp8 ? fused_kernel<true>(g, 1) : fused_kernel<false>(g, row_tiles(g, n_q));
   const int smem = decode_smem(g, n_q, cap);
   if (set_max_dynamic_smem(kern, smem) != cudaSuccess) {
     cudaGetLastError();
@@ -1737,7 +1757,7 @@ cudaError_t launch_decode_fused(const Geom& g, int batch, int n_q, int cap, int 
   p.nsel_w = si.nsel;
   const int smem = decode_smem(g, n_q, cap);
   const void* kern =
-      f8.on ? fused_kernel<true>(g.di, 1) : fused_kernel<false>(g.di, row_tiles(g, n_q));
+      f8.on ? fused_kernel<true>(g, 1) : fused_kernel<false>(g, row_tiles(g, n_q));
   const cudaError_t e = set_max_dynamic_smem(kern, smem);
   if (e != cudaSuccess) return e;
   return launch_decode_kernel(kern, dim3(nsplit, batch, g.Hkv), smem, nsplit, st, mk, mv, p);

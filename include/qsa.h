@@ -111,6 +111,18 @@ unsigned long long qsa_kernel_launch_count(void);
  * Returns QSA_ERR_INVALID_ARG for count outside [0, 4]. */
 qsa_status qsa_set_stage_events(void* const* events, int count);
 
+/* Debug counter of visited keys for the calling host thread (the keys_visited
+ * count of the llama.cpp PR #27739 page's QSA commit text, 16400 sparse against
+ * 24016 dense in its worked example). With counter != NULL (device memory, 8
+ * bytes, owned and zeroed by the caller) the attention kernels of later
+ * qsa_prefill / qsa_decode* / qsa_decode_attend / qsa_cp_attend calls on this
+ * thread add to *counter the number of (query, head, key) triples they attend
+ * over, counted where each kernel decides which keys a row sees: for a correct
+ * sparse consumer that is sum over queries of Hq * (min(k, nc) * B + tail),
+ * whatever extra work the kernel's tiles execute. NULL turns it off (the
+ * default; the counting adds one register and one atomic per warp). */
+void qsa_set_keys_visited(unsigned long long* counter);
+
 /* ---------------------------------------------------------------- prefill --
  * Packed variable-length prefill. Sequence b owns tokens
  * [cu_seqlens[b], cu_seqlens[b+1]); query token t at position p of its
