@@ -563,6 +563,17 @@ def gpu_leg(args, w, inp, steps, warmup, dist, dev, kv_format="bf16", paged=Fals
         step()
     torch.cuda.synchronize()
 
+    # the visited-keys debug counter over one more eager step, outside the timed
+    # region: the (query, head, key) triples the attention kernels attended over
+    ctr = torch.zeros(1, dtype=torch.int64, device=dev)
+    qsa.set_keys_visited(ctr)
+    try:
+        step()
+    finally:
+        qsa.set_keys_visited(None)
+    torch.cuda.synchronize()
+    res["keys_visited"] = int(ctr.item())
+
     def timed(run_once, stages):
         """Time the steps, each bracketed by CUDA events on the launching
         stream, with the L2 flush outside the events; returns per-step ms and,
@@ -690,9 +701,15 @@ def assemble(w, r, units, steps, dist, dev, peaks, peak_kind, kernel_file, kerne
               "median_ms_per_step": float(np.median(r["step_ms"])),
               "eager_median_ms_per_step": float(np.median(r["eager_ms"])),
               "selected_kv_tokens_per_step": units, "job_selected_kv_tokens_per_step": job_units}
+    ns = workload_units(w)[1]
+    visited = {"counted": r["keys_visited"], "expected": w.num_q_heads * units,
+               "dense": w.num_q_heads * int(sum(ns)),
+               "note": "one step with qsa_set_keys_visited on: (query, head, key) triples "
+                       "attended; expected = Hq * sum(min(k, nc) * B + tail), dense = Hq * "
+                       "sum(visible tokens)"}
     return {"value": value, "ms_per_step": total_ms / steps, "roofline": roof, "e2e": e2e,
             "clocks": r["clocks"], "gpu_launches": r["launches"], "cpu_baseline": cpu,
-            "selection_vs_oracle": agreement, "timing": timing}
+            "selection_vs_oracle": agreement, "keys_visited": visited, "timing": timing}
 
 
 def index_fn(w):
@@ -782,7 +799,8 @@ def run_ours(args, rank, world, dist):
             "dtype": w.dtype, "data": "synthetic (seeded numpy draws, shapes of the workload)",
             "config": cfg, "roofline": head["roofline"], "cpu_baseline": head["cpu_baseline"],
             "e2e": head["e2e"], "gpu_launches": head["gpu_launches"], "clocks": head["clocks"],
-            "selection_vs_oracle": head["selection_vs_oracle"], "timing": head["timing"],
+            "selection_vs_oracle": head["selection_vs_oracle"],
+            "keys_visited": head["keys_visited"], "timing": head["timing"],
             "shards": "one per rank: the workload's shapes, seed + 7919 * rank",
             "input_gen_s": gen_s[w.name], "impl": "ours"}
     if decode_objs:

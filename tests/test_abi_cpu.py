@@ -241,3 +241,12 @@ def test_append_rejects_bad_arguments():
     # an empty batch launches nothing
     assert lib.qsa_append(ctypes.byref(c), 0, 1, 4096, None, None, None, None, None, None, None,
                           None, None, 0, None, None) == _lib.QSA_OK
+
+
+def test_keys_visited_binding_refuses_bad_counters():
+    import block_sparse_attention_17_b200 as qsa
+    for bad in (torch.zeros(1, dtype=torch.int64), torch.zeros(2, dtype=torch.int64),
+                torch.zeros(1, dtype=torch.float32), 7):
+        with pytest.raises(ValueError):
+            qsa.set_keys_visited(bad)
+    qsa.set_keys_visited(None)   # off: no device needed
