@@ -82,6 +82,8 @@ def code_sha(text: str) -> str:
 def recorded_traffic(kernel_file: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
     the kernel code as it is now (code_sha prefix match); else None."""
+    if kernel_file is None:
+        return None
     src = os.path.join(ROOT, "block_sparse_attention_17_b200", "csrc", kernel_file)
     table = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not (os.path.exists(src) and os.path.exists(table)):
@@ -777,8 +779,9 @@ def run_ours(args, rank, world, dist):
                      dev, kv_format=args.kv, paged=args.paged)
         agree_d = (selection_agreement(wd, oracle_sel[wd.name], rd["sel"], rd["nsel"],
                                        index_fn(wd)) if wd.name in oracle_sel else None)
+        # (the recorded DRAM counters are those of the contiguous bf16 caches)
         obj = assemble(wd, rd, units_d, args.decode_steps, dist, dev, peaks, peak_kind,
-                       "qsa_decode_attn.cu",
+                       "qsa_decode_attn.cu" if args.kv == "bf16" and not args.paged else None,
                        "qsa decode step (selection + attention + merge, one kernel)",
                        cpu.get(wd.name), agree_d,
                        {"selected_kv_bytes": rd["alg"]["selected_kv_bytes"]})
