@@ -15,6 +15,21 @@
 
 #include "qsa_common.cuh"
 #include "qsa_kernels.h"
+#include <nvtx3/nvToolsExt.h>
+
+// An NVTX range over one library call or one of its stages (shown by Nsight
+// Systems and usable as an ncu filter; a no-op unless a tool is attached).
+namespace {
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+}  // namespace
+#define QSA_NVTX_CAT2(a, b) a##b
+#define QSA_NVTX_CAT(a, b) QSA_NVTX_CAT2(a, b)
+#define QSA_NVTX(name) NvtxRange QSA_NVTX_CAT(qsa_nvtx_range_, __LINE__)(name)
 
 using namespace qsa;
 
@@ -337,6 +352,7 @@ qsa_status qsa_prefill(const qsa_config* cfg, int batch, int total_tokens, int m
                        const void* iq, const void* ik, const float* iw, const void* gate,
                        void* out, float* lse, int32_t* sel, int32_t* nsel, float* pooled_out,
                        void* workspace, size_t workspace_bytes, void* stream) {
+  QSA_NVTX("qsa_prefill");
   g_err[0] = 0;
   qsa_status s = check_prefill_dims(cfg, batch, total_tokens, max_seqlen);
   if (s != QSA_OK) return s;
@@ -359,10 +375,14 @@ qsa_status qsa_prefill(const qsa_config* cfg, int batch, int total_tokens, int m
   int* sel_p = sel ? sel : w.sel;
   int* nsel_p = nsel ? nsel : w.nsel;
   stage_mark(0, st);
-  s = prefill_select_common(cfg, g, batch, total_tokens, max_seqlen, cu_seqlens, iq, ik, iw, w,
-                            pooled, sel_p, nsel_p, nullptr, st);
+  {
+    QSA_NVTX("pool + select");
+    s = prefill_select_common(cfg, g, batch, total_tokens, max_seqlen, cu_seqlens, iq, ik, iw, w,
+                              pooled, sel_p, nsel_p, nullptr, st);
+  }
   if (s != QSA_OK) return s;
   stage_mark(1, st);
+  QSA_NVTX("attention");
   if (cfg->dtype == QSA_BF16 && attn_prefill_tc_supported(g)) {
     const int max_nblk = (max_seqlen + g.B - 1) / g.B;
     QSA_CUDA(launch_attn_prefill_tc(g, cu_seqlens, batch, total_tokens, max_seqlen,
@@ -382,6 +402,7 @@ qsa_status qsa_select(const qsa_config* cfg, int batch, int total_tokens, int ma
                       const int32_t* cu_seqlens, const void* iq, const void* ik, const float* iw,
                       int32_t* sel, int32_t* nsel, float* scores, float* pooled_out,
                       void* workspace, size_t workspace_bytes, void* stream) {
+  QSA_NVTX("qsa_select");
   g_err[0] = 0;
   qsa_status s = check_prefill_dims(cfg, batch, total_tokens, max_seqlen);
   if (s != QSA_OK) return s;
@@ -491,6 +512,7 @@ qsa_status qsa_decode(const qsa_config* cfg, int batch, int n_q, int cap, const 
                       const void* ik_cache, const float* iw, const void* gate,
                       float* pooled_cache, void* out, float* lse, int32_t* sel, int32_t* nsel,
                       int32_t* dev_err, void* workspace, size_t workspace_bytes, void* stream) {
+  QSA_NVTX("qsa_decode");
   g_err[0] = 0;
   return decode_impl(cfg, batch, n_q, cap, kv_len, q, k_cache, v_cache, iq, ik_cache, iw, gate,
                      pooled_cache, out, lse, sel, nsel, dev_err, workspace, workspace_bytes,
@@ -504,6 +526,7 @@ qsa_status qsa_decode_fp8(const qsa_config* cfg, int batch, int n_q, int cap,
                           const void* gate, float* pooled_cache, void* out, float* lse,
                           int32_t* sel, int32_t* nsel, int32_t* dev_err, void* workspace,
                           size_t workspace_bytes, void* stream) {
+  QSA_NVTX("qsa_decode_fp8");
   g_err[0] = 0;
   qsa_status s = check_cfg(cfg);
   if (s != QSA_OK) return s;
@@ -529,6 +552,7 @@ qsa_status qsa_decode_attend(const qsa_config* cfg, int batch, int n_q, int cap,
                              const void* v_cache, const void* gate, const int32_t* sel,
                              const int32_t* nsel, void* out, float* lse, int32_t* dev_err,
                              void* workspace, size_t workspace_bytes, void* stream) {
+  QSA_NVTX("qsa_decode_attend");
   g_err[0] = 0;
   qsa_status s = check_decode_dims(cfg, batch, n_q, cap);
   if (s != QSA_OK) return s;
@@ -576,6 +600,7 @@ static qsa_status check_shard(const qsa_config* cfg, int batch, int n_q, int cap
 qsa_status qsa_cp_pool_build(const qsa_config* cfg, int batch, int cap, int block_lo,
                              const int32_t* kv_len, const void* ik_shard, float* pooled_shard,
                              int32_t* dev_err, void* stream) {
+  QSA_NVTX("qsa_cp_pool_build");
   g_err[0] = 0;
   qsa_status s = check_shard(cfg, batch, 1, cap, block_lo);
   if (s != QSA_OK) return s;
@@ -594,6 +619,7 @@ qsa_status qsa_cp_select(const qsa_config* cfg, int batch, int n_q, int cap, int
                          const float* iw, float* pooled_shard, float* cand_score,
                          int32_t* cand_id, int32_t* dev_err, void* workspace,
                          size_t workspace_bytes, void* stream) {
+  QSA_NVTX("qsa_cp_select");
   g_err[0] = 0;
   qsa_status s = check_shard(cfg, batch, n_q, cap, block_lo);
   if (s != QSA_OK) return s;
@@ -627,6 +653,7 @@ qsa_status qsa_cp_global_topk(const qsa_config* cfg, int batch, int n_q, int wor
                               const int32_t* kv_len, const float* cand_score,
                               const int32_t* cand_id, int32_t* sel, int32_t* nsel,
                               void* stream) {
+  QSA_NVTX("qsa_cp_global_topk");
   g_err[0] = 0;
   qsa_status s = check_cfg(cfg);
   if (s != QSA_OK) return s;
@@ -652,6 +679,7 @@ qsa_status qsa_cp_attend(const qsa_config* cfg, int batch, int n_q, int cap, int
                          const int32_t* nsel, float* part_out, float* part_lse,
                          int32_t* dev_err, void* workspace, size_t workspace_bytes,
                          void* stream) {
+  QSA_NVTX("qsa_cp_attend");
   g_err[0] = 0;
   qsa_status s = check_shard(cfg, batch, n_q, cap, block_lo);
   if (s != QSA_OK) return s;
@@ -691,6 +719,7 @@ qsa_status qsa_cp_attend(const qsa_config* cfg, int batch, int n_q, int cap, int
 qsa_status qsa_cp_merge(const qsa_config* cfg, int batch, int n_q, int world,
                         const float* part_out, const float* part_lse, void* out, float* lse,
                         void* stream) {
+  QSA_NVTX("qsa_cp_merge");
   g_err[0] = 0;
   qsa_status s = check_cfg(cfg);
   if (s != QSA_OK) return s;
@@ -722,6 +751,7 @@ qsa_status qsa_append(const qsa_config* cfg, int batch, int n_q, int cap, const 
                       const void* k_new, const void* v_new, const void* ik_new, void* k_cache,
                       void* v_cache, void* ik_cache, float* pooled_cache,
                       const int32_t* block_table, int num_pages, int32_t* dev_err, void* stream) {
+  QSA_NVTX("qsa_append");
   g_err[0] = 0;
   qsa_status s = check_decode_dims(cfg, batch, n_q, cap);
   if (s != QSA_OK) return s;
@@ -753,6 +783,7 @@ qsa_status qsa_decode_paged(const qsa_config* cfg, int batch, int n_q, int max_b
                             const void* gate, float* pooled_cache, void* out, float* lse,
                             int32_t* sel, int32_t* nsel, int32_t* dev_err, void* workspace,
                             size_t workspace_bytes, void* stream) {
+  QSA_NVTX("qsa_decode_paged");
   g_err[0] = 0;
   qsa_status s = check_cfg(cfg);
   if (s != QSA_OK) return s;
@@ -771,6 +802,7 @@ qsa_status qsa_select_decode(const qsa_config* cfg, int batch, int n_q, int cap,
                              const float* iw, float* pooled_cache, int32_t* sel, int32_t* nsel,
                              float* scores, int32_t* dev_err, void* workspace,
                              size_t workspace_bytes, void* stream) {
+  QSA_NVTX("qsa_select_decode");
   g_err[0] = 0;
   qsa_status s = check_decode_dims(cfg, batch, n_q, cap);
   if (s != QSA_OK) return s;
@@ -792,6 +824,7 @@ qsa_status qsa_select_decode(const qsa_config* cfg, int batch, int n_q, int cap,
 qsa_status qsa_pool_build(const qsa_config* cfg, int batch, int cap, const int32_t* kv_len,
                           const void* ik_cache, float* pooled_cache, int32_t* dev_err,
                           void* stream) {
+  QSA_NVTX("qsa_pool_build");
   g_err[0] = 0;
   qsa_status s = check_decode_dims(cfg, batch, 1, cap);
   if (s != QSA_OK) return s;
@@ -809,6 +842,7 @@ qsa_status qsa_pool_build_paged(const qsa_config* cfg, int batch, int max_blocks
                                 const int32_t* block_table, int num_pages,
                                 const int32_t* kv_len, const void* ik_pages,
                                 float* pooled_cache, int32_t* dev_err, void* stream) {
+  QSA_NVTX("qsa_pool_build_paged");
   g_err[0] = 0;
   qsa_status s = check_cfg(cfg);
   if (s != QSA_OK) return s;
