@@ -120,7 +120,9 @@ qsa_status qsa_set_stage_events(void* const* events, int count);
  * over, counted where each kernel decides which keys a row sees: for a correct
  * sparse consumer that is sum over queries of Hq * (min(k, nc) * B + tail),
  * whatever extra work the kernel's tiles execute. NULL turns it off (the
- * default; the counting adds one register and one atomic per warp). */
+ * default; the counting adds one register and one atomic per warp). The
+ * pointer is baked into the launches: a CUDA graph captured while it is set
+ * keeps adding to it on every replay. */
 void qsa_set_keys_visited(unsigned long long* counter);
 
 /* ---------------------------------------------------------------- prefill --
