@@ -349,24 +349,25 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
       }
       tc_fence_after();
       float pm = -INFINITY;
-      {
-        uint32_t v[64];
-        tmem_ld32(tS + 64 * hf, v);
-        tmem_ld32(tS + 64 * hf + 32, v + 32);
-        tmem_wait_ld();
-        if (any_vis) {
+      if (any_vis) {   // (warp-uniform: the TMEM loads are warp-collective)
+        // the thread's 64 S columns in two halves of 32 (register pressure)
+        float cm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t v[32];
+          tmem_ld32(tS + 64 * hf + 32 * half, v);
+          tmem_wait_ld();
           if (partial) {
 #pragma unroll
-            for (int i = 0; i < 64; ++i)
-              if (i >= lim) v[i] = __float_as_uint(-INFINITY);
+            for (int i = 0; i < 32; ++i)
+              if (32 * half + i >= lim) v[i] = __float_as_uint(-INFINITY);
           }
-          float cm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-          for (int i = 0; i < 64; i += 2)
+          for (int i = 0; i < 32; i += 2)
             cm[(i >> 1) & 3] =
                 fmax3(cm[(i >> 1) & 3], __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
-          pm = lim > 0 ? fmax3(cm[0], cm[1], fmaxf(cm[2], cm[3])) : -INFINITY;
         }
+        pm = lim > 0 ? fmax3(cm[0], cm[1], fmaxf(cm[2], cm[3])) : -INFINITY;
       }
       if (!exchange(j, pm)) {
         ok = false;
@@ -382,34 +383,40 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
       // P of this half is packed over the first 32 of its own 64 S columns,
       // so the two halves never touch each other's S
       float2 s2a = make_float2(0.f, 0.f), s2b = make_float2(0.f, 0.f);
-      uint32_t v[64];
       if (!any_vis) {
+        uint32_t z[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = 0u;
+        for (int i = 0; i < 32; ++i) z[i] = 0u;
+        tmem_st32(tS + 64 * hf, z);
       } else {
-        tmem_ld32(tS + 64 * hf, v);
-        tmem_ld32(tS + 64 * hf + 32, v + 32);
-        tmem_wait_ld();
-        if (partial) {
-#pragma unroll
-          for (int i = 0; i < 64; ++i)
-            if (i >= lim) v[i] = __float_as_uint(-INFINITY);
-        }
         // rows that do not see these columns subtract +inf: exp2(-inf) = 0
         const float nref = lim > 0 ? -ref : -INFINITY;
         const float2 sc2 = make_float2(sc, sc), nref2 = make_float2(nref, nref);
+        // in two halves of 32 columns: half h's P pairs land in packed columns
+        // 16 h .. 16 h + 15, whose S was read by half 0 already
 #pragma unroll
-        for (int i = 0; i < 64; i += 2) {
-          const float2 x = ffma2(make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])),
-                                 sc2, nref2);
-          const float2 pp = ((i >> 1) & 7) < kPolyPairsOf8
-                                ? exp2_poly2(x)
-                                : make_float2(ex2_approx(x.x), ex2_approx(x.y));
-          if ((i & 2) == 0) s2a = fadd2(s2a, pp); else s2b = fadd2(s2b, pp);
-          v[i >> 1] = pack_bf16(pp.x, pp.y);   // pair i/2 lands at index i/2 <= i
+        for (int half = 0; half < 2; ++half) {
+          uint32_t v[32], pk[16];
+          tmem_ld32(tS + 64 * hf + 32 * half, v);
+          tmem_wait_ld();
+          if (partial) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (32 * half + i >= lim) v[i] = __float_as_uint(-INFINITY);
+          }
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            const float2 x = ffma2(make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])),
+                                   sc2, nref2);
+            const float2 pp = ((i >> 1) & 7) < kPolyPairsOf8
+                                  ? exp2_poly2(x)
+                                  : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            if ((i & 2) == 0) s2a = fadd2(s2a, pp); else s2b = fadd2(s2b, pp);
+            pk[i >> 1] = pack_bf16(pp.x, pp.y);
+          }
+          tmem_st16(tS + 64 * hf + 16 * half, pk);
         }
       }
-      tmem_st32(tS + 64 * hf, v);
       l = l * alpha + ((s2a.x + s2a.y) + (s2b.x + s2b.y));
       if (j > 0 && __any_sync(kFull, alpha != 1.f)) {
         if (!__all_sync(kFull, mbar_wait(&o_done[t], (j - 1) & 1, abort_flag))) {
