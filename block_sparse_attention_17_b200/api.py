@@ -9,6 +9,7 @@ from __future__ import annotations
 
 import ctypes
 import math
+import threading
 from dataclasses import dataclass
 from typing import Optional
 
@@ -58,16 +59,21 @@ class QSAConfig:
                                int(self.rope_dim), float(self.rope_theta))
 
 
+_thread = threading.local()   # this host thread's visited-keys counter (its device)
+
+
 def set_keys_visited(counter: Optional[torch.Tensor]) -> None:
     """Debug counter of visited keys for this host thread (qsa_set_keys_visited):
     counter is a one-element int64 CUDA tensor the caller zeroes; the attention
     kernels of later calls add the (query, head, key) triples they attend over.
-    None turns it off."""
+    Calls on another GPU than the counter's are refused while it is set. None
+    turns it off."""
     if counter is not None:
         if not (isinstance(counter, torch.Tensor) and counter.is_cuda and
                 counter.dtype == torch.int64 and counter.numel() == 1):
             raise ValueError("counter must be a one-element int64 CUDA tensor")
     _lib.lib().qsa_set_keys_visited(None if counter is None else ctypes.c_void_p(counter.data_ptr()))
+    _thread.keys_visited_device = None if counter is None else counter.device
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -102,6 +108,9 @@ def _one_device(dev, stream=None, **tensors):
                              "call must be on the same GPU")
     if stream is not None and stream.device != dev:
         raise ValueError(f"stream is on {stream.device}, expected {dev}")
+    kvd = getattr(_thread, "keys_visited_device", None)
+    if kvd is not None and kvd != dev:
+        raise ValueError(f"the visited-keys counter is on {kvd}, the call on {dev}")
 
 
 def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]):

@@ -122,7 +122,8 @@ qsa_status qsa_set_stage_events(void* const* events, int count);
  * whatever extra work the kernel's tiles execute. NULL turns it off (the
  * default; the counting adds one register and one atomic per warp). The
  * pointer is baked into the launches: a CUDA graph captured while it is set
- * keeps adding to it on every replay. */
+ * keeps adding to it on every replay. The counter must be memory of the GPU
+ * the calls run on. */
 void qsa_set_keys_visited(unsigned long long* counter);
 
 /* ---------------------------------------------------------------- prefill --
