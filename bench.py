@@ -640,8 +640,46 @@ def gpu_leg(args, w, inp, steps, warmup, dist, dev, kv_format="bf16", paged=Fals
                graph=graph is not None)
 
     # end to end through the public API: pinned host inputs -> device, the
-    # call, result -> host, all inside the timed region
-    if not args.no_e2e:
+    # call, result -> host, all inside the timed region. A decode step's inputs
+    # (the query-side tensors and the new K, V and indexer-key rows) travel as
+    # one packed pinned buffer, one copy; qsa_append writes the new rows into the
+    # caches (and pools the block they complete) and qsa_decode runs the step.
+    if not args.no_e2e and w.kind == "decode" and append is not None:
+        out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        pieces = [(n, host[n]) for n in in_names] + \
+                 [(n, hsrc) for n, (_, hsrc, _) in zip(("k_new", "v_new", "ik_new"), append)]
+        offs, total = {}, 0
+        for n, t in pieces:
+            offs[n] = total
+            total += (t.numel() * t.element_size() + 255) // 256 * 256
+        pack_host = torch.empty(total, dtype=torch.uint8, pin_memory=True)
+        for n, t in pieces:
+            nb = t.numel() * t.element_size()
+            pack_host[offs[n]:offs[n] + nb].copy_(t.contiguous().view(-1).view(torch.uint8))
+        pack_dev = torch.empty(total, dtype=torch.uint8, device=dev)
+        dv = {n: pack_dev[offs[n]:offs[n] + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
+              for n, t in pieces}
+        kv_dev = dv["kv_len"]
+        e_st = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        e_en = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        for i in range(steps + 1):
+            flush.zero_()
+            if i > 0:
+                e_st[i - 1].record(stream)
+            pack_dev.copy_(pack_host, non_blocking=True)
+            qsa.append(cfg, dv["ik_new"], d["ik_cache"], pooled, kv_dev, k_new=dv["k_new"],
+                       v_new=dv["v_new"], k_cache=d["k_cache"], v_cache=d["v_cache"])
+            qsa.decode(cfg, dv["q"], d["k_cache"], d["v_cache"], dv["iq"], d["ik_cache"], dv["iw"],
+                       dv["gate"], pooled, kv_dev, out=out, sel=sel, nsel=nsel, workspace=ws)
+            out_host.copy_(out, non_blocking=True)
+            if i > 0:
+                e_en[i - 1].record(stream)
+        torch.cuda.synchronize()
+        res["e2e_ms"] = float(sum(e_st[i].elapsed_time(e_en[i]) for i in range(steps)))
+        res["h2d"], res["d2h"] = int(total), int(out_host.numel() * out_host.element_size())
+        res["e2e_note"] = ("one packed pinned copy of the step's inputs, qsa_append of the new "
+                           "K/V/indexer rows, qsa_decode, the output copied back")
+    elif not args.no_e2e:
         out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
         h2d = sum(host[n].numel() * host[n].element_size() for n in in_names)
         if append:
@@ -697,6 +735,8 @@ def assemble(w, r, units, steps, dist, dev, peaks, peak_kind, kernel_file, kerne
         e2e = {"value": job_units * steps / (e2e_ms / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
                "ms_per_step": e2e_ms / steps}
+        if "e2e_note" in r:
+            e2e["calls"] = r["e2e_note"]
     timing = {"timing": ("CUDA-graph replay of one library call per step" if r["graph"]
                          else "eager library call per step"),
               "eager_ms_per_step": float(np.mean(r["eager_ms"])),
